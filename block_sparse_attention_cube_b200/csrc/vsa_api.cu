@@ -1,0 +1,457 @@
+// C ABI of the library (declared in include/vsa.h): argument checks, error
+// reporting and the orchestration of the kernels of one attention call.
+// Every argument check runs on the host before anything is enqueued.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "vsa_internal.h"
+
+namespace vsa {
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+vsa_status fail(vsa_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+vsa_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(VSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+constexpr int64_t kMaxRows = (int64_t{1} << 31) - 1;
+
+vsa_status make_dims(const vsa_shape* s, Dims* d) {
+    if (!s) return fail(VSA_ERR_INVALID_ARGUMENT, "shape is NULL");
+    if (s->batch < 1 || s->heads < 1 || s->grid_t < 1 || s->grid_h < 1 || s->grid_w < 1)
+        return fail(VSA_ERR_INVALID_ARGUMENT, "batch, heads and grid dims must be >= 1 (got B=%d H=%d grid=%dx%dx%d)",
+                    s->batch, s->heads, s->grid_t, s->grid_h, s->grid_w);
+    if (s->head_dim < 1) return fail(VSA_ERR_INVALID_ARGUMENT, "head_dim must be >= 1 (got %d)", s->head_dim);
+    if (s->head_dim != 64 && s->head_dim != 128)
+        return fail(VSA_ERR_UNSUPPORTED, "head_dim %d is not supported (64 or 128)", s->head_dim);
+    d->B = s->batch;
+    d->H = s->heads;
+    d->D = s->head_dim;
+    d->T = s->grid_t;
+    d->X = s->grid_h;
+    d->Y = s->grid_w;
+    d->Ct = (d->T + kCube - 1) / kCube;
+    d->Cx = (d->X + kCube - 1) / kCube;
+    d->Cy = (d->Y + kCube - 1) / kCube;
+    const int64_t C = static_cast<int64_t>(d->Ct) * d->Cx * d->Cy;
+    if (C > (int64_t{1} << 24)) return fail(VSA_ERR_INVALID_ARGUMENT, "grid too large (%lld cubes)", (long long)C);
+    d->C = static_cast<int>(C);
+    d->N = static_cast<int64_t>(d->T) * d->X * d->Y;
+    d->Npad = C * kCubeTokens;
+    d->rows = static_cast<int64_t>(d->B) * d->H * d->Npad;
+    if (static_cast<int64_t>(d->B) * d->H > 65535)
+        return fail(VSA_ERR_UNSUPPORTED, "batch*heads = %lld exceeds 65535", (long long)d->B * d->H);
+    if (d->rows > kMaxRows)
+        return fail(VSA_ERR_INVALID_ARGUMENT, "B*H*Npad = %lld rows exceeds 2^31-1", (long long)d->rows);
+    return VSA_OK;
+}
+
+vsa_status need_ptr(const void* p, const char* name) {
+    if (!p) return fail(VSA_ERR_INVALID_ARGUMENT, "%s is NULL", name);
+    if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return fail(VSA_ERR_MISALIGNED, "%s is not 16-byte aligned", name);
+    return VSA_OK;
+}
+
+vsa_status opt_ptr(const void* p, const char* name) { return p ? need_ptr(p, name) : VSA_OK; }
+
+struct Range {
+    const void* p;
+    size_t bytes;
+    const char* name;
+};
+
+bool overlap(const Range& a, const Range& b) {
+    if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+    return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+vsa_status check_disjoint(std::initializer_list<Range> ins, std::initializer_list<Range> outs) {
+    for (const Range& o : outs) {
+        for (const Range& i : ins)
+            if (overlap(o, i)) return fail(VSA_ERR_INVALID_ARGUMENT, "output %s overlaps input %s", o.name, i.name);
+        for (const Range& o2 : outs)
+            if (&o2 != &o && overlap(o, o2)) return fail(VSA_ERR_INVALID_ARGUMENT, "outputs %s and %s overlap", o.name, o2.name);
+    }
+    return VSA_OK;
+}
+
+// The kernels are built for sm_100a only.
+vsa_status check_device() {
+    static int checked[64] = {};   // 0 unknown, 1 ok, 2 unsupported
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev >= 0 && dev < 64 && checked[dev] == 1) return VSA_OK;
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+        return cuda_fail(e, "cudaDeviceGetAttribute");
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+        return cuda_fail(e, "cudaDeviceGetAttribute");
+    if (major != 10 || minor != 0) {
+        if (dev >= 0 && dev < 64) checked[dev] = 2;
+        return fail(VSA_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library runs on sm_100a only", dev, major, minor);
+    }
+    if (dev >= 0 && dev < 64) checked[dev] = 1;
+    return VSA_OK;
+}
+
+cudaStream_t as_stream(vsa_stream_t s) { return static_cast<cudaStream_t>(s); }
+
+size_t tiled_bytes(const Dims& d) { return static_cast<size_t>(d.rows) * d.D * 2; }
+size_t token_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.N * d.H * d.D * 2; }
+size_t gate_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.N * d.H * 2; }
+size_t pooled_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C * d.D * 4; }
+size_t score_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C * d.C * 4; }
+size_t idx_bytes(const Dims& d, int k) { return static_cast<size_t>(d.B) * d.H * d.C * k * 4; }
+
+constexpr size_t kAlign = 256;
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Workspace of vsa_forward: qt | kt | vt | o_fine | qbar | kbar | vbar | o_coarse | scores | idx.
+// The merged output (combine) reuses qt, which is dead after the fine stage.
+struct Carve {
+    uint16_t *qt, *kt, *vt, *of;
+    float *qbar, *kbar, *vbar, *oc, *scores;
+    int32_t* idx;
+    size_t bytes;
+};
+
+Carve carve(const Dims& d, int k, void* ws) {
+    Carve c{};
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    size_t off = 0;
+    auto take = [&](size_t n) {
+        uint8_t* p = b ? b + off : nullptr;
+        off += up(n);
+        return p;
+    };
+    c.qt = reinterpret_cast<uint16_t*>(take(tiled_bytes(d)));
+    c.kt = reinterpret_cast<uint16_t*>(take(tiled_bytes(d)));
+    c.vt = reinterpret_cast<uint16_t*>(take(tiled_bytes(d)));
+    c.of = reinterpret_cast<uint16_t*>(take(tiled_bytes(d)));
+    c.qbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
+    c.kbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
+    c.vbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
+    c.oc = reinterpret_cast<float*>(take(pooled_bytes(d)));
+    c.scores = reinterpret_cast<float*>(take(score_bytes(d)));
+    c.idx = reinterpret_cast<int32_t*>(take(idx_bytes(d, k)));
+    c.bytes = off;
+    return c;
+}
+
+vsa_status check_scale(float scale) {
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return fail(VSA_ERR_INVALID_ARGUMENT, "scale must be finite and > 0 (got %g)", static_cast<double>(scale));
+    return VSA_OK;
+}
+
+vsa_status check_k(const Dims& d, int32_t k) {
+    if (k < 1 || k > d.C) return fail(VSA_ERR_INVALID_ARGUMENT, "top-k %d outside [1, C=%d]", k, d.C);
+    return VSA_OK;
+}
+
+#define VSA_TRY(expr)                      \
+    do {                                   \
+        const vsa_status st_ = (expr);     \
+        if (st_ != VSA_OK) return st_;     \
+    } while (0)
+
+#define VSA_CUDA(expr, where)                               \
+    do {                                                    \
+        const cudaError_t e_ = (expr);                      \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+    } while (0)
+
+// Body of vsa_forward once the arguments are checked.
+vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* gc,
+                       const uint16_t* gf, int topk, float scale, void* ws, uint16_t* out, cudaStream_t s) {
+    const Carve c = carve(d, topk, ws);
+    const bool dense = topk == d.C && gc == nullptr && gf == nullptr;
+    Bf16Triple t{{q, k, v}, {c.qt, c.kt, c.vt}, 3};
+    VSA_CUDA(launch_tile(d, t, s), "tile launch");
+    if (dense) {
+        const char* why = nullptr;
+        cudaError_t e = launch_fine(d, c.qt, c.kt, c.vt, nullptr, d.C, scale, c.of, nullptr, s, &why);
+        if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "fine launch");
+        VSA_CUDA(launch_untile(d, c.of, out, s), "untile launch");
+        return VSA_OK;
+    }
+    const uint16_t* pin[3] = {c.qt, c.kt, c.vt};
+    float* pout[3] = {c.qbar, c.kbar, c.vbar};
+    VSA_CUDA(launch_pool(d, pin, pout, 3, s), "pool launch");
+    VSA_CUDA(launch_coarse(d, c.qbar, c.kbar, c.vbar, scale, c.scores, c.oc, s), "coarse launch");
+    VSA_CUDA(launch_topk(d, c.scores, topk, c.idx, s), "topk launch");
+    const char* why = nullptr;
+    cudaError_t e = launch_fine(d, c.qt, c.kt, c.vt, c.idx, topk, scale, c.of, nullptr, s, &why);
+    if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "fine launch");
+    uint16_t* o_tiled = c.qt;   // qt is no longer read after the fine stage
+    VSA_CUDA(launch_combine(d, c.oc, c.of, gc, gf, o_tiled, s), "combine launch");
+    VSA_CUDA(launch_untile(d, o_tiled, out, s), "untile launch");
+    return VSA_OK;
+}
+
+}  // namespace
+
+int sm_count() {
+    static int counts[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!counts[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
+}  // namespace vsa
+
+using namespace vsa;
+
+extern "C" {
+
+int32_t vsa_abi_version(void) { return VSA_ABI_VERSION; }
+
+const char* vsa_status_string(vsa_status st) {
+    switch (st) {
+        case VSA_OK: return "VSA_OK";
+        case VSA_ERR_INVALID_ARGUMENT: return "VSA_ERR_INVALID_ARGUMENT";
+        case VSA_ERR_UNSUPPORTED: return "VSA_ERR_UNSUPPORTED";
+        case VSA_ERR_MISALIGNED: return "VSA_ERR_MISALIGNED";
+        case VSA_ERR_WORKSPACE: return "VSA_ERR_WORKSPACE";
+        case VSA_ERR_CUDA: return "VSA_ERR_CUDA";
+        case VSA_ERR_TIMEOUT: return "VSA_ERR_TIMEOUT";
+    }
+    return "VSA_ERR_UNKNOWN";
+}
+
+const char* vsa_last_error(void) { return g_last_error; }
+
+vsa_status vsa_shape_info(const vsa_shape* shape, int64_t* npad, int32_t* num_cubes) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    if (npad) *npad = d.Npad;
+    if (num_cubes) *num_cubes = d.C;
+    return VSA_OK;
+}
+
+vsa_status vsa_tile(const vsa_shape* shape, const vsa_bf16* x, vsa_bf16* xt, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(need_ptr(x, "x"));
+    VSA_TRY(need_ptr(xt, "xt"));
+    VSA_TRY(check_disjoint({{x, token_bytes(d), "x"}}, {{xt, tiled_bytes(d), "xt"}}));
+    VSA_TRY(check_device());
+    Bf16Triple t{{x, nullptr, nullptr}, {xt, nullptr, nullptr}, 1};
+    VSA_CUDA(launch_tile(d, t, as_stream(stream)), "tile launch");
+    return VSA_OK;
+}
+
+vsa_status vsa_untile(const vsa_shape* shape, const vsa_bf16* xt, vsa_bf16* x, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(need_ptr(xt, "xt"));
+    VSA_TRY(need_ptr(x, "x"));
+    VSA_TRY(check_disjoint({{xt, tiled_bytes(d), "xt"}}, {{x, token_bytes(d), "x"}}));
+    VSA_TRY(check_device());
+    VSA_CUDA(launch_untile(d, xt, x, as_stream(stream)), "untile launch");
+    return VSA_OK;
+}
+
+vsa_status vsa_pool(const vsa_shape* shape, const vsa_bf16* xt, float* xbar, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(need_ptr(xt, "xt"));
+    VSA_TRY(need_ptr(xbar, "xbar"));
+    VSA_TRY(check_disjoint({{xt, tiled_bytes(d), "xt"}}, {{xbar, pooled_bytes(d), "xbar"}}));
+    VSA_TRY(check_device());
+    const uint16_t* in[1] = {xt};
+    float* out[1] = {xbar};
+    VSA_CUDA(launch_pool(d, in, out, 1, as_stream(stream)), "pool launch");
+    return VSA_OK;
+}
+
+vsa_status vsa_coarse(const vsa_shape* shape, const float* qbar, const float* kbar, const float* vbar, float scale,
+                      float* scores, float* o_coarse, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(need_ptr(qbar, "qbar"));
+    VSA_TRY(need_ptr(kbar, "kbar"));
+    VSA_TRY(need_ptr(vbar, "vbar"));
+    VSA_TRY(need_ptr(scores, "scores"));
+    VSA_TRY(need_ptr(o_coarse, "o_coarse"));
+    VSA_TRY(check_scale(scale));
+    const size_t pb = pooled_bytes(d);
+    VSA_TRY(check_disjoint({{qbar, pb, "qbar"}, {kbar, pb, "kbar"}, {vbar, pb, "vbar"}},
+                           {{scores, score_bytes(d), "scores"}, {o_coarse, pb, "o_coarse"}}));
+    VSA_TRY(check_device());
+    VSA_CUDA(launch_coarse(d, qbar, kbar, vbar, scale, scores, o_coarse, as_stream(stream)), "coarse launch");
+    return VSA_OK;
+}
+
+vsa_status vsa_topk(const vsa_shape* shape, const float* scores, int32_t k, int32_t* idx, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(check_k(d, k));
+    VSA_TRY(need_ptr(scores, "scores"));
+    VSA_TRY(need_ptr(idx, "idx"));
+    if (d.C > 49152) return fail(VSA_ERR_UNSUPPORTED, "top-k supports at most 49152 cubes (got %d)", d.C);
+    VSA_TRY(check_disjoint({{scores, score_bytes(d), "scores"}}, {{idx, idx_bytes(d, k), "idx"}}));
+    VSA_TRY(check_device());
+    VSA_CUDA(launch_topk(d, scores, k, idx, as_stream(stream)), "topk launch");
+    return VSA_OK;
+}
+
+vsa_status vsa_fine(const vsa_shape* shape, const vsa_bf16* qt, const vsa_bf16* kt, const vsa_bf16* vt,
+                    const int32_t* idx, int32_t k, float scale, vsa_bf16* o_fine, float* lse, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    if (idx) VSA_TRY(check_k(d, k));
+    VSA_TRY(need_ptr(qt, "qt"));
+    VSA_TRY(need_ptr(kt, "kt"));
+    VSA_TRY(need_ptr(vt, "vt"));
+    VSA_TRY(opt_ptr(idx, "idx"));
+    VSA_TRY(need_ptr(o_fine, "o_fine"));
+    VSA_TRY(opt_ptr(lse, "lse"));
+    VSA_TRY(check_scale(scale));
+    const size_t tb = tiled_bytes(d);
+    VSA_TRY(check_disjoint({{qt, tb, "qt"}, {kt, tb, "kt"}, {vt, tb, "vt"}, {idx, idx ? idx_bytes(d, k) : 0, "idx"}},
+                           {{o_fine, tb, "o_fine"}, {lse, lse ? static_cast<size_t>(d.rows) * 4 : 0, "lse"}}));
+    VSA_TRY(check_device());
+    const char* why = nullptr;
+    cudaError_t e = launch_fine(d, qt, kt, vt, idx, k, scale, o_fine, lse, as_stream(stream), &why);
+    if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "fine launch");
+    return VSA_OK;
+}
+
+vsa_status vsa_combine(const vsa_shape* shape, const float* o_coarse, const vsa_bf16* o_fine, const vsa_bf16* g_coarse,
+                       const vsa_bf16* g_fine, vsa_bf16* o_tiled, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(need_ptr(o_coarse, "o_coarse"));
+    VSA_TRY(need_ptr(o_fine, "o_fine"));
+    VSA_TRY(opt_ptr(g_coarse, "g_coarse"));
+    VSA_TRY(opt_ptr(g_fine, "g_fine"));
+    VSA_TRY(need_ptr(o_tiled, "o_tiled"));
+    const size_t tb = tiled_bytes(d), gb = gate_bytes(d);
+    VSA_TRY(check_disjoint({{o_coarse, pooled_bytes(d), "o_coarse"}, {o_fine, tb, "o_fine"},
+                            {g_coarse, g_coarse ? gb : 0, "g_coarse"}, {g_fine, g_fine ? gb : 0, "g_fine"}},
+                           {{o_tiled, tb, "o_tiled"}}));
+    VSA_TRY(check_device());
+    VSA_CUDA(launch_combine(d, o_coarse, o_fine, g_coarse, g_fine, o_tiled, as_stream(stream)), "combine launch");
+    return VSA_OK;
+}
+
+size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk) {
+    Dims d{};
+    if (make_dims(shape, &d) != VSA_OK || topk < 1 || topk > d.C) return 0;
+    return carve(d, topk, nullptr).bytes;
+}
+
+vsa_status vsa_forward(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                       const vsa_bf16* g_coarse, const vsa_bf16* g_fine, int32_t topk, float scale, void* workspace,
+                       size_t workspace_bytes, vsa_bf16* out, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(check_k(d, topk));
+    VSA_TRY(check_scale(scale));
+    VSA_TRY(need_ptr(q, "q"));
+    VSA_TRY(need_ptr(k, "k"));
+    VSA_TRY(need_ptr(v, "v"));
+    VSA_TRY(opt_ptr(g_coarse, "g_coarse"));
+    VSA_TRY(opt_ptr(g_fine, "g_fine"));
+    VSA_TRY(need_ptr(out, "out"));
+    if (d.C > 49152) return fail(VSA_ERR_UNSUPPORTED, "top-k supports at most 49152 cubes (got %d)", d.C);
+    const size_t need = carve(d, topk, nullptr).bytes;
+    if (!workspace) return fail(VSA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0)
+        return fail(VSA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    if (workspace_bytes < need)
+        return fail(VSA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, need);
+    const size_t tb = token_bytes(d), gb = gate_bytes(d);
+    VSA_TRY(check_disjoint({{q, tb, "q"}, {k, tb, "k"}, {v, tb, "v"}, {g_coarse, g_coarse ? gb : 0, "g_coarse"},
+                            {g_fine, g_fine ? gb : 0, "g_fine"}},
+                           {{out, tb, "out"}, {workspace, need, "workspace"}}));
+    VSA_TRY(check_device());
+    return run_forward(d, q, k, v, g_coarse, g_fine, topk, scale, workspace, out, as_stream(stream));
+}
+
+size_t vsa_workspace_bytes_host(const vsa_shape* shape, int32_t topk) {
+    Dims d{};
+    if (make_dims(shape, &d) != VSA_OK || topk < 1 || topk > d.C) return 0;
+    return carve(d, topk, nullptr).bytes + 4 * up(token_bytes(d)) + 2 * up(gate_bytes(d));
+}
+
+vsa_status vsa_forward_host(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                            const vsa_bf16* g_coarse, const vsa_bf16* g_fine, int32_t topk, float scale,
+                            void* workspace, size_t workspace_bytes, vsa_bf16* out, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(check_k(d, topk));
+    VSA_TRY(check_scale(scale));
+    if (!q || !k || !v || !out) return fail(VSA_ERR_INVALID_ARGUMENT, "q, k, v and out must be non-NULL host pointers");
+    if (d.C > 49152) return fail(VSA_ERR_UNSUPPORTED, "top-k supports at most 49152 cubes (got %d)", d.C);
+    const size_t fwd = carve(d, topk, nullptr).bytes;
+    const size_t tb = token_bytes(d), gb = gate_bytes(d);
+    const size_t need = fwd + 4 * up(tb) + 2 * up(gb);
+    if (!workspace) return fail(VSA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0)
+        return fail(VSA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    if (workspace_bytes < need)
+        return fail(VSA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, need);
+    VSA_TRY(check_device());
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    uint16_t* dq = reinterpret_cast<uint16_t*>(w + fwd);
+    uint16_t* dk = reinterpret_cast<uint16_t*>(w + fwd + up(tb));
+    uint16_t* dv = reinterpret_cast<uint16_t*>(w + fwd + 2 * up(tb));
+    uint16_t* dout = reinterpret_cast<uint16_t*>(w + fwd + 3 * up(tb));
+    uint16_t* dgc = g_coarse ? reinterpret_cast<uint16_t*>(w + fwd + 4 * up(tb)) : nullptr;
+    uint16_t* dgf = g_fine ? reinterpret_cast<uint16_t*>(w + fwd + 4 * up(tb) + up(gb)) : nullptr;
+    cudaStream_t s = as_stream(stream);
+    VSA_CUDA(cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, s), "copy q to device");
+    VSA_CUDA(cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, s), "copy k to device");
+    VSA_CUDA(cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, s), "copy v to device");
+    if (dgc) VSA_CUDA(cudaMemcpyAsync(dgc, g_coarse, gb, cudaMemcpyHostToDevice, s), "copy g_coarse to device");
+    if (dgf) VSA_CUDA(cudaMemcpyAsync(dgf, g_fine, gb, cudaMemcpyHostToDevice, s), "copy g_fine to device");
+    VSA_TRY(run_forward(d, dq, dk, dv, dgc, dgf, topk, scale, workspace, dout, s));
+    VSA_CUDA(cudaMemcpyAsync(out, dout, tb, cudaMemcpyDeviceToHost, s), "copy out to host");
+    return VSA_OK;
+}
+
+vsa_status vsa_device_status(vsa_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int* w = status_word();
+    if (!w) return fail(VSA_ERR_CUDA, "watchdog word unavailable");
+    int value = 0;
+    if ((e = cudaMemcpy(&value, w, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "read watchdog word");
+    const int zero = 0;
+    if ((e = cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice)) != cudaSuccess)
+        return cuda_fail(e, "clear watchdog word");
+    if (value == VSA_ERR_TIMEOUT) return fail(VSA_ERR_TIMEOUT, "a device-side wait gave up (work incomplete)");
+    return VSA_OK;
+}
+
+vsa_status vsa_debug_wait_probe(uint64_t limit_ns, vsa_stream_t stream) {
+    if (limit_ns < 1000000ull || limit_ns > 10000000000ull)
+        return fail(VSA_ERR_INVALID_ARGUMENT, "limit_ns %llu outside [1 ms, 10 s]", (unsigned long long)limit_ns);
+    VSA_TRY(check_device());
+    VSA_CUDA(launch_wait_probe(limit_ns, as_stream(stream)), "wait probe launch");
+    return VSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,242 @@
+// Coarse stage and cube selection (Wan2.2 teardown, zharfai.com, section
+// "Video sparse attention selects cubes", part 1: cheap block-level attention
+// over the mean-pooled cubes that ranks the candidate key cubes, of which
+// each query cube keeps the top-k).
+//
+// The coarse scores decide the selection, so they are computed in float32 on
+// the CUDA cores (a deterministic sequential sum over the channels), not on
+// the bf16/tf32 tensor paths whose rounding would reorder near-equal cubes.
+#include <cfloat>
+
+#include "vsa_internal.h"
+
+namespace vsa {
+namespace {
+
+constexpr int kTile = 64;   // output tile edge
+constexpr int kBK = 16;     // reduction slice
+constexpr int kThreads = 256;
+
+// scores[bh][i][j] = scale * sum_d qbar[bh][i][d] * kbar[bh][j][d]
+__global__ void __launch_bounds__(kThreads) coarse_scores_kernel(int C, int D, const float* __restrict__ qbar,
+                                                                 const float* __restrict__ kbar, float scale,
+                                                                 float* __restrict__ scores) {
+    __shared__ float As[kBK][kTile + 4];
+    __shared__ float Bs[kBK][kTile + 4];
+    const int bh = blockIdx.z;
+    const int i0 = blockIdx.y * kTile, j0 = blockIdx.x * kTile;
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const float* Q = qbar + static_cast<int64_t>(bh) * C * D;
+    const float* K = kbar + static_cast<int64_t>(bh) * C * D;
+    float acc[4][4] = {};
+    for (int d0 = 0; d0 < D; d0 += kBK) {
+        // 64 rows x 16 channels of each operand; 4 elements per thread each
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int idx = threadIdx.x + e * kThreads;
+            const int r = idx / kBK, cc = idx % kBK;
+            const int gi = i0 + r, gj = j0 + r;
+            As[cc][r] = gi < C ? Q[static_cast<int64_t>(gi) * D + d0 + cc] : 0.f;
+            Bs[cc][r] = gj < C ? K[static_cast<int64_t>(gj) * D + d0 + cc] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < kBK; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a[r] = As[kk][ty + 16 * r];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) b[c] = Bs[kk][tx + 16 * c];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+        }
+        __syncthreads();
+    }
+    float* S = scores + static_cast<int64_t>(bh) * C * C;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int gi = i0 + ty + 16 * r;
+        if (gi >= C) continue;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int gj = j0 + tx + 16 * c;
+            if (gj < C) S[static_cast<int64_t>(gi) * C + gj] = scale * acc[r][c];
+        }
+    }
+}
+
+// o_coarse[bh][i] = sum_j softmax(scores[bh][i][:])_j * vbar[bh][j]
+// A block owns 64 query rows: it first reduces the row maxima and
+// denominators, then accumulates P * Vbar over key slices of 16.
+template <int D>
+__global__ void __launch_bounds__(kThreads) coarse_pv_kernel(int C, const float* __restrict__ scores,
+                                                             const float* __restrict__ vbar,
+                                                             float* __restrict__ o_coarse) {
+    constexpr int CPT = D / 16;   // output columns per thread
+    __shared__ float row_max[kTile], row_inv[kTile];
+    __shared__ float Ps[kBK][kTile + 4];
+    __shared__ float Vs[kBK][D];
+    const int bh = blockIdx.y;
+    const int i0 = blockIdx.x * kTile;
+    const float* S = scores + static_cast<int64_t>(bh) * C * C;
+    const float* V = vbar + static_cast<int64_t>(bh) * C * D;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int r = warp; r < kTile; r += kThreads / 32) {
+        const int gi = i0 + r;
+        float m = -FLT_MAX, l = 0.f;
+        if (gi < C) {
+            const float* row = S + static_cast<int64_t>(gi) * C;
+            for (int j = lane; j < C; j += 32) m = fmaxf(m, row[j]);
+#pragma unroll
+            for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            for (int j = lane; j < C; j += 32) l += expf(row[j] - m);
+#pragma unroll
+            for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+        }
+        if (lane == 0) {
+            row_max[r] = m;
+            row_inv[r] = l > 0.f ? 1.0f / l : 0.f;
+        }
+    }
+    __syncthreads();
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    float acc[4][CPT] = {};
+    for (int j0 = 0; j0 < C; j0 += kBK) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int idx = threadIdx.x + e * kThreads;   // 64 rows x 16 keys
+            const int r = idx / kBK, cc = idx % kBK;
+            const int gi = i0 + r, gj = j0 + cc;
+            Ps[cc][r] = (gi < C && gj < C) ? expf(S[static_cast<int64_t>(gi) * C + gj] - row_max[r]) : 0.f;
+        }
+        for (int idx = threadIdx.x; idx < kBK * D; idx += kThreads) {
+            const int kk = idx / D, cc = idx % D;
+            const int gj = j0 + kk;
+            Vs[kk][cc] = gj < C ? V[static_cast<int64_t>(gj) * D + cc] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < kBK; ++kk) {
+            float a[4], b[CPT];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a[r] = Ps[kk][ty + 16 * r];
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) b[c] = Vs[kk][tx + 16 * c];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+        }
+        __syncthreads();
+    }
+    float* O = o_coarse + static_cast<int64_t>(bh) * C * D;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int li = ty + 16 * r, gi = i0 + li;
+        if (gi >= C) continue;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) O[static_cast<int64_t>(gi) * D + tx + 16 * c] = acc[r][c] * row_inv[li];
+    }
+}
+
+// Order-preserving map float -> uint32 (larger float, larger key); -0 is
+// folded onto +0 so that equal scores compare equal.
+__device__ __forceinline__ uint32_t order_key(float f) {
+    if (f == 0.0f) f = 0.0f;
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One warp per (b, h, query cube) row.  The k-th largest key T is built bit
+// by bit from the top (largest T with at least k keys >= T); the row is then
+// scanned in index order, keeping every key > T and the lowest-index keys
+// equal to T until k are kept, so the output is ascending by construction.
+__global__ void __launch_bounds__(kThreads) topk_kernel(int64_t rows, int C, int k, const float* __restrict__ scores,
+                                                        int32_t* __restrict__ idx) {
+    extern __shared__ uint32_t keys_all[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t* keys = keys_all + static_cast<int64_t>(warp) * C;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
+    for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + warp; row < rows; row += warps) {
+        const float* s = scores + row * C;
+        for (int j = lane; j < C; j += 32) keys[j] = order_key(__ldcs(s + j));
+        __syncwarp();
+        uint32_t T = 0u;
+        for (int bit = 31; bit >= 0; --bit) {
+            const uint32_t cand = T | (1u << bit);
+            int cnt = 0;
+            for (int j0 = 0; j0 < C; j0 += 32) {
+                const int j = j0 + lane;
+                cnt += __popc(__ballot_sync(0xffffffffu, j < C && keys[j] >= cand));
+            }
+            if (cnt >= k) T = cand;
+        }
+        int gt = 0;
+        for (int j0 = 0; j0 < C; j0 += 32) {
+            const int j = j0 + lane;
+            gt += __popc(__ballot_sync(0xffffffffu, j < C && keys[j] > T));
+        }
+        const int need_eq = k - gt;
+        int out = 0, eq_seen = 0;
+        int32_t* dst = idx + row * k;
+        for (int j0 = 0; j0 < C && out < k; j0 += 32) {
+            const int j = j0 + lane;
+            const uint32_t key = j < C ? keys[j] : 0u;
+            const bool is_gt = j < C && key > T;
+            const bool is_eq = j < C && key == T;
+            const uint32_t eq_mask = __ballot_sync(0xffffffffu, is_eq);
+            const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
+            const bool take = is_gt || (is_eq && eq_rank < need_eq);
+            const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
+            if (take) dst[out + __popc(take_mask & lt_mask)] = j;
+            out += __popc(take_mask);
+            eq_seen += __popc(eq_mask);
+        }
+        __syncwarp();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
+                          float* scores, float* o_coarse, cudaStream_t s) {
+    const int bh = d.B * d.H;
+    const int tiles = (d.C + kTile - 1) / kTile;
+    coarse_scores_kernel<<<dim3(tiles, tiles, bh), kThreads, 0, s>>>(d.C, d.D, qbar, kbar, scale, scores);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (d.D == 128) coarse_pv_kernel<128><<<dim3(tiles, bh), kThreads, 0, s>>>(d.C, scores, vbar, o_coarse);
+    else coarse_pv_kernel<64><<<dim3(tiles, bh), kThreads, 0, s>>>(d.C, scores, vbar, o_coarse);
+    return cudaGetLastError();
+}
+
+// Largest C the selection kernel keeps in shared memory (one row per warp).
+constexpr int kTopkMaxC = 49152;
+
+int topk_warps_per_block(int C) {
+    int w = 8;
+    while (w > 1 && static_cast<int64_t>(w) * C * 4 > 200 * 1024) w >>= 1;
+    return w;
+}
+
+cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx, cudaStream_t s) {
+    if (d.C > kTopkMaxC) return cudaErrorInvalidValue;
+    const int64_t rows = static_cast<int64_t>(d.B) * d.H * d.C;
+    const int wpb = topk_warps_per_block(d.C);
+    const size_t smem = static_cast<size_t>(wpb) * d.C * 4;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t blocks_needed = (rows + wpb - 1) / wpb;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
+    topk_kernel<<<grid, wpb * 32, smem, s>>>(rows, d.C, k, scores, idx);
+    return cudaGetLastError();
+}
+
+}  // namespace vsa

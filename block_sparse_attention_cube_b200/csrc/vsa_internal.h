@@ -1,0 +1,58 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "vsa.h"
+
+namespace vsa {
+
+constexpr int kCube = 4;
+constexpr int kCubeTokens = 64;
+
+// Sizes derived from a vsa_shape (see include/vsa.h for the layouts).
+struct Dims {
+    int B, H, D;
+    int T, X, Y;        // token grid
+    int Ct, Cx, Cy;     // cubes per axis
+    int C;              // cubes
+    int64_t N;          // real tokens per batch element
+    int64_t Npad;       // padded tokens per batch element = C * 64
+    int64_t rows;       // B * H * Npad rows of the tiled layout
+};
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Watchdog word of the current device (device address, cached per device).
+int* status_word();
+
+// Upper bound on any device-side wait, in nanoseconds.
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+// ---- launches; each returns the launch error (cudaSuccess when enqueued)
+struct Bf16Triple {
+    const uint16_t* src[3];
+    uint16_t* dst[3];
+    int count;
+};
+
+cudaError_t launch_tile(const Dims& d, const Bf16Triple& t, cudaStream_t s);
+cudaError_t launch_untile(const Dims& d, const uint16_t* xt, uint16_t* x, cudaStream_t s);
+cudaError_t launch_pool(const Dims& d, const uint16_t* const* xt, float* const* xbar, int count, cudaStream_t s);
+cudaError_t launch_combine(const Dims& d, const float* o_coarse, const uint16_t* o_fine, const uint16_t* g_coarse,
+                           const uint16_t* g_fine, uint16_t* o_tiled, cudaStream_t s);
+cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
+                          float* scores, float* o_coarse, cudaStream_t s);
+cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx, cudaStream_t s);
+
+// Fine stage.  Returns cudaErrorInvalidValue (with *why set) when a tensor
+// map cannot be encoded.
+cudaError_t launch_fine(const Dims& d, const uint16_t* qt, const uint16_t* kt, const uint16_t* vt,
+                        const int32_t* idx, int k, float scale, uint16_t* o_fine, float* lse, cudaStream_t s,
+                        const char** why);
+
+cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t s);
+
+}  // namespace vsa

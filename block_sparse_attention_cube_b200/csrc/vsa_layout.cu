@@ -1,0 +1,234 @@
+// Memory-bound steps of the path: cube-major tiling with zero padding, its
+// inverse, the cube mean-pool and the gated merge.
+//
+// All four kernels work on "cube tasks" (tensor, b, h, cube) with a
+// grid-stride loop over a grid sized as a multiple of the SM count; a block
+// of 256 threads moves one cube (64 rows of D bf16) per task with 16-byte
+// vector accesses.  The cube-major order is the one of the Wan2.2 teardown
+// (zharfai.com), section "Video sparse attention selects cubes": 4x4x4 cubes
+// of 64 tokens on a grid padded per axis to a multiple of 4.
+#include <cuda_bf16.h>
+
+#include "vsa_internal.h"
+
+namespace vsa {
+namespace {
+
+constexpr int kBlock = 256;
+
+struct CubeTask {
+    int tensor;
+    int64_t bh;   // b * H + h
+    int b, h, c;
+    int ct, cx, cy;
+};
+
+__device__ __forceinline__ CubeTask decode_task(int64_t task, const Dims& d) {
+    const int64_t per_tensor = static_cast<int64_t>(d.B) * d.H * d.C;
+    CubeTask t;
+    t.tensor = static_cast<int>(task / per_tensor);
+    const int64_t r = task - t.tensor * per_tensor;
+    t.c = static_cast<int>(r % d.C);
+    t.bh = r / d.C;
+    t.h = static_cast<int>(t.bh % d.H);
+    t.b = static_cast<int>(t.bh / d.H);
+    t.ct = t.c / (d.Cx * d.Cy);
+    t.cx = (t.c / d.Cy) % d.Cx;
+    t.cy = t.c % d.Cy;
+    return t;
+}
+
+// Source token of offset o inside the cube, or -1 for a padded position.
+__device__ __forceinline__ int64_t token_of(const Dims& d, const CubeTask& t, int o) {
+    const int tt = t.ct * kCube + (o >> 4);
+    const int xx = t.cx * kCube + ((o >> 2) & 3);
+    const int yy = t.cy * kCube + (o & 3);
+    if (tt >= d.T || xx >= d.X || yy >= d.Y) return -1;
+    return (static_cast<int64_t>(tt) * d.X + xx) * d.Y + yy;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBlock) tile_kernel(Dims d, Bf16Triple io) {
+    constexpr int CH = D / 8;                   // 16-byte chunks per row
+    constexpr int PER = kCubeTokens * CH / kBlock;
+    const int64_t total = static_cast<int64_t>(d.B) * d.H * d.C * io.count;
+    for (int64_t task = blockIdx.x; task < total; task += gridDim.x) {
+        const CubeTask t = decode_task(task, d);
+        const uint4* src = reinterpret_cast<const uint4*>(io.src[t.tensor]);
+        uint4* dst = reinterpret_cast<uint4*>(io.dst[t.tensor]);
+        const int64_t out_row0 = t.bh * d.Npad + static_cast<int64_t>(t.c) * kCubeTokens;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int q = threadIdx.x + i * kBlock;
+            const int o = q / CH, j = q % CH;
+            const int64_t n = token_of(d, t, o);
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (n >= 0) v = __ldcs(src + ((static_cast<int64_t>(t.b) * d.N + n) * d.H + t.h) * CH + j);
+            dst[(out_row0 + o) * CH + j] = v;
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBlock) untile_kernel(Dims d, const uint16_t* __restrict__ xt,
+                                                        uint16_t* __restrict__ x) {
+    constexpr int CH = D / 8;
+    constexpr int PER = kCubeTokens * CH / kBlock;
+    const int64_t total = static_cast<int64_t>(d.B) * d.H * d.C;
+    const uint4* src = reinterpret_cast<const uint4*>(xt);
+    uint4* dst = reinterpret_cast<uint4*>(x);
+    for (int64_t task = blockIdx.x; task < total; task += gridDim.x) {
+        const CubeTask t = decode_task(task, d);
+        const int64_t in_row0 = t.bh * d.Npad + static_cast<int64_t>(t.c) * kCubeTokens;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int q = threadIdx.x + i * kBlock;
+            const int o = q / CH, j = q % CH;
+            const int64_t n = token_of(d, t, o);
+            if (n < 0) continue;
+            const uint4 v = __ldcs(src + (in_row0 + o) * CH + j);
+            __stcs(dst + ((static_cast<int64_t>(t.b) * d.N + n) * d.H + t.h) * CH + j, v);
+        }
+    }
+}
+
+// One warp per cube: lanes split a row into 16-byte chunks, rows are spread
+// over the warp's lane groups, partial sums are combined with shuffles.
+struct PoolIO {
+    const uint16_t* src[3];
+    float* dst[3];
+    int count;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kBlock) pool_kernel(Dims d, PoolIO io) {
+    constexpr int LPR = D / 8;          // lanes per row
+    constexpr int RPI = 32 / LPR;       // rows per warp iteration
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / LPR, j = lane % LPR;
+    const int64_t total = static_cast<int64_t>(d.B) * d.H * d.C * io.count;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kBlock / 32);
+    for (int64_t task = static_cast<int64_t>(blockIdx.x) * (kBlock / 32) + threadIdx.x / 32; task < total;
+         task += warps) {
+        const CubeTask t = decode_task(task, d);
+        const uint4* src = reinterpret_cast<const uint4*>(io.src[t.tensor]);
+        const int64_t row0 = t.bh * d.Npad + static_cast<int64_t>(t.c) * kCubeTokens;
+        const int nt = min(kCube, d.T - t.ct * kCube);
+        const int nx = min(kCube, d.X - t.cx * kCube);
+        const int ny = min(kCube, d.Y - t.cy * kCube);
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 4
+        for (int o = sub; o < kCubeTokens; o += RPI) {
+            if ((o >> 4) >= nt || ((o >> 2) & 3) >= nx || (o & 3) >= ny) continue;
+            const uint4 v = __ldcs(src + (row0 + o) * LPR + j);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc[2 * e] += __uint_as_float(w[e] << 16);
+                acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+            }
+        }
+#pragma unroll
+        for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+        }
+        if (sub == 0) {
+            const float inv = 1.0f / static_cast<float>(nt * nx * ny);
+            float4* out = reinterpret_cast<float4*>(io.dst[t.tensor] + (t.bh * d.C + t.c) * D + j * 8);
+            out[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+            out[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBlock) combine_kernel(Dims d, const float* __restrict__ o_coarse,
+                                                         const uint16_t* __restrict__ o_fine,
+                                                         const uint16_t* __restrict__ g_coarse,
+                                                         const uint16_t* __restrict__ g_fine,
+                                                         uint16_t* __restrict__ o_tiled) {
+    constexpr int CH = D / 8;
+    constexpr int PER = kCubeTokens * CH / kBlock;
+    const int64_t total = static_cast<int64_t>(d.B) * d.H * d.C;
+    const uint4* of = reinterpret_cast<const uint4*>(o_fine);
+    uint4* out = reinterpret_cast<uint4*>(o_tiled);
+    for (int64_t task = blockIdx.x; task < total; task += gridDim.x) {
+        const CubeTask t = decode_task(task, d);
+        const int64_t row0 = t.bh * d.Npad + static_cast<int64_t>(t.c) * kCubeTokens;
+        const float4* oc = reinterpret_cast<const float4*>(o_coarse + (t.bh * d.C + t.c) * D);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int q = threadIdx.x + i * kBlock;
+            const int o = q / CH, j = q % CH;
+            const int64_t n = token_of(d, t, o);
+            uint4 r = make_uint4(0u, 0u, 0u, 0u);
+            if (n >= 0) {
+                const int64_t g = (static_cast<int64_t>(t.b) * d.N + n) * d.H + t.h;
+                const float gc = g_coarse ? __uint_as_float(static_cast<uint32_t>(g_coarse[g]) << 16) : 0.f;
+                const float gf = g_fine ? __uint_as_float(static_cast<uint32_t>(g_fine[g]) << 16) : 1.f;
+                const float4 c0 = __ldg(oc + 2 * j), c1 = __ldg(oc + 2 * j + 1);
+                const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                const uint4 f = __ldcs(of + (row0 + o) * CH + j);
+                const uint32_t fw[4] = {f.x, f.y, f.z, f.w};
+                uint32_t ow[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float lo = gc * cv[2 * e] + gf * __uint_as_float(fw[e] << 16);
+                    const float hi = gc * cv[2 * e + 1] + gf * __uint_as_float(fw[e] & 0xFFFF0000u);
+                    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+                    ow[e] = *reinterpret_cast<const uint32_t*>(&p);
+                }
+                r = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            }
+            out[(row0 + o) * CH + j] = r;
+        }
+    }
+}
+
+int grid_for(int64_t tasks, int per_sm) {
+    const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
+    return static_cast<int>(tasks < cap ? (tasks > 0 ? tasks : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_tile(const Dims& d, const Bf16Triple& t, cudaStream_t s) {
+    const int grid = grid_for(static_cast<int64_t>(d.B) * d.H * d.C * t.count, 8);
+    if (d.D == 128) tile_kernel<128><<<grid, kBlock, 0, s>>>(d, t);
+    else tile_kernel<64><<<grid, kBlock, 0, s>>>(d, t);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_untile(const Dims& d, const uint16_t* xt, uint16_t* x, cudaStream_t s) {
+    const int grid = grid_for(static_cast<int64_t>(d.B) * d.H * d.C, 8);
+    if (d.D == 128) untile_kernel<128><<<grid, kBlock, 0, s>>>(d, xt, x);
+    else untile_kernel<64><<<grid, kBlock, 0, s>>>(d, xt, x);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pool(const Dims& d, const uint16_t* const* xt, float* const* xbar, int count, cudaStream_t s) {
+    PoolIO io{};
+    for (int i = 0; i < count; ++i) {
+        io.src[i] = xt[i];
+        io.dst[i] = xbar[i];
+    }
+    io.count = count;
+    const int64_t warps = static_cast<int64_t>(d.B) * d.H * d.C * count;
+    const int grid = grid_for((warps + 7) / 8, 8);
+    if (d.D == 128) pool_kernel<128><<<grid, kBlock, 0, s>>>(d, io);
+    else pool_kernel<64><<<grid, kBlock, 0, s>>>(d, io);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const Dims& d, const float* o_coarse, const uint16_t* o_fine, const uint16_t* g_coarse,
+                           const uint16_t* g_fine, uint16_t* o_tiled, cudaStream_t s) {
+    const int grid = grid_for(static_cast<int64_t>(d.B) * d.H * d.C, 8);
+    if (d.D == 128) combine_kernel<128><<<grid, kBlock, 0, s>>>(d, o_coarse, o_fine, g_coarse, g_fine, o_tiled);
+    else combine_kernel<64><<<grid, kBlock, 0, s>>>(d, o_coarse, o_fine, g_coarse, g_fine, o_tiled);
+    return cudaGetLastError();
+}
+
+}  // namespace vsa

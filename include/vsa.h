@@ -1,0 +1,230 @@
+/*
+ * vsa.h — C ABI of the B200 (sm_100a) cube-based Video Sparse Attention library.
+ *
+ * The library computes self-attention of a video diffusion transformer over a
+ * 3D latent token grid, in two forms:
+ *
+ *   dense:  O = softmax(Q K^T / sqrt(d)) V, bidirectional (no causal mask).
+ *           Wan2.1 acceleration article (bafh001.com), section 4.2 "replace
+ *           the attention kernel with a fused implementation".
+ *   VSA:    the grid is cut into 4x4x4 cubes of 64 tokens (padded per axis to
+ *           a multiple of 4); a coarse attention over mean-pooled cubes ranks
+ *           key cubes; each query cube keeps its top-k key cubes; a fine
+ *           token-level attention runs over those cubes only; the output is
+ *           the gated sum of the coarse and fine results.
+ *           Wan2.2 real-time inference teardown (zharfai.com), section
+ *           "Video sparse attention selects cubes".
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  * Grid: T x X x Y tokens (frames x height x width); token index
+ *    n = (t*X + x)*Y + y.  Padded grid Tp x Xp x Yp with each axis rounded up
+ *    to a multiple of 4; Npad = Tp*Xp*Yp; C = Npad/64 cubes.
+ *  * Token layout ("BNHD"): element (b, n, h, d) of a [B, N, H, D] array at
+ *    ((b*N + n)*H + h)*D + d, as a DiT's q/k/v projections produce it.
+ *  * Cube-major layout ("tiled"): [B, H, Npad, D]; position p = c*64 + o with
+ *    cube c = ((t/4)*(Xp/4) + x/4)*(Yp/4) + y/4 and offset
+ *    o = ((t%4)*4 + x%4)*4 + y%4.  Positions with t >= T, x >= X or y >= Y
+ *    are padding.
+ *  * bf16 values are passed as uint16_t bit patterns (vsa_bf16).
+ *  * Every pointer argument is a DEVICE pointer owned by the caller, except in
+ *    vsa_forward_host where the tensors are HOST pointers.  The library never
+ *    allocates or frees memory and keeps no device state other than one
+ *    watchdog status word per device.
+ *  * Every device pointer must be 16-byte aligned; input and output ranges of
+ *    one call must not overlap.
+ *  * `stream` is a cudaStream_t passed as an opaque pointer (NULL = the
+ *    legacy default stream).  All work is enqueued asynchronously on it.
+ *  * Errors in the arguments are reported synchronously, before anything is
+ *    enqueued, by the returned status; vsa_last_error() then gives a one-line
+ *    reason (thread-local).  A failed launch returns VSA_ERR_CUDA.  A device
+ *    wait that exceeded its limit is reported later by vsa_device_status().
+ *  * Supported: head_dim 64 or 128; 1 <= top-k <= C; B*H*Npad < 2^31.
+ *    Only sm_100a devices run the kernels; there is no fallback path.
+ */
+#ifndef VSA_B200_H
+#define VSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VSA_ABI_VERSION 1
+
+typedef uint16_t vsa_bf16;
+typedef void* vsa_stream_t;
+
+typedef struct vsa_shape {
+    int32_t batch;     /* B */
+    int32_t heads;     /* H */
+    int32_t head_dim;  /* D: 64 or 128 */
+    int32_t grid_t;    /* T: latent frames */
+    int32_t grid_h;    /* X: token rows per frame */
+    int32_t grid_w;    /* Y: token columns per frame */
+} vsa_shape;
+
+typedef enum vsa_status {
+    VSA_OK = 0,
+    VSA_ERR_INVALID_ARGUMENT = 1, /* a size, count or pointer is out of range */
+    VSA_ERR_UNSUPPORTED = 2,      /* valid request this build does not run (head_dim, device) */
+    VSA_ERR_MISALIGNED = 3,       /* a pointer is not 16-byte aligned */
+    VSA_ERR_WORKSPACE = 4,        /* workspace missing or smaller than vsa_workspace_bytes() */
+    VSA_ERR_CUDA = 5,             /* a CUDA runtime call or kernel launch failed */
+    VSA_ERR_TIMEOUT = 6           /* a device-side wait gave up (see vsa_device_status) */
+} vsa_status;
+
+/* ABI version of the loaded library (VSA_ABI_VERSION). */
+int32_t vsa_abi_version(void);
+
+/* Static text for a status code. */
+const char* vsa_status_string(vsa_status status);
+
+/* One-line reason for the last non-OK status returned on this host thread. */
+const char* vsa_last_error(void);
+
+/* Derived sizes of a shape: padded token count Npad and cube count C.
+ * Returns VSA_ERR_INVALID_ARGUMENT for a malformed shape. */
+vsa_status vsa_shape_info(const vsa_shape* shape, int64_t* npad, int32_t* num_cubes);
+
+/*
+ * vsa_tile — cube-major permutation with zero padding (step "pad and cut the
+ * grid into 4x4x4 cubes", teardown section "Video sparse attention selects
+ * cubes": 21x30x52 is padded to 24x32x52 = 39,936 tokens, 624 cubes).
+ *   x   [B, N, H, D] bf16, token layout (read).
+ *   xt  [B, H, Npad, D] bf16, tiled layout (written); padded rows are zero.
+ */
+vsa_status vsa_tile(const vsa_shape* shape, const vsa_bf16* x, vsa_bf16* xt, vsa_stream_t stream);
+
+/*
+ * vsa_untile — inverse of vsa_tile on the real tokens; padded rows are dropped.
+ *   xt  [B, H, Npad, D] bf16 tiled (read);  x [B, N, H, D] bf16 (written).
+ */
+vsa_status vsa_untile(const vsa_shape* shape, const vsa_bf16* xt, vsa_bf16* x, vsa_stream_t stream);
+
+/*
+ * vsa_pool — one representative vector per cube: the mean of the cube's real
+ * tokens (teardown, "Video sparse attention selects cubes", part 1 "coarse
+ * attention": each cube's query or key vectors are averaged into one).
+ *   xt    [B, H, Npad, D] bf16 tiled (read; padded rows are not read).
+ *   xbar  [B, H, C, D] float32 (written).
+ */
+vsa_status vsa_pool(const vsa_shape* shape, const vsa_bf16* xt, float* xbar, vsa_stream_t stream);
+
+/*
+ * vsa_coarse — block-level attention over the pooled cubes (same section,
+ * part 1): scores = scale * qbar kbar^T, o_coarse = softmax_rows(scores) vbar.
+ * float32 arithmetic on CUDA cores.
+ *   qbar, kbar, vbar  [B, H, C, D] float32 (read).
+ *   scores            [B, H, C, C] float32 (written): row = query cube.
+ *   o_coarse          [B, H, C, D] float32 (written).
+ */
+vsa_status vsa_coarse(const vsa_shape* shape, const float* qbar, const float* kbar, const float* vbar,
+                      float scale, float* scores, float* o_coarse, vsa_stream_t stream);
+
+/*
+ * vsa_topk — per query cube, the k key cubes with the highest coarse score
+ * (same section: the candidates are ranked and the top-k kept; 78 of 624 at
+ * 87.5% sparsity).  Equal scores go to the lower cube index; each row of the
+ * result is in ascending cube order.  Bit-exact for a given scores array.
+ *   scores  [B, H, C, C] float32 (read).   idx [B, H, C, k] int32 (written).
+ */
+vsa_status vsa_topk(const vsa_shape* shape, const float* scores, int32_t k, int32_t* idx, vsa_stream_t stream);
+
+/*
+ * vsa_fine — token-level attention of every 64-token query cube over the
+ * tokens of its selected key cubes (same section, part 2 "fine attention"),
+ * padded key tokens excluded, online softmax in float32 (teardown section
+ * "Fixed-max softmax is a numerical contract"), QK^T and PV on the tensor
+ * cores in bf16 with float32 accumulation.
+ *   qt, kt, vt  [B, H, Npad, D] bf16 tiled (read).  Padded rows of vt must be
+ *               finite (vsa_tile writes zeros); padded rows of kt may hold
+ *               anything finite.
+ *   idx         [B, H, C, k] int32 cube indices in [0, C), or NULL for all C
+ *               cubes in order (dense attention).  A cube listed twice is
+ *               attended twice.  Out-of-range entries are treated as an empty
+ *               cube (no memory outside the tensors is read).
+ *   k           entries per row of idx (ignored, taken as C, when idx is NULL).
+ *   scale       softmax scale, normally 1/sqrt(D).
+ *   o_fine      [B, H, Npad, D] bf16 (written).  Rows of padded query
+ *               positions are written but carry no meaning.
+ *   lse         [B, H, Npad] float32 natural-log sum of exp(scale*q.k) over
+ *               the attended keys (written), or NULL.
+ */
+vsa_status vsa_fine(const vsa_shape* shape, const vsa_bf16* qt, const vsa_bf16* kt, const vsa_bf16* vt,
+                    const int32_t* idx, int32_t k, float scale, vsa_bf16* o_fine, float* lse,
+                    vsa_stream_t stream);
+
+/*
+ * vsa_combine — gated merge (same section, part 3): per token and head,
+ * O = g_coarse * o_coarse[cube] + g_fine * o_fine, float32 arithmetic, bf16
+ * result.  Padded positions are written as zero.
+ *   o_coarse  [B, H, C, D] float32;  o_fine [B, H, Npad, D] bf16 tiled.
+ *   g_coarse, g_fine  [B, N, H] bf16 in token layout, or NULL (g_coarse = 0,
+ *                     g_fine = 1).
+ *   o_tiled   [B, H, Npad, D] bf16 (written).
+ */
+vsa_status vsa_combine(const vsa_shape* shape, const float* o_coarse, const vsa_bf16* o_fine,
+                       const vsa_bf16* g_coarse, const vsa_bf16* g_fine, vsa_bf16* o_tiled,
+                       vsa_stream_t stream);
+
+/* Bytes of device workspace vsa_forward needs for this shape and top-k
+ * (0 for a malformed shape). */
+size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
+
+/*
+ * vsa_forward — the whole attention call on one stream:
+ *   tile(q,k,v) -> pool -> coarse -> topk -> fine -> combine -> untile.
+ * When topk == C and both gates are NULL the call is dense attention and runs
+ * tile -> fine (all cubes) -> untile.
+ *   q, k, v      [B, N, H, D] bf16 token layout (read).
+ *   g_coarse, g_fine  [B, N, H] bf16 or NULL (see vsa_combine).
+ *   workspace    device buffer of at least vsa_workspace_bytes(shape, topk),
+ *                256-byte aligned; its contents on return are unspecified.
+ *   out          [B, N, H, D] bf16 (written).
+ */
+vsa_status vsa_forward(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                       const vsa_bf16* g_coarse, const vsa_bf16* g_fine, int32_t topk, float scale,
+                       void* workspace, size_t workspace_bytes, vsa_bf16* out, vsa_stream_t stream);
+
+/* Bytes of device workspace vsa_forward_host needs: vsa_workspace_bytes plus
+ * device staging for the inputs and the output. */
+size_t vsa_workspace_bytes_host(const vsa_shape* shape, int32_t topk);
+
+/*
+ * vsa_forward_host — vsa_forward on HOST tensors: copies q, k, v and the
+ * gates host->device (one cudaMemcpyAsync each), runs the call, copies the
+ * output device->host, all on `stream`.  Host buffers should be pinned for
+ * the copies to be asynchronous; the call returns once the work is enqueued
+ * and `out` is valid after the stream is synchronized.
+ *   q, k, v, g_coarse, g_fine, out: HOST pointers (gates may be NULL).
+ *   workspace: DEVICE buffer of vsa_workspace_bytes_host(shape, topk) bytes.
+ */
+vsa_status vsa_forward_host(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                            const vsa_bf16* g_coarse, const vsa_bf16* g_fine, int32_t topk, float scale,
+                            void* workspace, size_t workspace_bytes, vsa_bf16* out, vsa_stream_t stream);
+
+/*
+ * vsa_device_status — synchronizes `stream`, then reads and clears the
+ * current device's watchdog word.  Returns VSA_ERR_TIMEOUT if a kernel of
+ * this library gave up on a device-side wait since the last read (its output
+ * is then incomplete), VSA_ERR_CUDA if the synchronization failed, else VSA_OK.
+ */
+vsa_status vsa_device_status(vsa_stream_t stream);
+
+/*
+ * vsa_debug_wait_probe — diagnostic for the watchdog: launches one block that
+ * waits on a shared-memory barrier nothing arrives on, with the library's
+ * bounded wait, giving up after `limit_ns` nanoseconds (1 ms .. 10 s) and
+ * recording VSA_ERR_TIMEOUT for vsa_device_status().  Faults nothing and
+ * leaves the context usable.
+ */
+vsa_status vsa_debug_wait_probe(uint64_t limit_ns, vsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_B200_H */

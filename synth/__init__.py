@@ -20,23 +20,30 @@ The 480p grid (21 latent frames of 30x52 patches, 40 heads of width 128) is
 the workload of the Wan2.2 real-time inference teardown (zharfai.com),
 section "Why video attention becomes the bottleneck".
 
-Recipe (numpy ``Generator(Philox(seed))``, seed = 20261202 + 100*id + b for
-batch element b; draw order phases, Q noise, K noise, V, g_coarse, g_fine;
-all normals drawn as float32, every tensor rounded to bf16 with
-round-to-nearest-even):
+Recipe.  Batch element b of workload id W uses the numpy SeedSequence
+20261202 + 100*W + b, spawned into six children for phases, Q noise, K
+noise, V, g_coarse and g_fine; each of Q noise, K noise and V is spawned once
+more into one child per head, and every child drives its own
+``Generator(Philox(child))`` (so heads can be drawn in parallel).  Normals
+are drawn as float32; every tensor is rounded to bf16 with
+round-to-nearest-even.
 
 * iid workloads: Q, K, V ~ N(0, 1).
 * field workloads: Q = 0.5*N(0,1) + sin(0.3t + 0.2x + 0.1y + phi[h, d]) and
   K likewise with the SAME phases phi[h, d] ~ U(0, 2*pi) (one phase per head
-  and channel); V ~ N(0, 1).
+  and channel); V ~ N(0, 1).  The field is evaluated in float32 as
+  sin(a)cos(phi) + cos(a)sin(phi) with sin(a), cos(a), cos(phi), sin(phi)
+  taken from float64 and rounded to float32.
 * gates g_coarse, g_fine ~ U(0, 1), one per token and head, [B, N, H].
 
 bf16 tensors are returned as ``uint16`` bit patterns.
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
 import dataclasses
 import math
+import os
 from typing import Dict, Tuple
 
 import numpy as np
@@ -96,36 +103,64 @@ def _token_coords(grid: Tuple[int, int, int]) -> Tuple[np.ndarray, np.ndarray, n
     return n // (x * y), (n // y) % x, n % y
 
 
+def _rng(seq: np.random.SeedSequence) -> np.random.Generator:
+    return np.random.Generator(np.random.Philox(seq))
+
+
+def _workers() -> int:
+    return max(1, min(32, os.cpu_count() or 1))
+
+
 def make_batch_element(w: Workload, b: int, heads: slice | None = None) -> Dict[str, np.ndarray]:
     """Draw one batch element: q, k, v as uint16 [N, H, D]; g_coarse, g_fine as uint16 [N, H]."""
-    rng = np.random.Generator(np.random.Philox(w.seed(b)))
+    import torch
+
     n, h, d = w.tokens, w.heads, w.head_dim
+    s_phi, s_q, s_k, s_v, s_gc, s_gf = np.random.SeedSequence(w.seed(b)).spawn(6)
+    phi = _rng(s_phi).uniform(0.0, 2.0 * math.pi, size=(h, d)).astype(np.float32) if w.field else None
+    per_head = {name: seq.spawn(h) for name, seq in (("q", s_q), ("k", s_k), ("v", s_v))}
+    hsel = list(range(h) if heads is None else range(h)[heads])
+    noise = {name: np.empty((len(hsel), n, d), dtype=np.float32) for name in ("q", "k", "v")}
+
+    def draw(job):
+        name, j, hh = job
+        _rng(per_head[name][hh]).standard_normal(out=noise[name][j], dtype=np.float32)
+
+    jobs = [(name, j, hh) for name in ("q", "k", "v") for j, hh in enumerate(hsel)]
+    with cf.ThreadPoolExecutor(max_workers=_workers()) as ex:
+        list(ex.map(draw, jobs))
+    out = {}
     if w.field:
-        phi = rng.uniform(0.0, 2.0 * math.pi, size=(h, d)).astype(np.float32)
-    qn = rng.standard_normal((n, h, d), dtype=np.float32)
-    kn = rng.standard_normal((n, h, d), dtype=np.float32)
-    v = rng.standard_normal((n, h, d), dtype=np.float32)
-    gc = rng.uniform(0.0, 1.0, size=(n, h)).astype(np.float32)
-    gf = rng.uniform(0.0, 1.0, size=(n, h)).astype(np.float32)
-    if w.field:
+        # sin(a + phi) = sin(a) cos(phi) + cos(a) sin(phi), a = 0.3t + 0.2x + 0.1y, in float32
         tt, xx, yy = _token_coords(w.grid)
-        base = (0.3 * tt + 0.2 * xx + 0.1 * yy).astype(np.float32)
-        field = np.sin(base[:, None, None] + phi[None, :, :])
-        q = np.float32(0.5) * qn + field
-        k = np.float32(0.5) * kn + field
-        del field
-    else:
-        q, k = qn, kn
-    out = {
-        "q": f32_to_bf16_bits(q),
-        "k": f32_to_bf16_bits(k),
-        "v": f32_to_bf16_bits(v),
-        "g_coarse": f32_to_bf16_bits(gc),
-        "g_fine": f32_to_bf16_bits(gf),
-    }
-    if heads is not None:
-        out = {key: np.ascontiguousarray(a[:, heads]) for key, a in out.items()}
+        a = 0.3 * tt + 0.2 * xx + 0.1 * yy
+        sa = torch.from_numpy(np.sin(a).astype(np.float32))[None, :, None]
+        ca = torch.from_numpy(np.cos(a).astype(np.float32))[None, :, None]
+        ph = phi[hsel].astype(np.float64)
+        cphi = torch.from_numpy(np.cos(ph).astype(np.float32))[:, None, :]
+        sphi = torch.from_numpy(np.sin(ph).astype(np.float32))[:, None, :]
+        field = torch.empty((len(hsel), n, d), dtype=torch.float32)
+        torch.mul(sa, cphi, out=field)
+        field.addcmul_(ca, sphi)
+    for name in ("q", "k", "v"):
+        x = torch.from_numpy(noise[name])
+        if w.field and name != "v":
+            x.mul_(0.5).add_(field)
+        o = torch.empty((n, len(hsel), d), dtype=torch.bfloat16)
+        o.copy_(x.permute(1, 0, 2))                     # round to nearest even, token-major layout
+        out[name] = o.view(torch.int16).numpy().view(np.uint16)
+    del noise
+    gc = _rng(s_gc).uniform(0.0, 1.0, size=(n, h)).astype(np.float32)
+    gf = _rng(s_gf).uniform(0.0, 1.0, size=(n, h)).astype(np.float32)
+    out["g_coarse"] = np.ascontiguousarray(f32_to_bf16_bits(gc)[:, hsel])
+    out["g_fine"] = np.ascontiguousarray(f32_to_bf16_bits(gf)[:, hsel])
     return out
+
+
+def bf16_bits_torch(x) -> np.ndarray:
+    """torch's float32 -> bf16 conversion (round to nearest, ties to even), contiguous, as bits."""
+    import torch
+    return x.to(torch.bfloat16).contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
 def make_inputs(w: Workload, heads: slice | None = None) -> Dict[str, np.ndarray]:

@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* the in-tree library loads and exports every function include/vsa.h declares;
+* malformed arguments are rejected synchronously with the documented status,
+  before anything touches a device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_cube_b200 as vsa
+from block_sparse_attention_cube_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA = 1, 2, 3, 4, 5
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "vsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vsa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    declared = _declared_functions()
+    assert len(declared) >= 16
+    assert declared == sorted(_lib.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(_lib.LIB_PATH)
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_abi_version_and_status_strings():
+    assert vsa.abi_version() == 1
+    for code, name in _lib.STATUS_NAMES.items():
+        assert _lib.load().vsa_status_string(code).decode() == name
+
+
+def _shape(b=1, h=2, d=128, grid=(8, 8, 8)):
+    return vsa.Shape(b, h, d, grid).c()
+
+
+def test_shape_info():
+    assert vsa.shape_info(vsa.Shape(1, 40, 128, (21, 30, 52))) == (39936, 624)
+    assert vsa.shape_info(vsa.Shape(2, 40, 128, (21, 45, 80))) == (92160, 1440)
+    assert vsa.shape_info(vsa.Shape(1, 4, 128, (7, 15, 16))) == (2048, 32)
+
+
+@pytest.mark.parametrize("shape,code", [
+    (_shape(b=0), INVALID), (_shape(h=0), INVALID), (_shape(grid=(0, 8, 8)), INVALID),
+    (_shape(d=0), INVALID), (_shape(d=96), UNSUPPORTED), (_shape(d=256), UNSUPPORTED),
+    (_shape(b=1, h=200, grid=(256, 256, 256)), INVALID),           # more than 2^31 tiled rows
+    (_shape(b=300, h=300, grid=(4, 4, 4)), UNSUPPORTED),           # batch*heads above the grid limit
+])
+def test_shape_errors(shape, code):
+    st = vsa.raw_call("vsa_tile", ctypes.byref(shape), ctypes.c_void_p(4096), ctypes.c_void_p(1 << 40), None)
+    assert st == code, vsa.last_error()
+    assert vsa.last_error()
+
+
+def test_null_and_misaligned_pointers():
+    s = _shape()
+    assert vsa.raw_call("vsa_tile", ctypes.byref(s), None, ctypes.c_void_p(4096), None) == INVALID
+    assert "x is NULL" in vsa.last_error()
+    assert vsa.raw_call("vsa_tile", ctypes.byref(s), ctypes.c_void_p(4104), ctypes.c_void_p(1 << 40), None) == MISALIGNED
+    assert vsa.raw_call("vsa_shape_info", None, None, None) == INVALID
+
+
+def test_overlapping_input_and_output_rejected():
+    s = _shape()
+    base = 1 << 40
+    st = vsa.raw_call("vsa_tile", ctypes.byref(s), ctypes.c_void_p(base), ctypes.c_void_p(base + 1024), None)
+    assert st == INVALID and "overlaps" in vsa.last_error()
+
+
+@pytest.mark.parametrize("k", [0, -1, 9])
+def test_topk_out_of_range(k):
+    s = _shape()   # 8 cubes
+    st = vsa.raw_call("vsa_topk", ctypes.byref(s), ctypes.c_void_p(1 << 40), k, ctypes.c_void_p(1 << 41), None)
+    assert st == INVALID and "top-k" in vsa.last_error()
+
+
+@pytest.mark.parametrize("scale", [0.0, -1.0, float("inf"), float("nan")])
+def test_bad_scale(scale):
+    s = _shape()
+    p = [ctypes.c_void_p((1 << 40) + i * (1 << 32)) for i in range(5)]
+    st = vsa.raw_call("vsa_fine", ctypes.byref(s), p[0], p[1], p[2], None, 0, scale, p[3], None, None)
+    assert st == INVALID and "scale" in vsa.last_error()
+
+
+def test_workspace_checks():
+    s = _shape()
+    need = vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 2)
+    assert need > 0
+    assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 0) == 0
+    assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 9) == 0
+    assert vsa.raw_call("vsa_workspace_bytes_host", ctypes.byref(s), 2) > need
+    p = [ctypes.c_void_p((1 << 40) + i * (1 << 32)) for i in range(6)]
+    args = (ctypes.byref(s), p[0], p[1], p[2], None, None, 2, 0.125)
+    assert vsa.raw_call("vsa_forward", *args, None, need, p[3], None) == WORKSPACE
+    assert vsa.raw_call("vsa_forward", *args, p[4], need - 1, p[3], None) == WORKSPACE
+    assert vsa.raw_call("vsa_forward", *args, ctypes.c_void_p(p[4].value + 16), need, p[3], None) == MISALIGNED
+
+
+def test_workspace_size_480p_matches_layout():
+    # tiled q,k,v,o_fine (4 x 39936*40*128*2 B) + pooled q,k,v,o_coarse (4 x 624*40*128*4 B)
+    # + scores (624*624*40*4 B) + idx (624*40*32*4 B), each rounded up to 256 B
+    s = vsa.Shape(1, 40, 128, (21, 30, 52)).c()
+    up = lambda n: (n + 255) // 256 * 256
+    expect = 4 * up(39936 * 40 * 128 * 2) + 4 * up(624 * 40 * 128 * 4) + up(624 * 624 * 40 * 4) + up(624 * 40 * 32 * 4)
+    assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 32) == expect
+
+
+def test_probe_limit_checked_before_device():
+    assert vsa.raw_call("vsa_debug_wait_probe", 10, None) == INVALID
+    assert vsa.raw_call("vsa_debug_wait_probe", 10**12, None) == INVALID

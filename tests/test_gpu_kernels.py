@@ -1,0 +1,309 @@
+"""GPU parity of every step of the path against the fp64 oracle, on sizes the
+oracle runs in full (several cubes, padded and unpadded grids, ragged pairs)
+and on the edge cases of the method."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_cube_b200 as vsa
+import synth
+from oracle import vsa_oracle as O
+from tests._util import (COARSE_REL_L2, LSE_ABS, bf16_bits, check_close, check_heads, from_dev, near_tie_ok,
+                         to_dev)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["tiny_8x8x8", "tiny_8x8x8_all", "padded_7x15x16"]
+EDGE_SHAPES = {
+    # name: (batch, heads, head_dim, grid, topk)
+    "odd_cubes_4x4x12": (1, 3, 128, (4, 4, 12), 2),       # C = 3: last pair has one cube
+    "single_cube_3x2x4": (1, 2, 128, (3, 2, 4), 1),       # C = 1, partial cube
+    "ragged_9x6x5_d64": (2, 2, 64, (9, 6, 5), 4),         # B = 2, d = 64, partial cubes on every axis
+    "wide_5x9x30": (1, 2, 128, (5, 9, 30), 7),            # C = 2*3*8 = 48, odd k
+}
+
+
+def _workload(name):
+    if name in synth.WORKLOADS:
+        return synth.WORKLOADS[name]
+    b, h, d, grid, k = EDGE_SHAPES[name]
+    return synth.custom_workload(name, b, h, d, grid, k, field=True, wid=91 + list(EDGE_SHAPES).index(name))
+
+
+def _shape(w):
+    return vsa.Shape(w.batch, w.heads, w.head_dim, w.grid)
+
+
+@pytest.fixture(scope="module", params=SMALL + list(EDGE_SHAPES))
+def case(request):
+    w = _workload(request.param)
+    x = synth.make_inputs(w)
+    dev = {k: to_dev(v) for k, v in x.items()}
+    f64 = {k: O.bf16_to_f64(v) for k, v in x.items()}
+    return w, x, dev, f64
+
+
+def test_tile_bit_exact_and_roundtrip(case):
+    w, x, dev, _ = case
+    s = _shape(w)
+    for name in ("q", "k", "v"):
+        xt = vsa.tile(dev[name], s)
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_bits(xt), O.tile(x[name], w.grid)), name
+        back = vsa.untile(xt, s)
+        assert np.array_equal(bf16_bits(back), x[name]), name
+
+
+def test_pool_matches_oracle(case):
+    w, _, dev, f64 = case
+    s = _shape(w)
+    for name in ("q", "k", "v"):
+        got = from_dev(vsa.pool(vsa.tile(dev[name], s), s))
+        ref = O.pool(O.tile(f64[name], w.grid), w.grid)
+        np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-6)
+
+
+def test_coarse_on_shared_inputs(case):
+    """vsa_coarse on float32 pooled vectors the test generates, against the oracle's coarse step."""
+    w, _, _, f64 = case
+    s = _shape(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    bars32 = [O.pool(O.tile(f64[n], w.grid), w.grid).astype(np.float32) for n in ("q", "k", "v")]
+    scores, oc = vsa.coarse(*(torch.from_numpy(b).cuda() for b in bars32), s, scale)
+    r_scores, r_oc = O.coarse(*(b.astype(np.float64) for b in bars32), scale)
+    g_scores, g_oc = from_dev(scores), from_dev(oc)
+    np.testing.assert_allclose(g_scores, r_scores, rtol=0, atol=1e-5 * max(1.0, np.abs(r_scores).max()))
+    assert np.linalg.norm(g_oc - r_oc) / np.linalg.norm(r_oc) <= COARSE_REL_L2
+
+
+def test_topk_bit_exact_on_shared_scores(case):
+    """vsa_topk on float32 score arrays the test generates (many exact ties, signed zeros)."""
+    w = case[0]
+    s = _shape(w)
+    _, C = vsa.shape_info(s)
+    rng = np.random.default_rng(11)
+    shape = (w.batch, w.heads, C, C)
+    arrays = [rng.integers(-3, 4, size=shape).astype(np.float32),
+              (rng.standard_normal(shape) * 0.1).astype(np.float32),
+              np.where(rng.random(shape) < 0.5, np.float32(-0.0), np.float32(0.0))]
+    for a in arrays:
+        for k in sorted({1, w.topk, C}):
+            g = vsa.topk(torch.from_numpy(a).cuda(), s, k).cpu().numpy()
+            assert np.array_equal(g, O.topk(a.astype(np.float64), k)), k
+
+
+def test_selection_matches_oracle(case):
+    """The GPU's own pool -> coarse -> top-k against the oracle's, up to documented near-ties."""
+    w, _, dev, f64 = case
+    s = _shape(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    bars = [vsa.pool(vsa.tile(dev[n], s), s) for n in ("q", "k", "v")]
+    scores, oc = vsa.coarse(*bars, s, scale)
+    g_idx = vsa.topk(scores, s, w.topk).cpu().numpy()
+    ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, w.topk)
+    ok = near_tie_ok(g_idx, ora["idx"], ora["scores"], w.topk)
+    assert ok.all(), f"{(~ok).sum()} rows differ beyond the near-tie rule"
+    np.testing.assert_allclose(from_dev(scores), ora["scores"], rtol=0,
+                               atol=1e-5 * max(1.0, np.abs(ora["scores"]).max()))
+    rel = np.linalg.norm(from_dev(oc) - ora["o_coarse"]) / np.linalg.norm(ora["o_coarse"])
+    assert rel <= COARSE_REL_L2, rel
+
+
+def test_fine_sparse_matches_oracle(case):
+    """The fine kernel on the oracle's own selection against the oracle's fine step."""
+    w, _, dev, f64 = case
+    s = _shape(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, w.topk, scale)
+    qt, kt, vt = (vsa.tile(dev[n], s) for n in ("q", "k", "v"))
+    o, lse = vsa.fine(qt, kt, vt, s, torch.from_numpy(ora["idx"]).cuda(), scale)
+    check_heads(from_dev(o), ora["o_fine"], w.grid, "o_fine")
+    valid = O.key_valid_mask(w.grid)
+    err = np.abs(from_dev(lse)[:, :, valid] - ora["lse"][:, :, valid]).max()
+    assert err <= LSE_ABS, err
+
+
+def test_dense_matches_oracle(case):
+    w, _, dev, f64 = case
+    s = _shape(w)
+    qt, kt, vt = (vsa.tile(dev[n], s) for n in ("q", "k", "v"))
+    o, lse = vsa.fine(qt, kt, vt, s, None)
+    out = from_dev(vsa.untile(o, s))
+    r_out, r_lse = O.dense(f64["q"], f64["k"], f64["v"], w.grid)
+    for b in range(w.batch):
+        for h in range(w.heads):
+            check_close(out[b, :, h], r_out[b, :, h], f"dense[b={b},h={h}]")
+    g_lse = from_dev(lse)
+    g_lse_tok = O.untile(g_lse[..., None], w.grid)[..., 0]
+    assert np.abs(g_lse_tok - r_lse).max() <= LSE_ABS
+    # the whole call in dense mode (top-k = C, no gates) gives the same bits
+    npad, C = vsa.shape_info(s)
+    out2 = vsa.forward(dev["q"], dev["k"], dev["v"], s, C)
+    assert np.array_equal(bf16_bits(out2), bf16_bits(vsa.untile(o, s)))
+
+
+def _compare_call(w, dev, f64, k, scale, gates=True):
+    """The whole call against the oracle's, excluding only query cubes whose
+    selection differs through a documented near-tie."""
+    s = _shape(w)
+    gc, gf = (dev["g_coarse"], dev["g_fine"]) if gates else (None, None)
+    out = vsa.forward(dev["q"], dev["k"], dev["v"], s, k, scale, gc, gf)
+    bars = [vsa.pool(vsa.tile(dev[n], s), s) for n in ("q", "k", "v")]
+    g_idx = vsa.topk(vsa.coarse(*bars, s, scale)[0], s, k).cpu().numpy()
+    ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, k, scale,
+                    f64["g_coarse"] if gates else None, f64["g_fine"] if gates else None)
+    agree = np.all(g_idx == ora["idx"], axis=-1)                     # [B, H, C]
+    assert near_tie_ok(g_idx, ora["idx"], ora["scores"], k).all()
+    src = O.tile_source_index(w.grid)
+    got = from_dev(out)
+    for b in range(w.batch):
+        for h in range(w.heads):
+            keep = np.zeros(src.size, bool)
+            for c in np.nonzero(agree[b, h])[0]:
+                keep[c * 64:(c + 1) * 64] = True
+            toks = src[keep & (src >= 0)]
+            assert toks.size > 0.9 * w.tokens
+            check_close(got[b, toks, h], ora["out"][b, toks, h], f"out[b={b},h={h}] k={k}")
+
+
+def test_forward_matches_oracle(case):
+    w, _, dev, f64 = case
+    _compare_call(w, dev, f64, w.topk, 1 / math.sqrt(w.head_dim))
+
+
+def test_combine_matches_oracle(case):
+    w, _, dev, f64 = case
+    s = _shape(w)
+    rng = np.random.default_rng(5)
+    npad, C = vsa.shape_info(s)
+    oc = torch.from_numpy(rng.normal(size=(w.batch, w.heads, C, w.head_dim)).astype(np.float32)).cuda()
+    of_bits = synth.f32_to_bf16_bits(rng.normal(size=(w.batch, w.heads, npad, w.head_dim)).astype(np.float32))
+    of = to_dev(of_bits)
+    for gc, gf in ((dev["g_coarse"], dev["g_fine"]), (None, None), (dev["g_coarse"], None)):
+        got = from_dev(vsa.combine(oc, of, s, gc, gf))
+        ref = O.combine(oc.cpu().numpy().astype(np.float64), O.bf16_to_f64(of_bits),
+                        None if gc is None else f64["g_coarse"], None if gf is None else f64["g_fine"], w.grid)
+        # one bf16 rounding of a float32 value
+        np.testing.assert_allclose(got, ref, rtol=2 ** -8, atol=1e-6)
+
+
+# ---------------------------------------------------------------- edge cases
+def _run_fine(w, x, idx=None, scale=None):
+    s = _shape(w)
+    d = {k: to_dev(v) for k, v in x.items()}
+    qt, kt, vt = (vsa.tile(d[n], s) for n in ("q", "k", "v"))
+    return qt, kt, vt, s
+
+
+def test_zero_query_selects_first_cubes_and_averages_values():
+    w = synth.WORKLOADS["padded_7x15x16"]
+    x = synth.make_inputs(w)
+    x["q"] = np.zeros_like(x["q"])
+    qt, kt, vt, s = _run_fine(w, x)
+    bars = [vsa.pool(t, s) for t in (qt, kt, vt)]
+    scores, _ = vsa.coarse(*bars, s)
+    idx = vsa.topk(scores, s, 5)
+    first5 = np.broadcast_to(np.arange(5, dtype=np.int32), idx.shape)
+    assert np.array_equal(idx.cpu().numpy(), first5)
+    o, lse = vsa.fine(qt, kt, vt, s, idx)
+    r_o, r_lse = O.fine(*(O.tile(O.bf16_to_f64(x[n]), w.grid) for n in ("q", "k", "v")), first5,
+                        1 / math.sqrt(128), w.grid)
+    check_heads(from_dev(o), r_o, w.grid, "o_fine(q=0)")
+
+
+def test_constant_values_give_ones():
+    w = synth.WORKLOADS["padded_7x15x16"]
+    x = synth.make_inputs(w)
+    x["v"] = np.full_like(x["v"], 0x3F80)   # bf16 1.0
+    qt, kt, vt, s = _run_fine(w, x)
+    o, _ = vsa.fine(qt, kt, vt, s, None)
+    got = from_dev(o)[:, :, O.key_valid_mask(w.grid)]
+    assert np.abs(got - 1.0).max() <= 2 ** -8
+
+
+def test_overflow_scores_stay_finite():
+    """q.k/sqrt(d) near 150-200: an unshifted fp32 exp overflows; the online softmax must not."""
+    w = synth.WORKLOADS["padded_7x15x16"]
+    x = synth.make_inputs(w)
+    for n in ("q", "k"):
+        x[n] = synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(x[n]) * 16.0)
+    f64 = {k: O.bf16_to_f64(v) for k, v in x.items()}
+    qt, kt, vt, s = _run_fine(w, x)
+    o, lse = vsa.fine(qt, kt, vt, s, None)
+    r_o, r_lse = O.fine(*(O.tile(f64[n], w.grid) for n in ("q", "k", "v")), None, 1 / math.sqrt(128), w.grid)
+    valid = O.key_valid_mask(w.grid)
+    assert r_lse[:, :, valid].max() > 100
+    check_heads(from_dev(o), r_o, w.grid, "o_fine(overflow)")
+    assert np.abs(from_dev(lse)[:, :, valid] - r_lse[:, :, valid]).max() <= LSE_ABS
+
+
+def test_padded_key_rows_are_masked():
+    """Large finite values written into the padded rows of the tiled K do not change the result."""
+    w = synth.WORKLOADS["padded_7x15x16"]
+    x = synth.make_inputs(w)
+    qt, kt, vt, s = _run_fine(w, x)
+    o1, l1 = vsa.fine(qt, kt, vt, s, None)
+    pad = torch.from_numpy(~O.key_valid_mask(w.grid)).cuda()
+    kt2 = kt.clone()
+    kt2[:, :, pad, :] = 1.0e4
+    o2, l2 = vsa.fine(qt, kt2, vt, s, None)
+    valid = torch.from_numpy(O.key_valid_mask(w.grid)).cuda()
+    assert torch.equal(o1[:, :, valid], o2[:, :, valid])
+    assert torch.equal(l1[:, :, valid], l2[:, :, valid])
+
+
+def test_duplicate_and_out_of_range_indices():
+    """A listed-twice cube is attended twice; an out-of-range entry is an empty cube."""
+    w = synth.WORKLOADS["padded_7x15x16"]
+    x = synth.make_inputs(w)
+    f64 = {k: O.bf16_to_f64(v) for k, v in x.items()}
+    qt, kt, vt, s = _run_fine(w, x)
+    npad, C = vsa.shape_info(s)
+    rng = np.random.default_rng(3)
+    idx = np.sort(rng.integers(0, C, size=(1, w.heads, C, 6)), axis=-1).astype(np.int32)
+    idx[..., 1] = idx[..., 0]                      # a duplicate in every row
+    bad = idx.copy()
+    bad[..., -1] = C + 7                           # and an out-of-range entry
+    tq = [O.tile(f64[n], w.grid) for n in ("q", "k", "v")]
+    o, lse = vsa.fine(qt, kt, vt, s, torch.from_numpy(idx).cuda())
+    r_o, r_lse = O.fine(*tq, idx, 1 / math.sqrt(128), w.grid)
+    check_heads(from_dev(o), r_o, w.grid, "o_fine(dup)")
+    o2, _ = vsa.fine(qt, kt, vt, s, torch.from_numpy(bad).cuda())
+    r_o2, _ = O.fine(*tq, bad[..., :-1], 1 / math.sqrt(128), w.grid)
+    check_heads(from_dev(o2), r_o2, w.grid, "o_fine(out of range)")
+
+
+def test_k_equals_one_and_k_equals_c():
+    w = synth.WORKLOADS["padded_7x15x16"]
+    x = synth.make_inputs(w)
+    f64 = {k: O.bf16_to_f64(v) for k, v in x.items()}
+    d = {k: to_dev(v) for k, v in x.items()}
+    npad, C = vsa.shape_info(_shape(w))
+    for k in (1, C):
+        _compare_call(w, d, f64, k, 1 / math.sqrt(128))
+
+
+def test_repeated_calls_are_deterministic():
+    w = synth.WORKLOADS["padded_7x15x16"]
+    x = synth.make_inputs(w)
+    d = {k: to_dev(v) for k, v in x.items()}
+    s = _shape(w)
+    a = vsa.forward(d["q"], d["k"], d["v"], s, w.topk, None, d["g_coarse"], d["g_fine"])
+    b = vsa.forward(d["q"], d["k"], d["v"], s, w.topk, None, d["g_coarse"], d["g_fine"])
+    assert torch.equal(a, b)
+
+
+def test_forward_host_matches_device_forward():
+    w = synth.WORKLOADS["padded_7x15x16"]
+    x = synth.make_inputs(w)
+    d = {k: to_dev(v) for k, v in x.items()}
+    h = {k: d[k].cpu().pin_memory() for k in d}
+    s = _shape(w)
+    ref = vsa.forward(d["q"], d["k"], d["v"], s, w.topk, None, d["g_coarse"], d["g_fine"])
+    ws = vsa.alloc_workspace(s, w.topk, host_io=True)
+    out = torch.empty_like(h["q"]).pin_memory()
+    vsa.forward_host(h["q"], h["k"], h["v"], s, w.topk, ws, out, None, h["g_coarse"], h["g_fine"])
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(out, ref.cpu())
