@@ -6,7 +6,8 @@ objects are linked into one shared library with the CUDA runtime linked
 statically, so the library loads on a host without a GPU driver (its entry
 points then return VSA_ERR_CUDA) and needs nothing beyond libc at load time.
 
-Usage: ``python -m block_sparse_attention_cube_b200.build_lib [--force] [--ptxas-v]``
+Usage: ``python block_sparse_attention_cube_b200/build_lib.py [--force] [--ptxas-v]`` (run it as a
+file: importing the package loads the library this script builds).
 """
 from __future__ import annotations
 
