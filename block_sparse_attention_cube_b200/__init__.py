@@ -182,6 +182,28 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, shape: Shape, top
     return out
 
 
+def forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, shape: Shape, topk_k: int,
+                    scale: Optional[float] = None, g_coarse: Optional[torch.Tensor] = None,
+                    g_fine: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """vsa_forward_noalloc: the whole call on the library's static device workspace.
+
+    For callers that cannot allocate device memory (see include/vsa.h); the
+    output buffer is still the caller's (allocated here only when omitted).
+    Shapes whose workspace exceeds VSA_NOALLOC_WORKSPACE_BYTES raise VsaError.
+    """
+    scale = default_scale(shape) if scale is None else scale
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_L.vsa_forward_noalloc(ctypes.byref(shape.c()), _ptr(q, torch.bfloat16, "q"),
+                                  _ptr(k, torch.bfloat16, "k"), _ptr(v, torch.bfloat16, "v"),
+                                  _ptr(g_coarse, torch.bfloat16, "g_coarse"), _ptr(g_fine, torch.bfloat16, "g_fine"),
+                                  topk_k, scale, _ptr(out, torch.bfloat16, "out"), _stream()))
+    return out
+
+
+NOALLOC_WORKSPACE_BYTES = 32 << 20
+
+
 def _host_ptr(t: Optional[torch.Tensor], name: str) -> Optional[int]:
     if t is None:
         return None

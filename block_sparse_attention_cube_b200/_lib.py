@@ -46,6 +46,7 @@ SIGNATURES = {
     "vsa_forward": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _I32, _F32, _P, _SZ, _P, _P]),
     "vsa_workspace_bytes_host": (_SZ, [_SP, _I32]),
     "vsa_forward_host": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _I32, _F32, _P, _SZ, _P, _P]),
+    "vsa_forward_noalloc": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _I32, _F32, _P, _P]),
     "vsa_device_status": (ctypes.c_int, [_P]),
     "vsa_debug_wait_probe": (ctypes.c_int, [ctypes.c_uint64, _P]),
 }
@@ -55,7 +56,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise ImportError(
             f"CUDA library {path} is missing; build it with "
-            "`python -m block_sparse_attention_cube_b200.build_lib` (there is no CPU fallback)")
+            "`python block_sparse_attention_cube_b200/build_lib.py` (there is no CPU fallback)")
     lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

@@ -217,6 +217,8 @@ int sm_count() {
     return counts[dev];
 }
 
+vsa_status set_last_error(vsa_status st, const char* message) { return fail(st, "%s", message); }
+
 }  // namespace vsa
 
 using namespace vsa;

@@ -22,6 +22,9 @@ struct Dims {
     int64_t rows;       // B * H * Npad rows of the tiled layout
 };
 
+// Records `message` as this thread's vsa_last_error() text and returns `st`.
+vsa_status set_last_error(vsa_status st, const char* message);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 

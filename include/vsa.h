@@ -206,6 +206,35 @@ vsa_status vsa_forward_host(const vsa_shape* shape, const vsa_bf16* q, const vsa
                             const vsa_bf16* g_coarse, const vsa_bf16* g_fine, int32_t topk, float scale,
                             void* workspace, size_t workspace_bytes, vsa_bf16* out, vsa_stream_t stream);
 
+/* Size of the static device workspace used by vsa_forward_noalloc (32 MiB). */
+#define VSA_NOALLOC_WORKSPACE_BYTES ((size_t)32 << 20)
+
+/*
+ * vsa_forward_noalloc — vsa_forward for callers that cannot allocate device
+ * memory.  The pages have no counterpart; this is an interface convenience.
+ * Examples are a plugin that a host runtime hands only its input and output
+ * buffers, a runtime whose memory pool owns the device and forbids
+ * out-of-band cudaMalloc (which synchronizes the device and fragments the
+ * pool), and real-time code that must not allocate after start-up.
+ * Arguments are those of vsa_forward without the workspace: q, k, v, gates
+ * and out are caller-owned DEVICE buffers.  The workspace is a static
+ * device array of VSA_NOALLOC_WORKSPACE_BYTES inside the library, so the
+ * call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine).  Each GPU on which the library's module is loaded holds that
+ * array until the process exits.
+ *   - A shape whose vsa_workspace_bytes() exceeds VSA_NOALLOC_WORKSPACE_BYTES
+ *     is rejected with VSA_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents (nothing in it needs to start at zero).  Calls that overlap on
+ *     the GPU race on it: serialize them (one stream, or events).
+ */
+vsa_status vsa_forward_noalloc(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                               const vsa_bf16* g_coarse, const vsa_bf16* g_fine, int32_t topk, float scale,
+                               vsa_bf16* out, vsa_stream_t stream);
+
 /*
  * vsa_device_status — synchronizes `stream`, then reads and clears the
  * current device's watchdog word.  Returns VSA_ERR_TIMEOUT if a kernel of
