@@ -290,7 +290,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     dense_ms_max = reduce_max(dense_ms, world)
 
     # ---- per-stage breakdown (same kernels through the per-stage entry points)
-    names = ["tile", "pool", "coarse", "topk", "fine", "combine", "untile"]
+    names = ["tile", "pool", "coarse", "topk+group", "fine", "combine", "untile"]
     acc = {n: [] for n in names}
     acc["fine_dense"] = []
     for it in range(args.warmup + args.steps):
@@ -303,8 +303,9 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         scores, oc = vsa.coarse(*bars, s, scale)
         e[3].record(stream)
         idx = vsa.topk(scores, s, w.topk)
+        order = vsa.group(scores, s)
         e[4].record(stream)
-        of, _ = vsa.fine(qt, kt, vt, s, idx, scale, want_lse=False)
+        of, _ = vsa.fine(qt, kt, vt, s, idx, scale, want_lse=False, order=order)
         e[5].record(stream)
         ot = vsa.combine(oc, of, s, d["g_coarse"], d["g_fine"])
         e[6].record(stream)
@@ -317,7 +318,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
             for j, n in enumerate(names):
                 acc[n].append(e[j].elapsed_time(e[j + 1]))
             acc["fine_dense"].append(e[7].elapsed_time(e[8]))
-        del qt, kt, vt, bars, scores, oc, idx, of, ot
+        del qt, kt, vt, bars, scores, oc, idx, order, of, ot
     stage_ms = {n: round(statistics.mean(v), 4) for n, v in acc.items()}
 
     # ---- end to end through vsa_forward_host (pinned host buffers, copies inside the timed region)
@@ -379,7 +380,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                      "per_launch": "4*B*H*Npad*k*64*D executed flops (64x64 cube tiles of the k selected cubes)"},
         "e2e": {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "vsa_forward_host (pinned host q/k/v/gates in, host out)"},
-        "gpu_launches": 11 * args.steps,
+        "gpu_launches": 12 * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
         "context": {"pages_dense_call_ms_b200": 17.0, "pages_vsa_kernel_ms_b200_k78": 4.719,

@@ -127,15 +127,29 @@ def topk(scores: torch.Tensor, shape: Shape, k: int) -> torch.Tensor:
     return idx
 
 
+def group(scores: torch.Tensor, shape: Shape) -> torch.Tensor:
+    """Work order for fine(): per head, query cubes with similar selections next to each other."""
+    _, c = shape_info(shape)
+    order = torch.empty((shape.batch, shape.heads, c), dtype=torch.int32, device=scores.device)
+    _check(_L.vsa_group(ctypes.byref(shape.c()), _ptr(scores, torch.float32, "scores"),
+                        _ptr(order, torch.int32, "order"), _stream()))
+    return order
+
+
 def fine(qt: torch.Tensor, kt: torch.Tensor, vt: torch.Tensor, shape: Shape, idx: Optional[torch.Tensor] = None,
-         scale: Optional[float] = None, want_lse: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    """Fine attention over the selected cubes (idx [B,H,C,k] int32, or None for all cubes)."""
+         scale: Optional[float] = None, want_lse: bool = True,
+         order: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Fine attention over the selected cubes (idx [B,H,C,k] int32, or None for all cubes).
+
+    `order` ([B,H,C] int32 permutation, e.g. from group()) sets the work order only.
+    """
     scale = default_scale(shape) if scale is None else scale
     k = int(idx.shape[-1]) if idx is not None else 0
     o = torch.empty_like(qt)
     lse = torch.empty(qt.shape[:3], dtype=torch.float32, device=qt.device) if want_lse else None
     _check(_L.vsa_fine(ctypes.byref(shape.c()), _ptr(qt, torch.bfloat16, "qt"), _ptr(kt, torch.bfloat16, "kt"),
-                       _ptr(vt, torch.bfloat16, "vt"), _ptr(idx, torch.int32, "idx"), k, scale,
+                       _ptr(vt, torch.bfloat16, "vt"), _ptr(idx, torch.int32, "idx"), k,
+                       _ptr(order, torch.int32, "order"), scale,
                        _ptr(o, torch.bfloat16, "o_fine"), _ptr(lse, torch.float32, "lse"), _stream()))
     return o, lse
 

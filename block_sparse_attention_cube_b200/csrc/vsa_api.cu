@@ -116,16 +116,18 @@ size_t gate_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.N * d.H *
 size_t pooled_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C * d.D * 4; }
 size_t score_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C * d.C * 4; }
 size_t idx_bytes(const Dims& d, int k) { return static_cast<size_t>(d.B) * d.H * d.C * k * 4; }
+size_t order_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C * 4; }
 
 constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Workspace of vsa_forward: qt | kt | vt | o_fine | qbar | kbar | vbar | o_coarse | scores | idx.
+// Workspace of vsa_forward: qt | kt | vt | o_fine | qbar | kbar | vbar | o_coarse | scores | idx | order.
 // The merged output (combine) reuses qt, which is dead after the fine stage.
 struct Carve {
     uint16_t *qt, *kt, *vt, *of;
     float *qbar, *kbar, *vbar, *oc, *scores;
     int32_t* idx;
+    int32_t* order;
     size_t bytes;
 };
 
@@ -148,6 +150,7 @@ Carve carve(const Dims& d, int k, void* ws) {
     c.oc = reinterpret_cast<float*>(take(pooled_bytes(d)));
     c.scores = reinterpret_cast<float*>(take(score_bytes(d)));
     c.idx = reinterpret_cast<int32_t*>(take(idx_bytes(d, k)));
+    c.order = reinterpret_cast<int32_t*>(take(order_bytes(d)));
     c.bytes = off;
     return c;
 }
@@ -184,7 +187,7 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
     VSA_CUDA(launch_tile(d, t, s), "tile launch");
     if (dense) {
         const char* why = nullptr;
-        cudaError_t e = launch_fine(d, c.qt, c.kt, c.vt, nullptr, d.C, scale, c.of, nullptr, s, &why);
+        cudaError_t e = launch_fine(d, c.qt, c.kt, c.vt, nullptr, d.C, nullptr, scale, c.of, nullptr, s, &why);
         if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "fine launch");
         VSA_CUDA(launch_untile(d, c.of, out, s), "untile launch");
         return VSA_OK;
@@ -194,8 +197,13 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
     VSA_CUDA(launch_pool(d, pin, pout, 3, s), "pool launch");
     VSA_CUDA(launch_coarse(d, c.qbar, c.kbar, c.vbar, scale, c.scores, c.oc, s), "coarse launch");
     VSA_CUDA(launch_topk(d, c.scores, topk, c.idx, s), "topk launch");
+    const int32_t* order = nullptr;
+    if (d.C <= kGroupMaxC) {
+        VSA_CUDA(launch_group(d, c.scores, c.order, s), "group launch");
+        order = c.order;
+    }
     const char* why = nullptr;
-    cudaError_t e = launch_fine(d, c.qt, c.kt, c.vt, c.idx, topk, scale, c.of, nullptr, s, &why);
+    cudaError_t e = launch_fine(d, c.qt, c.kt, c.vt, c.idx, topk, order, scale, c.of, nullptr, s, &why);
     if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "fine launch");
     uint16_t* o_tiled = c.qt;   // qt is no longer read after the fine stage
     VSA_CUDA(launch_combine(d, c.oc, c.of, gc, gf, o_tiled, s), "combine launch");
@@ -317,8 +325,21 @@ vsa_status vsa_topk(const vsa_shape* shape, const float* scores, int32_t k, int3
     return VSA_OK;
 }
 
+vsa_status vsa_group(const vsa_shape* shape, const float* scores, int32_t* order, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(need_ptr(scores, "scores"));
+    VSA_TRY(need_ptr(order, "order"));
+    if (d.C > kGroupMaxC) return fail(VSA_ERR_UNSUPPORTED, "grouping supports at most %d cubes (got %d)", kGroupMaxC, d.C);
+    VSA_TRY(check_disjoint({{scores, score_bytes(d), "scores"}}, {{order, order_bytes(d), "order"}}));
+    VSA_TRY(check_device());
+    VSA_CUDA(launch_group(d, scores, order, as_stream(stream)), "group launch");
+    return VSA_OK;
+}
+
 vsa_status vsa_fine(const vsa_shape* shape, const vsa_bf16* qt, const vsa_bf16* kt, const vsa_bf16* vt,
-                    const int32_t* idx, int32_t k, float scale, vsa_bf16* o_fine, float* lse, vsa_stream_t stream) {
+                    const int32_t* idx, int32_t k, const int32_t* order, float scale, vsa_bf16* o_fine, float* lse,
+                    vsa_stream_t stream) {
     Dims d{};
     VSA_TRY(make_dims(shape, &d));
     if (idx) VSA_TRY(check_k(d, k));
@@ -326,15 +347,17 @@ vsa_status vsa_fine(const vsa_shape* shape, const vsa_bf16* qt, const vsa_bf16* 
     VSA_TRY(need_ptr(kt, "kt"));
     VSA_TRY(need_ptr(vt, "vt"));
     VSA_TRY(opt_ptr(idx, "idx"));
+    VSA_TRY(opt_ptr(order, "order"));
     VSA_TRY(need_ptr(o_fine, "o_fine"));
     VSA_TRY(opt_ptr(lse, "lse"));
     VSA_TRY(check_scale(scale));
     const size_t tb = tiled_bytes(d);
-    VSA_TRY(check_disjoint({{qt, tb, "qt"}, {kt, tb, "kt"}, {vt, tb, "vt"}, {idx, idx ? idx_bytes(d, k) : 0, "idx"}},
+    VSA_TRY(check_disjoint({{qt, tb, "qt"}, {kt, tb, "kt"}, {vt, tb, "vt"}, {idx, idx ? idx_bytes(d, k) : 0, "idx"},
+                            {order, order ? order_bytes(d) : 0, "order"}},
                            {{o_fine, tb, "o_fine"}, {lse, lse ? static_cast<size_t>(d.rows) * 4 : 0, "lse"}}));
     VSA_TRY(check_device());
     const char* why = nullptr;
-    cudaError_t e = launch_fine(d, qt, kt, vt, idx, k, scale, o_fine, lse, as_stream(stream), &why);
+    cudaError_t e = launch_fine(d, qt, kt, vt, idx, k, order, scale, o_fine, lse, as_stream(stream), &why);
     if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "fine launch");
     return VSA_OK;
 }

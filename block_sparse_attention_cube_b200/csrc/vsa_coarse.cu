@@ -199,7 +199,90 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(int64_t rows, int C, int
     }
 }
 
+// Work-order for the fine stage: per (b, h), the query cubes sorted by the
+// indices of their three highest-scoring key cubes (ties to the lower index),
+// so that consecutive cubes, which the fine kernel processes as a group of
+// four sharing one key/value stream, tend to select the same key cubes.  The
+// result is a permutation of [0, C); it changes the schedule only, never the
+// output.  One block per (b, h); C <= kGroupMaxC.
+constexpr int kGroupThreads = 512;
+
+__device__ __forceinline__ void top3_insert(uint64_t (&t)[3], uint64_t v) {
+    if (v > t[2]) {
+        if (v > t[1]) {
+            t[2] = t[1];
+            if (v > t[0]) {
+                t[1] = t[0];
+                t[0] = v;
+            } else {
+                t[1] = v;
+            }
+        } else {
+            t[2] = v;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kGroupThreads) group_kernel(int C, int cpow2, const float* __restrict__ scores,
+                                                              int32_t* __restrict__ order) {
+    __shared__ uint64_t keys[kGroupMaxC];
+    const int bh = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float* S = scores + static_cast<int64_t>(bh) * C * C;
+    for (int i = warp; i < C; i += kGroupThreads / 32) {
+        const float* row = S + static_cast<int64_t>(i) * C;
+        uint64_t t[3] = {0ull, 0ull, 0ull};
+        for (int j = lane; j < C; j += 32)   // key: score order, then lower index first
+            top3_insert(t, (static_cast<uint64_t>(order_key(row[j])) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(j)));
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            uint64_t o[3];
+#pragma unroll
+            for (int e = 0; e < 3; ++e) o[e] = __shfl_xor_sync(0xffffffffu, t[e], off);
+#pragma unroll
+            for (int e = 0; e < 3; ++e) top3_insert(t, o[e]);
+        }
+        if (lane == 0) {
+            uint64_t sig = static_cast<uint64_t>(i);
+#pragma unroll
+            for (int e = 0; e < 3; ++e) {
+                const uint64_t c = t[e] ? (0xFFFFFFFFu - static_cast<uint32_t>(t[e] & 0xFFFFFFFFu)) : 0xFFFFu;
+                sig |= (c & 0xFFFFu) << (48 - 16 * e);
+            }
+            keys[i] = sig;
+        }
+    }
+    for (int i = C + threadIdx.x; i < cpow2; i += kGroupThreads) keys[i] = ~0ull;
+    __syncthreads();
+    for (int k2 = 2; k2 <= cpow2; k2 <<= 1) {
+        for (int j = k2 >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < cpow2; i += kGroupThreads) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const uint64_t a = keys[i], b = keys[ixj];
+                    const bool up = (i & k2) == 0;
+                    if ((a > b) == up) {
+                        keys[i] = b;
+                        keys[ixj] = a;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int r = threadIdx.x; r < C; r += kGroupThreads)
+        order[static_cast<int64_t>(bh) * C + r] = static_cast<int32_t>(keys[r] & 0xFFFFu);
+}
+
 }  // namespace
+
+cudaError_t launch_group(const Dims& d, const float* scores, int32_t* order, cudaStream_t s) {
+    if (d.C > kGroupMaxC) return cudaErrorInvalidValue;
+    int cpow2 = 1;
+    while (cpow2 < d.C) cpow2 <<= 1;
+    group_kernel<<<d.B * d.H, kGroupThreads, 0, s>>>(d.C, cpow2, scores, order);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
                           float* scores, float* o_coarse, cudaStream_t s) {

@@ -50,11 +50,17 @@ cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, c
                           float* scores, float* o_coarse, cudaStream_t s);
 cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx, cudaStream_t s);
 
-// Fine stage.  Returns cudaErrorInvalidValue (with *why set) when a tensor
-// map cannot be encoded.
+// Work order of the fine stage from the coarse scores (C <= kGroupMaxC).
+constexpr int kGroupMaxC = 4096;
+cudaError_t launch_group(const Dims& d, const float* scores, int32_t* order, cudaStream_t s);
+
+// Fine stage.  `order` (may be null) is a per-head permutation of the query
+// cubes; groups of four consecutive entries share one key/value stream.
+// Returns cudaErrorInvalidValue (with *why set) when a tensor map cannot be
+// encoded.
 cudaError_t launch_fine(const Dims& d, const uint16_t* qt, const uint16_t* kt, const uint16_t* vt,
-                        const int32_t* idx, int k, float scale, uint16_t* o_fine, float* lse, cudaStream_t s,
-                        const char** why);
+                        const int32_t* idx, int k, const int32_t* order, float scale, uint16_t* o_fine,
+                        float* lse, cudaStream_t s, const char** why);
 
 cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t s);
 

@@ -42,7 +42,8 @@ def main(argv=None) -> int:
     npad, C = vsa.shape_info(s)
     scale = 1.0 / math.sqrt(w.head_dim)
     dense = w.topk == C
-    names = ["tile", "fine", "untile"] if dense else ["tile", "pool", "coarse", "topk", "fine", "combine", "untile"]
+    names = ["tile", "fine", "untile"] if dense else ["tile", "pool", "coarse", "topk+group", "fine", "combine",
+                                                       "untile"]
     if a.dense_too:
         names.append("fine_dense")
     times = {n: [] for n in names}
@@ -70,8 +71,9 @@ def main(argv=None) -> int:
             scores, oc = vsa.coarse(*bars, s, scale)
             mark()
             idx = vsa.topk(scores, s, w.topk)
+            order = vsa.group(scores, s)
             mark()
-            of, _ = vsa.fine(qt, kt, vt, s, idx, scale, want_lse=False)
+            of, _ = vsa.fine(qt, kt, vt, s, idx, scale, want_lse=False, order=order)
             mark()
             ot = vsa.combine(oc, of, s, d["g_coarse"], d["g_fine"])
             mark()

@@ -134,6 +134,18 @@ vsa_status vsa_coarse(const vsa_shape* shape, const float* qbar, const float* kb
 vsa_status vsa_topk(const vsa_shape* shape, const float* scores, int32_t k, int32_t* idx, vsa_stream_t stream);
 
 /*
+ * vsa_group — work order for vsa_fine (a schedule, not a step of the method):
+ * per (b, h), the query cubes sorted by the indices of their three
+ * highest-scoring key cubes (ties to the lower index).  Consecutive entries
+ * then tend to select the same key cubes, and vsa_fine processes groups of
+ * four consecutive entries over one shared key/value stream.  The output of
+ * vsa_fine does not depend on the order.
+ *   scores  [B, H, C, C] float32 (read).   order [B, H, C] int32 (written): a
+ *           permutation of [0, C) per (b, h).   Requires C <= 4096.
+ */
+vsa_status vsa_group(const vsa_shape* shape, const float* scores, int32_t* order, vsa_stream_t stream);
+
+/*
  * vsa_fine — token-level attention of every 64-token query cube over the
  * tokens of its selected key cubes (same section, part 2 "fine attention"),
  * padded key tokens excluded, online softmax in float32 (teardown section
@@ -147,6 +159,11 @@ vsa_status vsa_topk(const vsa_shape* shape, const float* scores, int32_t k, int3
  *               attended twice.  Out-of-range entries are treated as an empty
  *               cube (no memory outside the tensors is read).
  *   k           entries per row of idx (ignored, taken as C, when idx is NULL).
+ *   order       [B, H, C] int32 per-head permutation of the query cubes that
+ *               sets the work order (groups of four consecutive entries share
+ *               one key/value stream; see vsa_group), or NULL for 0..C-1.  An
+ *               entry outside [0, C) is skipped; a cube missing from `order`
+ *               leaves its output rows unwritten.
  *   scale       softmax scale, normally 1/sqrt(D).
  *   o_fine      [B, H, Npad, D] bf16 (written).  Rows of padded query
  *               positions are written but carry no meaning.
@@ -154,8 +171,8 @@ vsa_status vsa_topk(const vsa_shape* shape, const float* scores, int32_t k, int3
  *               the attended keys (written), or NULL.
  */
 vsa_status vsa_fine(const vsa_shape* shape, const vsa_bf16* qt, const vsa_bf16* kt, const vsa_bf16* vt,
-                    const int32_t* idx, int32_t k, float scale, vsa_bf16* o_fine, float* lse,
-                    vsa_stream_t stream);
+                    const int32_t* idx, int32_t k, const int32_t* order, float scale, vsa_bf16* o_fine,
+                    float* lse, vsa_stream_t stream);
 
 /*
  * vsa_combine — gated merge (same section, part 3): per token and head,
@@ -176,7 +193,8 @@ size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
 
 /*
  * vsa_forward — the whole attention call on one stream:
- *   tile(q,k,v) -> pool -> coarse -> topk -> fine -> combine -> untile.
+ *   tile(q,k,v) -> pool -> coarse -> topk -> group -> fine -> combine -> untile
+ * (the grouping step is skipped when C > 4096).
  * When topk == C and both gates are NULL the call is dense attention and runs
  * tile -> fine (all cubes) -> untile.
  *   q, k, v      [B, N, H, D] bf16 token layout (read).

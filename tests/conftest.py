@@ -11,6 +11,7 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
     config.addinivalue_line("markers", "slow: large-size parity case (still part of -m gpu)")
+    config.addinivalue_line("markers", "expects_timeout: the test makes a device-side wait give up on purpose")
 
 
 def pytest_collection_modifyitems(config, items):
@@ -27,3 +28,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _no_device_timeout(request):
+    """After every GPU test: no kernel of the library gave up on a device-side wait."""
+    yield
+    if "gpu" not in request.keywords or request.node.get_closest_marker("expects_timeout"):
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import block_sparse_attention_cube_b200 as vsa
+    vsa.device_status()

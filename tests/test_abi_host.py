@@ -90,7 +90,7 @@ def test_topk_out_of_range(k):
 def test_bad_scale(scale):
     s = _shape()
     p = [ctypes.c_void_p((1 << 40) + i * (1 << 32)) for i in range(5)]
-    st = vsa.raw_call("vsa_fine", ctypes.byref(s), p[0], p[1], p[2], None, 0, scale, p[3], None, None)
+    st = vsa.raw_call("vsa_fine", ctypes.byref(s), p[0], p[1], p[2], None, 0, None, scale, p[3], None, None)
     assert st == INVALID and "scale" in vsa.last_error()
 
 
@@ -110,13 +110,22 @@ def test_workspace_checks():
 
 def test_workspace_size_480p_matches_layout():
     # tiled q,k,v,o_fine (4 x 39936*40*128*2 B) + pooled q,k,v,o_coarse (4 x 624*40*128*4 B)
-    # + scores (624*624*40*4 B) + idx (624*40*32*4 B), each rounded up to 256 B
+    # + scores (624*624*40*4 B) + idx (624*40*32*4 B) + order (624*40*4 B), each rounded up to 256 B
     s = vsa.Shape(1, 40, 128, (21, 30, 52)).c()
     up = lambda n: (n + 255) // 256 * 256
-    expect = 4 * up(39936 * 40 * 128 * 2) + 4 * up(624 * 40 * 128 * 4) + up(624 * 624 * 40 * 4) + up(624 * 40 * 32 * 4)
+    expect = 4 * up(39936 * 40 * 128 * 2) + 4 * up(624 * 40 * 128 * 4) + up(624 * 624 * 40 * 4) + up(624 * 40 * 32 * 4) \
+        + up(624 * 40 * 4)
     assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 32) == expect
 
 
 def test_probe_limit_checked_before_device():
     assert vsa.raw_call("vsa_debug_wait_probe", 10, None) == INVALID
     assert vsa.raw_call("vsa_debug_wait_probe", 10**12, None) == INVALID
+
+
+def test_group_limits_checked_before_device():
+    s = vsa.Shape(1, 2, 128, (40, 40, 44)).c()     # 10*10*11 = 1100 cubes: fine
+    big = vsa.Shape(1, 2, 128, (80, 80, 44)).c()   # 20*20*11 = 4400 cubes: above the grouping limit
+    p = [ctypes.c_void_p((1 << 40) + i * (1 << 34)) for i in range(2)]
+    assert vsa.raw_call("vsa_group", ctypes.byref(big), p[0], p[1], None) == UNSUPPORTED
+    assert vsa.raw_call("vsa_group", ctypes.byref(s), None, p[1], None) == INVALID

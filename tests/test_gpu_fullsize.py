@@ -39,7 +39,7 @@ def run(request):
         bars = [vsa.pool(t, s) for t in (qt, kt, vt)]
         scores, oc = vsa.coarse(*bars, s, scale)
         idx = vsa.topk(scores, s, w.topk)
-        o, lse = vsa.fine(qt, kt, vt, s, idx, scale)
+        o, lse = vsa.fine(qt, kt, vt, s, idx, scale, order=vsa.group(scores, s))
         stage_out = vsa.untile(vsa.combine(oc, o, s, gc, gf), s)
         r["bars"] = [b.cpu() for b in bars]
         r["scores"] = scores.cpu()

@@ -307,3 +307,43 @@ def test_forward_host_matches_device_forward():
     vsa.forward_host(h["q"], h["k"], h["v"], s, w.topk, ws, out, None, h["g_coarse"], h["g_fine"])
     torch.cuda.current_stream().synchronize()
     assert torch.equal(out, ref.cpu())
+
+
+def test_group_is_a_permutation_and_does_not_change_the_output(case):
+    """vsa_group only reorders the work: fine() with its order is bit-identical to fine() without."""
+    w, _, dev, _ = case
+    s = _shape(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    qt, kt, vt = (vsa.tile(dev[n], s) for n in ("q", "k", "v"))
+    bars = [vsa.pool(t, s) for t in (qt, kt, vt)]
+    scores, _ = vsa.coarse(*bars, s, scale)
+    idx = vsa.topk(scores, s, w.topk)
+    order = vsa.group(scores, s)
+    _, C = vsa.shape_info(s)
+    o = order.cpu().numpy()
+    assert np.array_equal(np.sort(o, axis=-1), np.broadcast_to(np.arange(C, dtype=np.int32), o.shape))
+    o1, l1 = vsa.fine(qt, kt, vt, s, idx, scale)
+    o2, l2 = vsa.fine(qt, kt, vt, s, idx, scale, order=order)
+    rev = torch.flip(order, dims=[-1]).contiguous()
+    o3, l3 = vsa.fine(qt, kt, vt, s, idx, scale, order=rev)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert torch.equal(o1, o3) and torch.equal(l1, l3)
+    # dense attention with a shuffled order as well
+    perm = torch.from_numpy(np.random.default_rng(0).permuted(np.broadcast_to(np.arange(C, dtype=np.int32),
+                                                                              o.shape), axis=-1).copy()).cuda()
+    d1, dl1 = vsa.fine(qt, kt, vt, s, None, scale)
+    d2, dl2 = vsa.fine(qt, kt, vt, s, None, scale, order=perm)
+    assert torch.equal(d1, d2) and torch.equal(dl1, dl2)
+
+
+def test_group_keys_follow_top_scores():
+    """On hand-made scores the order is the sort by each row's top-3 key cubes."""
+    w = synth.custom_workload("group_8", 1, 1, 128, (8, 8, 8), 2)
+    s = _shape(w)
+    _, C = vsa.shape_info(s)
+    rng = np.random.default_rng(4)
+    sc = rng.standard_normal((1, 1, C, C)).astype(np.float32)
+    top = np.argsort(-sc[0, 0], axis=-1, kind="stable")[:, :3]
+    expect = sorted(range(C), key=lambda i: (top[i, 0], top[i, 1], top[i, 2], i))
+    got = vsa.group(torch.from_numpy(sc).cuda(), s).cpu().numpy()[0, 0]
+    assert got.tolist() == expect

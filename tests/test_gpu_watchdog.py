@@ -8,7 +8,7 @@ import block_sparse_attention_cube_b200 as vsa
 import synth
 from tests._util import to_dev
 
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.expects_timeout]
 
 
 def test_wait_probe_times_out_and_context_survives():
