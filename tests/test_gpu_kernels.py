@@ -310,30 +310,39 @@ def test_forward_host_matches_device_forward():
 
 
 def test_group_is_a_permutation_and_does_not_change_the_output(case):
-    """vsa_group only reorders the work: fine() with its order is bit-identical to fine() without."""
-    w, _, dev, _ = case
+    """vsa_group only reorders the work.  Any order gives a valid result: the
+    fine kernel pairs a row's key cubes into 128-key steps as the group's
+    union dictates, which changes only the rounding order, so each order is
+    compared with the oracle (its own selection) within the usual tolerances."""
+    w, _, dev, f64 = case
     s = _shape(w)
     scale = 1 / math.sqrt(w.head_dim)
     qt, kt, vt = (vsa.tile(dev[n], s) for n in ("q", "k", "v"))
     bars = [vsa.pool(t, s) for t in (qt, kt, vt)]
     scores, _ = vsa.coarse(*bars, s, scale)
-    idx = vsa.topk(scores, s, w.topk)
     order = vsa.group(scores, s)
     _, C = vsa.shape_info(s)
     o = order.cpu().numpy()
     assert np.array_equal(np.sort(o, axis=-1), np.broadcast_to(np.arange(C, dtype=np.int32), o.shape))
-    o1, l1 = vsa.fine(qt, kt, vt, s, idx, scale)
-    o2, l2 = vsa.fine(qt, kt, vt, s, idx, scale, order=order)
+    ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, w.topk, scale)
+    idx = torch.from_numpy(ora["idx"]).cuda()
     rev = torch.flip(order, dims=[-1]).contiguous()
-    o3, l3 = vsa.fine(qt, kt, vt, s, idx, scale, order=rev)
-    assert torch.equal(o1, o2) and torch.equal(l1, l2)
-    assert torch.equal(o1, o3) and torch.equal(l1, l3)
-    # dense attention with a shuffled order as well
-    perm = torch.from_numpy(np.random.default_rng(0).permuted(np.broadcast_to(np.arange(C, dtype=np.int32),
-                                                                              o.shape), axis=-1).copy()).cuda()
-    d1, dl1 = vsa.fine(qt, kt, vt, s, None, scale)
-    d2, dl2 = vsa.fine(qt, kt, vt, s, None, scale, order=perm)
-    assert torch.equal(d1, d2) and torch.equal(dl1, dl2)
+    shuffled = torch.from_numpy(np.random.default_rng(0).permuted(
+        np.broadcast_to(np.arange(C, dtype=np.int32), o.shape), axis=-1).copy()).cuda()
+    valid = O.key_valid_mask(w.grid)
+    for name, ordr in (("identity", None), ("group", order), ("reversed", rev), ("shuffled", shuffled)):
+        of, lse = vsa.fine(qt, kt, vt, s, idx, scale, order=ordr)
+        check_heads(from_dev(of), ora["o_fine"], w.grid, f"o_fine[{name}]")
+        assert np.abs(from_dev(lse)[:, :, valid] - ora["lse"][:, :, valid]).max() <= LSE_ABS, name
+    r_d, r_dl = O.fine(*(O.tile(f64[n], w.grid) for n in ("q", "k", "v")), None, scale, w.grid)
+    for ordr in (None, shuffled):
+        d1, dl1 = vsa.fine(qt, kt, vt, s, None, scale, order=ordr)
+        check_heads(from_dev(d1), r_d, w.grid, "dense")
+        assert np.abs(from_dev(dl1)[:, :, valid] - r_dl[:, :, valid]).max() <= LSE_ABS
+    # dense attention walks every cube in the same pairs whatever the order: bit-identical
+    d1, _ = vsa.fine(qt, kt, vt, s, None, scale)
+    d2, _ = vsa.fine(qt, kt, vt, s, None, scale, order=shuffled)
+    assert torch.equal(d1, d2)
 
 
 def test_group_keys_follow_top_scores():
