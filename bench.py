@@ -289,36 +289,31 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     vsa_ms_max = reduce_max(vsa_ms, world)
     dense_ms_max = reduce_max(dense_ms, world)
 
-    # ---- per-stage breakdown (same kernels through the per-stage entry points)
-    names = ["tile", "pool", "coarse", "topk+group", "fine", "combine", "untile"]
+    # ---- per-stage breakdown: the launches of vsa_forward, one by one through the entry points
+    names = ["pool", "coarse", "topk", "group", "fine"]
     acc = {n: [] for n in names}
     acc["fine_dense"] = []
     for it in range(args.warmup + args.steps):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
         e[0].record(stream)
-        qt, kt, vt = (vsa.tile(d[n], s) for n in ("q", "k", "v"))
+        bars = vsa.pool_qkv(d["q"], d["k"], d["v"], s)
         e[1].record(stream)
-        bars = [vsa.pool(t, s) for t in (qt, kt, vt)]
-        e[2].record(stream)
         scores, oc = vsa.coarse(*bars, s, scale)
-        e[3].record(stream)
+        e[2].record(stream)
         idx = vsa.topk(scores, s, w.topk)
+        e[3].record(stream)
         order = vsa.group(scores, s)
         e[4].record(stream)
-        of, _ = vsa.fine(qt, kt, vt, s, idx, scale, want_lse=False, order=order)
+        vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, order, oc, d["g_coarse"], d["g_fine"], out=out)
         e[5].record(stream)
-        ot = vsa.combine(oc, of, s, d["g_coarse"], d["g_fine"])
+        vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out_d)
         e[6].record(stream)
-        vsa.untile(ot, s, out=out)
-        e[7].record(stream)
-        vsa.fine(qt, kt, vt, s, None, scale, want_lse=False)
-        e[8].record(stream)
         torch.cuda.synchronize()
         if it >= args.warmup:
             for j, n in enumerate(names):
                 acc[n].append(e[j].elapsed_time(e[j + 1]))
-            acc["fine_dense"].append(e[7].elapsed_time(e[8]))
-        del qt, kt, vt, bars, scores, oc, idx, order, of, ot
+            acc["fine_dense"].append(e[5].elapsed_time(e[6]))
+        del bars, scores, oc, idx, order
     stage_ms = {n: round(statistics.mean(v), 4) for n, v in acc.items()}
 
     # ---- end to end through vsa_forward_host (pinned host buffers, copies inside the timed region)
@@ -345,7 +340,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     peaks, peaks_src = load_peaks()
     bf16_peak = float(peaks["bf16_tflops"])
     fine_flops = executed_fine_flops(w.batch, w.heads, npad, w.topk, w.head_dim)
-    dense_flops = executed_fine_flops(w.batch, w.heads, npad, C, w.head_dim)
+    nblk = (w.tokens + 63) // 64   # dense attention walks blocks of 64 consecutive real tokens
+    dense_flops = dense_equivalent_flops(w.batch, w.heads, 64 * nblk, w.head_dim)
     fine_tflops = fine_flops / (stage_ms["fine"] * 1e-3) / 1e12
     dense_tflops = dense_flops / (stage_ms["fine_dense"] * 1e-3) / 1e12
     fine_src = os.path.join(ROOT, "block_sparse_attention_cube_b200", "csrc", "vsa_fine.cu")
@@ -372,15 +368,17 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                  "dense_equivalent_tflops": round(dense_equivalent_flops(w.batch, w.heads, w.tokens, w.head_dim)
                                                   / (stage_ms["fine"] * 1e-3) / 1e12, 1)},
         "dense_fine": {"executed_tflop": round(dense_flops / 1e12, 3), "tflops": round(dense_tflops, 1),
-                       "frac_bf16_peak": round(dense_tflops / bf16_peak, 4)},
-        "roofline": {"kernel": "fine_kernel (VSA, top-k 32)", "bound": "tensor", "achieved": round(fine_tflops, 2),
+                       "frac_bf16_peak": round(dense_tflops / bf16_peak, 4),
+                       "per_launch": "4*B*H*(64*ceil(N/64))^2*D: blocks of 64 real tokens, no padding"},
+        "roofline": {"kernel": "fine_kernel<128, cubes, fused> (VSA, top-k 32)", "bound": "tensor",
+                     "achieved": round(fine_tflops, 2),
                      "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(fine_tflops / bf16_peak, 4),
                      "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)" if peaks_src == "measured"
                      else "fallback 1.59 PFLOP/s", "traffic": traffic,
                      "per_launch": "4*B*H*Npad*k*64*D executed flops (64x64 cube tiles of the k selected cubes)"},
         "e2e": {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "vsa_forward_host (pinned host q/k/v/gates in, host out)"},
-        "gpu_launches": 12 * args.steps,
+        "gpu_launches": 6 * args.steps,   # VSA: pool, coarse, top-k, group, fine; dense: fine
         "clocks": clocks,
         "cpu_baseline": cpu,
         "context": {"pages_dense_call_ms_b200": 17.0, "pages_vsa_kernel_ms_b200_k78": 4.719,

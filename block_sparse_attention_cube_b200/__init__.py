@@ -163,6 +163,35 @@ def combine(o_coarse: torch.Tensor, o_fine: torch.Tensor, shape: Shape, g_coarse
     return out
 
 
+def pool_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+             shape: Shape) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Cube means of q, k, v ([B,N,H,D] token layout) in one launch: three [B,H,C,D] float32 tensors."""
+    _, c = shape_info(shape)
+    outs = [torch.empty((shape.batch, shape.heads, c, shape.head_dim), dtype=torch.float32, device=q.device)
+            for _ in range(3)]
+    _check(_L.vsa_pool_qkv(ctypes.byref(shape.c()), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                           _ptr(v, torch.bfloat16, "v"), *(_ptr(o, torch.float32, n) for o, n in
+                                                            zip(outs, ("qbar", "kbar", "vbar"))), _stream()))
+    return outs[0], outs[1], outs[2]
+
+
+def fine_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, shape: Shape, idx: Optional[torch.Tensor] = None,
+               scale: Optional[float] = None, order: Optional[torch.Tensor] = None,
+               o_coarse: Optional[torch.Tensor] = None, g_coarse: Optional[torch.Tensor] = None,
+               g_fine: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Fine attention + gated merge on the token layout, written as [B,N,H,D] (idx None: dense attention)."""
+    scale = default_scale(shape) if scale is None else scale
+    kk = int(idx.shape[-1]) if idx is not None else 0
+    if out is None:
+        out = torch.empty_like(q)
+    _check(_L.vsa_fine_fused(ctypes.byref(shape.c()), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                             _ptr(v, torch.bfloat16, "v"), _ptr(idx, torch.int32, "idx"), kk,
+                             _ptr(order, torch.int32, "order"), scale, _ptr(o_coarse, torch.float32, "o_coarse"),
+                             _ptr(g_coarse, torch.bfloat16, "g_coarse"), _ptr(g_fine, torch.bfloat16, "g_fine"),
+                             _ptr(out, torch.bfloat16, "out"), _stream()))
+    return out
+
+
 def workspace_bytes(shape: Shape, k: int) -> int:
     return int(_L.vsa_workspace_bytes(ctypes.byref(shape.c()), k))
 
@@ -182,7 +211,7 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, shape: Shape, top
             scale: Optional[float] = None, g_coarse: Optional[torch.Tensor] = None,
             g_fine: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
             out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """The whole VSA call (dense attention when topk_k == C and both gates are None)."""
+    """The whole VSA call: pool_qkv -> coarse -> topk -> group -> fine_fused (topk_k == C: dense fine stage)."""
     scale = default_scale(shape) if scale is None else scale
     if workspace is None:
         workspace = alloc_workspace(shape, topk_k, device=q.device)

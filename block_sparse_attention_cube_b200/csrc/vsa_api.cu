@@ -121,17 +121,19 @@ size_t order_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C 
 constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Workspace of vsa_forward: qt | kt | vt | o_fine | qbar | kbar | vbar | o_coarse | scores | idx | order.
-// The merged output (combine) reuses qt, which is dead after the fine stage.
+// Workspace of vsa_forward: qbar | kbar | vbar | o_coarse | scores | idx | order.
+// Q, K and V are read in the caller's [B, N, H, D] layout (the fine stage
+// gathers cubes with TMA), so no tiled copies are kept.  With every cube
+// selected the fine stage is dense attention and needs none of it; the
+// coarse buffers are then used only when a coarse gate is given.
 struct Carve {
-    uint16_t *qt, *kt, *vt, *of;
     float *qbar, *kbar, *vbar, *oc, *scores;
     int32_t* idx;
     int32_t* order;
     size_t bytes;
 };
 
-Carve carve(const Dims& d, int k, void* ws) {
+Carve carve(const Dims& d, int k, bool coarse_gate, void* ws) {
     Carve c{};
     uint8_t* b = static_cast<uint8_t*>(ws);
     size_t off = 0;
@@ -140,18 +142,19 @@ Carve carve(const Dims& d, int k, void* ws) {
         off += up(n);
         return p;
     };
-    c.qt = reinterpret_cast<uint16_t*>(take(tiled_bytes(d)));
-    c.kt = reinterpret_cast<uint16_t*>(take(tiled_bytes(d)));
-    c.vt = reinterpret_cast<uint16_t*>(take(tiled_bytes(d)));
-    c.of = reinterpret_cast<uint16_t*>(take(tiled_bytes(d)));
-    c.qbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
-    c.kbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
-    c.vbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
-    c.oc = reinterpret_cast<float*>(take(pooled_bytes(d)));
-    c.scores = reinterpret_cast<float*>(take(score_bytes(d)));
-    c.idx = reinterpret_cast<int32_t*>(take(idx_bytes(d, k)));
-    c.order = reinterpret_cast<int32_t*>(take(order_bytes(d)));
-    c.bytes = off;
+    const bool sparse = k < d.C;
+    if (sparse || coarse_gate) {
+        c.qbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
+        c.kbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
+        c.vbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
+        c.oc = reinterpret_cast<float*>(take(pooled_bytes(d)));
+        c.scores = reinterpret_cast<float*>(take(score_bytes(d)));
+    }
+    if (sparse) {
+        c.idx = reinterpret_cast<int32_t*>(take(idx_bytes(d, k)));
+        c.order = reinterpret_cast<int32_t*>(take(order_bytes(d)));
+    }
+    c.bytes = off > kAlign ? off : kAlign;
     return c;
 }
 
@@ -178,37 +181,56 @@ vsa_status check_k(const Dims& d, int32_t k) {
         if (e_ != cudaSuccess) return cuda_fail(e_, where); \
     } while (0)
 
+// The fused fine stage once the arguments are checked: cube gathers when a
+// selection is given, blocks of consecutive real tokens for dense attention.
+vsa_status run_fine_fused(const Dims& d, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                          const int32_t* idx, int topk, const int32_t* order, float scale, const float* o_coarse,
+                          const uint16_t* gc, const uint16_t* gf, uint16_t* out, cudaStream_t s) {
+    FineArgs a{};
+    a.mode = idx ? kFineCubesFused : kFineTokensFused;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.idx = idx;
+    a.k_sel = topk;
+    a.order = idx ? order : nullptr;
+    a.scale = scale;
+    a.out = out;
+    a.o_coarse = o_coarse;
+    a.g_coarse = o_coarse ? gc : nullptr;
+    a.g_fine = gf;
+    const char* why = nullptr;
+    cudaError_t e = launch_fine(d, a, s, &why);
+    if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "fine launch");
+    return VSA_OK;
+}
+
 // Body of vsa_forward once the arguments are checked.
+//  * top-k < C:  pool (Q, K, V read in place) -> coarse -> top-k -> work order
+//                -> fine with cube gathers and the merge + untiling in its epilogue;
+//  * top-k == C: every cube is selected, so the fine stage is dense attention
+//                over the real tokens (blocks of 64 consecutive tokens, no
+//                padding); pool -> coarse run only when a coarse gate is given.
 vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* gc,
                        const uint16_t* gf, int topk, float scale, void* ws, uint16_t* out, cudaStream_t s) {
-    const Carve c = carve(d, topk, ws);
-    const bool dense = topk == d.C && gc == nullptr && gf == nullptr;
-    Bf16Triple t{{q, k, v}, {c.qt, c.kt, c.vt}, 3};
-    VSA_CUDA(launch_tile(d, t, s), "tile launch");
-    if (dense) {
-        const char* why = nullptr;
-        cudaError_t e = launch_fine(d, c.qt, c.kt, c.vt, nullptr, d.C, nullptr, scale, c.of, nullptr, s, &why);
-        if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "fine launch");
-        VSA_CUDA(launch_untile(d, c.of, out, s), "untile launch");
-        return VSA_OK;
+    const bool sparse = topk < d.C;
+    const Carve c = carve(d, topk, gc != nullptr, ws);
+    if (sparse || gc != nullptr) {
+        const uint16_t* pin[3] = {q, k, v};
+        float* pout[3] = {c.qbar, c.kbar, c.vbar};
+        VSA_CUDA(launch_pool_tokens(d, pin, pout, 3, s), "pool launch");
+        VSA_CUDA(launch_coarse(d, c.qbar, c.kbar, c.vbar, scale, c.scores, c.oc, s), "coarse launch");
     }
-    const uint16_t* pin[3] = {c.qt, c.kt, c.vt};
-    float* pout[3] = {c.qbar, c.kbar, c.vbar};
-    VSA_CUDA(launch_pool(d, pin, pout, 3, s), "pool launch");
-    VSA_CUDA(launch_coarse(d, c.qbar, c.kbar, c.vbar, scale, c.scores, c.oc, s), "coarse launch");
-    VSA_CUDA(launch_topk(d, c.scores, topk, c.idx, s), "topk launch");
     const int32_t* order = nullptr;
-    if (d.C <= kGroupMaxC) {
-        VSA_CUDA(launch_group(d, c.scores, c.order, s), "group launch");
-        order = c.order;
+    if (sparse) {
+        VSA_CUDA(launch_topk(d, c.scores, topk, c.idx, s), "topk launch");
+        if (d.C <= kGroupMaxC) {
+            VSA_CUDA(launch_group(d, c.scores, c.order, s), "group launch");
+            order = c.order;
+        }
     }
-    const char* why = nullptr;
-    cudaError_t e = launch_fine(d, c.qt, c.kt, c.vt, c.idx, topk, order, scale, c.of, nullptr, s, &why);
-    if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "fine launch");
-    uint16_t* o_tiled = c.qt;   // qt is no longer read after the fine stage
-    VSA_CUDA(launch_combine(d, c.oc, c.of, gc, gf, o_tiled, s), "combine launch");
-    VSA_CUDA(launch_untile(d, o_tiled, out, s), "untile launch");
-    return VSA_OK;
+    return run_fine_fused(d, q, k, v, sparse ? c.idx : nullptr, topk, order, scale, gc ? c.oc : nullptr, gc, gf,
+                          out, s);
 }
 
 }  // namespace
@@ -356,8 +378,19 @@ vsa_status vsa_fine(const vsa_shape* shape, const vsa_bf16* qt, const vsa_bf16* 
                             {order, order ? order_bytes(d) : 0, "order"}},
                            {{o_fine, tb, "o_fine"}, {lse, lse ? static_cast<size_t>(d.rows) * 4 : 0, "lse"}}));
     VSA_TRY(check_device());
+    FineArgs a{};
+    a.mode = kFineTiled;
+    a.q = qt;
+    a.k = kt;
+    a.v = vt;
+    a.idx = idx;
+    a.k_sel = k;
+    a.order = order;
+    a.scale = scale;
+    a.out = o_fine;
+    a.lse = lse;
     const char* why = nullptr;
-    cudaError_t e = launch_fine(d, qt, kt, vt, idx, k, order, scale, o_fine, lse, as_stream(stream), &why);
+    cudaError_t e = launch_fine(d, a, as_stream(stream), &why);
     if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "fine launch");
     return VSA_OK;
 }
@@ -380,10 +413,57 @@ vsa_status vsa_combine(const vsa_shape* shape, const float* o_coarse, const vsa_
     return VSA_OK;
 }
 
+vsa_status vsa_pool_qkv(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                        float* qbar, float* kbar, float* vbar, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(need_ptr(q, "q"));
+    VSA_TRY(need_ptr(k, "k"));
+    VSA_TRY(need_ptr(v, "v"));
+    VSA_TRY(need_ptr(qbar, "qbar"));
+    VSA_TRY(need_ptr(kbar, "kbar"));
+    VSA_TRY(need_ptr(vbar, "vbar"));
+    const size_t tb = token_bytes(d), pb = pooled_bytes(d);
+    VSA_TRY(check_disjoint({{q, tb, "q"}, {k, tb, "k"}, {v, tb, "v"}},
+                           {{qbar, pb, "qbar"}, {kbar, pb, "kbar"}, {vbar, pb, "vbar"}}));
+    VSA_TRY(check_device());
+    const uint16_t* in[3] = {q, k, v};
+    float* out[3] = {qbar, kbar, vbar};
+    VSA_CUDA(launch_pool_tokens(d, in, out, 3, as_stream(stream)), "pool launch");
+    return VSA_OK;
+}
+
+vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                          const int32_t* idx, int32_t topk, const int32_t* order, float scale,
+                          const float* o_coarse, const vsa_bf16* g_coarse, const vsa_bf16* g_fine, vsa_bf16* out,
+                          vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    if (idx) VSA_TRY(check_k(d, topk));
+    VSA_TRY(need_ptr(q, "q"));
+    VSA_TRY(need_ptr(k, "k"));
+    VSA_TRY(need_ptr(v, "v"));
+    VSA_TRY(opt_ptr(idx, "idx"));
+    VSA_TRY(opt_ptr(order, "order"));
+    VSA_TRY(opt_ptr(o_coarse, "o_coarse"));
+    VSA_TRY(opt_ptr(g_coarse, "g_coarse"));
+    VSA_TRY(opt_ptr(g_fine, "g_fine"));
+    VSA_TRY(need_ptr(out, "out"));
+    VSA_TRY(check_scale(scale));
+    const size_t tb = token_bytes(d), gb = gate_bytes(d);
+    VSA_TRY(check_disjoint({{q, tb, "q"}, {k, tb, "k"}, {v, tb, "v"}, {idx, idx ? idx_bytes(d, topk) : 0, "idx"},
+                            {order, order ? order_bytes(d) : 0, "order"},
+                            {o_coarse, o_coarse ? pooled_bytes(d) : 0, "o_coarse"},
+                            {g_coarse, g_coarse ? gb : 0, "g_coarse"}, {g_fine, g_fine ? gb : 0, "g_fine"}},
+                           {{out, tb, "out"}}));
+    VSA_TRY(check_device());
+    return run_fine_fused(d, q, k, v, idx, topk, order, scale, o_coarse, g_coarse, g_fine, out, as_stream(stream));
+}
+
 size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk) {
     Dims d{};
     if (make_dims(shape, &d) != VSA_OK || topk < 1 || topk > d.C) return 0;
-    return carve(d, topk, nullptr).bytes;
+    return carve(d, topk, true, nullptr).bytes;
 }
 
 vsa_status vsa_forward(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
@@ -400,7 +480,7 @@ vsa_status vsa_forward(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16
     VSA_TRY(opt_ptr(g_fine, "g_fine"));
     VSA_TRY(need_ptr(out, "out"));
     if (d.C > 49152) return fail(VSA_ERR_UNSUPPORTED, "top-k supports at most 49152 cubes (got %d)", d.C);
-    const size_t need = carve(d, topk, nullptr).bytes;
+    const size_t need = carve(d, topk, g_coarse != nullptr, nullptr).bytes;
     if (!workspace) return fail(VSA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0)
         return fail(VSA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
@@ -417,7 +497,7 @@ vsa_status vsa_forward(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16
 size_t vsa_workspace_bytes_host(const vsa_shape* shape, int32_t topk) {
     Dims d{};
     if (make_dims(shape, &d) != VSA_OK || topk < 1 || topk > d.C) return 0;
-    return carve(d, topk, nullptr).bytes + 4 * up(token_bytes(d)) + 2 * up(gate_bytes(d));
+    return carve(d, topk, true, nullptr).bytes + 4 * up(token_bytes(d)) + 2 * up(gate_bytes(d));
 }
 
 vsa_status vsa_forward_host(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
@@ -429,7 +509,7 @@ vsa_status vsa_forward_host(const vsa_shape* shape, const vsa_bf16* q, const vsa
     VSA_TRY(check_scale(scale));
     if (!q || !k || !v || !out) return fail(VSA_ERR_INVALID_ARGUMENT, "q, k, v and out must be non-NULL host pointers");
     if (d.C > 49152) return fail(VSA_ERR_UNSUPPORTED, "top-k supports at most 49152 cubes (got %d)", d.C);
-    const size_t fwd = carve(d, topk, nullptr).bytes;
+    const size_t fwd = carve(d, topk, true, nullptr).bytes;
     const size_t tb = token_bytes(d), gb = gate_bytes(d);
     const size_t need = fwd + 4 * up(tb) + 2 * up(gb);
     if (!workspace) return fail(VSA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);

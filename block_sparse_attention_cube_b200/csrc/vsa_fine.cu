@@ -5,28 +5,39 @@
 // to the tokens of the key/value cubes selected for it; padded key tokens are
 // excluded.  With every cube selected this is dense bidirectional attention
 // softmax(q k^T / sqrt(d)) v (Wan2.1 acceleration article, bafh001.com,
-// section 4.2).
+// section 4.2), which does not depend on the token order at all.
 //
 // Design (re-derived for B200, not taken from the pages' Hopper/Triton
 // kernels):
-//  * Work item = (b, h, group of four query cubes).  The four cubes form two
-//    128-row tiles (the M = 128 of one tcgen05.mma), A = cubes 0-1 and
-//    B = cubes 2-3 of the group, which share one K/V stream: the item walks
-//    the merged, ordered union of the four selection lists, two key cubes
-//    (128 keys, the N of QK^T) per step.  Rows of a cube that did not select
-//    one of the step's cubes mask that cube's 64 columns; a tile none of whose
-//    cubes selected either cube skips the step (no MMA, no softmax).  Dense
-//    attention selects every cube for every row, so nothing is masked or
-//    skipped.  Groups are four consecutive entries of an optional per-head
-//    permutation of the query cubes (vsa_group orders cubes with similar
-//    selections next to each other).
+//  * A "block" is 64 tokens of one (batch, head).  Three ways to fetch one
+//    with TMA (one 64-row x 128-byte box per 64 channels):
+//      tiled  - a cube of the cube-major tiled tensor [B, H, Npad, D];
+//      cubes  - the same cube gathered straight from the projection layout
+//               [B, N, H, D] by a 5-D box (64 channels x 4 y x 4 x x 4 t),
+//               padded positions zero-filled by the copy engine, so no
+//               tiling pass is needed;
+//      tokens - 64 consecutive tokens of [B, N, H, D] (dense attention over
+//               the real tokens only, no padding).
+//  * Work item = (b, h, group of four query blocks).  The four blocks form
+//    two 128-row tiles (the M = 128 of one tcgen05.mma), A = blocks 0-1 and
+//    B = blocks 2-3, which share one K/V stream: the item walks the merged,
+//    ordered union of the four selection lists, two key blocks (128 keys,
+//    the N of QK^T) per step.  Rows of a block that did not select one of the
+//    step's blocks mask that block's 64 columns; a tile none of whose blocks
+//    selected either block skips the step.  Dense attention selects every
+//    block for every row.  Groups are four consecutive entries of an optional
+//    per-head permutation of the query cubes (vsa_group orders cubes with
+//    similar selections next to each other).
 //  * Roles (warp specialisation, teardown section "Blackwell changes the
-//    optimisation problem"): warp 0 issues TMA loads (the Q group, then the
-//    step's K cubes through a 3-deep ring and V cubes through a separate
-//    2-deep ring, so K slots recycle as soon as QK^T is done); warp 1
-//    allocates all 512 tensor-memory columns and one thread issues the MMAs;
-//    warps 2..5 run the softmax and epilogue of tile A and warps 6..9 those
-//    of tile B, one query row per thread (warp w reads TMEM lane quarter w%4).
+//    optimisation problem"): warp 0 walks the selections and issues TMA (the
+//    Q group, then the step's K blocks through a 3-deep ring and V blocks
+//    through a 2-deep ring, so K slots recycle as soon as QK^T is done); for
+//    sparse selections it publishes each step (its two key blocks and which
+//    query blocks selected them) in an 8-deep shared-memory ring, so no
+//    other role repeats the walk.  Warp 1 allocates all 512 tensor-memory
+//    columns and one thread issues the MMAs; warps 2..5 run the softmax and
+//    epilogue of tile A and warps 6..9 those of tile B, one query row per
+//    thread (warp w reads TMEM lane quarter w%4).
 //  * Tensor memory, per tile: one 128x128 fp32 score buffer and a 128xD fp32
 //    output accumulator.  The softmax writes P (bf16) over the first 64
 //    columns of the scores it read and PV takes its A operand from there.
@@ -35,15 +46,18 @@
 //    per step, S_A(i), PV_B(i-1), S_B(i), PV_A(i), lets each tile's softmax
 //    run while the tensor cores work on the other tile.
 //  * Softmax: online, in the log2 domain.  The running maximum starts at the
-//    row's first tile maximum and moves only when a step's probabilities would
-//    exceed 2^64 (the bound that keeps every later sum finite); moving it
-//    rescales the accumulator, the denominator and any P already stored.  The
-//    scores of step i arrive only after the tile's PV of step i-1 completed,
-//    so the accumulator is stable then.  P is rounded to bf16; the
-//    denominator sums the float32 probabilities; exponent arguments use
-//    packed f32x2 FMA.  Teardown section "Fixed-max
-//    softmax is a numerical contract": subtracting any common constant leaves
-//    softmax unchanged; here the constant is bounded so no exponent overflows.
+//    maximum of the row's first scores and moves only when a half step's
+//    probabilities would exceed 2^64 (the bound that keeps every later sum
+//    finite); moving it rescales the accumulator, the denominator and any P
+//    already stored.  The scores of step i arrive only after the tile's PV
+//    of step i-1 completed, so the accumulator is stable then.  P is rounded
+//    to bf16; the denominator sums the float32 probabilities.  Teardown
+//    section "Fixed-max softmax is a numerical contract": subtracting any
+//    common constant leaves softmax unchanged; here the constant is bounded
+//    so no exponent overflows.
+//  * Epilogue: O / l either to the tiled output (plus log-sum-exp), or, fused,
+//    the gated merge of part 3 of the method, g_c * O_c[cube] + g_f * O / l,
+//    written straight to the token's row of [B, N, H, D] (the untiling).
 //  * Persistent CTAs (teardown section "Persistent kernel removes repeated
 //    start-up cost"): one CTA per SM walks the work items of consecutive
 //    heads, so the K/V of a head stay in L2 while its query groups use them.
@@ -72,12 +86,14 @@ using namespace ptx;
 constexpr int kThreads = 320;          // producer warp, MMA warp, 2 x 4 softmax warps
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
+constexpr int kRing = 8;               // published steps (sparse selections)
 constexpr uint32_t kQTileBytes = 32768;   // 128 rows x 256 B (two 128-B column halves)
-constexpr uint32_t kKVBytes = 32768;      // two cubes: [d 0-63: cube a, cube b][d 64-127: cube a, cube b]
+constexpr uint32_t kKVBytes = 32768;      // two blocks: [d 0-63: block a, block b][d 64-127: block a, block b]
 constexpr uint32_t kOffQ = 0;                                  // [2 tiles]
 constexpr uint32_t kOffK = kOffQ + 2 * kQTileBytes;            // [kKStages]
 constexpr uint32_t kOffV = kOffK + kKStages * kKVBytes;        // [kVStages]
-constexpr uint32_t kOffBar = kOffV + kVStages * kKVBytes;
+constexpr uint32_t kOffRec = kOffV + kVStages * kKVBytes;      // [kRing] x 16 B
+constexpr uint32_t kOffBar = kOffRec + kRing * 16;
 // barrier slots
 constexpr int kBarQFull = 0;
 constexpr int kBarQEmpty = 1;
@@ -88,25 +104,39 @@ constexpr int kBarVEmpty = kBarVFull + kVStages;
 constexpr int kBarSFull = kBarVEmpty + kVStages;    // [tile]
 constexpr int kBarPFull = kBarSFull + 2;            // [tile]
 constexpr int kBarPVDone = kBarPFull + 2;           // [tile]
-constexpr int kBarDrain = kBarPVDone + 2;
+constexpr int kBarRecFull = kBarPVDone + 2;         // [kRing]
+constexpr int kBarRecEmpty = kBarRecFull + kRing;   // [kRing]
+constexpr int kBarDrain = kBarRecEmpty + kRing;
 constexpr int kNumBars = kBarDrain + 1;
+constexpr uint32_t kRecConsumers = 1 + 8;           // the MMA thread and the eight softmax warps
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem slot (4 B) + abort flag (4 B)
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;     // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTileCols = 256;   // per tile: S at +0 (P over its first 64 columns), O at +128
 constexpr uint32_t kColO = 128;
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s for draining after an abort
+static_assert(kSmemBytes <= 232448, "shared memory over the 227 KB per-block limit");
+
+enum LoadMode : int { kLoadTiled = 0, kLoadCubes = 1, kLoadTokens = 2 };
 
 struct FineParams {
-    const int32_t* idx;     // [B, H, C, k] or nullptr (all cubes)
+    const int32_t* idx;     // [B, H, C, k] or nullptr (every block)
     const int32_t* order;   // [B, H, C] permutation of query cubes, or nullptr (identity)
-    uint16_t* o;            // [B, H, Npad, D]
-    float* lse;             // [B, H, Npad] or nullptr
-    int k;
+    uint16_t* o;            // tiled O [B, H, Npad, D], or the merged output [B, N, H, D] (fused)
+    float* lse;             // [B, H, Npad] or nullptr (tiled output only)
+    const float* o_coarse;  // [B, H, C, D] or nullptr (fused only; no coarse term)
+    const uint16_t* g_coarse;   // [B, N, H] or nullptr (gate 0)
+    const uint16_t* g_fine;     // [B, N, H] or nullptr (gate 1)
+    int k;                  // selections per query block (nblk when idx is nullptr)
+    int B, H;
+    int nblk;               // blocks per head: C (cube modes) or ceil(N / 64) (token mode)
     int C, Ct, Cx, Cy, T, X, Y;
-    int ngroups;            // ceil(C / 4)
+    int64_t N;
+    int ngroups;            // ceil(nblk / 4)
     uint64_t magic_cxcy;    // floor(2^48 / (Cx*Cy)) + 1: exact j / (Cx*Cy) for j < 2^24
     uint64_t magic_cy;      // floor(2^48 / Cy) + 1
+    uint64_t magic_cx;      // floor(2^48 / Cx) + 1
+    uint64_t mask_t, mask_x, mask_y;   // real offsets of a cube in the last cube layer along t, x, y
     int64_t Npad;
     int64_t items;
     int32_t oob_row;        // a row index outside the tiled tensors (TMA fills zeros)
@@ -119,52 +149,70 @@ __device__ __forceinline__ uint32_t div_magic(uint32_t j, uint64_t magic) {
     return static_cast<uint32_t>((static_cast<uint64_t>(j) * magic) >> 48);
 }
 
-// The four query cubes of one work item (slot j < 0 when absent).
+// The four query blocks of one work item (slot j < 0 when absent).
 struct Item {
     int64_t bh;
-    int cube[4];
-    uint32_t present;   // bit j set when slot j holds a query cube
+    int b, h;
+    int blk[4];
+    uint32_t present;   // bit j set when slot j holds a query block
 };
 
 __device__ __forceinline__ Item decode_item(int64_t it, const FineParams& p) {
     Item r;
     const int g = static_cast<int>(it % p.ngroups);
     r.bh = it / p.ngroups;
+    r.b = static_cast<int>(r.bh / p.H);
+    r.h = static_cast<int>(r.bh - static_cast<int64_t>(r.b) * p.H);
     r.present = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int pos = 4 * g + j;
         int c = -1;
-        if (pos < p.C) {
+        if (pos < p.nblk) {
             c = p.order ? __ldg(p.order + r.bh * p.C + pos) : pos;
-            if (c < 0 || c >= p.C) c = -1;
+            if (c < 0 || c >= p.nblk) c = -1;
         }
-        r.cube[j] = c;
+        r.blk[j] = c;
         r.present |= (c >= 0 ? 1u : 0u) << j;
     }
     return r;
 }
 
-// Ordered union of the selection lists of the group's query cubes, two cubes
-// per step.  Entries outside [0, C) are visited as the empty cube C.  Every
-// entry of every list is consumed exactly once, duplicates included.  In
-// `flags`, bit j (cube a) or bit 4 + j (cube b) is set when slot j's list
-// holds that cube; cube b is -1 (empty, no flags) when the union runs out.
+// One step of an item: key blocks a and b (b = -1 when the union ran out; an
+// index outside [0, nblk) is the empty block), bit j (block a) or 4 + j
+// (block b) of `flags` set when query slot j selected it, `last` on the
+// item's final step.
+struct StepRec {
+    int32_t ca, cb;
+    uint32_t flags;
+    uint32_t last;
+};
+
+__device__ __forceinline__ StepRec dense_step(int s, uint32_t present, int nblk) {
+    StepRec r;
+    r.ca = 2 * s;
+    r.cb = 2 * s + 1 < nblk ? 2 * s + 1 : -1;
+    r.flags = present | (r.cb >= 0 ? present << 4 : 0u);
+    r.last = 2 * s + 2 >= nblk ? 1u : 0u;
+    return r;
+}
+
+// Ordered union of the selection lists of the group's query blocks, two
+// blocks per step (run by the producer lane only).  Entries outside [0, C)
+// are visited as the empty block C.  Every entry of every list is consumed
+// exactly once, duplicates included.
 struct GroupWalk {
     const int32_t* lst[4];
     int pos[4];
     int k, C;
     uint32_t present;
-    bool dense;
 
     __device__ __forceinline__ int head(int j) const {
-        if (!((present >> j) & 1u)) return INT_MAX;
-        if (dense) return pos[j] < C ? pos[j] : INT_MAX;
-        if (pos[j] >= k) return INT_MAX;
+        if (!((present >> j) & 1u) || pos[j] >= k) return INT_MAX;
         const int v = __ldg(lst[j] + pos[j]);
         return (v < 0 || v >= C) ? C : v;
     }
-    __device__ __forceinline__ bool next1(int& cube, uint32_t& flags) {
+    __device__ __forceinline__ bool next1(int& blk, uint32_t& flags) {
         int h[4];
         int m = INT_MAX;
 #pragma unroll
@@ -173,7 +221,7 @@ struct GroupWalk {
             m = min(m, h[j]);
         }
         if (m == INT_MAX) return false;
-        cube = m;
+        blk = m;
         flags = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -184,57 +232,85 @@ struct GroupWalk {
         }
         return true;
     }
-    __device__ __forceinline__ bool next(int& cube_a, int& cube_b, uint32_t& flags) {
+    __device__ __forceinline__ bool done() const {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (((present >> j) & 1u) && pos[j] < k) return false;
+        return true;
+    }
+    // Next step of the union; false once it is exhausted.
+    __device__ __forceinline__ bool next(StepRec& r) {
         uint32_t fa, fb = 0;
-        if (!next1(cube_a, fa)) return false;
-        if (!next1(cube_b, fb)) {
-            cube_b = -1;
+        int a, b;
+        if (!next1(a, fa)) return false;
+        if (!next1(b, fb)) {
+            b = -1;
             fb = 0;
         }
-        flags = fa | (fb << 4);
+        r.ca = a;
+        r.cb = b;
+        r.flags = fa | (fb << 4);
+        r.last = done() ? 1u : 0u;
         return true;
     }
 };
 
 __device__ __forceinline__ GroupWalk make_walk(const Item& item, const FineParams& p) {
     GroupWalk w;
-    w.dense = p.idx == nullptr;
     w.k = p.k;
     w.C = p.C;
     w.present = item.present;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         w.pos[j] = 0;
-        w.lst[j] = (w.dense || item.cube[j] < 0)
-                       ? nullptr
-                       : p.idx + (item.bh * p.C + item.cube[j]) * static_cast<int64_t>(p.k);
+        w.lst[j] = item.blk[j] < 0 ? p.idx : p.idx + (item.bh * p.C + item.blk[j]) * static_cast<int64_t>(p.k);
     }
     return w;
 }
 
 __device__ __forceinline__ bool tile_active(uint32_t flags, int t) { return (flags & (0x33u << (2 * t))) != 0u; }
 
-// Bit o is set when offset o of cube j holds a real token.
-__device__ __forceinline__ uint64_t cube_key_mask(int j, const FineParams& p) {
-    if (j < 0 || j >= p.C) return 0ull;
-    const uint32_t ct = div_magic(static_cast<uint32_t>(j), p.magic_cxcy);
-    const uint32_t rem = static_cast<uint32_t>(j) - ct * static_cast<uint32_t>(p.Cx * p.Cy);
-    const uint32_t cx = div_magic(rem, p.magic_cy);
-    const uint32_t cy = rem - cx * static_cast<uint32_t>(p.Cy);
-    const int nt = min(4, p.T - 4 * static_cast<int>(ct));
-    const int nx = min(4, p.X - 4 * static_cast<int>(cx));
-    const int ny = min(4, p.Y - 4 * static_cast<int>(cy));
-    if ((nt & nx & ny) == 4) return ~0ull;
-    const uint64_t my = static_cast<uint64_t>((1u << ny) - 1u) * 0x1111111111111111ull;
-    const uint32_t ex = (0xFFFFu >> (16 - 4 * nx));                  // nx nibbles of 0xF
-    const uint64_t mx = static_cast<uint64_t>(ex) * 0x0001000100010001ull;
-    const uint64_t mt = (nt == 4) ? ~0ull : ((1ull << (16 * nt)) - 1ull);
-    return my & mx & mt;
+// Bit o is set when offset o of key block j holds a real token.
+template <int LM>
+__device__ __forceinline__ uint64_t key_mask(int j, const FineParams& p) {
+    if (j < 0 || j >= p.nblk) return 0ull;
+    if (LM == kLoadTokens) {
+        const int64_t left = p.N - 64ll * j;
+        return left >= 64 ? ~0ull : ((1ull << left) - 1ull);
+    }
+    uint64_t m = ~0ull;
+    const uint32_t q = div_magic(static_cast<uint32_t>(j), p.magic_cy);          // j / Cy
+    if (static_cast<int>(static_cast<uint32_t>(j) - q * static_cast<uint32_t>(p.Cy)) == p.Cy - 1) m &= p.mask_y;
+    const uint32_t ct = div_magic(q, p.magic_cx);                                  // j / (Cx*Cy)
+    if (static_cast<int>(q - ct * static_cast<uint32_t>(p.Cx)) == p.Cx - 1) m &= p.mask_x;
+    if (static_cast<int>(ct) == p.Ct - 1) m &= p.mask_t;
+    return m;
 }
 
-__device__ __forceinline__ int32_t tile_row(int64_t bh, int cube, const FineParams& p) {
-    if (cube < 0 || cube >= p.C) return p.oob_row;
-    return static_cast<int32_t>(bh * p.Npad + static_cast<int64_t>(cube) * 64);
+// One 64-row x 64-channel box of block j (channels [d0, d0 + 64)) into dst.
+// Blocks outside [0, nblk) are fetched from fully out-of-range coordinates,
+// which the copy engine fills with zeros (and still counts in full).
+template <int LM, int D>
+__device__ __forceinline__ void load_block(const CUtensorMap* m, uint32_t dst, int j, int d0, uint32_t bar,
+                                           const Item& it, const FineParams& p) {
+    const bool valid = j >= 0 && j < p.nblk;
+    if (LM == kLoadTiled) {
+        const int32_t row = valid ? static_cast<int32_t>(it.bh * p.Npad + static_cast<int64_t>(j) * 64) : p.oob_row;
+        tma_load_2d(dst, m, d0, row, bar);
+    } else if (LM == kLoadCubes) {
+        if (valid) {
+            const uint32_t q = div_magic(static_cast<uint32_t>(j), p.magic_cy);
+            const uint32_t ct = div_magic(q, p.magic_cx);
+            const int cy = j - static_cast<int>(q) * p.Cy;
+            const int cx = static_cast<int>(q) - static_cast<int>(ct) * p.Cx;
+            tma_load_5d(dst, m, it.h * D + d0, 4 * cy, 4 * cx, 4 * static_cast<int>(ct), it.b, bar);
+        } else {
+            tma_load_5d(dst, m, d0, 0, 0, 0, p.B, bar);
+        }
+    } else {
+        if (valid) tma_load_3d(dst, m, it.h * D + d0, 64 * j, it.b, bar);
+        else tma_load_3d(dst, m, d0, 0, p.B, bar);
+    }
 }
 
 // Scores of columns whose bit in `vm` is clear become -inf.
@@ -257,29 +333,9 @@ __device__ __forceinline__ float max64(const uint32_t (&s)[64]) {
 
 constexpr float kSumLimit = 18446744073709551616.0f;   // 2^64: bound on any probability
 
-// Maximum over both cubes' masked scores of this row: cube a in columns
-// [taddr, taddr + 64) (skipped when vm_a is 0), cube b in [taddr + 64, taddr + 128).
-// Warp-collective TMEM loads; used on a row's first step and on overflow only,
-// so kept out of line.
-__device__ __noinline__ float tile_max(uint32_t taddr, uint64_t vm_a, uint64_t vm_b) {
-    uint32_t s[64];
-    float m = -INFINITY;
-    if (vm_a) {
-        tmem_ld64_wait(taddr, s);
-        mask64(s, vm_a);
-        m = max64(s);
-    }
-    tmem_ld64_wait(taddr + 64u, s);
-    mask64(s, vm_b);
-    return fmaxf(m, max64(s));
-}
-
-// Probabilities 2^(s*c - m) of one cube's 64 masked scores: returned packed as
-// 32 bf16 pairs in pk, their float32 sum as the result.
-__device__ __forceinline__ float probs_half(uint32_t taddr, uint64_t vm, float c, float m, uint32_t (&pk)[32]) {
-    uint32_t s[64];
-    tmem_ld64_wait(taddr, s);
-    mask64(s, vm);
+// Probabilities 2^(s*c - m) of 64 masked scores: packed as 32 bf16 pairs in
+// pk, their float32 sum returned.
+__device__ __forceinline__ float probs64(const uint32_t (&s)[64], float c, float m, uint32_t (&pk)[32]) {
     const uint64_t c2 = f32x2(c, c), nm2 = f32x2(-m, -m);
     uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -309,7 +365,7 @@ __device__ __forceinline__ void scale_tmem_f32(uint32_t taddr, int chunks, float
     }
 }
 
-// Multiply 32 columns of bf16 pairs (this row's stored P of one cube) by alpha.
+// Multiply 32 columns of bf16 pairs (this row's stored P of one block) by alpha.
 __device__ __forceinline__ void scale_tmem_bf16(uint32_t taddr, float alpha) {
     uint32_t o[32];
     tmem_ld32_wait(taddr, o);
@@ -319,39 +375,43 @@ __device__ __forceinline__ void scale_tmem_bf16(uint32_t taddr, float alpha) {
     tmem_st32(taddr, o);
 }
 
-// Rare path of a cube half whose probabilities overflowed for some row of the
-// warp: those rows move their maximum to the tile maximum and rescale O, l and
-// (for half 1) the stored P of half 0; every row then recomputes the half and
-// stores its P.  Warp-collective; returns the row's new sum.
-struct RowState {
-    float sum, m, l;   // the half's new sum, the row maximum and denominator after the move
-};
-
+// Softmax of one half step (64 key columns, block a for h = 0, block b for
+// h = 1) of this thread's row: reads the scores from tensor memory, stores P
+// as bf16 pairs over columns [32h, 32h + 32) and adds the probabilities to
+// l_run.  `vm` is warp-uniform (every row of a warp belongs to one query
+// block).  Warp-collective.
 template <int D>
-__device__ __noinline__ RowState move_max_and_redo(uint32_t tcol, int h, uint64_t vm_a, uint64_t vm_b, float c,
-                                                   bool over, bool row_active, float m_run, float l_run) {
-    // half 1: only cube b's scores count (half 0's columns hold P by now)
-    const float tmax = (h ? tile_max(tcol, 0ull, vm_b) : tile_max(tcol, vm_a, vm_b)) * c;
-    float alpha = 1.f;
-    if (over) {
-        const float m_new = fmaxf(m_run, tmax);
-        alpha = ex2_approx(m_run - m_new);
-        l_run *= alpha;
-        m_run = m_new;
-    }
-    // the tile's previous PV completed before these scores were committed
-    scale_tmem_f32(tcol + kColO, D / 32, alpha);
-    if (h == 1) scale_tmem_bf16(tcol, alpha);   // half 0's P is already stored
+__device__ __forceinline__ void softmax_half(uint32_t tcol, int h, uint64_t vm, float c, float& m_run,
+                                             float& l_run) {
     uint32_t pk[32];
-    float sum = 0.f;
-    if (row_active) {
-        sum = probs_half(tcol + 64u * h, h ? vm_b : vm_a, c, m_run, pk);
+    if (vm != 0ull) {
+        uint32_t s[64];
+        tmem_ld64_wait(tcol + 64u * h, s);
+        mask64(s, vm);
+        if (m_run == -INFINITY) m_run = max64(s) * c;   // the row's first scores
+        float sum = probs64(s, c, m_run, pk);
+        const bool over = !(sum <= kSumLimit);
+        if (__any_sync(0xffffffffu, over)) {
+            // rare: the maximum fell far behind; rows that overflowed move it
+            // to this half's maximum and rescale what they accumulated so far
+            float alpha = 1.f;
+            if (over) {
+                const float m_new = fmaxf(m_run, max64(s) * c);
+                alpha = ex2_approx(m_run - m_new);
+                m_run = m_new;
+                l_run *= alpha;
+                sum = probs64(s, c, m_run, pk);
+            }
+            // the tile's previous PV completed before these scores were committed
+            scale_tmem_f32(tcol + kColO, D / 32, alpha);
+            if (h == 1) scale_tmem_bf16(tcol, alpha);   // half 0's P is already stored
+        }
+        l_run += sum;
     } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) pk[j] = 0u;
     }
     tmem_st32(tcol + 32u * h, pk);
-    return RowState{sum, m_run, l_run};
 }
 
 // Shared-memory descriptor for a 1024-byte-aligned 128-byte-swizzled operand:
@@ -360,7 +420,20 @@ __device__ __forceinline__ uint64_t desc_at(uint64_t fixed, uint32_t saddr) {
     return fixed | static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
 }
 
-template <int D>
+// Position of a ring (or stage) counter: slot and phase parity.
+struct RingPos {
+    int slot;
+    uint32_t phase;
+    template <int N>
+    __device__ __forceinline__ void advance() {
+        if (++slot == N) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
+template <int D, int LM, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
 fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const FineParams p) {
@@ -373,7 +446,9 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     auto bar = [&](int i) -> uint32_t { return base + kOffBar + 8u * static_cast<uint32_t>(i); };
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+    StepRec* ring = reinterpret_cast<StepRec*>(smem + kOffRec);
     const BoundedWait bw{abort_flag, p.status, p.limit_ns};
+    const bool dense = p.idx == nullptr;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -389,8 +464,12 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(kBarSFull + t), 1);
-            mbar_init(bar(kBarPFull + t), 128);
+            mbar_init(bar(kBarPFull + t), 4);   // one arrival per softmax warp of the tile
             mbar_init(bar(kBarPVDone + t), 1);
+        }
+        for (int r = 0; r < kRing; ++r) {
+            mbar_init(bar(kBarRecFull + r), 1);
+            mbar_init(bar(kBarRecEmpty + r), kRecConsumers);
         }
         mbar_init(bar(kBarDrain), 1);
         fence_mbar_init();
@@ -408,48 +487,56 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t tmem = *tmem_slot;
 
     constexpr uint32_t kBytesQ = 4u * 64u * D * 2u;   // one Q group load
-    constexpr uint32_t kBytesKV = 2u * 64u * D * 2u;  // one step's two K (or V) cubes
+    constexpr uint32_t kBytesKV = 2u * 64u * D * 2u;  // one step's two K (or V) blocks
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ walk + TMA producer
         if (lane == 0) {
             uint32_t q_issued = 0, k_issued[kKStages] = {}, v_issued[kVStages] = {};
-            int64_t g = 0;
+            RingPos kp{0, 0}, vp{0, 0}, rp{0, 0};
             int n_item = 0;
             bool ok = true;
-            // two cubes into one stage: [d 0-63: a | b][d 64-127: a | b], 8 KB per box
-            auto load_pair = [&](const CUtensorMap* m, uint32_t dst, int32_t ra, int32_t rb, uint32_t b) {
-                tma_load_2d(dst, m, 0, ra, b);
-                tma_load_2d(dst + 8192, m, 0, rb, b);
-                if (D == 128) {
-                    tma_load_2d(dst + 16384, m, 64, ra, b);
-                    tma_load_2d(dst + 24576, m, 64, rb, b);
-                }
-            };
             for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
                 const Item item = decode_item(it, p);
+                auto load_pair = [&](const CUtensorMap* m, uint32_t dst, int ja, int jb, uint32_t b) {
+                    load_block<LM, D>(m, dst, ja, 0, b, item, p);
+                    load_block<LM, D>(m, dst + 8192, jb, 0, b, item, p);
+                    if (D == 128) {
+                        load_block<LM, D>(m, dst + 16384, ja, 64, b, item, p);
+                        load_block<LM, D>(m, dst + 24576, jb, 64, b, item, p);
+                    }
+                };
                 if (!(ok = bw.wait(bar(kBarQEmpty), (n_item & 1) ^ 1))) break;
                 mbar_arrive_expect_tx(bar(kBarQFull), kBytesQ);
                 ++q_issued;
                 for (int t = 0; t < 2; ++t)
-                    load_pair(&tm_q, base + kOffQ + t * kQTileBytes, tile_row(item.bh, item.cube[2 * t], p),
-                              tile_row(item.bh, item.cube[2 * t + 1], p), bar(kBarQFull));
+                    load_pair(&tm_q, base + kOffQ + t * kQTileBytes, item.blk[2 * t], item.blk[2 * t + 1],
+                              bar(kBarQFull));
                 GroupWalk w = make_walk(item, p);
-                int ca, cb;
-                uint32_t flags;
-                while (w.next(ca, cb, flags)) {
-                    const int32_t ra = tile_row(item.bh, ca, p), rb = tile_row(item.bh, cb, p);
-                    const int ks = static_cast<int>(g % kKStages);
-                    if (!(ok = bw.wait(bar(kBarKEmpty + ks), static_cast<uint32_t>((g / kKStages) & 1) ^ 1u))) break;
-                    mbar_arrive_expect_tx(bar(kBarKFull + ks), kBytesKV);
-                    ++k_issued[ks];
-                    load_pair(&tm_k, base + kOffK + ks * kKVBytes, ra, rb, bar(kBarKFull + ks));
-                    const int vs = static_cast<int>(g % kVStages);
-                    if (!(ok = bw.wait(bar(kBarVEmpty + vs), static_cast<uint32_t>((g / kVStages) & 1) ^ 1u))) break;
-                    mbar_arrive_expect_tx(bar(kBarVFull + vs), kBytesKV);
-                    ++v_issued[vs];
-                    load_pair(&tm_v, base + kOffV + vs * kKVBytes, ra, rb, bar(kBarVFull + vs));
-                    ++g;
+                for (int s = 0;; ++s) {
+                    StepRec r;
+                    if (dense) {
+                        r = dense_step(s, item.present, p.nblk);
+                    } else {
+                        // an item none of whose slots holds a query block (an order
+                        // entry out of range) still publishes one empty step
+                        if (!w.next(r)) r = StepRec{-1, -1, 0u, 1u};
+                        if (!(ok = bw.wait(bar(kBarRecEmpty + rp.slot), rp.phase ^ 1u))) break;
+                        ring[rp.slot] = r;
+                        mbar_arrive(bar(kBarRecFull + rp.slot));   // release: the record is visible
+                        rp.advance<kRing>();
+                    }
+                    if (!(ok = bw.wait(bar(kBarKEmpty + kp.slot), kp.phase ^ 1u))) break;
+                    mbar_arrive_expect_tx(bar(kBarKFull + kp.slot), kBytesKV);
+                    ++k_issued[kp.slot];
+                    load_pair(&tm_k, base + kOffK + kp.slot * kKVBytes, r.ca, r.cb, bar(kBarKFull + kp.slot));
+                    kp.advance<kKStages>();
+                    if (!(ok = bw.wait(bar(kBarVEmpty + vp.slot), vp.phase ^ 1u))) break;
+                    mbar_arrive_expect_tx(bar(kBarVFull + vp.slot), kBytesKV);
+                    ++v_issued[vp.slot];
+                    load_pair(&tm_v, base + kOffV + vp.slot * kKVBytes, r.ca, r.cb, bar(kBarVFull + vp.slot));
+                    vp.advance<kVStages>();
+                    if (r.last) break;
                 }
             }
             if (!ok) {
@@ -473,11 +560,11 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);     // P (TMEM, K-major) x V (MN-major)
             const uint64_t fix_k = smem_desc_sw128(0, 16u, 1024u);         // K-major, 8-row groups 1 KB apart
             const uint64_t fix_v = smem_desc_sw128(0, 16384u, 1024u);      // MN-major, d halves 16 KB apart
-            int64_t g = 0;
-            uint32_t n_s[2] = {0, 0}, n_p[2] = {0, 0};   // per-tile S and PV steps issued
+            RingPos kp{0, 0}, vp{0, 0}, rp{0, 0};
+            uint32_t n_p[2] = {0, 0};   // per-tile PV steps issued
             int n_item = 0;
             bool ok = true, issued_any = false;
-            bool acc[2] = {false, false};                 // O of the tile already holds this item's sum
+            bool acc[2] = {false, false};   // O of the tile already holds this item's sum
             auto issue_s = [&](int t, int ks) {
                 const uint32_t qa = base + kOffQ + t * kQTileBytes;
                 const uint32_t kb = base + kOffK + ks * kKVBytes;
@@ -488,16 +575,14 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                                 kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(kBarSFull + t));
-                ++n_s[t];
                 issued_any = true;
             };
-            // PV of tile t for the step whose V sits in stage vs (waits for its P and V)
-            auto issue_pv = [&](int t, int64_t gs) -> bool {
-                const int vs = static_cast<int>(gs % kVStages);
+            // PV of tile t for the step whose V sits in stage v (waits for its P and V)
+            auto issue_pv = [&](int t, RingPos v) -> bool {
                 if (!bw.wait(bar(kBarPFull + t), n_p[t] & 1u)) return false;
-                if (!bw.wait(bar(kBarVFull + vs), static_cast<uint32_t>((gs / kVStages) & 1))) return false;
+                if (!bw.wait(bar(kBarVFull + v.slot), v.phase)) return false;
                 tc_fence_after();
-                const uint32_t vb = base + kOffV + vs * kKVBytes;
+                const uint32_t vb = base + kOffV + v.slot * kKVBytes;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_bf16_ts(tmem + t * kTileCols + kColO, tmem + t * kTileCols + 8u * kk,
@@ -508,33 +593,42 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 return true;
             };
             for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
-                const Item item = decode_item(it, p);
+                const uint32_t present = dense ? decode_item(it, p).present : 0u;
                 if (!(ok = bw.wait(bar(kBarQFull), n_item & 1))) break;
                 acc[0] = acc[1] = false;
-                GroupWalk w = make_walk(item, p);
-                int ca, cb;
-                uint32_t flags;
                 bool pend_b = false;   // PV of tile B for the previous step still to issue
-                int64_t g_prev = -1;
-                while (w.next(ca, cb, flags)) {
-                    const int ks = static_cast<int>(g % kKStages);
-                    if (!(ok = bw.wait(bar(kBarKFull + ks), static_cast<uint32_t>((g / kKStages) & 1)))) break;
+                bool have_prev = false;
+                RingPos v_prev{0, 0};
+                for (int s = 0;; ++s) {
+                    StepRec r;
+                    if (dense) {
+                        r = dense_step(s, present, p.nblk);
+                    } else {
+                        if (!(ok = bw.wait(bar(kBarRecFull + rp.slot), rp.phase))) break;
+                        r = ring[rp.slot];
+                        mbar_arrive(bar(kBarRecEmpty + rp.slot));
+                        rp.advance<kRing>();
+                    }
+                    if (!(ok = bw.wait(bar(kBarKFull + kp.slot), kp.phase))) break;
                     tc_fence_after();
-                    const bool act_a = tile_active(flags, 0), act_b = tile_active(flags, 1);
-                    if (act_a) issue_s(0, ks);                                  // S_A(i)
-                    if (pend_b && !(ok = issue_pv(1, g_prev))) break;           // PV_B(i-1)
-                    if (g_prev >= 0) mma_commit(bar(kBarVEmpty + static_cast<int>(g_prev % kVStages)));
-                    if (act_b) issue_s(1, ks);                                  // S_B(i)
-                    mma_commit(bar(kBarKEmpty + ks));
-                    if (act_a && !(ok = issue_pv(0, g))) break;                 // PV_A(i)
+                    const bool act_a = tile_active(r.flags, 0), act_b = tile_active(r.flags, 1);
+                    if (act_a) issue_s(0, kp.slot);                               // S_A(i)
+                    if (pend_b && !(ok = issue_pv(1, v_prev))) break;             // PV_B(i-1)
+                    if (have_prev) mma_commit(bar(kBarVEmpty + v_prev.slot));
+                    if (act_b) issue_s(1, kp.slot);                               // S_B(i)
+                    mma_commit(bar(kBarKEmpty + kp.slot));
+                    kp.advance<kKStages>();
+                    if (act_a && !(ok = issue_pv(0, vp))) break;                  // PV_A(i)
                     pend_b = act_b;
-                    g_prev = g;
-                    ++g;
+                    have_prev = true;
+                    v_prev = vp;
+                    vp.advance<kVStages>();
+                    if (r.last) break;
                 }
                 if (!ok) break;
                 mma_commit(bar(kBarQEmpty));
-                if (pend_b && !(ok = issue_pv(1, g_prev))) break;
-                if (g_prev >= 0) mma_commit(bar(kBarVEmpty + static_cast<int>(g_prev % kVStages)));
+                if (pend_b && !(ok = issue_pv(1, v_prev))) break;
+                if (have_prev) mma_commit(bar(kBarVEmpty + v_prev.slot));
             }
             if (issued_any) {
                 // all MMAs of this CTA complete before tensor memory is freed
@@ -543,20 +637,20 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 while (!mbar_try_wait(bar(kBarDrain), 0) && globaltimer() - t0 < kDrainLimitNs) {
                 }
             }
-            (void)n_s;
         }
     } else {
         // ------------------------------------------------------------ softmax + epilogue
         const int tile = (warp - 2) >> 2;        // 0: warps 2..5, 1: warps 6..9
         const int q = warp & 3;                  // TMEM lane quarter of this warp
         const int row = q * 32 + lane;           // query row of the tile, 0..127
-        const int slot = 2 * tile + (q >> 1);    // query-cube slot of the group
+        const int slot = 2 * tile + (q >> 1);    // query-block slot of the group
         const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
         const uint32_t tcol = tmem + tile * kTileCols + lane_addr;
         const uint32_t bar_sfull = bar(kBarSFull + tile), bar_pfull = bar(kBarPFull + tile);
         const uint32_t bar_pvdone = bar(kBarPVDone + tile);
         const float c = p.c_log2;
         uint32_t n = 0;   // steps this tile has taken part in (same count as the MMA issuer's)
+        RingPos rp{0, 0};
         bool ok = true;
         auto wait_all = [&](uint32_t b, uint32_t par) -> bool {
             const bool mine = bw.wait(b, par);
@@ -564,82 +658,133 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         };
         for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x) {
             const Item item = decode_item(it, p);
-            GroupWalk w = make_walk(item, p);
             float m_run = -INFINITY, l_run = 0.f;
             uint32_t steps = 0;
-            int ca, cb;
-            uint32_t flags;
-            while (w.next(ca, cb, flags)) {
-                if (!tile_active(flags, tile)) continue;      // the tile skips this step
-                if (!(ok = wait_all(bar_sfull, n & 1u))) break;
-                tc_fence_after();
-                // warp-uniform: this warp's rows belong to one query cube
-                const uint64_t vm_a = ((flags >> slot) & 1u) ? cube_key_mask(ca, p) : 0ull;
-                const uint64_t vm_b = ((flags >> (4 + slot)) & 1u) ? cube_key_mask(cb, p) : 0ull;
-                const bool row_active = (vm_a | vm_b) != 0ull;   // warp-uniform
-                // the row's first step with keys: the running maximum starts at the tile maximum
-                if (row_active && m_run == -INFINITY) {
-                    m_run = tile_max(tcol, vm_a, vm_b) * c;
-                    l_run = 0.f;
+            for (int s = 0;; ++s) {
+                StepRec r;
+                if (dense) {
+                    r = dense_step(s, item.present, p.nblk);
+                } else {
+                    if (!(ok = wait_all(bar(kBarRecFull + rp.slot), rp.phase))) break;
+                    r = ring[rp.slot];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(kBarRecEmpty + rp.slot));
+                    rp.advance<kRing>();
                 }
-                // P per cube half h, from the scores in columns [64h, 64h + 64), stored as bf16
-                // pairs over columns [32h, 32h + 32).  A half whose probabilities would exceed
-                // 2^64 (the lazy maximum fell far behind) moves the maximum up first; the
-                // scores of both halves are intact until half 0's P is stored.
-#pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t pk[32];
-                    float sum = 0.f;
-                    const uint64_t vm = h ? vm_b : vm_a;
-                    if (row_active) sum = probs_half(tcol + 64u * h, vm, c, m_run, pk);
-                    const bool over = !(sum <= kSumLimit);
-                    if (__any_sync(0xffffffffu, over)) {
-                        const RowState r = move_max_and_redo<D>(tcol, h, vm_a, vm_b, c, over, row_active, m_run, l_run);
-                        sum = r.sum;
-                        m_run = r.m;
-                        l_run = r.l;
-                    } else {
-                        if (!row_active) {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) pk[j] = 0u;
-                        }
-                        tmem_st32(tcol + 32u * h, pk);
-                    }
-                    l_run += sum;
+                if (tile_active(r.flags, tile)) {
+                    // warp-uniform: this warp's rows belong to one query block
+                    const uint64_t vm_a = ((r.flags >> slot) & 1u) ? key_mask<LM>(r.ca, p) : 0ull;
+                    const uint64_t vm_b = ((r.flags >> (4 + slot)) & 1u) ? key_mask<LM>(r.cb, p) : 0ull;
+                    if (!(ok = wait_all(bar_sfull, n & 1u))) break;
+                    tc_fence_after();
+                    softmax_half<D>(tcol, 0, vm_a, c, m_run, l_run);
+                    softmax_half<D>(tcol, 1, vm_b, c, m_run, l_run);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_pfull);
+                    ++n;
+                    ++steps;
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar_pfull);
-                ++n;
-                ++steps;
+                if (r.last) break;
             }
             if (!ok) break;
-            if (steps == 0) continue;   // the tile holds no query cube of this group
-            // ---------------- epilogue: O / l and log-sum-exp of this tile's rows
+            if (steps == 0) continue;   // the tile holds no query block of this group
+            // ---------------- epilogue of this tile's rows
             // PV(n-2) completed before S(n-1) was committed, so this parity cannot alias
             if (!(ok = wait_all(bar_pvdone, (n - 1) & 1u))) break;
             tc_fence_after();
-            const int cube_row = item.cube[slot];
-            const bool store = cube_row >= 0;
-            const int64_t grow = item.bh * p.Npad + static_cast<int64_t>(store ? cube_row : 0) * 64 + (row & 63);
+            const int blk = item.blk[slot];
+            const int o_ = row & 63;
             const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+            if (!FUSED) {
+                const bool store = blk >= 0;
+                const int64_t grow = item.bh * p.Npad + static_cast<int64_t>(store ? blk : 0) * 64 + o_;
 #pragma unroll 1
-            for (int ch = 0; ch < D / 32; ++ch) {
-                uint32_t o[32];
-                tmem_ld32_wait(tcol + kColO + 32u * ch, o);
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32_wait(tcol + kColO + 32u * ch, o);
+                    if (store) {
+                        uint32_t w16[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            w16[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv_l,
+                                                 __uint_as_float(o[2 * j + 1]) * inv_l);
+                        uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + 32 * ch);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(w16[4 * v], w16[4 * v + 1], w16[4 * v + 2], w16[4 * v + 3]);
+                    }
+                }
+                if (store && p.lse != nullptr)
+                    p.lse[grow] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+            } else {
+                // token of this row, and the cube whose coarse output it merges
+                int64_t tok = -1;
+                int cube = 0;
+                if (blk >= 0) {
+                    if (LM == kLoadTokens) {
+                        tok = 64ll * blk + o_;
+                        if (tok >= p.N) {
+                            tok = -1;
+                        } else if (p.o_coarse != nullptr) {
+                            const int64_t xy = static_cast<int64_t>(p.X) * p.Y;
+                            const int tt = static_cast<int>(tok / xy);
+                            const int rem = static_cast<int>(tok - tt * xy);
+                            const int xx = rem / p.Y, yy = rem - (rem / p.Y) * p.Y;
+                            cube = ((tt >> 2) * p.Cx + (xx >> 2)) * p.Cy + (yy >> 2);
+                        }
+                    } else {
+                        const uint32_t qd = div_magic(static_cast<uint32_t>(blk), p.magic_cy);
+                        const uint32_t ct = div_magic(qd, p.magic_cx);
+                        const int cy = blk - static_cast<int>(qd) * p.Cy;
+                        const int cx = static_cast<int>(qd) - static_cast<int>(ct) * p.Cx;
+                        const int tt = 4 * static_cast<int>(ct) + (o_ >> 4);
+                        const int xx = 4 * cx + ((o_ >> 2) & 3), yy = 4 * cy + (o_ & 3);
+                        if (tt < p.T && xx < p.X && yy < p.Y)
+                            tok = (static_cast<int64_t>(tt) * p.X + xx) * p.Y + yy;
+                        cube = blk;
+                    }
+                }
+                const bool store = tok >= 0;
+                float gc = 0.f, gf = 1.f;
+                const float* ocr = nullptr;
+                const int64_t grow = (static_cast<int64_t>(item.b) * p.N + (store ? tok : 0)) * p.H + item.h;
                 if (store) {
-                    uint32_t w16[16];
+                    if (p.g_coarse) gc = __uint_as_float(static_cast<uint32_t>(__ldg(p.g_coarse + grow)) << 16);
+                    if (p.g_fine) gf = __uint_as_float(static_cast<uint32_t>(__ldg(p.g_fine + grow)) << 16);
+                    if (p.o_coarse) ocr = p.o_coarse + (item.bh * p.C + cube) * D;
+                }
+                const float sf = gf * inv_l;
+#pragma unroll 1
+                for (int ch = 0; ch < D / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32_wait(tcol + kColO + 32u * ch, o);
+                    if (store) {
+                        float v[32];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        w16[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv_l, __uint_as_float(o[2 * j + 1]) * inv_l);
-                    uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + 32 * ch);
+                        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(o[j]) * sf;
+                        if (ocr != nullptr) {
+                            const float4* oc4 = reinterpret_cast<const float4*>(ocr + 32 * ch);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(w16[4 * v], w16[4 * v + 1], w16[4 * v + 2], w16[4 * v + 3]);
+                            for (int j = 0; j < 8; ++j) {
+                                const float4 cv = __ldg(oc4 + j);
+                                v[4 * j] = fmaf(gc, cv.x, v[4 * j]);
+                                v[4 * j + 1] = fmaf(gc, cv.y, v[4 * j + 1]);
+                                v[4 * j + 2] = fmaf(gc, cv.z, v[4 * j + 2]);
+                                v[4 * j + 3] = fmaf(gc, cv.w, v[4 * j + 3]);
+                            }
+                        }
+                        uint32_t w16[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) w16[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                        uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + 32 * ch);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(w16[4 * v4], w16[4 * v4 + 1], w16[4 * v4 + 2], w16[4 * v4 + 3]);
+                    }
                 }
             }
-            if (store && p.lse != nullptr)
-                p.lse[grow] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
             tc_fence_before();
         }
     }
@@ -682,31 +827,75 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-bool encode_rows(CUtensorMap* m, const void* ptr, int D, int64_t rows) {
+// bf16 tensor map with a 64-channel (128-byte, swizzled) innermost box edge.
+bool encode_map(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                const cuuint32_t* box) {
     auto fn = encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2u};
-    const cuuint32_t box[2] = {64u, 64u};
-    const cuuint32_t estr[2] = {1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(ptr), dims,
+              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
-cudaError_t set_smem_attr() {
+// Tiled [rows, D]: box 64 channels x 64 rows.
+bool encode_tiled(CUtensorMap* m, const void* ptr, const Dims& d) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d.D), static_cast<cuuint64_t>(d.rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d.D) * 2u};
+    const cuuint32_t box[2] = {64u, 64u};
+    return encode_map(m, ptr, 2, dims, strides, box);
+}
+
+// Projection layout [B, N, H, D] seen as (H*D channels, Y, X, T, B): box
+// 64 channels x 4 x 4 x 4 tokens = one cube in cube-major offset order.
+bool encode_cubes(CUtensorMap* m, const void* ptr, const Dims& d) {
+    const cuuint64_t hd = static_cast<cuuint64_t>(d.H) * d.D;
+    const cuuint64_t dims[5] = {hd, static_cast<cuuint64_t>(d.Y), static_cast<cuuint64_t>(d.X),
+                                static_cast<cuuint64_t>(d.T), static_cast<cuuint64_t>(d.B)};
+    const cuuint64_t row = hd * 2u;
+    const cuuint64_t strides[4] = {row, row * d.Y, row * d.Y * d.X, row * static_cast<cuuint64_t>(d.N)};
+    const cuuint32_t box[5] = {64u, 4u, 4u, 4u, 1u};
+    return encode_map(m, ptr, 5, dims, strides, box);
+}
+
+// Projection layout [B, N, H, D] seen as (H*D channels, N, B): box
+// 64 channels x 64 consecutive tokens.
+bool encode_tokens(CUtensorMap* m, const void* ptr, const Dims& d) {
+    const cuuint64_t hd = static_cast<cuuint64_t>(d.H) * d.D;
+    const cuuint64_t dims[3] = {hd, static_cast<cuuint64_t>(d.N), static_cast<cuuint64_t>(d.B)};
+    const cuuint64_t strides[2] = {hd * 2u, hd * 2u * static_cast<cuuint64_t>(d.N)};
+    const cuuint32_t box[3] = {64u, 64u, 1u};
+    return encode_map(m, ptr, 3, dims, strides, box);
+}
+
+template <int D, int LM, bool FUSED>
+cudaError_t launch_instance(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const FineParams& p, int grid, cudaStream_t s) {
     static int done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(fine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
-    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
-    return e;
+    if (!(dev >= 0 && dev < 64 && done[dev])) {
+        cudaError_t e = cudaFuncSetAttribute(fine_kernel<D, LM, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemBytes));
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) done[dev] = 1;
+    }
+    fine_kernel<D, LM, FUSED><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
+    return cudaGetLastError();
 }
 
 uint64_t magic48(uint32_t d) { return ((uint64_t{1} << 48) / d) + 1; }
+
+// Real offsets o = (t%4)*16 + (x%4)*4 + y%4 of a cube whose extent along one
+// axis is n (< 4 only in the last cube layer of that axis).
+uint64_t axis_mask(int axis, int n) {
+    uint64_t m = 0;
+    for (int o = 0; o < 64; ++o) {
+        const int e = axis == 0 ? (o >> 4) : axis == 1 ? ((o >> 2) & 3) : (o & 3);
+        if (e < n) m |= 1ull << o;
+    }
+    return m;
+}
 
 }  // namespace
 
@@ -724,21 +913,36 @@ int* status_word() {
     return ptrs[dev];
 }
 
-cudaError_t launch_fine(const Dims& d, const uint16_t* qt, const uint16_t* kt, const uint16_t* vt,
-                        const int32_t* idx, int k, const int32_t* order, float scale, uint16_t* o_fine,
-                        float* lse, cudaStream_t s, const char** why) {
+cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const char** why) {
     CUtensorMap tq, tk, tv;
-    if (!encode_rows(&tq, qt, d.D, d.rows) || !encode_rows(&tk, kt, d.D, d.rows) ||
-        !encode_rows(&tv, vt, d.D, d.rows)) {
-        if (why) *why = "cuTensorMapEncodeTiled failed for a tiled Q/K/V tensor";
+    bool enc = false;
+    const int mode = a.mode;
+    if (mode == kFineTiled) {
+        enc = encode_tiled(&tq, a.q, d) && encode_tiled(&tk, a.k, d) && encode_tiled(&tv, a.v, d);
+    } else if (mode == kFineCubesFused) {
+        enc = encode_cubes(&tq, a.q, d) && encode_cubes(&tk, a.k, d) && encode_cubes(&tv, a.v, d);
+    } else if (mode == kFineTokensFused) {
+        enc = encode_tokens(&tq, a.q, d) && encode_tokens(&tk, a.k, d) && encode_tokens(&tv, a.v, d);
+    } else {
+        if (why) *why = "unknown fine-stage mode";
+        return cudaErrorInvalidValue;
+    }
+    if (!enc) {
+        if (why) *why = "cuTensorMapEncodeTiled failed for a Q/K/V tensor";
         return cudaErrorInvalidValue;
     }
     FineParams p{};
-    p.idx = idx;
-    p.order = order;
-    p.o = o_fine;
-    p.lse = lse;
-    p.k = idx ? k : d.C;
+    p.idx = a.idx;
+    p.order = a.order;
+    p.o = a.out;
+    p.lse = a.lse;
+    p.o_coarse = a.o_coarse;
+    p.g_coarse = a.g_coarse;
+    p.g_fine = a.g_fine;
+    p.B = d.B;
+    p.H = d.H;
+    p.nblk = mode == kFineTokensFused ? static_cast<int>((d.N + 63) / 64) : d.C;
+    p.k = a.idx ? a.k_sel : p.nblk;
     p.C = d.C;
     p.Ct = d.Ct;
     p.Cx = d.Cx;
@@ -746,13 +950,18 @@ cudaError_t launch_fine(const Dims& d, const uint16_t* qt, const uint16_t* kt, c
     p.T = d.T;
     p.X = d.X;
     p.Y = d.Y;
-    p.ngroups = (d.C + 3) / 4;
+    p.N = d.N;
+    p.ngroups = (p.nblk + 3) / 4;
     p.magic_cxcy = magic48(static_cast<uint32_t>(d.Cx * d.Cy));
     p.magic_cy = magic48(static_cast<uint32_t>(d.Cy));
+    p.magic_cx = magic48(static_cast<uint32_t>(d.Cx));
+    p.mask_t = axis_mask(0, d.T - 4 * (d.Ct - 1));
+    p.mask_x = axis_mask(1, d.X - 4 * (d.Cx - 1));
+    p.mask_y = axis_mask(2, d.Y - 4 * (d.Cy - 1));
     p.Npad = d.Npad;
     p.items = static_cast<int64_t>(d.B) * d.H * p.ngroups;
     p.oob_row = static_cast<int32_t>(d.rows);
-    p.c_log2 = scale * 1.4426950408889634f;
+    p.c_log2 = a.scale * 1.4426950408889634f;
     p.status = status_word();
     p.limit_ns = kWaitLimitNs;
     if (!p.status) {
@@ -760,15 +969,14 @@ cudaError_t launch_fine(const Dims& d, const uint16_t* qt, const uint16_t* kt, c
         return cudaErrorInvalidValue;
     }
     const int grid = static_cast<int>(p.items < sm_count() ? p.items : sm_count());
-    cudaError_t e;
     if (d.D == 128) {
-        if ((e = set_smem_attr<128>()) != cudaSuccess) return e;
-        fine_kernel<128><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
-    } else {
-        if ((e = set_smem_attr<64>()) != cudaSuccess) return e;
-        fine_kernel<64><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, p);
+        if (mode == kFineTiled) return launch_instance<128, kLoadTiled, false>(tq, tk, tv, p, grid, s);
+        if (mode == kFineCubesFused) return launch_instance<128, kLoadCubes, true>(tq, tk, tv, p, grid, s);
+        return launch_instance<128, kLoadTokens, true>(tq, tk, tv, p, grid, s);
     }
-    return cudaGetLastError();
+    if (mode == kFineTiled) return launch_instance<64, kLoadTiled, false>(tq, tk, tv, p, grid, s);
+    if (mode == kFineCubesFused) return launch_instance<64, kLoadCubes, true>(tq, tk, tv, p, grid, s);
+    return launch_instance<64, kLoadTokens, true>(tq, tk, tv, p, grid, s);
 }
 
 cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t s) {

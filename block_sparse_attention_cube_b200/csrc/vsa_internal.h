@@ -54,13 +54,38 @@ cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx,
 constexpr int kGroupMaxC = 4096;
 cudaError_t launch_group(const Dims& d, const float* scores, int32_t* order, cudaStream_t s);
 
-// Fine stage.  `order` (may be null) is a per-head permutation of the query
-// cubes; groups of four consecutive entries share one key/value stream.
-// Returns cudaErrorInvalidValue (with *why set) when a tensor map cannot be
-// encoded.
-cudaError_t launch_fine(const Dims& d, const uint16_t* qt, const uint16_t* kt, const uint16_t* vt,
-                        const int32_t* idx, int k, const int32_t* order, float scale, uint16_t* o_fine,
-                        float* lse, cudaStream_t s, const char** why);
+// Fine stage.  Modes:
+//  kFineTiled       - q/k/v tiled [B, H, Npad, D]; out = tiled O_f (+ lse when non-null);
+//  kFineCubesFused  - q/k/v in the projection layout [B, N, H, D], cubes gathered by TMA;
+//                     out = g_c * O_c[cube] + g_f * O_f in [B, N, H, D] (o_coarse/g_coarse/g_fine
+//                     may be null: no coarse term / gate 1);
+//  kFineTokensFused - as kFineCubesFused but attending over blocks of 64 consecutive real
+//                     tokens (dense attention only: idx must be null).
+// `order` (may be null) is a per-head permutation of the query cubes; groups
+// of four consecutive entries share one key/value stream.  Returns
+// cudaErrorInvalidValue (with *why set) when a tensor map cannot be encoded.
+enum FineMode : int { kFineTiled = 0, kFineCubesFused = 1, kFineTokensFused = 2 };
+
+struct FineArgs {
+    int mode;
+    const uint16_t *q, *k, *v;
+    const int32_t* idx;     // [B, H, C, k] or null (every block)
+    int k_sel;
+    const int32_t* order;   // [B, H, C] or null
+    float scale;
+    uint16_t* out;
+    float* lse;             // kFineTiled only
+    const float* o_coarse;  // fused modes only
+    const uint16_t* g_coarse;
+    const uint16_t* g_fine;
+};
+
+cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const char** why);
+
+// Cube mean-pool read straight from the projection layout [B, N, H, D]
+// (same fp32 summation order as launch_pool on the tiled tensor).
+cudaError_t launch_pool_tokens(const Dims& d, const uint16_t* const* x, float* const* xbar, int count,
+                               cudaStream_t s);
 
 cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t s);
 

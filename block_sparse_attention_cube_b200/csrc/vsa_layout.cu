@@ -144,6 +144,65 @@ __global__ void __launch_bounds__(kBlock) pool_kernel(Dims d, PoolIO io) {
     }
 }
 
+// The same pool read straight from the projection layout [B, N, H, D], so a
+// forward call needs no tiled copy.  Tasks run (tensor, b, cube, head) with
+// the head fastest: the warps of a block read neighbouring heads of the same
+// tokens, 256 contiguous bytes per row.  Each output channel is summed in the
+// same order as pool_kernel (per lane group in offset order, then the same
+// shuffle tree), so both give identical float32 means.
+template <int D>
+__global__ void __launch_bounds__(kBlock) pool_tokens_kernel(Dims d, PoolIO io) {
+    constexpr int LPR = D / 8;          // lanes per row
+    constexpr int RPI = 32 / LPR;       // rows per warp iteration
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / LPR, j = lane % LPR;
+    const int64_t per_tensor = static_cast<int64_t>(d.B) * d.H * d.C;
+    const int64_t total = per_tensor * io.count;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kBlock / 32);
+    for (int64_t task = static_cast<int64_t>(blockIdx.x) * (kBlock / 32) + threadIdx.x / 32; task < total;
+         task += warps) {
+        const int tensor = static_cast<int>(task / per_tensor);
+        const int64_t r = task - tensor * per_tensor;
+        const int h = static_cast<int>(r % d.H);
+        const int64_t bc = r / d.H;
+        const int c = static_cast<int>(bc % d.C);
+        const int b = static_cast<int>(bc / d.C);
+        const int ct = c / (d.Cx * d.Cy), cx = (c / d.Cy) % d.Cx, cy = c % d.Cy;
+        const uint4* src = reinterpret_cast<const uint4*>(io.src[tensor]);
+        const int nt = min(kCube, d.T - ct * kCube);
+        const int nx = min(kCube, d.X - cx * kCube);
+        const int ny = min(kCube, d.Y - cy * kCube);
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 4
+        for (int o = sub; o < kCubeTokens; o += RPI) {
+            const int ot = o >> 4, ox = (o >> 2) & 3, oy = o & 3;
+            if (ot >= nt || ox >= nx || oy >= ny) continue;
+            const int64_t n = (static_cast<int64_t>(ct * kCube + ot) * d.X + cx * kCube + ox) * d.Y + cy * kCube + oy;
+            const uint4 v = __ldcs(src + ((static_cast<int64_t>(b) * d.N + n) * d.H + h) * LPR + j);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                acc[2 * e] += __uint_as_float(w[e] << 16);
+                acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+            }
+        }
+#pragma unroll
+        for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+        }
+        if (sub == 0) {
+            const float inv = 1.0f / static_cast<float>(nt * nx * ny);
+            const int64_t bh = static_cast<int64_t>(b) * d.H + h;
+            float4* out = reinterpret_cast<float4*>(io.dst[tensor] + (bh * d.C + c) * D + j * 8);
+            out[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+            out[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+        }
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kBlock) combine_kernel(Dims d, const float* __restrict__ o_coarse,
                                                          const uint16_t* __restrict__ o_fine,
@@ -220,6 +279,21 @@ cudaError_t launch_pool(const Dims& d, const uint16_t* const* xt, float* const* 
     const int grid = grid_for((warps + 7) / 8, 8);
     if (d.D == 128) pool_kernel<128><<<grid, kBlock, 0, s>>>(d, io);
     else pool_kernel<64><<<grid, kBlock, 0, s>>>(d, io);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pool_tokens(const Dims& d, const uint16_t* const* x, float* const* xbar, int count,
+                               cudaStream_t s) {
+    PoolIO io{};
+    for (int i = 0; i < count; ++i) {
+        io.src[i] = x[i];
+        io.dst[i] = xbar[i];
+    }
+    io.count = count;
+    const int64_t warps = static_cast<int64_t>(d.B) * d.H * d.C * count;
+    const int grid = grid_for((warps + 7) / 8, 8);
+    if (d.D == 128) pool_tokens_kernel<128><<<grid, kBlock, 0, s>>>(d, io);
+    else pool_tokens_kernel<64><<<grid, kBlock, 0, s>>>(d, io);
     return cudaGetLastError();
 }
 

@@ -2,11 +2,13 @@
 
     python -m block_sparse_attention_cube_b200.run_case --workload wan480p_vsa_k32 --iters 3
 
-Each iteration runs tile -> pool -> coarse -> top-k -> fine -> combine -> untile
-through the C ABI (tile -> fine -> untile when top-k covers every cube), with
-CUDA events between the stages.  `--dense-too` adds a dense fine launch on the
-same tiled tensors.  Useful on its own and as a small, fixed case to put
-under a profiler.
+Each iteration runs the launches of vsa_forward one by one through the C ABI,
+pool_qkv -> coarse -> top-k -> group -> fine_fused (fine_fused alone, dense,
+when top-k covers every cube), with CUDA events between the stages.
+`--dense-too` adds a dense fine_fused launch on the same inputs.  `--staged`
+runs the unfused per-step path instead (tile -> pool -> coarse -> top-k ->
+group -> fine -> combine -> untile).  Useful on its own and as a small, fixed
+case to put under a profiler.
 """
 from __future__ import annotations
 
@@ -34,6 +36,7 @@ def main(argv=None) -> int:
     ap.add_argument("--workload", default="wan480p_vsa_k32", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--dense-too", action="store_true")
+    ap.add_argument("--staged", action="store_true")
     a = ap.parse_args(argv)
     w = synth.WORKLOADS[a.workload]
     x = synth.make_inputs(w)
@@ -42,8 +45,11 @@ def main(argv=None) -> int:
     npad, C = vsa.shape_info(s)
     scale = 1.0 / math.sqrt(w.head_dim)
     dense = w.topk == C
-    names = ["tile", "fine", "untile"] if dense else ["tile", "pool", "coarse", "topk+group", "fine", "combine",
-                                                       "untile"]
+    if a.staged:
+        names = ["tile", "fine", "untile"] if dense else ["tile", "pool", "coarse", "topk+group", "fine", "combine",
+                                                           "untile"]
+    else:
+        names = ["fine"] if dense else ["pool", "coarse", "topk", "group", "fine"]
     if a.dense_too:
         names.append("fine_dense")
     times = {n: [] for n in names}
@@ -58,30 +64,49 @@ def main(argv=None) -> int:
             i += 1
 
         mark()
-        qt, kt, vt = (vsa.tile(d[n], s) for n in ("q", "k", "v"))
-        mark()
-        if dense:
-            of, _ = vsa.fine(qt, kt, vt, s, None, scale, want_lse=False)
+        if a.staged:
+            qt, kt, vt = (vsa.tile(d[n], s) for n in ("q", "k", "v"))
             mark()
-            vsa.untile(of, s)
-            mark()
+            if dense:
+                of, _ = vsa.fine(qt, kt, vt, s, None, scale, want_lse=False)
+                mark()
+                vsa.untile(of, s)
+                mark()
+            else:
+                bars = [vsa.pool(t, s) for t in (qt, kt, vt)]
+                mark()
+                scores, oc = vsa.coarse(*bars, s, scale)
+                mark()
+                idx = vsa.topk(scores, s, w.topk)
+                order = vsa.group(scores, s)
+                mark()
+                of, _ = vsa.fine(qt, kt, vt, s, idx, scale, want_lse=False, order=order)
+                mark()
+                ot = vsa.combine(oc, of, s, d["g_coarse"], d["g_fine"])
+                mark()
+                vsa.untile(ot, s)
+                mark()
+            if a.dense_too:
+                vsa.fine(qt, kt, vt, s, None, scale, want_lse=False)
+                mark()
         else:
-            bars = [vsa.pool(t, s) for t in (qt, kt, vt)]
-            mark()
-            scores, oc = vsa.coarse(*bars, s, scale)
-            mark()
-            idx = vsa.topk(scores, s, w.topk)
-            order = vsa.group(scores, s)
-            mark()
-            of, _ = vsa.fine(qt, kt, vt, s, idx, scale, want_lse=False, order=order)
-            mark()
-            ot = vsa.combine(oc, of, s, d["g_coarse"], d["g_fine"])
-            mark()
-            vsa.untile(ot, s)
-            mark()
-        if a.dense_too:
-            vsa.fine(qt, kt, vt, s, None, scale, want_lse=False)
-            mark()
+            if dense:
+                vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale)
+                mark()
+            else:
+                bars = vsa.pool_qkv(d["q"], d["k"], d["v"], s)
+                mark()
+                scores, oc = vsa.coarse(*bars, s, scale)
+                mark()
+                idx = vsa.topk(scores, s, w.topk)
+                mark()
+                order = vsa.group(scores, s)
+                mark()
+                vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, order, oc, d["g_coarse"], d["g_fine"])
+                mark()
+            if a.dense_too:
+                vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale)
+                mark()
         torch.cuda.synchronize()
         for j, n in enumerate(names):
             times[n].append(ev[j].elapsed_time(ev[j + 1]))

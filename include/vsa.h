@@ -187,20 +187,58 @@ vsa_status vsa_combine(const vsa_shape* shape, const float* o_coarse, const vsa_
                        const vsa_bf16* g_coarse, const vsa_bf16* g_fine, vsa_bf16* o_tiled,
                        vsa_stream_t stream);
 
+/*
+ * vsa_pool_qkv — the cube mean-pool of vsa_pool applied to q, k and v in one
+ * launch, read straight from the token layout (no tiled copy).  Each mean is
+ * summed in the same float32 order as vsa_pool on the tiled tensor, so the two
+ * give identical bits.  Same section, part 1.
+ *   q, k, v           [B, N, H, D] bf16 token layout (read).
+ *   qbar, kbar, vbar  [B, H, C, D] float32 (written).
+ */
+vsa_status vsa_pool_qkv(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                        float* qbar, float* kbar, float* vbar, vsa_stream_t stream);
+
+/*
+ * vsa_fine_fused — the fine stage (part 2) and the gated merge (part 3) in
+ * one kernel, on the token layout: key/value cubes are gathered from q, k, v
+ * by the copy engine (padded positions read as zeros, so no vsa_tile pass),
+ * and each query row's result g_coarse * o_coarse[cube] + g_fine * O_fine is
+ * written to its token's row of `out` (no vsa_combine / vsa_untile pass).
+ * O_fine is not rounded to bf16 before the merge.
+ * With idx == NULL every key is attended (dense attention, the Wan2.1
+ * article's section 4.2): the kernel then walks blocks of 64 consecutive real
+ * tokens instead of cubes, so no padded position is computed at all.
+ *   q, k, v    [B, N, H, D] bf16 token layout (read).
+ *   idx, k, order, scale   as in vsa_fine (idx NULL: dense; order then unused).
+ *   o_coarse   [B, H, C, D] float32, or NULL (no coarse term; g_coarse ignored).
+ *   g_coarse, g_fine  [B, N, H] bf16 or NULL (g_coarse = 0, g_fine = 1).
+ *   out        [B, N, H, D] bf16 (written at every real token).
+ */
+vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
+                          const int32_t* idx, int32_t topk, const int32_t* order, float scale,
+                          const float* o_coarse, const vsa_bf16* g_coarse, const vsa_bf16* g_fine,
+                          vsa_bf16* out, vsa_stream_t stream);
+
 /* Bytes of device workspace vsa_forward needs for this shape and top-k
  * (0 for a malformed shape). */
 size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
 
 /*
- * vsa_forward — the whole attention call on one stream:
- *   tile(q,k,v) -> pool -> coarse -> topk -> group -> fine -> combine -> untile
- * (the grouping step is skipped when C > 4096).
- * When topk == C and both gates are NULL the call is dense attention and runs
- * tile -> fine (all cubes) -> untile.
+ * vsa_forward — the whole attention call on one stream, as five launches:
+ *   vsa_pool_qkv -> vsa_coarse -> vsa_topk -> vsa_group -> vsa_fine_fused
+ * (the grouping step is skipped when C > 4096).  The result equals
+ *   tile -> pool -> coarse -> topk -> group -> fine -> combine -> untile
+ * up to the bf16 rounding of O_fine that the staged path makes.
+ * When topk == C every cube is selected and the fine stage is dense attention
+ * over the real tokens: vsa_fine_fused with idx == NULL, preceded by
+ * vsa_pool_qkv -> vsa_coarse only when g_coarse is given.  With both gates
+ * NULL that is dense attention in one launch.
  *   q, k, v      [B, N, H, D] bf16 token layout (read).
  *   g_coarse, g_fine  [B, N, H] bf16 or NULL (see vsa_combine).
  *   workspace    device buffer of at least vsa_workspace_bytes(shape, topk),
- *                256-byte aligned; its contents on return are unspecified.
+ *                256-byte aligned (that size covers both gates; a call without
+ *                g_coarse at topk == C needs only 256 bytes); its contents on
+ *                return are unspecified.
  *   out          [B, N, H, D] bf16 (written).
  */
 vsa_status vsa_forward(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,

@@ -109,13 +109,16 @@ def test_workspace_checks():
 
 
 def test_workspace_size_480p_matches_layout():
-    # tiled q,k,v,o_fine (4 x 39936*40*128*2 B) + pooled q,k,v,o_coarse (4 x 624*40*128*4 B)
-    # + scores (624*624*40*4 B) + idx (624*40*32*4 B) + order (624*40*4 B), each rounded up to 256 B
+    # Q, K, V are read in place, so the workspace holds only the pooled q,k,v and o_coarse
+    # (4 x 624*40*128*4 B), the scores (624*624*40*4 B), idx (624*40*32*4 B) and the work order
+    # (624*40*4 B), each rounded up to 256 B
     s = vsa.Shape(1, 40, 128, (21, 30, 52)).c()
     up = lambda n: (n + 255) // 256 * 256
-    expect = 4 * up(39936 * 40 * 128 * 2) + 4 * up(624 * 40 * 128 * 4) + up(624 * 624 * 40 * 4) + up(624 * 40 * 32 * 4) \
-        + up(624 * 40 * 4)
+    expect = 4 * up(624 * 40 * 128 * 4) + up(624 * 624 * 40 * 4) + up(624 * 40 * 32 * 4) + up(624 * 40 * 4)
     assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 32) == expect
+    # every cube selected: dense attention; the coarse buffers are for a coarse gate only
+    assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 624) == 4 * up(624 * 40 * 128 * 4) + \
+        up(624 * 624 * 40 * 4)
 
 
 def test_probe_limit_checked_before_device():

@@ -1,7 +1,7 @@
 """Parity at the full Wan 480p / 720p sizes, in the launch configuration the
 benchmark times (the whole call on one stream), checked on sampled heads and
 query cubes that the oracle computes one by one, plus properties that hold at
-any size (tile round trip, whole call == the stages run one by one)."""
+any size (tile round trip, whole call == the per-step path up to rounding)."""
 import math
 
 import numpy as np
@@ -45,7 +45,17 @@ def run(request):
         r["scores"] = scores.cpu()
         r["oc"] = oc.cpu()
         r["idx"] = idx.cpu().numpy()
-    r["stage_equal"] = torch.equal(stage_out, r["out"])
+    fused, staged = r["out"].float(), stage_out.float()
+    if dense:
+        # different block order (64 consecutive real tokens instead of cubes): a different
+        # but equally valid rounding order, so the oracle tolerance applies
+        err = fused - staged
+        r["stage_close"] = bool(err.abs().max() <= 2e-2) and bool(err.norm() <= 5e-3 * staged.norm())
+    else:
+        # identical selections and steps; only the staged path's bf16 rounding of O_f differs
+        ulp = lambda t: torch.exp2(torch.floor(torch.log2(t.abs().clamp_min(2.0 ** -100))) - 7)
+        of_tok = vsa.untile(o, s).float()
+        r["stage_close"] = bool(((fused - staged).abs() <= ulp(staged) + 0.5 * ulp(of_tok) + 1e-6).all())
     r["qt_rows"] = qt
     r["o_fine"] = o.cpu()
     r["lse"] = lse.cpu()
@@ -68,7 +78,7 @@ def _sample_cubes(C, n=12, seed=0):
 
 def test_roundtrip_and_stage_equivalence(run):
     assert run["rt_ok"]
-    assert run["stage_equal"], "vsa_forward differs from the same kernels run stage by stage"
+    assert run["stage_close"], "vsa_forward differs from the per-step path beyond rounding"
 
 
 def test_tile_sampled_rows(run):

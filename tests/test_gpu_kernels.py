@@ -138,10 +138,48 @@ def test_dense_matches_oracle(case):
     g_lse = from_dev(lse)
     g_lse_tok = O.untile(g_lse[..., None], w.grid)[..., 0]
     assert np.abs(g_lse_tok - r_lse).max() <= LSE_ABS
-    # the whole call in dense mode (top-k = C, no gates) gives the same bits
+    # the whole call with top-k = C and no gates: dense attention over blocks of
+    # 64 consecutive real tokens read in place (no tiling, no padding)
     npad, C = vsa.shape_info(s)
-    out2 = vsa.forward(dev["q"], dev["k"], dev["v"], s, C)
-    assert np.array_equal(bf16_bits(out2), bf16_bits(vsa.untile(o, s)))
+    out2 = from_dev(vsa.forward(dev["q"], dev["k"], dev["v"], s, C))
+    for b in range(w.batch):
+        for h in range(w.heads):
+            check_close(out2[b, :, h], r_out[b, :, h], f"dense forward[b={b},h={h}]")
+
+
+def test_forward_matches_the_stages_run_one_by_one(case):
+    """vsa_forward (pool read in place, cube gathers, merge in the fine epilogue) against
+    tile -> pool -> coarse -> top-k -> group -> fine -> combine -> untile through the
+    per-step entry points.  The selections are identical (the same float32 pooling order);
+    the outputs differ only by the bf16 rounding of O_f that the staged path makes."""
+    w, _, dev, _ = case
+    s = _shape(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    gc, gf = dev["g_coarse"], dev["g_fine"]
+    qt, kt, vt = (vsa.tile(dev[n], s) for n in ("q", "k", "v"))
+    bars = [vsa.pool(t, s) for t in (qt, kt, vt)]
+    scores, oc = vsa.coarse(*bars, s, scale)
+    idx = vsa.topk(scores, s, w.topk)
+    order = vsa.group(scores, s)
+    of, _ = vsa.fine(qt, kt, vt, s, idx, scale, order=order)
+    staged = from_dev(vsa.untile(vsa.combine(oc, of, s, gc, gf), s))
+    fused = from_dev(vsa.forward(dev["q"], dev["k"], dev["v"], s, w.topk, scale, gc, gf))
+    assert np.array_equal(vsa.topk(vsa.coarse(*[vsa.pool(t, s) for t in (qt, kt, vt)], s, scale)[0], s,
+                                   w.topk).cpu().numpy(), idx.cpu().numpy())
+    _, C = vsa.shape_info(s)
+    if w.topk == C:
+        # every cube selected: the forward call attends over blocks of consecutive real tokens,
+        # a different but equally valid summation order, so the oracle tolerance applies
+        for b in range(w.batch):
+            for h in range(w.heads):
+                check_close(fused[b, :, h], staged[b, :, h], f"forward vs stages[b={b},h={h}]")
+        return
+    # apart by at most the staged path's extra rounding of O_f (half a bf16 unit of O_f, times
+    # g_f <= 1) plus one unit of the result (the two final roundings)
+    ulp = lambda a: 2.0 ** (np.floor(np.log2(np.maximum(np.abs(a), 2.0 ** -100))) - 7)
+    of_tok = from_dev(vsa.untile(of, s))
+    bound = ulp(staged) + 0.5 * ulp(of_tok) + 1e-6
+    assert np.all(np.abs(fused - staged) <= bound), "fused forward differs from the staged path beyond rounding"
 
 
 def _compare_call(w, dev, f64, k, scale, gates=True):
@@ -356,3 +394,60 @@ def test_group_keys_follow_top_scores():
     expect = sorted(range(C), key=lambda i: (top[i, 0], top[i, 1], top[i, 2], i))
     got = vsa.group(torch.from_numpy(sc).cuda(), s).cpu().numpy()[0, 0]
     assert got.tolist() == expect
+
+
+# ---------------------------------------------------------------- fused pipeline entry points
+def test_pool_qkv_bit_identical_to_pool_of_tiles(case):
+    """Pooling straight from the token layout sums in the same order as pooling the tiled copy."""
+    w, _, dev, _ = case
+    s = _shape(w)
+    bars = vsa.pool_qkv(dev["q"], dev["k"], dev["v"], s)
+    for name, got in zip(("q", "k", "v"), bars):
+        assert torch.equal(got, vsa.pool(vsa.tile(dev[name], s), s)), name
+
+
+def test_fine_fused_sparse_matches_oracle(case):
+    """Cube gathers from the token layout + merge in the epilogue, on the oracle's selection."""
+    w, _, dev, f64 = case
+    s = _shape(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, w.topk, scale, f64["g_coarse"], f64["g_fine"])
+    idx = torch.from_numpy(ora["idx"]).cuda()
+    # fine output alone (no coarse term, g_fine = 1), written in token layout
+    got = from_dev(vsa.fine_fused(dev["q"], dev["k"], dev["v"], s, idx, scale))
+    ref = O.untile(ora["o_fine"], w.grid)
+    for b in range(w.batch):
+        for h in range(w.heads):
+            check_close(got[b, :, h], ref[b, :, h], f"fine_fused[b={b},h={h}]")
+    # with the oracle's coarse output and both gates: the whole merged result
+    oc = torch.from_numpy(ora["o_coarse"].astype(np.float32)).cuda()
+    got = from_dev(vsa.fine_fused(dev["q"], dev["k"], dev["v"], s, idx, scale, None, oc, dev["g_coarse"],
+                                  dev["g_fine"]))
+    for b in range(w.batch):
+        for h in range(w.heads):
+            check_close(got[b, :, h], ora["out"][b, :, h], f"fine_fused merged[b={b},h={h}]")
+
+
+def test_fine_fused_dense_matches_oracle(case):
+    """Dense attention over blocks of 64 consecutive real tokens (a ragged last block)."""
+    w, _, dev, f64 = case
+    s = _shape(w)
+    r_out, _ = O.dense(f64["q"], f64["k"], f64["v"], w.grid)
+    got = from_dev(vsa.fine_fused(dev["q"], dev["k"], dev["v"], s, None))
+    for b in range(w.batch):
+        for h in range(w.heads):
+            check_close(got[b, :, h], r_out[b, :, h], f"dense fused[b={b},h={h}]")
+
+
+def test_fine_fused_writes_only_real_tokens_and_ignores_order_for_dense():
+    w = synth.WORKLOADS["padded_7x15x16"]
+    x = synth.make_inputs(w)
+    d = {k: to_dev(v) for k, v in x.items()}
+    s = _shape(w)
+    sentinel = torch.full_like(d["q"], float("nan"))
+    out = vsa.fine_fused(d["q"], d["k"], d["v"], s, None, out=sentinel.clone())
+    assert not torch.isnan(out).any()          # every real token's row was written
+    npad, C = vsa.shape_info(s)
+    rev = torch.arange(C - 1, -1, -1, dtype=torch.int32, device="cuda").expand(w.batch, w.heads, C).contiguous()
+    out2 = vsa.fine_fused(d["q"], d["k"], d["v"], s, None, order=rev)
+    assert torch.equal(out, out2)
