@@ -290,7 +290,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     dense_ms_max = reduce_max(dense_ms, world)
 
     # ---- per-stage breakdown: the launches of vsa_forward, one by one through the entry points
-    names = ["pool", "coarse", "topk", "group", "fine"]
+    names = ["pool", "coarse", "topk_order", "fine"]
     acc = {n: [] for n in names}
     acc["fine_dense"] = []
     for it in range(args.warmup + args.steps):
@@ -300,19 +300,17 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         e[1].record(stream)
         scores, oc = vsa.coarse(*bars, s, scale)
         e[2].record(stream)
-        idx = vsa.topk(scores, s, w.topk)
+        idx, order = vsa.topk_order(scores, s, w.topk)
         e[3].record(stream)
-        order = vsa.group(scores, s)
-        e[4].record(stream)
         vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, order, oc, d["g_coarse"], d["g_fine"], out=out)
-        e[5].record(stream)
+        e[4].record(stream)
         vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out_d)
-        e[6].record(stream)
+        e[5].record(stream)
         torch.cuda.synchronize()
         if it >= args.warmup:
             for j, n in enumerate(names):
                 acc[n].append(e[j].elapsed_time(e[j + 1]))
-            acc["fine_dense"].append(e[5].elapsed_time(e[6]))
+            acc["fine_dense"].append(e[4].elapsed_time(e[5]))
         del bars, scores, oc, idx, order
     stage_ms = {n: round(statistics.mean(v), 4) for n, v in acc.items()}
 
@@ -378,7 +376,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                      "per_launch": "4*B*H*Npad*k*64*D executed flops (64x64 cube tiles of the k selected cubes)"},
         "e2e": {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "vsa_forward_host (pinned host q/k/v/gates in, host out)"},
-        "gpu_launches": 6 * args.steps,   # VSA: pool, coarse, top-k, group, fine; dense: fine
+        "gpu_launches": 8 * args.steps,   # VSA: pool, coarse (2), top-k, order sort, fine; dense: fine
         "clocks": clocks,
         "cpu_baseline": cpu,
         "context": {"pages_dense_call_ms_b200": 17.0, "pages_vsa_kernel_ms_b200_k78": 4.719,

@@ -163,6 +163,18 @@ def combine(o_coarse: torch.Tensor, o_fine: torch.Tensor, shape: Shape, g_coarse
     return out
 
 
+def topk_order(scores: torch.Tensor, shape: Shape, k: int) -> Tuple[torch.Tensor, torch.Tensor]:
+    """topk() and group() from one pass over the scores (C <= 2048): (idx [B,H,C,k], order [B,H,C])."""
+    _, c = shape_info(shape)
+    idx = torch.empty((shape.batch, shape.heads, c, k), dtype=torch.int32, device=scores.device)
+    order = torch.empty((shape.batch, shape.heads, c), dtype=torch.int32, device=scores.device)
+    sig = torch.empty((shape.batch, shape.heads, c), dtype=torch.int64, device=scores.device)
+    _check(_L.vsa_topk_order(ctypes.byref(shape.c()), _ptr(scores, torch.float32, "scores"), k,
+                             _ptr(idx, torch.int32, "idx"), _ptr(order, torch.int32, "order"),
+                             _ptr(sig, torch.int64, "sig_scratch"), _stream()))
+    return idx, order
+
+
 def pool_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
              shape: Shape) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Cube means of q, k, v ([B,N,H,D] token layout) in one launch: three [B,H,C,D] float32 tensors."""

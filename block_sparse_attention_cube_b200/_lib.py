@@ -44,6 +44,7 @@ SIGNATURES = {
     "vsa_fine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _I32, _P, _F32, _P, _P, _P]),
     "vsa_combine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P]),
     "vsa_pool_qkv": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P]),
+    "vsa_topk_order": (ctypes.c_int, [_SP, _P, _I32, _P, _P, _P, _P]),
     "vsa_fine_fused": (ctypes.c_int, [_SP, _P, _P, _P, _P, _I32, _P, _F32, _P, _P, _P, _P, _P]),
     "vsa_workspace_bytes": (_SZ, [_SP, _I32]),
     "vsa_forward": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _I32, _F32, _P, _SZ, _P, _P]),

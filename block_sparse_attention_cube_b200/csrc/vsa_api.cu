@@ -121,7 +121,7 @@ size_t order_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C 
 constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Workspace of vsa_forward: qbar | kbar | vbar | o_coarse | scores | idx | order.
+// Workspace of vsa_forward: qbar | kbar | vbar | o_coarse | scores | idx | order | sig.
 // Q, K and V are read in the caller's [B, N, H, D] layout (the fine stage
 // gathers cubes with TMA), so no tiled copies are kept.  With every cube
 // selected the fine stage is dense attention and needs none of it; the
@@ -130,6 +130,7 @@ struct Carve {
     float *qbar, *kbar, *vbar, *oc, *scores;
     int32_t* idx;
     int32_t* order;
+    uint64_t* sig;   // work-order signatures, when top-k computes them (C <= kTopkRegMaxC)
     size_t bytes;
 };
 
@@ -153,6 +154,7 @@ Carve carve(const Dims& d, int k, bool coarse_gate, void* ws) {
     if (sparse) {
         c.idx = reinterpret_cast<int32_t*>(take(idx_bytes(d, k)));
         c.order = reinterpret_cast<int32_t*>(take(order_bytes(d)));
+        if (d.C <= kTopkRegMaxC) c.sig = reinterpret_cast<uint64_t*>(take(2 * order_bytes(d)));
     }
     c.bytes = off > kAlign ? off : kAlign;
     return c;
@@ -223,10 +225,17 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
     }
     const int32_t* order = nullptr;
     if (sparse) {
-        VSA_CUDA(launch_topk(d, c.scores, topk, c.idx, s), "topk launch");
-        if (d.C <= kGroupMaxC) {
-            VSA_CUDA(launch_group(d, c.scores, c.order, s), "group launch");
+        if (d.C <= kTopkRegMaxC && d.C <= kGroupMaxC) {
+            // one pass over the scores gives the selection and the work-order keys
+            VSA_CUDA(launch_topk_sig(d, c.scores, topk, c.idx, c.sig, s), "topk launch");
+            VSA_CUDA(launch_group_sort(d, c.sig, c.order, s), "group launch");
             order = c.order;
+        } else {
+            VSA_CUDA(launch_topk(d, c.scores, topk, c.idx, s), "topk launch");
+            if (d.C <= kGroupMaxC) {
+                VSA_CUDA(launch_group(d, c.scores, c.order, s), "group launch");
+                order = c.order;
+            }
         }
     }
     return run_fine_fused(d, q, k, v, sparse ? c.idx : nullptr, topk, order, scale, gc ? c.oc : nullptr, gc, gf,
@@ -410,6 +419,26 @@ vsa_status vsa_combine(const vsa_shape* shape, const float* o_coarse, const vsa_
                            {{o_tiled, tb, "o_tiled"}}));
     VSA_TRY(check_device());
     VSA_CUDA(launch_combine(d, o_coarse, o_fine, g_coarse, g_fine, o_tiled, as_stream(stream)), "combine launch");
+    return VSA_OK;
+}
+
+vsa_status vsa_topk_order(const vsa_shape* shape, const float* scores, int32_t k, int32_t* idx, int32_t* order,
+                          uint64_t* sig_scratch, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(check_k(d, k));
+    VSA_TRY(need_ptr(scores, "scores"));
+    VSA_TRY(need_ptr(idx, "idx"));
+    VSA_TRY(need_ptr(order, "order"));
+    VSA_TRY(need_ptr(sig_scratch, "sig_scratch"));
+    if (d.C > kTopkRegMaxC || d.C > kGroupMaxC)
+        return fail(VSA_ERR_UNSUPPORTED, "vsa_topk_order supports at most %d cubes (got %d)", kTopkRegMaxC, d.C);
+    VSA_TRY(check_disjoint({{scores, score_bytes(d), "scores"}},
+                           {{idx, idx_bytes(d, k), "idx"}, {order, order_bytes(d), "order"},
+                            {sig_scratch, 2 * order_bytes(d), "sig_scratch"}}));
+    VSA_TRY(check_device());
+    VSA_CUDA(launch_topk_sig(d, scores, k, idx, sig_scratch, as_stream(stream)), "topk launch");
+    VSA_CUDA(launch_group_sort(d, sig_scratch, order, as_stream(stream)), "group launch");
     return VSA_OK;
 }
 

@@ -149,6 +149,36 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+__device__ __forceinline__ void top3_insert(uint64_t (&t)[3], uint64_t v) {
+    if (v > t[2]) {
+        if (v > t[1]) {
+            t[2] = t[1];
+            if (v > t[0]) {
+                t[1] = t[0];
+                t[0] = v;
+            } else {
+                t[1] = v;
+            }
+        } else {
+            t[2] = v;
+        }
+    }
+}
+
+// Work-order key of query cube i from its three best key cubes t[0..2]
+// (score order, lower index first; 0xFFFF for an absent entry): the three
+// cube indices, then i, so sorting the keys groups cubes with similar
+// selections and is a permutation.
+__device__ __forceinline__ uint64_t group_signature(const uint64_t (&t)[3], uint32_t i) {
+    uint64_t sg = static_cast<uint64_t>(i);
+#pragma unroll
+    for (int e = 0; e < 3; ++e) {
+        const uint64_t c = t[e] ? (0xFFFFFFFFu - static_cast<uint32_t>(t[e] & 0xFFFFFFFFu)) : 0xFFFFu;
+        sg |= (c & 0xFFFFu) << (48 - 16 * e);
+    }
+    return sg;
+}
+
 // One warp per (b, h, query cube) row.  The k-th largest key T is built bit
 // by bit from the top (largest T with at least k keys >= T); the row is then
 // scanned in index order, keeping every key > T and the lowest-index keys
@@ -199,6 +229,90 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(int64_t rows, int C, int
     }
 }
 
+// Top-k with the row held in registers (KPL keys per lane, key j in lane
+// j % 32, slot j / 32), for C <= 32 * KPL.  The k-th largest key T is built
+// bit by bit from the top with warp sums (redux) of per-lane counts; the row
+// is then scanned in index order exactly as topk_kernel does, so both give
+// the same selection.  When `sig` is non-null the row's work-order signature
+// (its three best key cubes, see group_kernel) is written as well, from the
+// same registers.
+template <int KPL>
+__global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C, int k, const float* __restrict__ scores,
+                                                            int32_t* __restrict__ idx, uint64_t* __restrict__ sig) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
+    for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + warp; row < rows; row += warps) {
+        const float* s = scores + row * C;
+        uint32_t key[KPL];
+#pragma unroll
+        for (int i = 0; i < KPL; ++i) {
+            const int j = lane + 32 * i;
+            key[i] = j < C ? order_key(__ldcs(s + j)) : 0u;   // 0 ranks below every real score
+        }
+        // T lies between a lower bound and the largest key, so it shares their
+        // leading bits: only the bits below the highest differing one are searched.
+        // Lower bound: the smallest lane maximum when k <= 32 (at least 32 keys
+        // reach it), else the smallest key.
+        uint32_t lane_max = 0u, lane_min = 0xFFFFFFFFu;
+#pragma unroll
+        for (int i = 0; i < KPL; ++i) {
+            lane_max = max(lane_max, key[i]);
+            if (lane + 32 * i < C) lane_min = min(lane_min, key[i]);
+        }
+        const uint32_t hi = __reduce_max_sync(0xffffffffu, lane_max);
+        const uint32_t lo = k <= 32 ? __reduce_min_sync(0xffffffffu, lane_max) : __reduce_min_sync(0xffffffffu, lane_min);
+        const uint32_t diff = hi ^ lo;
+        const int top = diff ? 31 - __clz(diff) : -1;          // highest differing bit
+        uint32_t T = top < 0 ? hi : (top >= 31 ? 0u : (hi & ~((2u << top) - 1u)));
+#pragma unroll 1
+        for (int bit = top; bit >= 0; --bit) {
+            const uint32_t cand = T | (1u << bit);
+            uint32_t cnt = 0;
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) cnt += key[i] >= cand ? 1u : 0u;
+            if (static_cast<int>(__reduce_add_sync(0xffffffffu, cnt)) >= k) T = cand;
+        }
+        uint32_t gt = 0;
+#pragma unroll
+        for (int i = 0; i < KPL; ++i) gt += key[i] > T ? 1u : 0u;
+        const int need_eq = k - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+        int out = 0, eq_seen = 0;
+        int32_t* dst = idx + row * k;
+#pragma unroll
+        for (int i = 0; i < KPL; ++i) {
+            const int j = lane + 32 * i;
+            const bool valid = j < C;
+            const bool is_gt = valid && key[i] > T;
+            const bool is_eq = valid && key[i] == T;
+            const uint32_t eq_mask = __ballot_sync(0xffffffffu, is_eq);
+            const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
+            const bool take = is_gt || (is_eq && eq_rank < need_eq);
+            const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
+            if (take) dst[out + __popc(take_mask & lt_mask)] = j;
+            out += __popc(take_mask);
+            eq_seen += __popc(eq_mask);
+        }
+        if (sig != nullptr) {
+            uint64_t t[3] = {0ull, 0ull, 0ull};
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) {
+                const int j = lane + 32 * i;
+                if (j < C) top3_insert(t, (static_cast<uint64_t>(key[i]) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(j)));
+            }
+#pragma unroll
+            for (int off = 16; off; off >>= 1) {
+                uint64_t o[3];
+#pragma unroll
+                for (int e = 0; e < 3; ++e) o[e] = __shfl_xor_sync(0xffffffffu, t[e], off);
+#pragma unroll
+                for (int e = 0; e < 3; ++e) top3_insert(t, o[e]);
+            }
+            if (lane == 0) sig[row] = group_signature(t, static_cast<uint32_t>(row % C));
+        }
+    }
+}
+
 // Work-order for the fine stage: per (b, h), the query cubes sorted by the
 // indices of their three highest-scoring key cubes (ties to the lower index),
 // so that consecutive cubes, which the fine kernel processes as a group of
@@ -207,20 +321,29 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(int64_t rows, int C, int
 // output.  One block per (b, h); C <= kGroupMaxC.
 constexpr int kGroupThreads = 512;
 
-__device__ __forceinline__ void top3_insert(uint64_t (&t)[3], uint64_t v) {
-    if (v > t[2]) {
-        if (v > t[1]) {
-            t[2] = t[1];
-            if (v > t[0]) {
-                t[1] = t[0];
-                t[0] = v;
-            } else {
-                t[1] = v;
+// Sorts keys[0, C) ascending (keys[C, cpow2) are padding set here) with a
+// bitonic network over the block and writes each key's low 16 bits (the
+// query cube) to order[0, C).
+__device__ __forceinline__ void sort_and_write(uint64_t* keys, int C, int cpow2, int32_t* __restrict__ order) {
+    for (int i = C + threadIdx.x; i < cpow2; i += kGroupThreads) keys[i] = ~0ull;
+    __syncthreads();
+    for (int k2 = 2; k2 <= cpow2; k2 <<= 1) {
+        for (int j = k2 >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < cpow2; i += kGroupThreads) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const uint64_t a = keys[i], b = keys[ixj];
+                    const bool up = (i & k2) == 0;
+                    if ((a > b) == up) {
+                        keys[i] = b;
+                        keys[ixj] = a;
+                    }
+                }
             }
-        } else {
-            t[2] = v;
+            __syncthreads();
         }
     }
+    for (int r = threadIdx.x; r < C; r += kGroupThreads) order[r] = static_cast<int32_t>(keys[r] & 0xFFFFu);
 }
 
 __global__ void __launch_bounds__(kGroupThreads) group_kernel(int C, int cpow2, const float* __restrict__ scores,
@@ -242,36 +365,19 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(int C, int cpow2, 
 #pragma unroll
             for (int e = 0; e < 3; ++e) top3_insert(t, o[e]);
         }
-        if (lane == 0) {
-            uint64_t sig = static_cast<uint64_t>(i);
-#pragma unroll
-            for (int e = 0; e < 3; ++e) {
-                const uint64_t c = t[e] ? (0xFFFFFFFFu - static_cast<uint32_t>(t[e] & 0xFFFFFFFFu)) : 0xFFFFu;
-                sig |= (c & 0xFFFFu) << (48 - 16 * e);
-            }
-            keys[i] = sig;
-        }
+        if (lane == 0) keys[i] = group_signature(t, static_cast<uint32_t>(i));
     }
-    for (int i = C + threadIdx.x; i < cpow2; i += kGroupThreads) keys[i] = ~0ull;
-    __syncthreads();
-    for (int k2 = 2; k2 <= cpow2; k2 <<= 1) {
-        for (int j = k2 >> 1; j > 0; j >>= 1) {
-            for (int i = threadIdx.x; i < cpow2; i += kGroupThreads) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const uint64_t a = keys[i], b = keys[ixj];
-                    const bool up = (i & k2) == 0;
-                    if ((a > b) == up) {
-                        keys[i] = b;
-                        keys[ixj] = a;
-                    }
-                }
-            }
-            __syncthreads();
-        }
-    }
-    for (int r = threadIdx.x; r < C; r += kGroupThreads)
-        order[static_cast<int64_t>(bh) * C + r] = static_cast<int32_t>(keys[r] & 0xFFFFu);
+    sort_and_write(keys, C, cpow2, order + static_cast<int64_t>(bh) * C);
+}
+
+// The work order from signatures already computed (topk_reg_kernel): one
+// block per (b, h) sorts them.
+__global__ void __launch_bounds__(kGroupThreads) group_sort_kernel(int C, int cpow2, const uint64_t* __restrict__ sig,
+                                                                   int32_t* __restrict__ order) {
+    __shared__ uint64_t keys[kGroupMaxC];
+    const int bh = blockIdx.x;
+    for (int i = threadIdx.x; i < C; i += kGroupThreads) keys[i] = sig[static_cast<int64_t>(bh) * C + i];
+    sort_and_write(keys, C, cpow2, order + static_cast<int64_t>(bh) * C);
 }
 
 }  // namespace
@@ -305,8 +411,40 @@ int topk_warps_per_block(int C) {
     return w;
 }
 
+namespace {
+
+// Register-resident selection for C <= 2048 (a warp holds the row, KPL keys per lane).
+template <int KPL>
+cudaError_t launch_topk_reg(int64_t rows, int C, int k, const float* scores, int32_t* idx, uint64_t* sig,
+                            cudaStream_t s) {
+    const int64_t blocks_needed = (rows + kThreads / 32 - 1) / (kThreads / 32);
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
+    topk_reg_kernel<KPL><<<grid, kThreads, 0, s>>>(rows, C, k, scores, idx, sig);
+    return cudaGetLastError();
+}
+
+cudaError_t topk_reg_dispatch(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig,
+                              cudaStream_t s) {
+    const int64_t rows = static_cast<int64_t>(d.B) * d.H * d.C;
+    const int kpl = (d.C + 31) / 32;
+    if (kpl <= 4) return launch_topk_reg<4>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 8) return launch_topk_reg<8>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 12) return launch_topk_reg<12>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 16) return launch_topk_reg<16>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 20) return launch_topk_reg<20>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 24) return launch_topk_reg<24>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 32) return launch_topk_reg<32>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 40) return launch_topk_reg<40>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 48) return launch_topk_reg<48>(rows, d.C, k, scores, idx, sig, s);
+    return launch_topk_reg<64>(rows, d.C, k, scores, idx, sig, s);
+}
+
+}  // namespace
+
 cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx, cudaStream_t s) {
     if (d.C > kTopkMaxC) return cudaErrorInvalidValue;
+    if (d.C <= kTopkRegMaxC) return topk_reg_dispatch(d, scores, k, idx, nullptr, s);
     const int64_t rows = static_cast<int64_t>(d.B) * d.H * d.C;
     const int wpb = topk_warps_per_block(d.C);
     const size_t smem = static_cast<size_t>(wpb) * d.C * 4;
@@ -319,6 +457,19 @@ cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx,
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
     topk_kernel<<<grid, wpb * 32, smem, s>>>(rows, d.C, k, scores, idx);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s) {
+    if (d.C > kTopkRegMaxC) return cudaErrorInvalidValue;
+    return topk_reg_dispatch(d, scores, k, idx, sig, s);
+}
+
+cudaError_t launch_group_sort(const Dims& d, const uint64_t* sig, int32_t* order, cudaStream_t s) {
+    if (d.C > kGroupMaxC) return cudaErrorInvalidValue;
+    int cpow2 = 1;
+    while (cpow2 < d.C) cpow2 <<= 1;
+    group_sort_kernel<<<d.B * d.H, kGroupThreads, 0, s>>>(d.C, cpow2, sig, order);
     return cudaGetLastError();
 }
 

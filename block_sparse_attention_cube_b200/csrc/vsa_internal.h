@@ -50,9 +50,16 @@ cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, c
                           float* scores, float* o_coarse, cudaStream_t s);
 cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx, cudaStream_t s);
 
+// Largest C whose rows the selection holds in registers; up to it, top-k can
+// also emit each row's work-order signature (uint64 [B, H, C]) in the same
+// pass, and launch_group_sort turns those into the order launch_group gives.
+constexpr int kTopkRegMaxC = 2048;
+cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s);
+
 // Work order of the fine stage from the coarse scores (C <= kGroupMaxC).
 constexpr int kGroupMaxC = 4096;
 cudaError_t launch_group(const Dims& d, const float* scores, int32_t* order, cudaStream_t s);
+cudaError_t launch_group_sort(const Dims& d, const uint64_t* sig, int32_t* order, cudaStream_t s);
 
 // Fine stage.  Modes:
 //  kFineTiled       - q/k/v tiled [B, H, Npad, D]; out = tiled O_f (+ lse when non-null);

@@ -145,62 +145,63 @@ __global__ void __launch_bounds__(kBlock) pool_kernel(Dims d, PoolIO io) {
 }
 
 // The same pool read straight from the projection layout [B, N, H, D], so a
-// forward call needs no tiled copy.  Tasks run (tensor, b, cube, head) with
-// the head fastest: the warps of a block read neighbouring heads of the same
-// tokens, 256 contiguous bytes per row.  Each output channel is summed in the
-// same order as pool_kernel (per lane group in offset order, then the same
-// shuffle tree), so both give identical float32 means.
+// forward call needs no tiled copy.  A token's H*D channels are contiguous,
+// so a block of kPoolThreads threads owns one (tensor, b, cube) and a range
+// of 16-byte channel chunks, one chunk per thread, and walks the cube's real
+// tokens: every token row it reads is kPoolThreads * 16 contiguous bytes.
+// Each channel is summed in the order of pool_kernel: R = 256 / D partial
+// sums over the offsets o with o % R == r, each in offset order, combined as
+// pool_kernel's shuffle tree does; both kernels give identical float32 means.
+constexpr int kPoolThreads = 128;
+
 template <int D>
-__global__ void __launch_bounds__(kBlock) pool_tokens_kernel(Dims d, PoolIO io) {
-    constexpr int LPR = D / 8;          // lanes per row
-    constexpr int RPI = 32 / LPR;       // rows per warp iteration
-    const int lane = threadIdx.x & 31;
-    const int sub = lane / LPR, j = lane % LPR;
-    const int64_t per_tensor = static_cast<int64_t>(d.B) * d.H * d.C;
-    const int64_t total = per_tensor * io.count;
-    const int64_t warps = static_cast<int64_t>(gridDim.x) * (kBlock / 32);
-    for (int64_t task = static_cast<int64_t>(blockIdx.x) * (kBlock / 32) + threadIdx.x / 32; task < total;
-         task += warps) {
-        const int tensor = static_cast<int>(task / per_tensor);
-        const int64_t r = task - tensor * per_tensor;
-        const int h = static_cast<int>(r % d.H);
-        const int64_t bc = r / d.H;
-        const int c = static_cast<int>(bc % d.C);
-        const int b = static_cast<int>(bc / d.C);
-        const int ct = c / (d.Cx * d.Cy), cx = (c / d.Cy) % d.Cx, cy = c % d.Cy;
-        const uint4* src = reinterpret_cast<const uint4*>(io.src[tensor]);
-        const int nt = min(kCube, d.T - ct * kCube);
-        const int nx = min(kCube, d.X - cx * kCube);
-        const int ny = min(kCube, d.Y - cy * kCube);
-        float acc[8];
+__global__ void __launch_bounds__(kPoolThreads) pool_tokens_kernel(Dims d, PoolIO io) {
+    constexpr int CH = D / 8;            // 16-byte chunks per head
+    constexpr int R = 256 / D;           // partial sums per channel (lane groups of pool_kernel)
+    const int q = blockIdx.y * kPoolThreads + threadIdx.x;   // chunk of the token row
+    if (q >= d.H * CH) return;
+    const int64_t bc = blockIdx.x;       // (tensor * B + b) * C + c
+    const int c = static_cast<int>(bc % d.C);
+    const int tb = static_cast<int>(bc / d.C);
+    const int tensor = tb / d.B, b = tb - tensor * d.B;
+    const int h = q / CH, j = q - h * CH;
+    const int ct = c / (d.Cx * d.Cy), cx = (c / d.Cy) % d.Cx, cy = c % d.Cy;
+    const int nt = min(kCube, d.T - ct * kCube);
+    const int nx = min(kCube, d.X - cx * kCube);
+    const int ny = min(kCube, d.Y - cy * kCube);
+    const int64_t row = static_cast<int64_t>(d.H) * CH;   // 16-byte chunks per token
+    const uint4* src = reinterpret_cast<const uint4*>(io.src[tensor]) + static_cast<int64_t>(b) * d.N * row + q;
+    const int64_t base_n = (static_cast<int64_t>(ct) * kCube * d.X + cx * kCube) * d.Y + cy * kCube;
+    float acc[R][8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll 4
-        for (int o = sub; o < kCubeTokens; o += RPI) {
-            const int ot = o >> 4, ox = (o >> 2) & 3, oy = o & 3;
-            if (ot >= nt || ox >= nx || oy >= ny) continue;
-            const int64_t n = (static_cast<int64_t>(ct * kCube + ot) * d.X + cx * kCube + ox) * d.Y + cy * kCube + oy;
-            const uint4 v = __ldcs(src + ((static_cast<int64_t>(b) * d.N + n) * d.H + h) * LPR + j);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                acc[2 * e] += __uint_as_float(w[e] << 16);
-                acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
-            }
-        }
+        for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
 #pragma unroll
-        for (int off = LPR; off < 32; off <<= 1) {
+    for (int o = 0; o < kCubeTokens; ++o) {
+        const int ot = o >> 4, ox = (o >> 2) & 3, oy = o & 3;
+        if (ot >= nt || ox >= nx || oy >= ny) continue;
+        const int64_t n = base_n + (static_cast<int64_t>(ot) * d.X + ox) * d.Y + oy;
+        const uint4 v = __ldcs(src + n * row);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
-        }
-        if (sub == 0) {
-            const float inv = 1.0f / static_cast<float>(nt * nx * ny);
-            const int64_t bh = static_cast<int64_t>(b) * d.H + h;
-            float4* out = reinterpret_cast<float4*>(io.dst[tensor] + (bh * d.C + c) * D + j * 8);
-            out[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-            out[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+        for (int e = 0; e < 4; ++e) {
+            acc[o % R][2 * e] += __uint_as_float(w[e] << 16);
+            acc[o % R][2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
         }
     }
+    float m[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        if (R == 1) m[e] = acc[0][e];
+        else if (R == 2) m[e] = acc[0][e] + acc[R - 1][e];
+        else m[e] = (acc[0][e] + acc[1 % R][e]) + (acc[2 % R][e] + acc[3 % R][e]);
+    }
+    const float inv = 1.0f / static_cast<float>(nt * nx * ny);
+    const int64_t bh = static_cast<int64_t>(b) * d.H + h;
+    float4* out = reinterpret_cast<float4*>(io.dst[tensor] + (bh * d.C + c) * D + j * 8);
+    out[0] = make_float4(m[0] * inv, m[1] * inv, m[2] * inv, m[3] * inv);
+    out[1] = make_float4(m[4] * inv, m[5] * inv, m[6] * inv, m[7] * inv);
 }
 
 template <int D>
@@ -290,10 +291,12 @@ cudaError_t launch_pool_tokens(const Dims& d, const uint16_t* const* x, float* c
         io.dst[i] = xbar[i];
     }
     io.count = count;
-    const int64_t warps = static_cast<int64_t>(d.B) * d.H * d.C * count;
-    const int grid = grid_for((warps + 7) / 8, 8);
-    if (d.D == 128) pool_tokens_kernel<128><<<grid, kBlock, 0, s>>>(d, io);
-    else pool_tokens_kernel<64><<<grid, kBlock, 0, s>>>(d, io);
+    const int64_t cubes = static_cast<int64_t>(count) * d.B * d.C;
+    const int slots = (d.H * (d.D / 8) + kPoolThreads - 1) / kPoolThreads;
+    if (cubes > 0x7FFFFFFFll || slots > 65535) return cudaErrorInvalidValue;
+    const dim3 grid(static_cast<unsigned>(cubes), static_cast<unsigned>(slots));
+    if (d.D == 128) pool_tokens_kernel<128><<<grid, kPoolThreads, 0, s>>>(d, io);
+    else pool_tokens_kernel<64><<<grid, kPoolThreads, 0, s>>>(d, io);
     return cudaGetLastError();
 }
 

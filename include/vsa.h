@@ -188,6 +188,22 @@ vsa_status vsa_combine(const vsa_shape* shape, const float* o_coarse, const vsa_
                        vsa_stream_t stream);
 
 /*
+ * vsa_topk_order — vsa_topk and vsa_group from one pass over the scores: the
+ * k best key cubes of every query cube (as vsa_topk) and the per-head work
+ * order (as vsa_group), identical to the two calls.  Two launches: the
+ * selection, which also writes each row's work-order key to sig_scratch,
+ * then a per-head sort of those keys.
+ *   scores       [B, H, C, C] float32 (read).
+ *   idx          [B, H, C, k] int32 (written).
+ *   order        [B, H, C] int32 (written).
+ *   sig_scratch  [B, H, C] uint64 caller scratch (overwritten).
+ * Supported for C <= 2048 (VSA_ERR_UNSUPPORTED otherwise; use vsa_topk and
+ * vsa_group, which vsa_forward then does as well).
+ */
+vsa_status vsa_topk_order(const vsa_shape* shape, const float* scores, int32_t k, int32_t* idx, int32_t* order,
+                          uint64_t* sig_scratch, vsa_stream_t stream);
+
+/*
  * vsa_pool_qkv — the cube mean-pool of vsa_pool applied to q, k and v in one
  * launch, read straight from the token layout (no tiled copy).  Each mean is
  * summed in the same float32 order as vsa_pool on the tiled tensor, so the two
@@ -224,9 +240,10 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
 size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
 
 /*
- * vsa_forward — the whole attention call on one stream, as five launches:
- *   vsa_pool_qkv -> vsa_coarse -> vsa_topk -> vsa_group -> vsa_fine_fused
- * (the grouping step is skipped when C > 4096).  The result equals
+ * vsa_forward — the whole attention call on one stream, as six launches:
+ *   vsa_pool_qkv -> vsa_coarse (2) -> vsa_topk_order (2) -> vsa_fine_fused
+ * (vsa_topk -> vsa_group instead when C > 2048; the grouping step is skipped
+ * when C > 4096).  The result equals
  *   tile -> pool -> coarse -> topk -> group -> fine -> combine -> untile
  * up to the bf16 rounding of O_fine that the staged path makes.
  * When topk == C every cube is selected and the fine stage is dense attention

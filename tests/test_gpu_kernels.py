@@ -451,3 +451,19 @@ def test_fine_fused_writes_only_real_tokens_and_ignores_order_for_dense():
     rev = torch.arange(C - 1, -1, -1, dtype=torch.int32, device="cuda").expand(w.batch, w.heads, C).contiguous()
     out2 = vsa.fine_fused(d["q"], d["k"], d["v"], s, None, order=rev)
     assert torch.equal(out, out2)
+
+
+def test_topk_order_equals_topk_and_group(case):
+    """The one-pass selection + work order gives exactly vsa_topk's and vsa_group's results."""
+    w, _, dev, _ = case
+    s = _shape(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    scores, _ = vsa.coarse(*vsa.pool_qkv(dev["q"], dev["k"], dev["v"], s), s, scale)
+    _, C = vsa.shape_info(s)
+    rng = np.random.default_rng(2)
+    tied = torch.from_numpy(rng.integers(-2, 3, size=(w.batch, w.heads, C, C)).astype(np.float32)).cuda()
+    for sc in (scores, tied):
+        for k in sorted({1, w.topk, C}):
+            idx, order = vsa.topk_order(sc, s, k)
+            assert torch.equal(idx, vsa.topk(sc, s, k)), k
+            assert torch.equal(order, vsa.group(sc, s)), k
