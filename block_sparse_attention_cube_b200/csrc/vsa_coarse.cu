@@ -18,11 +18,14 @@ constexpr int kBK = 16;     // reduction slice
 constexpr int kThreads = 256;
 
 // scores[bh][i][j] = scale * sum_d qbar[bh][i][d] * kbar[bh][j][d]
+// A 64x64 output tile per block; thread (ty, tx) owns rows 4ty..4ty+3 and
+// columns 4tx..4tx+3, reading four operands at a time from shared memory.
+// Each output is one sequential float32 fma chain over the channels.
 __global__ void __launch_bounds__(kThreads) coarse_scores_kernel(int C, int D, const float* __restrict__ qbar,
                                                                  const float* __restrict__ kbar, float scale,
                                                                  float* __restrict__ scores) {
-    __shared__ float As[kBK][kTile + 4];
-    __shared__ float Bs[kBK][kTile + 4];
+    __shared__ __align__(16) float As[kBK][kTile + 4];
+    __shared__ __align__(16) float Bs[kBK][kTile + 4];
     const int bh = blockIdx.z;
     const int i0 = blockIdx.y * kTile, j0 = blockIdx.x * kTile;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -30,7 +33,7 @@ __global__ void __launch_bounds__(kThreads) coarse_scores_kernel(int C, int D, c
     const float* K = kbar + static_cast<int64_t>(bh) * C * D;
     float acc[4][4] = {};
     for (int d0 = 0; d0 < D; d0 += kBK) {
-        // 64 rows x 16 channels of each operand; 4 elements per thread each
+        // 64 rows x 16 channels of each operand, stored channel-major; 4 elements per thread each
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int idx = threadIdx.x + e * kThreads;
@@ -42,48 +45,50 @@ __global__ void __launch_bounds__(kThreads) coarse_scores_kernel(int C, int D, c
         __syncthreads();
 #pragma unroll
         for (int kk = 0; kk < kBK; ++kk) {
-            float a[4], b[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) a[r] = As[kk][ty + 16 * r];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) b[c] = Bs[kk][tx + 16 * c];
+            const float4 a = *reinterpret_cast<const float4*>(&As[kk][4 * ty]);
+            const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][4 * tx]);
+            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
         }
         __syncthreads();
     }
     float* S = scores + static_cast<int64_t>(bh) * C * C;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const int gi = i0 + ty + 16 * r;
+        const int gi = i0 + 4 * ty + r;
         if (gi >= C) continue;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const int gj = j0 + tx + 16 * c;
+            const int gj = j0 + 4 * tx + c;
             if (gj < C) S[static_cast<int64_t>(gi) * C + gj] = scale * acc[r][c];
         }
     }
 }
 
 // o_coarse[bh][i] = sum_j softmax(scores[bh][i][:])_j * vbar[bh][j]
-// A block owns 64 query rows: it first reduces the row maxima and
-// denominators, then accumulates P * Vbar over key slices of 16.
+// A block owns kPvRows query rows: it reduces their row maxima and
+// denominators (a warp per row), then accumulates exp(S - max) * Vbar over
+// key slices of 16; thread (ty, tx) owns RPT rows and 4 output channels.
+constexpr int kPvRows = 32;
+
 template <int D>
 __global__ void __launch_bounds__(kThreads) coarse_pv_kernel(int C, const float* __restrict__ scores,
                                                              const float* __restrict__ vbar,
                                                              float* __restrict__ o_coarse) {
-    constexpr int CPT = D / 16;   // output columns per thread
-    __shared__ float row_max[kTile], row_inv[kTile];
-    __shared__ float Ps[kBK][kTile + 4];
-    __shared__ float Vs[kBK][D];
+    constexpr int TX = D / 4;                     // threads across the channels
+    constexpr int RPT = kPvRows * TX / kThreads;  // rows per thread
+    __shared__ float row_max[kPvRows], row_inv[kPvRows];
+    __shared__ __align__(16) float Ps[kBK][kPvRows + 4];
+    __shared__ __align__(16) float Vs[kBK][D];
     const int bh = blockIdx.y;
-    const int i0 = blockIdx.x * kTile;
+    const int i0 = blockIdx.x * kPvRows;
     const float* S = scores + static_cast<int64_t>(bh) * C * C;
     const float* V = vbar + static_cast<int64_t>(bh) * C * D;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int r = warp; r < kTile; r += kThreads / 32) {
+    for (int r = warp; r < kPvRows; r += kThreads / 32) {
         const int gi = i0 + r;
         float m = -FLT_MAX, l = 0.f;
         if (gi < C) {
@@ -101,43 +106,44 @@ __global__ void __launch_bounds__(kThreads) coarse_pv_kernel(int C, const float*
         }
     }
     __syncthreads();
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float acc[4][CPT] = {};
+    const int tx = threadIdx.x % TX, ty = threadIdx.x / TX;
+    float acc[RPT][4] = {};
     for (int j0 = 0; j0 < C; j0 += kBK) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int idx = threadIdx.x + e * kThreads;   // 64 rows x 16 keys
+        for (int idx = threadIdx.x; idx < kPvRows * kBK; idx += kThreads) {   // kPvRows rows x 16 keys
             const int r = idx / kBK, cc = idx % kBK;
             const int gi = i0 + r, gj = j0 + cc;
             Ps[cc][r] = (gi < C && gj < C) ? expf(S[static_cast<int64_t>(gi) * C + gj] - row_max[r]) : 0.f;
         }
-        for (int idx = threadIdx.x; idx < kBK * D; idx += kThreads) {
-            const int kk = idx / D, cc = idx % D;
+        for (int idx = threadIdx.x; idx < kBK * D / 4; idx += kThreads) {      // 16 keys x D channels
+            const int kk = idx / (D / 4), c4 = idx % (D / 4);
             const int gj = j0 + kk;
-            Vs[kk][cc] = gj < C ? V[static_cast<int64_t>(gj) * D + cc] : 0.f;
+            *reinterpret_cast<float4*>(&Vs[kk][4 * c4]) =
+                gj < C ? *reinterpret_cast<const float4*>(V + static_cast<int64_t>(gj) * D + 4 * c4)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         __syncthreads();
 #pragma unroll
         for (int kk = 0; kk < kBK; ++kk) {
-            float a[4], b[CPT];
+            float a[RPT];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) a[r] = Ps[kk][ty + 16 * r];
+            for (int r = 0; r < RPT; ++r) a[r] = Ps[kk][RPT * ty + r];
+            const float4 b = *reinterpret_cast<const float4*>(&Vs[kk][4 * tx]);
+            const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-            for (int c = 0; c < CPT; ++c) b[c] = Vs[kk][tx + 16 * c];
+            for (int r = 0; r < RPT; ++r)
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int c = 0; c < CPT; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], bv[c], acc[r][c]);
         }
         __syncthreads();
     }
     float* O = o_coarse + static_cast<int64_t>(bh) * C * D;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int li = ty + 16 * r, gi = i0 + li;
+    for (int r = 0; r < RPT; ++r) {
+        const int li = RPT * ty + r, gi = i0 + li;
         if (gi >= C) continue;
-#pragma unroll
-        for (int c = 0; c < CPT; ++c) O[static_cast<int64_t>(gi) * D + tx + 16 * c] = acc[r][c] * row_inv[li];
+        const float inv = row_inv[li];
+        *reinterpret_cast<float4*>(O + static_cast<int64_t>(gi) * D + 4 * tx) =
+            make_float4(acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv, acc[r][3] * inv);
     }
 }
 
@@ -397,8 +403,9 @@ cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, c
     coarse_scores_kernel<<<dim3(tiles, tiles, bh), kThreads, 0, s>>>(d.C, d.D, qbar, kbar, scale, scores);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if (d.D == 128) coarse_pv_kernel<128><<<dim3(tiles, bh), kThreads, 0, s>>>(d.C, scores, vbar, o_coarse);
-    else coarse_pv_kernel<64><<<dim3(tiles, bh), kThreads, 0, s>>>(d.C, scores, vbar, o_coarse);
+    const int pv_blocks = (d.C + kPvRows - 1) / kPvRows;
+    if (d.D == 128) coarse_pv_kernel<128><<<dim3(pv_blocks, bh), kThreads, 0, s>>>(d.C, scores, vbar, o_coarse);
+    else coarse_pv_kernel<64><<<dim3(pv_blocks, bh), kThreads, 0, s>>>(d.C, scores, vbar, o_coarse);
     return cudaGetLastError();
 }
 
