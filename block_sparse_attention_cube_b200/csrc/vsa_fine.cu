@@ -29,32 +29,36 @@
 //    per-head permutation of the query cubes (vsa_group orders cubes with
 //    similar selections next to each other).
 //  * Roles (warp specialisation, teardown section "Blackwell changes the
-//    optimisation problem"): warp 0 walks the selections and issues TMA (the
-//    Q group, then the step's K blocks through a 3-deep ring and V blocks
-//    through a 2-deep ring, so K slots recycle as soon as QK^T is done); for
-//    sparse selections it publishes each step (its two key blocks and which
-//    query blocks selected them) in an 8-deep shared-memory ring, so no
-//    other role repeats the walk.  Warp 1 allocates all 512 tensor-memory
-//    columns and one thread issues the MMAs; warps 2..5 run the softmax and
-//    epilogue of tile A and warps 6..9 those of tile B, one query row per
-//    thread (warp w reads TMEM lane quarter w%4).
+//    optimisation problem"): warp 16 walks the selections and issues TMA (the
+//    Q group, then the step's K blocks and V blocks through two 2-deep rings,
+//    so K slots recycle as soon as QK^T is done); for sparse selections it
+//    publishes each step (its two key blocks and which query blocks selected
+//    them) in an 8-deep shared-memory ring, so no other role repeats the
+//    walk.  Warp 17 allocates all 512 tensor-memory columns and one thread
+//    issues the MMAs.  Warps 0..15 run the softmax and epilogue, one query row
+//    per thread, two warps per TMEM lane quarter of a tile: one takes the
+//    first 64 of a step's 128 key columns, the other the last 64, so a tile's
+//    softmax runs as two halves in parallel (warp w reads lane quarter w%4).
+//    The two agree on each row's running maximum and add their row sums
+//    through a double-buffered shared slot guarded by a two-arrival mbarrier.
 //  * Tensor memory, per tile: one 128x128 fp32 score buffer and a 128xD fp32
-//    output accumulator.  The softmax writes P (bf16) over the first 64
-//    columns of the scores it read and PV takes its A operand from there.
-//    MMAs issued by one thread execute in order, so the next QK^T into the
-//    buffer is issued right after the PV that reads its P.  The issue order
-//    per step, S_A(i), PV_B(i-1), S_B(i), PV_A(i), lets each tile's softmax
-//    run while the tensor cores work on the other tile.
+//    output accumulator.  Each half's softmax writes its P (bf16 pairs) over
+//    the first 32 columns of its own 64 score columns, and PV takes its A
+//    operand from there.  MMAs issued by one thread execute in order, so the
+//    next QK^T into the buffer is issued right after the PV that reads its P.
+//    The issue order per step, S_A(i), PV_B(i-1), S_B(i), PV_A(i), lets each
+//    tile's softmax run while the tensor cores work on the other tile.
 //  * Softmax: online, in the log2 domain.  The running maximum starts at the
-//    maximum of the row's first scores and moves only when a half step's
-//    probabilities would exceed 2^64 (the bound that keeps every later sum
-//    finite); moving it rescales the accumulator, the denominator and any P
-//    already stored.  The scores of step i arrive only after the tile's PV
-//    of step i-1 completed, so the accumulator is stable then.  P is rounded
-//    to bf16; the denominator sums the float32 probabilities.  Teardown
-//    section "Fixed-max softmax is a numerical contract": subtracting any
-//    common constant leaves softmax unchanged; here the constant is bounded
-//    so no exponent overflows.
+//    maximum of the row's first scores (over both halves) and moves only when
+//    a step's probabilities in either half would exceed 2^64 (the bound that
+//    keeps every later sum finite); moving it rescales the accumulator and the
+//    denominators and recomputes the step, whose P is stored only once both
+//    halves agree.  The scores of step i arrive only after the tile's PV of
+//    step i-1 completed, so the accumulator is stable then.  P is rounded to
+//    bf16; the denominator sums the float32 probabilities.  Teardown section
+//    "Fixed-max softmax is a numerical contract": subtracting any common
+//    constant leaves softmax unchanged; here the constant is bounded so no
+//    exponent overflows.
 //  * Epilogue: O / l either to the tiled output (plus log-sum-exp), or, fused,
 //    the gated merge of part 3 of the method, g_c * O_c[cube] + g_f * O / l,
 //    written straight to the token's row of [B, N, H, D] (the untiling).
@@ -83,8 +87,10 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 320;          // producer warp, MMA warp, 2 x 4 softmax warps
-constexpr int kKStages = 3;
+constexpr int kThreads = 576;          // 2 tiles x 2 halves x 4 softmax warps, then the TMA and MMA warps
+constexpr int kTmaWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr int kRing = 8;               // published steps (sparse selections)
 constexpr uint32_t kQTileBytes = 32768;   // 128 rows x 256 B (two 128-B column halves)
@@ -93,7 +99,9 @@ constexpr uint32_t kOffQ = 0;                                  // [2 tiles]
 constexpr uint32_t kOffK = kOffQ + 2 * kQTileBytes;            // [kKStages]
 constexpr uint32_t kOffV = kOffK + kKStages * kKVBytes;        // [kVStages]
 constexpr uint32_t kOffRec = kOffV + kVStages * kKVBytes;      // [kRing] x 16 B
-constexpr uint32_t kOffBar = kOffRec + kRing * 16;
+constexpr uint32_t kOffXch = kOffRec + kRing * 16;             // [2 buffers][2 tiles][4 quarters][2 halves][32] floats
+constexpr uint32_t kXchBytes = 2 * 2 * 4 * 2 * 32 * 4;
+constexpr uint32_t kOffBar = kOffXch + kXchBytes;
 // barrier slots
 constexpr int kBarQFull = 0;
 constexpr int kBarQEmpty = 1;
@@ -106,9 +114,10 @@ constexpr int kBarPFull = kBarSFull + 2;            // [tile]
 constexpr int kBarPVDone = kBarPFull + 2;           // [tile]
 constexpr int kBarRecFull = kBarPVDone + 2;         // [kRing]
 constexpr int kBarRecEmpty = kBarRecFull + kRing;   // [kRing]
-constexpr int kBarDrain = kBarRecEmpty + kRing;
+constexpr int kBarPair = kBarRecEmpty + kRing;      // [tile * 4 + lane quarter]: the two half warps
+constexpr int kBarDrain = kBarPair + 8;
 constexpr int kNumBars = kBarDrain + 1;
-constexpr uint32_t kRecConsumers = 1 + 8;           // the MMA thread and the eight softmax warps
+constexpr uint32_t kRecConsumers = 1 + 16;          // the MMA thread and the sixteen softmax warps
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;   // tmem slot (4 B) + abort flag (4 B)
 constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;     // + alignment slack
 constexpr uint32_t kTmemCols = 512;
@@ -313,45 +322,7 @@ __device__ __forceinline__ void load_block(const CUtensorMap* m, uint32_t dst, i
     }
 }
 
-// Scores of columns whose bit in `vm` is clear become -inf.
-__device__ __forceinline__ void mask64(uint32_t (&s)[64], uint64_t vm) {
-    if (vm == ~0ull) return;
-    const uint32_t ninf = __float_as_uint(-INFINITY);
-#pragma unroll
-    for (int j = 0; j < 64; ++j)
-        if (!((vm >> j) & 1ull)) s[j] = ninf;
-}
-
-__device__ __forceinline__ float max64(const uint32_t (&s)[64]) {
-    float m[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m[i] = __uint_as_float(s[i]);
-#pragma unroll
-    for (int j = 8; j < 64; ++j) m[j & 7] = fmaxf(m[j & 7], __uint_as_float(s[j]));
-    return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
-}
-
 constexpr float kSumLimit = 18446744073709551616.0f;   // 2^64: bound on any probability
-
-// Probabilities 2^(s*c - m) of 64 masked scores: packed as 32 bf16 pairs in
-// pk, their float32 sum returned.
-__device__ __forceinline__ float probs64(const uint32_t (&s)[64], float c, float m, uint32_t (&pk)[32]) {
-    const uint64_t c2 = f32x2(c, c), nm2 = f32x2(-m, -m);
-    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const uint64_t t = fma_f32x2(f32x2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), c2, nm2);
-        float t0, t1;
-        f32x2_split(t, t0, t1);
-        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-        acc[j & 3] = add_f32x2(acc[j & 3], f32x2(p0, p1));
-        pk[j] = pack_bf16x2(p0, p1);
-    }
-    const uint64_t a2 = add_f32x2(add_f32x2(acc[0], acc[1]), add_f32x2(acc[2], acc[3]));
-    float lo, hi;
-    f32x2_split(a2, lo, hi);
-    return lo + hi;
-}
 
 // Multiply `chunks` x 32 float32 columns of this row's tensor memory by alpha.
 __device__ __forceinline__ void scale_tmem_f32(uint32_t taddr, int chunks, float alpha) {
@@ -365,53 +336,68 @@ __device__ __forceinline__ void scale_tmem_f32(uint32_t taddr, int chunks, float
     }
 }
 
-// Multiply 32 columns of bf16 pairs (this row's stored P of one block) by alpha.
-__device__ __forceinline__ void scale_tmem_bf16(uint32_t taddr, float alpha) {
-    uint32_t o[32];
-    tmem_ld32_wait(taddr, o);
+// Scores of columns whose bit in `vm` is clear become -inf (32 columns).
+__device__ __forceinline__ void mask32(uint32_t (&s)[32], uint32_t vm) {
+    if (vm == 0xFFFFFFFFu) return;
+    const uint32_t ninf = __float_as_uint(-INFINITY);
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-        o[j] = pack_bf16x2(__uint_as_float(o[j] << 16) * alpha, __uint_as_float(o[j] & 0xFFFF0000u) * alpha);
-    tmem_st32(taddr, o);
+        if (!((vm >> j) & 1u)) s[j] = ninf;
 }
 
-// Softmax of one half step (64 key columns, block a for h = 0, block b for
-// h = 1) of this thread's row: reads the scores from tensor memory, stores P
-// as bf16 pairs over columns [32h, 32h + 32) and adds the probabilities to
-// l_run.  `vm` is warp-uniform (every row of a warp belongs to one query
-// block).  Warp-collective.
-template <int D>
-__device__ __forceinline__ void softmax_half(uint32_t tcol, int h, uint64_t vm, float c, float& m_run,
-                                             float& l_run) {
-    uint32_t pk[32];
-    if (vm != 0ull) {
-        uint32_t s[64];
-        tmem_ld64_wait(tcol + 64u * h, s);
-        mask64(s, vm);
-        if (m_run == -INFINITY) m_run = max64(s) * c;   // the row's first scores
-        float sum = probs64(s, c, m_run, pk);
-        const bool over = !(sum <= kSumLimit);
-        if (__any_sync(0xffffffffu, over)) {
-            // rare: the maximum fell far behind; rows that overflowed move it
-            // to this half's maximum and rescale what they accumulated so far
-            float alpha = 1.f;
-            if (over) {
-                const float m_new = fmaxf(m_run, max64(s) * c);
-                alpha = ex2_approx(m_run - m_new);
-                m_run = m_new;
-                l_run *= alpha;
-                sum = probs64(s, c, m_run, pk);
-            }
-            // the tile's previous PV completed before these scores were committed
-            scale_tmem_f32(tcol + kColO, D / 32, alpha);
-            if (h == 1) scale_tmem_bf16(tcol, alpha);   // half 0's P is already stored
-        }
-        l_run += sum;
-    } else {
+__device__ __forceinline__ float max32(const uint32_t (&s)[32]) {
+    float m[8];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) pk[j] = 0u;
+    for (int i = 0; i < 8; ++i) m[i] = __uint_as_float(s[i]);
+#pragma unroll
+    for (int j = 8; j < 32; ++j) m[j & 7] = fmaxf(m[j & 7], __uint_as_float(s[j]));
+    return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
+// Probabilities 2^(s*c - m) of 32 masked scores: 16 bf16 pairs into pk, their
+// float32 sum returned.
+__device__ __forceinline__ float probs32(const uint32_t (&s)[32], float c, float m, uint32_t* pk) {
+    const uint64_t c2 = f32x2(c, c), nm2 = f32x2(-m, -m);
+    uint64_t acc[2] = {0ull, 0ull};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        const uint64_t t = fma_f32x2(f32x2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), c2, nm2);
+        float t0, t1;
+        f32x2_split(t, t0, t1);
+        const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+        acc[j & 1] = add_f32x2(acc[j & 1], f32x2(p0, p1));
+        pk[j] = pack_bf16x2(p0, p1);
     }
-    tmem_st32(tcol + 32u * h, pk);
+    float lo, hi;
+    f32x2_split(add_f32x2(acc[0], acc[1]), lo, hi);
+    return lo + hi;
+}
+
+// Masked maximum (times c) of this warp's 64 score columns at tS.  Warp-collective.
+__device__ __forceinline__ float half_max(uint32_t tS, uint64_t vm, float c) {
+    float m = -INFINITY;
+#pragma unroll 1
+    for (int ch = 0; ch < 2; ++ch) {
+        uint32_t sc[32];
+        tmem_ld32_wait(tS + 32u * ch, sc);
+        mask32(sc, static_cast<uint32_t>(vm >> (32 * ch)));
+        m = fmaxf(m, max32(sc));
+    }
+    return m * c;
+}
+
+// Probabilities of this warp's 64 score columns at tS, as 32 bf16 pairs in
+// pk; their float32 sum returned.  Warp-collective.
+__device__ __forceinline__ float half_probs(uint32_t tS, uint64_t vm, float c, float m, uint32_t (&pk)[32]) {
+    float sum = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+        uint32_t sc[32];
+        tmem_ld32_wait(tS + 32u * ch, sc);
+        mask32(sc, static_cast<uint32_t>(vm >> (32 * ch)));
+        sum += probs32(sc, c, m, pk + 16 * ch);
+    }
+    return sum;
 }
 
 // Shared-memory descriptor for a 1024-byte-aligned 128-byte-swizzled operand:
@@ -464,20 +450,21 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(kBarSFull + t), 1);
-            mbar_init(bar(kBarPFull + t), 4);   // one arrival per softmax warp of the tile
+            mbar_init(bar(kBarPFull + t), 8);   // one arrival per softmax warp of the tile
             mbar_init(bar(kBarPVDone + t), 1);
         }
         for (int r = 0; r < kRing; ++r) {
             mbar_init(bar(kBarRecFull + r), 1);
             mbar_init(bar(kBarRecEmpty + r), kRecConsumers);
         }
+        for (int i = 0; i < 8; ++i) mbar_init(bar(kBarPair + i), 2);
         mbar_init(bar(kBarDrain), 1);
         fence_mbar_init();
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(base + kOffMisc, kTmemCols);
         tmem_relinquish();
     }
@@ -489,7 +476,7 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     constexpr uint32_t kBytesQ = 4u * 64u * D * 2u;   // one Q group load
     constexpr uint32_t kBytesKV = 2u * 64u * D * 2u;  // one step's two K (or V) blocks
 
-    if (warp == 0) {
+    if (warp == kTmaWarp) {
         // ------------------------------------------------------------ walk + TMA producer
         if (lane == 0) {
             uint32_t q_issued = 0, k_issued[kKStages] = {}, v_issued[kVStages] = {};
@@ -553,7 +540,7 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 for (int s = 0; s < kVStages; ++s) drain(bar(kBarVFull + s), v_issued[s]);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);   // Q (K-major) x K^T (K-major)
@@ -585,7 +572,8 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 const uint32_t vb = base + kOffV + v.slot * kKVBytes;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16_ts(tmem + t * kTileCols + kColO, tmem + t * kTileCols + 8u * kk,
+                    // P of key half h sits in the first 32 columns of that half's scores
+                    mma_bf16_ts(tmem + t * kTileCols + kColO, tmem + t * kTileCols + (kk >> 2) * 64u + (kk & 3) * 8u,
                                 desc_at(fix_v, vb + kk * 2048u), idesc_o, (!acc[t] && kk == 0) ? 0u : 1u);
                 acc[t] = true;
                 mma_commit(bar(kBarPVDone + t));
@@ -638,27 +626,49 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
             }
         }
-    } else {
+    } else if (warp < kTmaWarp) {
         // ------------------------------------------------------------ softmax + epilogue
-        const int tile = (warp - 2) >> 2;        // 0: warps 2..5, 1: warps 6..9
+        // Warps 0..15.  Two warps share each TMEM lane quarter of a tile, one per
+        // 64-column half of a step's 128 scores, so a tile's softmax runs as two
+        // independent halves.  The pair agrees on each row's maximum (first scores,
+        // overflow) and adds its row sums through a double-buffered shared slot
+        // guarded by a two-arrival mbarrier (every wait bounded).
+        const int sidx = warp;
+        const int tile = sidx >> 3;              // 0: warps 0..7, 1: warps 8..15
+        const int half = (sidx >> 2) & 1;        // which 64 of the step's 128 key columns
         const int q = warp & 3;                  // TMEM lane quarter of this warp
         const int row = q * 32 + lane;           // query row of the tile, 0..127
         const int slot = 2 * tile + (q >> 1);    // query-block slot of the group
         const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
-        const uint32_t tcol = tmem + tile * kTileCols + lane_addr;
+        const uint32_t tS = tmem + tile * kTileCols + lane_addr + 64u * half;   // scores; P over its first 32 columns
+        const uint32_t tO = tmem + tile * kTileCols + lane_addr + kColO + (D / 2) * half;   // this warp's channels
         const uint32_t bar_sfull = bar(kBarSFull + tile), bar_pfull = bar(kBarPFull + tile);
         const uint32_t bar_pvdone = bar(kBarPVDone + tile);
+        const uint32_t bar_pair = bar(kBarPair + tile * 4 + q);
+        float* xbuf = reinterpret_cast<float*>(smem + kOffXch);
         const float c = p.c_log2;
-        uint32_t n = 0;   // steps this tile has taken part in (same count as the MMA issuer's)
+        uint32_t n = 0;    // steps this tile has taken part in (same count as the MMA issuer's)
+        uint32_t xn = 0;   // exchanges of this pair
         RingPos rp{0, 0};
         bool ok = true;
         auto wait_all = [&](uint32_t b, uint32_t par) -> bool {
             const bool mine = bw.wait(b, par);
             return __all_sync(0xffffffffu, mine);
         };
+        // Gives the partner warp this lane's value and returns the partner's for the same row.
+        auto exchange = [&](float mine, float& other) -> bool {
+            float* slot_base = xbuf + (((xn & 1u) * 2 + tile) * 4 + q) * 64;
+            slot_base[half * 32 + lane] = mine;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_pair);   // release: the warp's 32 values are visible
+            const bool got = wait_all(bar_pair, xn & 1u);
+            ++xn;
+            other = slot_base[(half ^ 1) * 32 + lane];
+            return got;
+        };
         for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x) {
             const Item item = decode_item(it, p);
-            float m_run = -INFINITY, l_run = 0.f;
+            float m_run = -INFINITY, l_run = 0.f;   // m_run is the same in both warps of the pair
             uint32_t steps = 0;
             for (int s = 0;; ++s) {
                 StepRec r;
@@ -675,10 +685,49 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     // warp-uniform: this warp's rows belong to one query block
                     const uint64_t vm_a = ((r.flags >> slot) & 1u) ? key_mask<LM>(r.ca, p) : 0ull;
                     const uint64_t vm_b = ((r.flags >> (4 + slot)) & 1u) ? key_mask<LM>(r.cb, p) : 0ull;
+                    const uint64_t vm = half ? vm_b : vm_a;
                     if (!(ok = wait_all(bar_sfull, n & 1u))) break;
                     tc_fence_after();
-                    softmax_half<D>(tcol, 0, vm_a, c, m_run, l_run);
-                    softmax_half<D>(tcol, 1, vm_b, c, m_run, l_run);
+                    uint32_t pk[32];
+                    if ((vm_a | vm_b) != 0ull) {   // the same in both warps of the pair
+                        if (__any_sync(0xffffffffu, m_run == -INFINITY)) {
+                            // the row's first scores: the maximum over both halves
+                            const float mx = vm ? half_max(tS, vm, c) : -INFINITY;
+                            float omx;
+                            if (!(ok = exchange(mx, omx))) break;
+                            if (m_run == -INFINITY) m_run = fmaxf(mx, omx);
+                        }
+                        float sum = 0.f;
+                        if (vm) {
+                            sum = half_probs(tS, vm, c, m_run, pk);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) pk[j] = 0u;
+                        }
+                        float osum;
+                        if (!(ok = exchange(sum, osum))) break;
+                        // A probability above 2^64 in either half (the maximum fell far
+                        // behind): both warps raise it to the step's maximum, rescale what
+                        // they accumulated (each its half of O) and recompute.  The scores
+                        // are intact, since no P of this step is stored yet.
+                        if (__any_sync(0xffffffffu, !(sum <= kSumLimit) || !(osum <= kSumLimit))) {
+                            const float mx = vm ? half_max(tS, vm, c) : -INFINITY;
+                            float omx;
+                            if (!(ok = exchange(mx, omx))) break;
+                            const float m_new = fmaxf(m_run, fmaxf(mx, omx));
+                            const float alpha = ex2_approx(m_run - m_new);
+                            m_run = m_new;
+                            l_run *= alpha;
+                            // the tile's previous PV completed before these scores were committed
+                            scale_tmem_f32(tO, D / 64, alpha);
+                            if (vm) sum = half_probs(tS, vm, c, m_run, pk);
+                        }
+                        l_run += sum;
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) pk[j] = 0u;
+                    }
+                    tmem_st32(tS, pk);
                     tmem_wait_st();
                     tc_fence_before();
                     __syncwarp();
@@ -689,35 +738,39 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 if (r.last) break;
             }
             if (!ok) break;
-            if (steps == 0) continue;   // the tile holds no query block of this group
-            // ---------------- epilogue of this tile's rows
+            if (steps == 0) continue;   // the tile holds no query block of this group (both warps)
+            // ---------------- epilogue of this warp's rows and channels
             // PV(n-2) completed before S(n-1) was committed, so this parity cannot alias
             if (!(ok = wait_all(bar_pvdone, (n - 1) & 1u))) break;
             tc_fence_after();
+            float ol;
+            if (!(ok = exchange(l_run, ol))) break;
+            const float l_tot = half ? (ol + l_run) : (l_run + ol);   // one order in both warps
             const int blk = item.blk[slot];
             const int o_ = row & 63;
-            const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+            const int d0 = (D / 2) * half;
+            const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
             if (!FUSED) {
                 const bool store = blk >= 0;
                 const int64_t grow = item.bh * p.Npad + static_cast<int64_t>(store ? blk : 0) * 64 + o_;
 #pragma unroll 1
-                for (int ch = 0; ch < D / 32; ++ch) {
+                for (int ch = 0; ch < D / 64; ++ch) {
                     uint32_t o[32];
-                    tmem_ld32_wait(tcol + kColO + 32u * ch, o);
+                    tmem_ld32_wait(tO + 32u * ch, o);
                     if (store) {
                         uint32_t w16[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
                             w16[j] = pack_bf16x2(__uint_as_float(o[2 * j]) * inv_l,
                                                  __uint_as_float(o[2 * j + 1]) * inv_l);
-                        uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + 32 * ch);
+                        uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + d0 + 32 * ch);
 #pragma unroll
                         for (int v = 0; v < 4; ++v)
                             dst[v] = make_uint4(w16[4 * v], w16[4 * v + 1], w16[4 * v + 2], w16[4 * v + 3]);
                     }
                 }
-                if (store && p.lse != nullptr)
-                    p.lse[grow] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+                if (store && half == 0 && p.lse != nullptr)
+                    p.lse[grow] = l_tot > 0.f ? (m_run + log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
             } else {
                 // token of this row, and the cube whose coarse output it merges
                 int64_t tok = -1;
@@ -757,15 +810,15 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                 }
                 const float sf = gf * inv_l;
 #pragma unroll 1
-                for (int ch = 0; ch < D / 32; ++ch) {
+                for (int ch = 0; ch < D / 64; ++ch) {
                     uint32_t o[32];
-                    tmem_ld32_wait(tcol + kColO + 32u * ch, o);
+                    tmem_ld32_wait(tO + 32u * ch, o);
                     if (store) {
                         float v[32];
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(o[j]) * sf;
                         if (ocr != nullptr) {
-                            const float4* oc4 = reinterpret_cast<const float4*>(ocr + 32 * ch);
+                            const float4* oc4 = reinterpret_cast<const float4*>(ocr + d0 + 32 * ch);
 #pragma unroll
                             for (int j = 0; j < 8; ++j) {
                                 const float4 cv = __ldg(oc4 + j);
@@ -778,7 +831,7 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                         uint32_t w16[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) w16[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-                        uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + 32 * ch);
+                        uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + d0 + 32 * ch);
 #pragma unroll
                         for (int v4 = 0; v4 < 4; ++v4)
                             dst[v4] = make_uint4(w16[4 * v4], w16[4 * v4 + 1], w16[4 * v4 + 2], w16[4 * v4 + 3]);
@@ -791,7 +844,7 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
