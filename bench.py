@@ -290,11 +290,11 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     dense_ms_max = reduce_max(dense_ms, world)
 
     # ---- per-stage breakdown: the launches of vsa_forward, one by one through the entry points
-    names = ["pool", "coarse", "topk_order", "fine"]
+    names = ["pool", "coarse", "topk_order", "schedule", "fine"]
     acc = {n: [] for n in names}
     acc["fine_dense"] = []
     for it in range(args.warmup + args.steps):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
         e[0].record(stream)
         bars = vsa.pool_qkv(d["q"], d["k"], d["v"], s)
         e[1].record(stream)
@@ -302,16 +302,19 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         e[2].record(stream)
         idx, order = vsa.topk_order(scores, s, w.topk)
         e[3].record(stream)
-        vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, order, oc, d["g_coarse"], d["g_fine"], out=out)
+        steps = vsa.schedule(idx, s, order)
         e[4].record(stream)
-        vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out_d)
+        vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, order, oc, d["g_coarse"], d["g_fine"], out=out,
+                       steps=steps)
         e[5].record(stream)
+        vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out_d)
+        e[6].record(stream)
         torch.cuda.synchronize()
         if it >= args.warmup:
             for j, n in enumerate(names):
                 acc[n].append(e[j].elapsed_time(e[j + 1]))
-            acc["fine_dense"].append(e[4].elapsed_time(e[5]))
-        del bars, scores, oc, idx, order
+            acc["fine_dense"].append(e[5].elapsed_time(e[6]))
+        del bars, scores, oc, idx, order, steps
     stage_ms = {n: round(statistics.mean(v), 4) for n, v in acc.items()}
 
     # ---- end to end through vsa_forward_host (pinned host buffers, copies inside the timed region)
@@ -376,7 +379,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                      "per_launch": "4*B*H*Npad*k*64*D executed flops (64x64 cube tiles of the k selected cubes)"},
         "e2e": {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "vsa_forward_host (pinned host q/k/v/gates in, host out)"},
-        "gpu_launches": 8 * args.steps,   # VSA: pool, coarse (2), top-k, order sort, fine; dense: fine
+        "gpu_launches": 9 * args.steps,   # VSA: pool, coarse (2), top-k, order sort, schedule, fine; dense: fine
         "clocks": clocks,
         "cpu_baseline": cpu,
         "context": {"pages_dense_call_ms_b200": 17.0, "pages_vsa_kernel_ms_b200_k78": 4.719,

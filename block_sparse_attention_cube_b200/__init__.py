@@ -187,20 +187,33 @@ def pool_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return outs[0], outs[1], outs[2]
 
 
+def schedule(idx: torch.Tensor, shape: Shape, order: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Precomputed steps of the fine stage for the selection idx [B,H,C,k] (and work order)."""
+    k = int(idx.shape[-1])
+    n = int(_L.vsa_schedule_bytes(ctypes.byref(shape.c()), k))
+    steps = torch.empty(max(n, 1), dtype=torch.uint8, device=idx.device)
+    _check(_L.vsa_schedule(ctypes.byref(shape.c()), _ptr(idx, torch.int32, "idx"), k,
+                           _ptr(order, torch.int32, "order"), _ptr(steps, torch.uint8, "steps"), _stream()))
+    return steps
+
+
 def fine_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, shape: Shape, idx: Optional[torch.Tensor] = None,
                scale: Optional[float] = None, order: Optional[torch.Tensor] = None,
                o_coarse: Optional[torch.Tensor] = None, g_coarse: Optional[torch.Tensor] = None,
-               g_fine: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Fine attention + gated merge on the token layout, written as [B,N,H,D] (idx None: dense attention)."""
+               g_fine: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+               steps: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Fine attention + gated merge on the token layout, written as [B,N,H,D] (idx None: dense attention).
+
+    `steps` (from schedule()) replaces the kernel's own walk of the selection."""
     scale = default_scale(shape) if scale is None else scale
     kk = int(idx.shape[-1]) if idx is not None else 0
     if out is None:
         out = torch.empty_like(q)
     _check(_L.vsa_fine_fused(ctypes.byref(shape.c()), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
                              _ptr(v, torch.bfloat16, "v"), _ptr(idx, torch.int32, "idx"), kk,
-                             _ptr(order, torch.int32, "order"), scale, _ptr(o_coarse, torch.float32, "o_coarse"),
-                             _ptr(g_coarse, torch.bfloat16, "g_coarse"), _ptr(g_fine, torch.bfloat16, "g_fine"),
-                             _ptr(out, torch.bfloat16, "out"), _stream()))
+                             _ptr(order, torch.int32, "order"), _ptr(steps, torch.uint8, "steps"), scale,
+                             _ptr(o_coarse, torch.float32, "o_coarse"), _ptr(g_coarse, torch.bfloat16, "g_coarse"),
+                             _ptr(g_fine, torch.bfloat16, "g_fine"), _ptr(out, torch.bfloat16, "out"), _stream()))
     return out
 
 

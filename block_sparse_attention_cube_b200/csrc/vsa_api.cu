@@ -121,7 +121,7 @@ size_t order_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C 
 constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Workspace of vsa_forward: qbar | kbar | vbar | o_coarse | scores | idx | order | sig.
+// Workspace of vsa_forward: qbar | kbar | vbar | o_coarse | scores | idx | order | sig | steps.
 // Q, K and V are read in the caller's [B, N, H, D] layout (the fine stage
 // gathers cubes with TMA), so no tiled copies are kept.  With every cube
 // selected the fine stage is dense attention and needs none of it; the
@@ -131,6 +131,7 @@ struct Carve {
     int32_t* idx;
     int32_t* order;
     uint64_t* sig;   // work-order signatures, when top-k computes them (C <= kTopkRegMaxC)
+    void* steps;     // the fine stage's precomputed steps (when schedule_supported)
     size_t bytes;
 };
 
@@ -155,6 +156,7 @@ Carve carve(const Dims& d, int k, bool coarse_gate, void* ws) {
         c.idx = reinterpret_cast<int32_t*>(take(idx_bytes(d, k)));
         c.order = reinterpret_cast<int32_t*>(take(order_bytes(d)));
         if (d.C <= kTopkRegMaxC) c.sig = reinterpret_cast<uint64_t*>(take(2 * order_bytes(d)));
+        if (schedule_supported(d, k)) c.steps = take(schedule_bytes(d, k));
     }
     c.bytes = off > kAlign ? off : kAlign;
     return c;
@@ -186,8 +188,9 @@ vsa_status check_k(const Dims& d, int32_t k) {
 // The fused fine stage once the arguments are checked: cube gathers when a
 // selection is given, blocks of consecutive real tokens for dense attention.
 vsa_status run_fine_fused(const Dims& d, const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                          const int32_t* idx, int topk, const int32_t* order, float scale, const float* o_coarse,
-                          const uint16_t* gc, const uint16_t* gf, uint16_t* out, cudaStream_t s) {
+                          const int32_t* idx, int topk, const int32_t* order, const void* steps, float scale,
+                          const float* o_coarse, const uint16_t* gc, const uint16_t* gf, uint16_t* out,
+                          cudaStream_t s) {
     FineArgs a{};
     a.mode = idx ? kFineCubesFused : kFineTokensFused;
     a.q = q;
@@ -196,6 +199,7 @@ vsa_status run_fine_fused(const Dims& d, const uint16_t* q, const uint16_t* k, c
     a.idx = idx;
     a.k_sel = topk;
     a.order = idx ? order : nullptr;
+    a.steps = idx ? steps : nullptr;
     a.scale = scale;
     a.out = out;
     a.o_coarse = o_coarse;
@@ -238,8 +242,13 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
             }
         }
     }
-    return run_fine_fused(d, q, k, v, sparse ? c.idx : nullptr, topk, order, scale, gc ? c.oc : nullptr, gc, gf,
-                          out, s);
+    const void* steps = nullptr;
+    if (sparse && c.steps != nullptr) {
+        VSA_CUDA(launch_schedule(d, c.idx, topk, order, c.steps, s), "schedule launch");
+        steps = c.steps;
+    }
+    return run_fine_fused(d, q, k, v, sparse ? c.idx : nullptr, topk, order, steps, scale, gc ? c.oc : nullptr, gc,
+                          gf, out, s);
 }
 
 }  // namespace
@@ -442,6 +451,30 @@ vsa_status vsa_topk_order(const vsa_shape* shape, const float* scores, int32_t k
     return VSA_OK;
 }
 
+size_t vsa_schedule_bytes(const vsa_shape* shape, int32_t topk) {
+    Dims d{};
+    if (make_dims(shape, &d) != VSA_OK || topk < 1 || topk > d.C) return 0;
+    return schedule_bytes(d, topk);
+}
+
+vsa_status vsa_schedule(const vsa_shape* shape, const int32_t* idx, int32_t topk, const int32_t* order, void* steps,
+                        vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(check_k(d, topk));
+    VSA_TRY(need_ptr(idx, "idx"));
+    VSA_TRY(opt_ptr(order, "order"));
+    VSA_TRY(need_ptr(steps, "steps"));
+    if (!schedule_supported(d, topk))
+        return fail(VSA_ERR_UNSUPPORTED, "vsa_schedule: C = %d, top-k = %d too large for its shared memory", d.C,
+                    topk);
+    VSA_TRY(check_disjoint({{idx, idx_bytes(d, topk), "idx"}, {order, order ? order_bytes(d) : 0, "order"}},
+                           {{steps, schedule_bytes(d, topk), "steps"}}));
+    VSA_TRY(check_device());
+    VSA_CUDA(launch_schedule(d, idx, topk, order, steps, as_stream(stream)), "schedule launch");
+    return VSA_OK;
+}
+
 vsa_status vsa_pool_qkv(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
                         float* qbar, float* kbar, float* vbar, vsa_stream_t stream) {
     Dims d{};
@@ -463,7 +496,7 @@ vsa_status vsa_pool_qkv(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf1
 }
 
 vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
-                          const int32_t* idx, int32_t topk, const int32_t* order, float scale,
+                          const int32_t* idx, int32_t topk, const int32_t* order, const void* steps, float scale,
                           const float* o_coarse, const vsa_bf16* g_coarse, const vsa_bf16* g_fine, vsa_bf16* out,
                           vsa_stream_t stream) {
     Dims d{};
@@ -474,6 +507,10 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
     VSA_TRY(need_ptr(v, "v"));
     VSA_TRY(opt_ptr(idx, "idx"));
     VSA_TRY(opt_ptr(order, "order"));
+    VSA_TRY(opt_ptr(steps, "steps"));
+    if (steps && !idx) return fail(VSA_ERR_INVALID_ARGUMENT, "steps given without idx");
+    if (steps && d.C > kScheduleMaxC)
+        return fail(VSA_ERR_UNSUPPORTED, "precomputed steps support at most %d cubes (got %d)", kScheduleMaxC, d.C);
     VSA_TRY(opt_ptr(o_coarse, "o_coarse"));
     VSA_TRY(opt_ptr(g_coarse, "g_coarse"));
     VSA_TRY(opt_ptr(g_fine, "g_fine"));
@@ -482,11 +519,13 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
     const size_t tb = token_bytes(d), gb = gate_bytes(d);
     VSA_TRY(check_disjoint({{q, tb, "q"}, {k, tb, "k"}, {v, tb, "v"}, {idx, idx ? idx_bytes(d, topk) : 0, "idx"},
                             {order, order ? order_bytes(d) : 0, "order"},
+                            {steps, steps ? schedule_bytes(d, topk) : 0, "steps"},
                             {o_coarse, o_coarse ? pooled_bytes(d) : 0, "o_coarse"},
                             {g_coarse, g_coarse ? gb : 0, "g_coarse"}, {g_fine, g_fine ? gb : 0, "g_fine"}},
                            {{out, tb, "out"}}));
     VSA_TRY(check_device());
-    return run_fine_fused(d, q, k, v, idx, topk, order, scale, o_coarse, g_coarse, g_fine, out, as_stream(stream));
+    return run_fine_fused(d, q, k, v, idx, topk, order, steps, scale, o_coarse, g_coarse, g_fine, out,
+                          as_stream(stream));
 }
 
 size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk) {

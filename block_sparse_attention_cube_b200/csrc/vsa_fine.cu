@@ -131,6 +131,8 @@ enum LoadMode : int { kLoadTiled = 0, kLoadCubes = 1, kLoadTokens = 2 };
 struct FineParams {
     const int32_t* idx;     // [B, H, C, k] or nullptr (every block)
     const int32_t* order;   // [B, H, C] permutation of query cubes, or nullptr (identity)
+    const uint2* steps;     // precomputed steps [items][steps_stride] (schedule_kernel), or nullptr (walk here)
+    int64_t steps_stride;
     uint16_t* o;            // tiled O [B, H, Npad, D], or the merged output [B, N, H, D] (fused)
     float* lse;             // [B, H, Npad] or nullptr (tiled output only)
     const float* o_coarse;  // [B, H, C, D] or nullptr (fused only; no coarse term)
@@ -275,6 +277,43 @@ __device__ __forceinline__ GroupWalk make_walk(const Item& item, const FineParam
         w.lst[j] = item.blk[j] < 0 ? p.idx : p.idx + (item.bh * p.C + item.blk[j]) * static_cast<int64_t>(p.k);
     }
     return w;
+}
+
+// Entries of the union in three passes: those only tile A's query blocks
+// selected, then only tile B's, then both tiles' (pairing like with like
+// leaves fewer tiles half-used in a step).
+struct TileWalk {
+    GroupWalk w0, w;
+    int pass;
+    __device__ __forceinline__ bool next_entry(int& blk, uint32_t& fl) {
+        for (;;) {
+            if (!w.next1(blk, fl)) {
+                if (++pass == 3) return false;
+                w = w0;
+                continue;
+            }
+            const int pat = ((fl & 3u) ? 1 : 0) | ((fl & 12u) ? 2 : 0);
+            if (pat == pass + 1) return true;
+        }
+    }
+};
+
+// A step record in global memory: x = block a | block b << 16 (0xFFFF: none),
+// y = flags | last << 31.
+__device__ __forceinline__ uint2 encode_step(const StepRec& r) {
+    const uint32_t a = r.ca < 0 ? 0xFFFFu : static_cast<uint32_t>(r.ca);
+    const uint32_t b = r.cb < 0 ? 0xFFFFu : static_cast<uint32_t>(r.cb);
+    return make_uint2(a | (b << 16), r.flags | (r.last << 31));
+}
+
+__device__ __forceinline__ StepRec decode_step(uint2 e) {
+    StepRec r;
+    const uint32_t a = e.x & 0xFFFFu, b = e.x >> 16;
+    r.ca = a == 0xFFFFu ? -1 : static_cast<int32_t>(a);
+    r.cb = b == 0xFFFFu ? -1 : static_cast<int32_t>(b);
+    r.flags = e.y & 0xFFu;
+    r.last = e.y >> 31;
+    return r;
 }
 
 __device__ __forceinline__ bool tile_active(uint32_t flags, int t) { return (flags & (0x33u << (2 * t))) != 0u; }
@@ -505,9 +544,18 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
                     if (dense) {
                         r = dense_step(s, item.present, p.nblk);
                     } else {
-                        // an item none of whose slots holds a query block (an order
-                        // entry out of range) still publishes one empty step
-                        if (!w.next(r)) r = StepRec{-1, -1, 0u, 1u};
+                        if (p.steps != nullptr) {
+                            // a record is trusted no further than the buffer's bounds: blocks
+                            // past the grid read as the empty cube, and the last slot ends the item
+                            r = decode_step(__ldg(p.steps + it * p.steps_stride + s));
+                            r.ca = min(r.ca, p.C);
+                            r.cb = min(r.cb, p.C);
+                            if (s + 1 >= p.steps_stride) r.last = 1u;
+                        } else if (!w.next(r)) {
+                            // an item none of whose slots holds a query block (an order
+                            // entry out of range) still publishes one empty step
+                            r = StepRec{-1, -1, 0u, 1u};
+                        }
                         if (!(ok = bw.wait(bar(kBarRecEmpty + rp.slot), rp.phase ^ 1u))) break;
                         ring[rp.slot] = r;
                         mbar_arrive(bar(kBarRecFull + rp.slot));   // release: the record is visible
@@ -850,6 +898,145 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
 }
 
+// Steps of one work item by the serial three-pass walk (TileWalk), written by
+// one thread: the general case, which also visits repeated entries of a list
+// as often as they appear.
+__device__ void schedule_serial(const Item& item, const FineParams& p, uint2* out) {
+    TileWalk tw;
+    tw.w0 = make_walk(item, p);
+    tw.w = tw.w0;
+    tw.pass = 0;
+    int blk = -1;
+    uint32_t fl = 0;
+    bool more = tw.next_entry(blk, fl);
+    if (!more) {   // no query block in the group (order entries out of range): one empty step
+        out[0] = encode_step(StepRec{-1, -1, 0u, 1u});
+        return;
+    }
+    for (int s = 0; more; ++s) {
+        StepRec r;
+        r.ca = blk;
+        r.flags = fl;
+        more = tw.next_entry(blk, fl);
+        r.cb = -1;
+        if (more) {
+            r.cb = blk;
+            r.flags |= fl << 4;
+            more = tw.next_entry(blk, fl);
+        }
+        r.last = more ? 0u : 1u;
+        out[s] = encode_step(r);
+    }
+}
+
+// Entries of a nibble word (cube 8w + n in nibble n, bit j set when query
+// slot j selected it), one bit per nibble: selected by slot 0 or 1 (tile A),
+// by slot 2 or 3 (tile B).
+__device__ __forceinline__ uint32_t nib_tile_a(uint32_t v) { return (v | (v >> 1)) & 0x11111111u; }
+__device__ __forceinline__ uint32_t nib_tile_b(uint32_t v) { return ((v >> 2) | (v >> 3)) & 0x11111111u; }
+
+// Steps of every work item of a sparse selection, precomputed so the fine
+// kernel's producer only reads them: the union of the group's four lists in
+// three classes (key cubes only tile A's query blocks selected, only tile B's,
+// both tiles'), ascending within a class, paired two per step.
+//
+// One warp per item.  The warp marks each list entry as a bit in a nibble per
+// cube (cubes 0..C, C standing for every out-of-range entry) in shared memory,
+// then scans the nibbles in cube order twice: once to count each class, once
+// to place each cube at its class's offset plus its rank, with warp prefix
+// sums over packed per-lane counts.  A list that holds a cube twice (never the
+// case for a top-k selection) sends the item to the serial walk.
+constexpr int kScheduleWarps = 4;
+
+__host__ __device__ __forceinline__ int schedule_words(int C) { return (C + 8) >> 3; }
+
+__global__ void __launch_bounds__(kScheduleWarps * 32) schedule_kernel(const FineParams p, uint2* __restrict__ steps) {
+    extern __shared__ uint32_t sched_smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int W = schedule_words(p.C), E = 4 * p.k;
+    uint32_t* nib = sched_smem + static_cast<int64_t>(warp) * (W + E);
+    uint32_t* ent = nib + W;
+    const int64_t it = static_cast<int64_t>(blockIdx.x) * kScheduleWarps + warp;
+    if (it >= p.items) return;   // warp-uniform
+    for (int i = lane; i < W; i += 32) nib[i] = 0u;
+    __syncwarp();
+    const Item item = decode_item(it, p);
+    uint2* out = steps + it * p.steps_stride;
+    if (item.present == 0u) {   // no query block in the group: one empty step
+        if (lane == 0) out[0] = encode_step(StepRec{-1, -1, 0u, 1u});
+        return;
+    }
+    bool dup = false;
+    for (int e = lane; e < E; e += 32) {
+        const int j = e / p.k, i = e - j * p.k;
+        if (!((item.present >> j) & 1u)) continue;
+        int x = __ldg(p.idx + (item.bh * p.C + item.blk[j]) * static_cast<int64_t>(p.k) + i);
+        if (x < 0 || x >= p.C) x = p.C;
+        const uint32_t bit = 1u << (j + 4 * (x & 7));
+        dup |= (atomicOr(nib + (x >> 3), bit) & bit) != 0u;
+    }
+    __syncwarp();
+    if (__any_sync(0xFFFFFFFFu, dup)) {
+        if (lane == 0) schedule_serial(item, p, out);
+        return;
+    }
+    // class totals
+    uint32_t t1 = 0, t2 = 0, t3 = 0;
+    for (int w0 = 0; w0 < W; w0 += 32) {
+        const uint32_t v = w0 + lane < W ? nib[w0 + lane] : 0u;
+        const uint32_t a = nib_tile_a(v), b = nib_tile_b(v);
+        t1 += __popc(a & ~b);
+        t2 += __popc(b & ~a);
+        t3 += __popc(a & b);
+    }
+    t1 = __reduce_add_sync(0xFFFFFFFFu, t1);
+    t2 = __reduce_add_sync(0xFFFFFFFFu, t2);
+    t3 = __reduce_add_sync(0xFFFFFFFFu, t3);
+    // placement: class base + cubes of the class in earlier words
+    uint32_t base[3] = {0u, t1, t1 + t2};
+    for (int w0 = 0; w0 < W; w0 += 32) {
+        const int wi = w0 + lane;
+        const uint32_t v = wi < W ? nib[wi] : 0u;
+        const uint32_t a = nib_tile_a(v), b = nib_tile_b(v);
+        // per-lane counts of the three classes in 10-bit fields (at most 8 each)
+        const uint32_t mine = __popc(a & ~b) | (__popc(b & ~a) << 10) | (__popc(a & b) << 20);
+        uint32_t incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - mine;
+        uint32_t pa = base[0] + (excl & 1023u), pb = base[1] + ((excl >> 10) & 1023u), pab = base[2] + (excl >> 20);
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            const uint32_t f = (v >> (4 * n)) & 15u;
+            if (f == 0u) continue;
+            const bool in_a = (f & 3u) != 0u, in_b = (f & 12u) != 0u;
+            const uint32_t at = in_a ? (in_b ? pab++ : pa++) : pb++;
+            ent[at] = static_cast<uint32_t>(8 * wi + n) | (f << 16);
+        }
+        const uint32_t tot = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        base[0] += tot & 1023u;
+        base[1] += (tot >> 10) & 1023u;
+        base[2] += tot >> 20;
+    }
+    __syncwarp();
+    const int U = static_cast<int>(t1 + t2 + t3);
+    const int nsteps = (U + 1) >> 1;
+    for (int st = lane; st < nsteps; st += 32) {
+        const uint32_t ea = ent[2 * st];
+        const bool has_b = 2 * st + 1 < U;
+        const uint32_t eb = has_b ? ent[2 * st + 1] : 0u;
+        StepRec r;
+        r.ca = static_cast<int32_t>(ea & 0xFFFFu);
+        r.cb = has_b ? static_cast<int32_t>(eb & 0xFFFFu) : -1;
+        r.flags = (ea >> 16) | (has_b ? (eb >> 16) << 4 : 0u);
+        r.last = st == nsteps - 1 ? 1u : 0u;
+        out[st] = encode_step(r);
+    }
+}
+
 __global__ void wait_probe_kernel(int* status, uint64_t limit_ns) {
     __shared__ __align__(8) uint64_t bar_storage;
     __shared__ int abort_flag;
@@ -966,27 +1153,14 @@ int* status_word() {
     return ptrs[dev];
 }
 
-cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const char** why) {
-    CUtensorMap tq, tk, tv;
-    bool enc = false;
+namespace {
+
+FineParams make_params(const Dims& d, const FineArgs& a) {
     const int mode = a.mode;
-    if (mode == kFineTiled) {
-        enc = encode_tiled(&tq, a.q, d) && encode_tiled(&tk, a.k, d) && encode_tiled(&tv, a.v, d);
-    } else if (mode == kFineCubesFused) {
-        enc = encode_cubes(&tq, a.q, d) && encode_cubes(&tk, a.k, d) && encode_cubes(&tv, a.v, d);
-    } else if (mode == kFineTokensFused) {
-        enc = encode_tokens(&tq, a.q, d) && encode_tokens(&tk, a.k, d) && encode_tokens(&tv, a.v, d);
-    } else {
-        if (why) *why = "unknown fine-stage mode";
-        return cudaErrorInvalidValue;
-    }
-    if (!enc) {
-        if (why) *why = "cuTensorMapEncodeTiled failed for a Q/K/V tensor";
-        return cudaErrorInvalidValue;
-    }
     FineParams p{};
     p.idx = a.idx;
     p.order = a.order;
+    p.steps = reinterpret_cast<const uint2*>(a.steps);
     p.o = a.out;
     p.lse = a.lse;
     p.o_coarse = a.o_coarse;
@@ -996,6 +1170,7 @@ cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const 
     p.H = d.H;
     p.nblk = mode == kFineTokensFused ? static_cast<int>((d.N + 63) / 64) : d.C;
     p.k = a.idx ? a.k_sel : p.nblk;
+    p.steps_stride = schedule_stride(p.k);
     p.C = d.C;
     p.Ct = d.Ct;
     p.Cx = d.Cx;
@@ -1017,6 +1192,62 @@ cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const 
     p.c_log2 = a.scale * 1.4426950408889634f;
     p.status = status_word();
     p.limit_ns = kWaitLimitNs;
+    return p;
+}
+
+}  // namespace
+
+size_t schedule_bytes(const Dims& d, int k) {
+    const int64_t items = static_cast<int64_t>(d.B) * d.H * ((d.C + 3) / 4);
+    return static_cast<size_t>(items) * static_cast<size_t>(schedule_stride(k)) * sizeof(uint2);
+}
+
+namespace {
+size_t schedule_smem(const Dims& d, int k) {
+    return static_cast<size_t>(kScheduleWarps) * (static_cast<size_t>(schedule_words(d.C)) + 4ull * k) * 4u;
+}
+}  // namespace
+
+bool schedule_supported(const Dims& d, int k) {
+    return d.C <= kScheduleMaxC && k >= 1 && k <= d.C && schedule_smem(d, k) <= 48u * 1024u;
+}
+
+cudaError_t launch_schedule(const Dims& d, const int32_t* idx, int k, const int32_t* order, void* steps,
+                            cudaStream_t s) {
+    if (!schedule_supported(d, k)) return cudaErrorInvalidValue;
+    FineArgs a{};
+    a.mode = kFineCubesFused;
+    a.idx = idx;
+    a.k_sel = k;
+    a.order = order;
+    const FineParams p = make_params(d, a);
+    const int64_t blocks = (p.items + kScheduleWarps - 1) / kScheduleWarps;
+    if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+    if (blocks == 0) return cudaSuccess;
+    schedule_kernel<<<static_cast<unsigned>(blocks), kScheduleWarps * 32, schedule_smem(d, k), s>>>(
+        p, static_cast<uint2*>(steps));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const char** why) {
+    CUtensorMap tq, tk, tv;
+    bool enc = false;
+    const int mode = a.mode;
+    if (mode == kFineTiled) {
+        enc = encode_tiled(&tq, a.q, d) && encode_tiled(&tk, a.k, d) && encode_tiled(&tv, a.v, d);
+    } else if (mode == kFineCubesFused) {
+        enc = encode_cubes(&tq, a.q, d) && encode_cubes(&tk, a.k, d) && encode_cubes(&tv, a.v, d);
+    } else if (mode == kFineTokensFused) {
+        enc = encode_tokens(&tq, a.q, d) && encode_tokens(&tk, a.k, d) && encode_tokens(&tv, a.v, d);
+    } else {
+        if (why) *why = "unknown fine-stage mode";
+        return cudaErrorInvalidValue;
+    }
+    if (!enc) {
+        if (why) *why = "cuTensorMapEncodeTiled failed for a Q/K/V tensor";
+        return cudaErrorInvalidValue;
+    }
+    FineParams p = make_params(d, a);
     if (!p.status) {
         if (why) *why = "watchdog word unavailable";
         return cudaErrorInvalidValue;

@@ -79,6 +79,7 @@ struct FineArgs {
     const int32_t* idx;     // [B, H, C, k] or null (every block)
     int k_sel;
     const int32_t* order;   // [B, H, C] or null
+    const void* steps;      // precomputed steps (launch_schedule) or null: the kernel walks the selection
     float scale;
     uint16_t* out;
     float* lse;             // kFineTiled only
@@ -88,6 +89,18 @@ struct FineArgs {
 };
 
 cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const char** why);
+
+// Precomputed steps of the fine stage's work items for a sparse selection
+// (idx [B, H, C, k], order [B, H, C] or null): 8 bytes per step, at most
+// 2k steps per item of four query cubes.  Cube indices travel in 16 bits, so
+// the fine kernel takes steps for C <= kScheduleMaxC; launch_schedule also
+// needs its shared memory (four warps x (C/8 + 1 + 4k) words) within 48 KB.
+constexpr int kScheduleMaxC = 65534;
+inline int64_t schedule_stride(int k) { return 2ll * k; }
+size_t schedule_bytes(const Dims& d, int k);
+bool schedule_supported(const Dims& d, int k);
+cudaError_t launch_schedule(const Dims& d, const int32_t* idx, int k, const int32_t* order, void* steps,
+                            cudaStream_t s);
 
 // Cube mean-pool read straight from the projection layout [B, N, H, D]
 // (same fp32 summation order as launch_pool on the tiled tensor).

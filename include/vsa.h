@@ -226,22 +226,45 @@ vsa_status vsa_pool_qkv(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf1
  * tokens instead of cubes, so no padded position is computed at all.
  *   q, k, v    [B, N, H, D] bf16 token layout (read).
  *   idx, k, order, scale   as in vsa_fine (idx NULL: dense; order then unused).
+ *   steps      vsa_schedule's output for this idx and order, or NULL (the
+ *              kernel then walks the selection itself, in index order).
  *   o_coarse   [B, H, C, D] float32, or NULL (no coarse term; g_coarse ignored).
  *   g_coarse, g_fine  [B, N, H] bf16 or NULL (g_coarse = 0, g_fine = 1).
  *   out        [B, N, H, D] bf16 (written at every real token).
  */
 vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
-                          const int32_t* idx, int32_t topk, const int32_t* order, float scale,
+                          const int32_t* idx, int32_t topk, const int32_t* order, const void* steps, float scale,
                           const float* o_coarse, const vsa_bf16* g_coarse, const vsa_bf16* g_fine,
                           vsa_bf16* out, vsa_stream_t stream);
+
+/* Bytes of the step list vsa_schedule writes for this shape and top-k. */
+size_t vsa_schedule_bytes(const vsa_shape* shape, int32_t topk);
+
+/*
+ * vsa_schedule — the fine stage's work, precomputed: for every group of four
+ * query cubes (four consecutive entries of `order`), the merged union of their
+ * selections, paired two key cubes per step, cubes that only the first two
+ * query cubes selected first, then those only the last two selected, then
+ * those both pairs selected (fewer half-used 128-row tiles).  The fine kernel
+ * given these steps does no list walking of its own; the result equals the
+ * kernel's own walk up to the order of the float32 sums.
+ *   idx, topk, order  as in vsa_fine (order may be NULL for 0..C-1).
+ *   steps             device buffer of vsa_schedule_bytes(shape, topk) (written).
+ * Returns VSA_ERR_UNSUPPORTED when its shared memory, 4 x (C/8 + 1 + 4 topk)
+ * 32-bit words, exceeds 48 KB (C = 624, topk = 32 needs 3.3 KB); vsa_forward
+ * then lets the fine kernel walk the selection itself.  A list that holds a
+ * cube twice is visited as often as it holds it.
+ */
+vsa_status vsa_schedule(const vsa_shape* shape, const int32_t* idx, int32_t topk, const int32_t* order,
+                        void* steps, vsa_stream_t stream);
 
 /* Bytes of device workspace vsa_forward needs for this shape and top-k
  * (0 for a malformed shape). */
 size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
 
 /*
- * vsa_forward — the whole attention call on one stream, as six launches:
- *   vsa_pool_qkv -> vsa_coarse (2) -> vsa_topk_order (2) -> vsa_fine_fused
+ * vsa_forward — the whole attention call on one stream, as seven launches:
+ *   vsa_pool_qkv -> vsa_coarse (2) -> vsa_topk_order (2) -> vsa_schedule -> vsa_fine_fused
  * (vsa_topk -> vsa_group instead when C > 2048; the grouping step is skipped
  * when C > 4096).  The result equals
  *   tile -> pool -> coarse -> topk -> group -> fine -> combine -> untile

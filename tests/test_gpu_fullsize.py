@@ -52,10 +52,15 @@ def run(request):
         err = fused - staged
         r["stage_close"] = bool(err.abs().max() <= 2e-2) and bool(err.norm() <= 5e-3 * staged.norm())
     else:
-        # identical selections and steps; only the staged path's bf16 rounding of O_f differs
-        ulp = lambda t: torch.exp2(torch.floor(torch.log2(t.abs().clamp_min(2.0 ** -100))) - 7)
-        of_tok = vsa.untile(o, s).float()
-        r["stage_close"] = bool(((fused - staged).abs() <= ulp(staged) + 0.5 * ulp(of_tok) + 1e-6).all())
+        # identical selections; the forward call's steps come in another (precomputed) order,
+        # so the oracle tolerance applies, per head
+        err = (fused - staged).float()
+        ok = True
+        for b in range(fused.shape[0]):
+            for h in range(fused.shape[2]):
+                e, ref = err[b, :, h], staged[b, :, h]
+                ok = ok and bool(e.abs().max() <= 2e-2) and bool(e.norm() <= 5e-3 * ref.norm())
+        r["stage_close"] = ok
     r["qt_rows"] = qt
     r["o_fine"] = o.cpu()
     r["lse"] = lse.cpu()

@@ -166,20 +166,23 @@ def test_forward_matches_the_stages_run_one_by_one(case):
     fused = from_dev(vsa.forward(dev["q"], dev["k"], dev["v"], s, w.topk, scale, gc, gf))
     assert np.array_equal(vsa.topk(vsa.coarse(*[vsa.pool(t, s) for t in (qt, kt, vt)], s, scale)[0], s,
                                    w.topk).cpu().numpy(), idx.cpu().numpy())
+    # the forward call walks its steps in a different order (precomputed, grouped by the tiles
+    # that use them; dense attention over blocks of consecutive real tokens), a different but
+    # equally valid summation order, so the oracle tolerance applies
+    for b in range(w.batch):
+        for h in range(w.heads):
+            check_close(fused[b, :, h], staged[b, :, h], f"forward vs stages[b={b},h={h}]")
+    # with the fine kernel's own walk (no precomputed steps) the two paths share every step,
+    # so they differ by at most the staged path's extra rounding of O_f (half a bf16 unit of
+    # O_f, times g_f <= 1) plus one unit of the result (the two final roundings)
     _, C = vsa.shape_info(s)
     if w.topk == C:
-        # every cube selected: the forward call attends over blocks of consecutive real tokens,
-        # a different but equally valid summation order, so the oracle tolerance applies
-        for b in range(w.batch):
-            for h in range(w.heads):
-                check_close(fused[b, :, h], staged[b, :, h], f"forward vs stages[b={b},h={h}]")
         return
-    # apart by at most the staged path's extra rounding of O_f (half a bf16 unit of O_f, times
-    # g_f <= 1) plus one unit of the result (the two final roundings)
+    walk = from_dev(vsa.fine_fused(dev["q"], dev["k"], dev["v"], s, idx, scale, order, oc, gc, gf))
     ulp = lambda a: 2.0 ** (np.floor(np.log2(np.maximum(np.abs(a), 2.0 ** -100))) - 7)
     of_tok = from_dev(vsa.untile(of, s))
     bound = ulp(staged) + 0.5 * ulp(of_tok) + 1e-6
-    assert np.all(np.abs(fused - staged) <= bound), "fused forward differs from the staged path beyond rounding"
+    assert np.all(np.abs(walk - staged) <= bound), "fused fine stage differs from the staged path beyond rounding"
 
 
 def _compare_call(w, dev, f64, k, scale, gates=True):
@@ -413,12 +416,14 @@ def test_fine_fused_sparse_matches_oracle(case):
     scale = 1 / math.sqrt(w.head_dim)
     ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, w.topk, scale, f64["g_coarse"], f64["g_fine"])
     idx = torch.from_numpy(ora["idx"]).cuda()
-    # fine output alone (no coarse term, g_fine = 1), written in token layout
-    got = from_dev(vsa.fine_fused(dev["q"], dev["k"], dev["v"], s, idx, scale))
+    # fine output alone (no coarse term, g_fine = 1), written in token layout, with the kernel's
+    # own walk and with precomputed steps
     ref = O.untile(ora["o_fine"], w.grid)
-    for b in range(w.batch):
-        for h in range(w.heads):
-            check_close(got[b, :, h], ref[b, :, h], f"fine_fused[b={b},h={h}]")
+    for steps in (None, vsa.schedule(idx, s)):
+        got = from_dev(vsa.fine_fused(dev["q"], dev["k"], dev["v"], s, idx, scale, steps=steps))
+        for b in range(w.batch):
+            for h in range(w.heads):
+                check_close(got[b, :, h], ref[b, :, h], f"fine_fused[b={b},h={h}] steps={steps is not None}")
     # with the oracle's coarse output and both gates: the whole merged result
     oc = torch.from_numpy(ora["o_coarse"].astype(np.float32)).cuda()
     got = from_dev(vsa.fine_fused(dev["q"], dev["k"], dev["v"], s, idx, scale, None, oc, dev["g_coarse"],
@@ -467,3 +472,58 @@ def test_topk_order_equals_topk_and_group(case):
             idx, order = vsa.topk_order(sc, s, k)
             assert torch.equal(idx, vsa.topk(sc, s, k)), k
             assert torch.equal(order, vsa.group(sc, s)), k
+
+
+def _decode_steps(raw: np.ndarray, items: int, stride: int):
+    e = raw.view(np.uint32).reshape(items, stride, 2)
+    a, b = (e[..., 0] & 0xFFFF).astype(np.int64), (e[..., 0] >> 16).astype(np.int64)
+    return a, b, (e[..., 1] & 0xFF).astype(np.int64), (e[..., 1] >> 31).astype(np.int64)
+
+
+def test_schedule_covers_every_selection_once(case):
+    """Bit-exact check of the precomputed steps: each item's steps visit every (query cube,
+    selected key cube) entry of its four lists exactly as often as the lists hold it, two key
+    cubes at most per step, tile-A-only cubes before tile-B-only cubes before shared ones,
+    ascending within each class, and the last flag only on the final step."""
+    w, _, dev, _ = case
+    s = _shape(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    scores, _ = vsa.coarse(*vsa.pool_qkv(dev["q"], dev["k"], dev["v"], s), s, scale)
+    _, C = vsa.shape_info(s)
+    k = w.topk
+    idx, order = vsa.topk_order(scores, s, k)
+    rng = np.random.default_rng(9)
+    dup = idx.cpu().numpy().copy()
+    if k >= 2:
+        dup[..., 1] = dup[..., 0]                       # duplicates must be visited twice
+    dup[..., -1] = np.where(rng.random(dup.shape[:-1]) < 0.2, C + 3, dup[..., -1])   # out of range: empty cube
+    for sel in (idx.cpu().numpy(), dup):
+        steps = vsa.schedule(torch.from_numpy(sel).cuda(), s, order).cpu().numpy()
+        groups = (C + 3) // 4
+        items, stride = w.batch * w.heads * groups, 2 * k
+        a, b, fl, last = _decode_steps(steps, items, stride)
+        o = order.cpu().numpy().reshape(-1, C)
+        for it in range(items):
+            bh, g = divmod(it, groups)
+            cubes = [o[bh, 4 * g + j] if 4 * g + j < C else -1 for j in range(4)]
+            want = {}
+            for j, c in enumerate(cubes):
+                if c < 0:
+                    continue
+                for kc in sel.reshape(-1, C, k)[bh, c]:
+                    key = (j, int(kc) if 0 <= kc < C else C)
+                    want[key] = want.get(key, 0) + 1
+            got, pats = {}, []
+            n = int(np.argmax(last[it] == 1)) + 1
+            assert last[it, :n].sum() == 1
+            for st in range(n):
+                for blk, f in ((a[it, st], fl[it, st] & 15), (b[it, st], fl[it, st] >> 4)):
+                    if blk == 0xFFFF:
+                        assert f == 0
+                        continue
+                    pats.append(((1 if f & 3 else 0) | (2 if f & 12 else 0), int(blk)))
+                    for j in range(4):
+                        if f >> j & 1:
+                            got[(j, int(blk))] = got.get((j, int(blk)), 0) + 1
+            assert got == want, it
+            assert pats == sorted(pats), it
