@@ -187,6 +187,27 @@ def pool_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     return outs[0], outs[1], outs[2]
 
 
+def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, shape: Shape, w_q: Optional[torch.Tensor] = None,
+                 w_k: Optional[torch.Tensor] = None, eps: float = 1e-6, theta: float = 10000.0,
+                 token_offset: int = 0, out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                 inplace: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Q/K RMSNorm over H*D then 3D RoPE of [B, n, H, D] rows of global tokens token_offset..+n-1.
+
+    Returns (q_out, k_out): new tensors, the given `out` pair, or q and k themselves when `inplace`."""
+    n = int(q.shape[1])
+    if inplace:
+        qo, ko = q, k
+    elif out is not None:
+        qo, ko = out
+    else:
+        qo, ko = torch.empty_like(q), torch.empty_like(k)
+    _check(_L.vsa_qk_norm_rope(ctypes.byref(shape.c()), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
+                               _ptr(w_q, torch.bfloat16, "w_q"), _ptr(w_k, torch.bfloat16, "w_k"), eps, theta,
+                               token_offset, n, _ptr(qo, torch.bfloat16, "q_out"), _ptr(ko, torch.bfloat16, "k_out"),
+                               _stream()))
+    return qo, ko
+
+
 def schedule(idx: torch.Tensor, shape: Shape, order: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Precomputed steps of the fine stage for the selection idx [B,H,C,k] (and work order)."""
     k = int(idx.shape[-1])

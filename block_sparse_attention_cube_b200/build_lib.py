@@ -25,7 +25,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libvsa_b200.so")
 
-SOURCES = ["vsa_api.cu", "vsa_layout.cu", "vsa_coarse.cu", "vsa_fine.cu", "vsa_noalloc.cu"]
+SOURCES = ["vsa_api.cu", "vsa_layout.cu", "vsa_coarse.cu", "vsa_fine.cu", "vsa_prenorm.cu", "vsa_noalloc.cu"]
 HEADERS = ["ptx_sm100.cuh", "vsa_internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -475,6 +475,50 @@ vsa_status vsa_schedule(const vsa_shape* shape, const int32_t* idx, int32_t topk
     return VSA_OK;
 }
 
+vsa_status vsa_qk_norm_rope(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* w_q,
+                            const vsa_bf16* w_k, float eps, float theta, int64_t token_offset, int64_t n_tokens,
+                            vsa_bf16* q_out, vsa_bf16* k_out, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    if (!(eps > 0.f) || !std::isfinite(eps)) return fail(VSA_ERR_INVALID_ARGUMENT, "eps must be finite and > 0");
+    if (!(theta > 1.f) || !std::isfinite(theta))
+        return fail(VSA_ERR_INVALID_ARGUMENT, "theta must be finite and > 1");
+    if (token_offset < 0 || n_tokens < 0)
+        return fail(VSA_ERR_INVALID_ARGUMENT, "token_offset and n_tokens must be >= 0");
+    if (static_cast<int64_t>(d.H) * d.D > kNormRopeMaxHD)
+        return fail(VSA_ERR_UNSUPPORTED, "vsa_qk_norm_rope needs H*D <= %d (got %d)", kNormRopeMaxHD, d.H * d.D);
+    if (n_tokens == 0) return VSA_OK;   // nothing to read or write
+    VSA_TRY(need_ptr(q, "q"));
+    VSA_TRY(need_ptr(k, "k"));
+    VSA_TRY(opt_ptr(w_q, "w_q"));
+    VSA_TRY(opt_ptr(w_k, "w_k"));
+    VSA_TRY(need_ptr(q_out, "q_out"));
+    VSA_TRY(need_ptr(k_out, "k_out"));
+    const size_t tb = static_cast<size_t>(d.B) * static_cast<size_t>(n_tokens) * d.H * d.D * 2;
+    const size_t wb = static_cast<size_t>(d.H) * d.D * 2;
+    // in place is q_out == q (and k_out == k); any other overlap is refused
+    const Range in_q{q, q == q_out ? 0 : tb, "q"}, in_k{k, k == k_out ? 0 : tb, "k"};
+    VSA_TRY(check_disjoint({in_q, in_k, {w_q, w_q ? wb : 0, "w_q"}, {w_k, w_k ? wb : 0, "w_k"}},
+                           {{q_out, tb, "q_out"}, {k_out, tb, "k_out"}}));
+    VSA_TRY(check_disjoint({{q_out, tb, "q_out"}}, {{k_out, tb, "k_out"}}));
+    if (q == q_out) VSA_TRY(check_disjoint({{q, tb, "q"}}, {{k_out, tb, "k_out"}}));
+    if (k == k_out) VSA_TRY(check_disjoint({{k, tb, "k"}}, {{q_out, tb, "q_out"}}));
+    VSA_TRY(check_device());
+    NormRopeArgs a{};
+    a.q = q;
+    a.k = k;
+    a.w_q = w_q;
+    a.w_k = w_k;
+    a.q_out = q_out;
+    a.k_out = k_out;
+    a.eps = eps;
+    a.theta = theta;
+    a.token_offset = token_offset;
+    a.n_tokens = n_tokens;
+    VSA_CUDA(launch_norm_rope(d, a, as_stream(stream)), "norm/rope launch");
+    return VSA_OK;
+}
+
 vsa_status vsa_pool_qkv(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
                         float* qbar, float* kbar, float* vbar, vsa_stream_t stream) {
     Dims d{};

@@ -102,6 +102,21 @@ bool schedule_supported(const Dims& d, int k);
 cudaError_t launch_schedule(const Dims& d, const int32_t* idx, int k, const int32_t* order, void* steps,
                             cudaStream_t s);
 
+// Pre-attention pass: Q/K RMSNorm over H*D channels, then 3D RoPE, on the
+// [B, n_tokens, H, D] rows of global tokens [token_offset, token_offset + n_tokens).
+struct NormRopeArgs {
+    const uint16_t* q;
+    const uint16_t* k;
+    const uint16_t* w_q;   // [H*D] or null (1)
+    const uint16_t* w_k;
+    uint16_t* q_out;       // may equal q
+    uint16_t* k_out;       // may equal k
+    float eps, theta;
+    int64_t token_offset, n_tokens;
+};
+constexpr int kNormRopeMaxHD = 8192;   // a lane holds at most 32 16-byte chunks of a row
+cudaError_t launch_norm_rope(const Dims& d, const NormRopeArgs& a, cudaStream_t s);
+
 // Cube mean-pool read straight from the projection layout [B, N, H, D]
 // (same fp32 summation order as launch_pool on the tiled tensor).
 cudaError_t launch_pool_tokens(const Dims& d, const uint16_t* const* x, float* const* xbar, int count,

@@ -204,6 +204,33 @@ vsa_status vsa_topk_order(const vsa_shape* shape, const float* scores, int32_t k
                           uint64_t* sig_scratch, vsa_stream_t stream);
 
 /*
+ * vsa_qk_norm_rope — the pre-attention pass of a Wan DiT block: RMSNorm of each
+ * token's query and key over all H*D channels, then the 3D rotary position
+ * embedding, in one read and one write of Q and K (WorldFoundry inference guide,
+ * "推理优化", exact-kernel table, row fused_rope; Wan2.2 teardown, zharfai.com,
+ * section "Fusion targets launch overhead and memory").
+ *   q, k           [B, n_tokens, H, D] bf16 (read): rows of global tokens
+ *                  token_offset .. token_offset + n_tokens - 1 (a sequence-
+ *                  parallel shard, or the whole sequence with offset 0).
+ *   w_q, w_k       [H*D] bf16 RMSNorm weights, or NULL (weight 1).
+ *   eps            > 0: y = x / sqrt(mean(x^2) + eps) * w, in float32.
+ *   theta          > 1: RoPE base.  The D/2 channel pairs (2i, 2i+1) of each
+ *                  head form three bands, for the token's t, x and y
+ *                  coordinates in that order (x and y floor(D/6) pairs each, t
+ *                  the rest); pair j of a band of P pairs turns by
+ *                  pos * theta^(-j/P) radians (angles in float64, rotation in
+ *                  float32), (a, b) -> (a cos - b sin, a sin + b cos).
+ *   q_out, k_out   [B, n_tokens, H, D] bf16 (written, rounded once); q_out may
+ *                  be q and k_out may be k (in place); no other overlap.
+ * Rows whose global token index is >= N (the padding that evens out shards)
+ * are written as zeros.  Needs H*D <= 8192 (VSA_ERR_UNSUPPORTED otherwise).
+ * With n_tokens = 0 nothing is read or written and the pointers may be NULL.
+ */
+vsa_status vsa_qk_norm_rope(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* w_q,
+                            const vsa_bf16* w_k, float eps, float theta, int64_t token_offset, int64_t n_tokens,
+                            vsa_bf16* q_out, vsa_bf16* k_out, vsa_stream_t stream);
+
+/*
  * vsa_pool_qkv — the cube mean-pool of vsa_pool applied to q, k and v in one
  * launch, read straight from the token layout (no tiled copy).  Each mean is
  * summed in the same float32 order as vsa_pool on the tiled tensor, so the two

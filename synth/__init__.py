@@ -174,3 +174,31 @@ def custom_workload(name: str, batch: int, heads: int, head_dim: int,
                     wid: int = 90) -> Workload:
     """A workload outside the named set (edge-case shapes for tests)."""
     return Workload(name, wid, batch, heads, head_dim, tuple(grid), topk, field)
+
+
+def make_projection_inputs(w: Workload, n_tokens: int | None = None, token_offset: int = 0) -> Dict[str, np.ndarray]:
+    """Raw (pre-normalisation) Q and K projections and RMSNorm weights for the pre-attention pass.
+
+    q_raw, k_raw: uint16 [B, n_tokens, H, D], the rows of global tokens token_offset .. +n_tokens-1
+    (rows past the grid, i.e. shard padding, are drawn like any other); w_q, w_k: uint16 [H*D].
+    Recipe: SeedSequence SEED_BASE + 100*wid + 50 + b spawns four children per batch element (Q row
+    scales, Q rows, K row scales, K rows); row r's scale is the r-th draw exp(0.7*N(0,1)) of its
+    scale stream and its H*D values the r-th block of its row stream, all float32, so a shard's rows
+    equal the same rows of the whole sequence; a row is its normals times its scale.  The weights
+    come from SeedSequence SEED_BASE + 100*wid + 49 as 1 + 0.25*N(0,1), Q's H*D values then K's.
+    All rounded to bf16 (RNE).  Meant for small and medium shapes (the draw is single-threaded)."""
+    n = w.tokens - token_offset if n_tokens is None else n_tokens
+    h, d = w.heads, w.head_dim
+    end = token_offset + n
+    out = {"q_raw": np.empty((w.batch, n, h, d), np.uint16), "k_raw": np.empty((w.batch, n, h, d), np.uint16)}
+    for b in range(w.batch):
+        kids = np.random.SeedSequence(SEED_BASE + 100 * (w.data_wid or w.wid) + 50 + b).spawn(4)
+        for key, s_scale, s_rows in (("q_raw", kids[0], kids[1]), ("k_raw", kids[2], kids[3])):
+            scale = np.exp(0.7 * _rng(s_scale).standard_normal(end, dtype=np.float32))[token_offset:]
+            x = _rng(s_rows).standard_normal((end, h * d), dtype=np.float32)[token_offset:]
+            out[key][b] = f32_to_bf16_bits(x * scale[:, None]).reshape(n, h, d)
+    s_w = np.random.SeedSequence(SEED_BASE + 100 * (w.data_wid or w.wid) + 49)
+    ww = 1.0 + 0.25 * _rng(s_w).standard_normal(2 * h * d, dtype=np.float32)
+    out["w_q"] = f32_to_bf16_bits(ww[:h * d])
+    out["w_k"] = f32_to_bf16_bits(ww[h * d:])
+    return out

@@ -134,3 +134,42 @@ def test_group_limits_checked_before_device():
     p = [ctypes.c_void_p((1 << 40) + i * (1 << 34)) for i in range(2)]
     assert vsa.raw_call("vsa_group", ctypes.byref(big), p[0], p[1], None) == UNSUPPORTED
     assert vsa.raw_call("vsa_group", ctypes.byref(s), None, p[1], None) == INVALID
+
+
+def _norm_rope_call(s, q, k, wq, wk, eps, theta, off, n, qo, ko):
+    return vsa.raw_call("vsa_qk_norm_rope", ctypes.byref(s), q, k, wq, wk, ctypes.c_float(eps), ctypes.c_float(theta),
+                        ctypes.c_int64(off), ctypes.c_int64(n), qo, ko, None)
+
+
+def _far(i):
+    return ctypes.c_void_p((1 << 40) + i * (1 << 32))
+
+
+@pytest.mark.parametrize("eps, theta, off, n, word", [
+    (0.0, 1e4, 0, 512, "eps"), (-1.0, 1e4, 0, 512, "eps"), (float("nan"), 1e4, 0, 512, "eps"),
+    (float("inf"), 1e4, 0, 512, "eps"), (1e-6, 1.0, 0, 512, "theta"), (1e-6, float("nan"), 0, 512, "theta"),
+    (1e-6, 1e4, -1, 512, "token_offset"), (1e-6, 1e4, 0, -5, "n_tokens")])
+def test_norm_rope_bad_scalars(eps, theta, off, n, word):
+    s = _shape()
+    st = _norm_rope_call(s, _far(0), _far(1), None, None, eps, theta, off, n, _far(2), _far(3))
+    assert st == INVALID and word in vsa.last_error()
+
+
+def test_norm_rope_pointer_checks():
+    s = _shape()
+    assert _norm_rope_call(s, None, _far(1), None, None, 1e-6, 1e4, 0, 8, _far(2), _far(3)) == INVALID
+    assert _norm_rope_call(s, _far(0), _far(1), ctypes.c_void_p((1 << 40) + 8), None, 1e-6, 1e4, 0, 8, _far(2),
+                           _far(3)) == MISALIGNED
+    # outputs may not overlap another tensor (only q_out == q and k_out == k are allowed)
+    st = _norm_rope_call(s, _far(0), _far(1), None, None, 1e-6, 1e4, 0, 8, _far(1), _far(3))
+    assert st == INVALID and "overlap" in vsa.last_error()
+    st = _norm_rope_call(s, _far(0), _far(1), None, None, 1e-6, 1e4, 0, 8, _far(2), _far(2))
+    assert st == INVALID and "overlap" in vsa.last_error()
+    st = _norm_rope_call(s, _far(0), _far(1), None, None, 1e-6, 1e4, 0, 8, _far(0), _far(0))
+    assert st == INVALID and "overlap" in vsa.last_error()
+
+
+def test_norm_rope_row_width_limit():
+    s = vsa.Shape(1, 65, 128, (4, 4, 4)).c()   # H*D = 8320 > 8192
+    st = _norm_rope_call(s, _far(0), _far(1), None, None, 1e-6, 1e4, 0, 64, _far(2), _far(3))
+    assert st == UNSUPPORTED and "H*D" in vsa.last_error()
