@@ -317,6 +317,22 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         del bars, scores, oc, idx, order, steps
     stage_ms = {n: round(statistics.mean(v), 4) for n, v in acc.items()}
 
+    # ---- the pre-attention pass (Q/K RMSNorm + 3D RoPE) on the same Q/K, timed on its own
+    wts = synth.make_projection_inputs(synth.custom_workload("weights", 1, w.heads, w.head_dim, (1, 1, 1), 1))
+    w_q, w_k = (torch.from_numpy(wts[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("w_q", "w_k"))
+    q_n, k_n = torch.empty_like(d["q"]), torch.empty_like(d["k"])
+    pre = []
+    for it in range(args.warmup + args.steps):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        vsa.qk_norm_rope(d["q"], d["k"], s, w_q, w_k, out=(q_n, k_n))
+        e[1].record(stream)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            pre.append(e[0].elapsed_time(e[1]))
+    pre_ms = reduce_max(statistics.mean(pre), world)
+    del q_n, k_n
+
     # ---- end to end through vsa_forward_host (pinned host buffers, copies inside the timed region)
     h = {k: v.cpu().pin_memory() for k, v in d.items()}
     h_out = torch.empty_like(h["q"]).pin_memory()
@@ -340,6 +356,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         return
     peaks, peaks_src = load_peaks()
     bf16_peak = float(peaks["bf16_tflops"])
+    hbm_peak = float(peaks["hbm_gbs"])
+    pre_bytes = 4 * w.batch * w.tokens * w.heads * w.head_dim * 2
     fine_flops = executed_fine_flops(w.batch, w.heads, npad, w.topk, w.head_dim)
     nblk = (w.tokens + 63) // 64   # dense attention walks blocks of 64 consecutive real tokens
     dense_flops = dense_equivalent_flops(w.batch, w.heads, 64 * nblk, w.head_dim)
@@ -377,6 +395,11 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                      "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)" if peaks_src == "measured"
                      else "fallback 1.59 PFLOP/s", "traffic": traffic,
                      "per_launch": "4*B*H*Npad*k*64*D executed flops (64x64 cube tiles of the k selected cubes)"},
+        "pre_attention": {"api": "vsa_qk_norm_rope (Q/K RMSNorm over H*D + 3D RoPE), timed on its own, not in value",
+                          "ms": round(pre_ms, 4), "bytes": pre_bytes, "bound": "hbm",
+                          "achieved_gbps": round(pre_bytes / (pre_ms * 1e-3) / 1e9, 1), "peak_gbps": hbm_peak,
+                          "frac": round(pre_bytes / (pre_ms * 1e-3) / 1e9 / hbm_peak, 4),
+                          "per_launch": "Q and K read once and written once: 4*B*N*H*D*2 bytes"},
         "e2e": {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "vsa_forward_host (pinned host q/k/v/gates in, host out)"},
         "gpu_launches": 9 * args.steps,   # VSA: pool, coarse (2), top-k, order sort, schedule, fine; dense: fine
