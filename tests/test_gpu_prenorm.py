@@ -137,3 +137,21 @@ def test_norm_rope_then_attention_matches_oracle():
     for h in range(w.heads):
         e = got[0, :, h] - ref[0, :, h]
         assert np.abs(e).max() <= 2e-2 and np.linalg.norm(e) <= 5e-3 * np.linalg.norm(ref[0, :, h]), h
+
+
+def test_sharded_forward_on_one_rank_is_the_plain_call():
+    """block_sparse_attention_cube_b200.sharding with one rank: the pre-attention pass at token offset 0
+    then the call on every head, bit-identical to calling the two entry points directly."""
+    from block_sparse_attention_cube_b200 import sharding as S
+    w = synth.WORKLOADS["padded_7x15x16"]
+    s = _shape(w)
+    x = synth.make_projection_inputs(w)
+    base = synth.make_inputs(w)
+    q, k, v = _dev(x["q_raw"]), _dev(x["k_raw"]), _dev(base["v"])
+    gc, gf = _dev(base["g_coarse"]), _dev(base["g_fine"])
+    wq, wk = _dev(x["w_q"]), _dev(x["w_k"])
+    scale = 1 / math.sqrt(w.head_dim)
+    got = S.sharded_forward(q, k, v, s, w.topk, scale, gc, gf, norm_rope={"w_q": wq, "w_k": wk})
+    qn, kn = vsa.qk_norm_rope(q, k, s, wq, wk)
+    ref = vsa.forward(qn, kn, v, s, w.topk, scale, gc, gf)
+    assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
