@@ -389,7 +389,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         "dense_fine": {"executed_tflop": round(dense_flops / 1e12, 3), "tflops": round(dense_tflops, 1),
                        "frac_bf16_peak": round(dense_tflops / bf16_peak, 4),
                        "per_launch": "4*B*H*(64*ceil(N/64))^2*D: blocks of 64 real tokens, no padding"},
-        "roofline": {"kernel": "fine_kernel<128, cubes, fused> (VSA, top-k 32)", "bound": "tensor",
+        "roofline": {"kernel": "fine_tile_kernel<128, cubes> (VSA, top-k 32)", "bound": "tensor",
                      "achieved": round(fine_tflops, 2),
                      "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(fine_tflops / bf16_peak, 4),
                      "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)" if peaks_src == "measured"
@@ -402,7 +402,9 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                           "per_launch": "Q and K read once and written once: 4*B*N*H*D*2 bytes"},
         "e2e": {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "vsa_forward_host (pinned host q/k/v/gates in, host out)"},
-        "gpu_launches": 9 * args.steps,   # VSA: pool, coarse (2), top-k, order sort, schedule, fine; dense: fine
+        # VSA: pool, coarse (2), top-k, order sort, schedule, fine (one-tile kernel) and the re-run guard
+        # (fine_kernel, which returns at once unless the one-tile kernel overflowed); dense: fine
+        "gpu_launches": 10 * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
         "context": {"pages_dense_call_ms_b200": 17.0, "pages_vsa_kernel_ms_b200_k78": 4.719,

@@ -121,7 +121,7 @@ size_t order_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C 
 constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Workspace of vsa_forward: qbar | kbar | vbar | o_coarse | scores | idx | order | sig | steps.
+// Workspace of vsa_forward: qbar | kbar | vbar | o_coarse | scores | idx | order | sig | steps | overflow.
 // Q, K and V are read in the caller's [B, N, H, D] layout (the fine stage
 // gathers cubes with TMA), so no tiled copies are kept.  With every cube
 // selected the fine stage is dense attention and needs none of it; the
@@ -132,6 +132,7 @@ struct Carve {
     int32_t* order;
     uint64_t* sig;   // work-order signatures, when top-k computes them (C <= kTopkRegMaxC)
     void* steps;     // the fine stage's precomputed steps (when schedule_supported)
+    int* overflow;   // the fine stage's overflow word
     size_t bytes;
 };
 
@@ -158,6 +159,7 @@ Carve carve(const Dims& d, int k, bool coarse_gate, void* ws) {
         if (d.C <= kTopkRegMaxC) c.sig = reinterpret_cast<uint64_t*>(take(2 * order_bytes(d)));
         if (schedule_supported(d, k)) c.steps = take(schedule_bytes(d, k));
     }
+    c.overflow = reinterpret_cast<int*>(take(sizeof(int)));
     c.bytes = off > kAlign ? off : kAlign;
     return c;
 }
@@ -190,8 +192,9 @@ vsa_status check_k(const Dims& d, int32_t k) {
 vsa_status run_fine_fused(const Dims& d, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                           const int32_t* idx, int topk, const int32_t* order, const void* steps, float scale,
                           const float* o_coarse, const uint16_t* gc, const uint16_t* gf, uint16_t* out,
-                          cudaStream_t s) {
+                          int* overflow, cudaStream_t s) {
     FineArgs a{};
+    a.overflow = overflow;
     a.mode = idx ? kFineCubesFused : kFineTokensFused;
     a.q = q;
     a.k = k;
@@ -248,7 +251,7 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
         steps = c.steps;
     }
     return run_fine_fused(d, q, k, v, sparse ? c.idx : nullptr, topk, order, steps, scale, gc ? c.oc : nullptr, gc,
-                          gf, out, s);
+                          gf, out, c.overflow, s);
 }
 
 }  // namespace
@@ -568,7 +571,7 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
                             {g_coarse, g_coarse ? gb : 0, "g_coarse"}, {g_fine, g_fine ? gb : 0, "g_fine"}},
                            {{out, tb, "out"}}));
     VSA_TRY(check_device());
-    return run_fine_fused(d, q, k, v, idx, topk, order, steps, scale, o_coarse, g_coarse, g_fine, out,
+    return run_fine_fused(d, q, k, v, idx, topk, order, steps, scale, o_coarse, g_coarse, g_fine, out, nullptr,
                           as_stream(stream));
 }
 

@@ -82,6 +82,7 @@
 namespace vsa {
 
 __device__ int g_vsa_status;   // watchdog word (VSA_OK or VSA_ERR_TIMEOUT)
+__device__ int g_vsa_overflow;   // fine_tile_kernel's overflow word for callers without a workspace
 
 namespace {
 
@@ -143,7 +144,8 @@ struct FineParams {
     int nblk;               // blocks per head: C (cube modes) or ceil(N / 64) (token mode)
     int C, Ct, Cx, Cy, T, X, Y;
     int64_t N;
-    int ngroups;            // ceil(nblk / 4)
+    int group;              // query blocks per work item: 4 (two tiles, fine_kernel) or 2 (one tile, fine_tile_kernel)
+    int ngroups;            // ceil(nblk / group)
     uint64_t magic_cxcy;    // floor(2^48 / (Cx*Cy)) + 1: exact j / (Cx*Cy) for j < 2^24
     uint64_t magic_cy;      // floor(2^48 / Cy) + 1
     uint64_t magic_cx;      // floor(2^48 / Cx) + 1
@@ -154,13 +156,15 @@ struct FineParams {
     float c_log2;           // scale * log2(e)
     int* status;
     uint64_t limit_ns;
+    int* overflow;          // fine_tile_kernel: set to 1 when a probability bound was exceeded (or nullptr)
+    const int* run_if;      // fine_kernel: return at once unless *run_if != 0 (or nullptr: always run)
 };
 
 __device__ __forceinline__ uint32_t div_magic(uint32_t j, uint64_t magic) {
     return static_cast<uint32_t>((static_cast<uint64_t>(j) * magic) >> 48);
 }
 
-// The four query blocks of one work item (slot j < 0 when absent).
+// The query blocks of one work item (slot j < 0 when absent; slots past p.group are absent).
 struct Item {
     int64_t bh;
     int b, h;
@@ -177,9 +181,9 @@ __device__ __forceinline__ Item decode_item(int64_t it, const FineParams& p) {
     r.present = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const int pos = 4 * g + j;
+        const int pos = p.group * g + j;
         int c = -1;
-        if (pos < p.nblk) {
+        if (j < p.group && pos < p.nblk) {
             c = p.order ? __ldg(p.order + r.bh * p.C + pos) : pos;
             if (c < 0 || c >= p.nblk) c = -1;
         }
@@ -467,6 +471,8 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const uint32_t base = (raw_u32 + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_u32);
 
+    // a re-run launched behind fine_tile_kernel does nothing unless that kernel's probabilities overflowed
+    if (p.run_if != nullptr && *p.run_if == 0) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto bar = [&](int i) -> uint32_t { return base + kOffBar + 8u * static_cast<uint32_t>(i); };
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffMisc);
@@ -898,6 +904,453 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
 }
 
+// ====================================================================== one-tile kernel
+// fine_tile_kernel: the fused fine stage with one 128-row tile per work item
+// (two query blocks) and three score buffers in tensor memory, so that three
+// steps of the same tile are in flight at once: while one group of softmax
+// warps turns step i's scores into probabilities, the tensor core computes
+// the scores of steps i+1 and i+2 into the other two buffers.  Two threads
+// issue the MMAs, one the QK^T products (S) and one the PV products, because
+// one thread issues an M128N128K16 MMA only every ~95 cycles, against ~68 for
+// the tensor core to run it.
+//
+// Roles (480 threads): warps 0-11 are three softmax groups of four warps
+// (group g owns score buffer g and takes the steps s with s % 3 == g; warp
+// 4g + q reads TMEM lane quarter q); warp 12 issues TMA (the tile's Q, then
+// per step two K blocks through a 3-deep ring and two V blocks through a
+// 2-deep ring); warp 13 allocates tensor memory and issues S(s) into buffer
+// s % 3 once PV(s - 3) has drained it; warp 14 issues PV(s) into the output
+// accumulator once group s % 3 has stored P(s).
+//
+// Tensor memory: buffers at columns 0, 128 and 256 (128 fp32 scores for a
+// step's 128 keys; P, as bf16 pairs, over the first 64 columns), the output
+// accumulator at 384.
+//
+// Softmax with a fixed maximum per row (Wan2.2 teardown, zharfai.com, section
+// "Fixed-max softmax is a numerical contract"): the maximum of a row's first
+// selected scores is kept for the whole item, so the three groups need no
+// exchange per step; each keeps its own partial row sum and the epilogue adds
+// the three.  A probability above 2^64 (a later score far above the first
+// maximum) or a non-finite sum raises the overflow word, and the caller then
+// runs fine_kernel, whose online maximum is rescaled per step, over the whole
+// stage again: the teardown's guard that re-runs a tile with online rescaling.
+constexpr int kTThreads = 480;
+constexpr int kTTmaWarp = 12;
+constexpr int kTSWarp = 13;
+constexpr int kTPVWarp = 14;
+constexpr int kTBufs = 3;
+constexpr int kTKStages = 3;
+constexpr int kTVStages = 2;
+constexpr uint32_t kTOffQ = 0;                                   // one tile: 128 rows x 256 B
+constexpr uint32_t kTOffK = kTOffQ + kQTileBytes;                // [kTKStages]
+constexpr uint32_t kTOffV = kTOffK + kTKStages * kKVBytes;       // [kTVStages]
+constexpr uint32_t kTOffM = kTOffV + kTVStages * kKVBytes;       // [128] each row's fixed maximum
+constexpr uint32_t kTOffL = kTOffM + 128 * 4;                    // [kTBufs][128] each group's row sums
+constexpr uint32_t kTOffBar = kTOffL + kTBufs * 128 * 4;
+constexpr int kTBarQFull = 0;
+constexpr int kTBarQEmpty = 1;
+constexpr int kTBarKFull = 2;                                    // [kTKStages]
+constexpr int kTBarKEmpty = kTBarKFull + kTKStages;
+constexpr int kTBarVFull = kTBarKEmpty + kTKStages;             // [kTVStages]
+constexpr int kTBarVEmpty = kTBarVFull + kTVStages;
+constexpr int kTBarSFull = kTBarVEmpty + kTVStages;             // [kTBufs]
+constexpr int kTBarPFull = kTBarSFull + kTBufs;                  // [kTBufs], four arrivals
+constexpr int kTBarPVDone = kTBarPFull + kTBufs;                 // [kTBufs]
+constexpr int kTBarMReady = kTBarPVDone + kTBufs;                // [2 query blocks], two arrivals
+constexpr int kTBarEpi = kTBarMReady + 2;                        // twelve arrivals
+constexpr int kTBarOFree = kTBarEpi + 1;                         // twelve arrivals
+constexpr int kTBarDrain = kTBarOFree + 1;                       // [2 issuers]
+constexpr int kTNumBars = kTBarDrain + 2;
+constexpr uint32_t kTOffMisc = kTOffBar + kTNumBars * 8;         // tmem slot (4 B) + abort flag (4 B)
+constexpr uint32_t kTSmemBytes = kTOffMisc + 16 + 1024;
+constexpr uint32_t kTColO = 384;
+static_assert(kTSmemBytes <= 232448, "shared memory over the 227 KB per-block limit");
+
+// Step s of item it: computed (dense) or read from the precomputed list.
+__device__ __forceinline__ StepRec tile_step(const FineParams& p, int64_t it, int s, uint32_t present) {
+    if (p.idx == nullptr) return dense_step(s, present, p.nblk);
+    StepRec r = decode_step(__ldg(p.steps + it * p.steps_stride + s));
+    r.ca = min(r.ca, p.C);
+    r.cb = min(r.cb, p.C);
+    if (s + 1 >= p.steps_stride) r.last = 1u;
+    return r;
+}
+
+template <int D, int LM>
+__global__ void __launch_bounds__(kTThreads, 1)
+fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const FineParams p) {
+    static_assert(LM == kLoadCubes || LM == kLoadTokens, "token-layout inputs only");
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t base = (raw_u32 + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_u32);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto bar = [&](int i) -> uint32_t { return base + kTOffBar + 8u * static_cast<uint32_t>(i); };
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kTOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kTOffMisc + 4);
+    float* m_row = reinterpret_cast<float*>(smem + kTOffM);
+    float* l_part = reinterpret_cast<float*>(smem + kTOffL);
+    const BoundedWait bw{abort_flag, p.status, p.limit_ns};
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bar(kTBarQFull), 1);
+        mbar_init(bar(kTBarQEmpty), 1);
+        for (int s = 0; s < kTKStages; ++s) {
+            mbar_init(bar(kTBarKFull + s), 1);
+            mbar_init(bar(kTBarKEmpty + s), 1);
+        }
+        for (int s = 0; s < kTVStages; ++s) {
+            mbar_init(bar(kTBarVFull + s), 1);
+            mbar_init(bar(kTBarVEmpty + s), 1);
+        }
+        for (int b = 0; b < kTBufs; ++b) {
+            mbar_init(bar(kTBarSFull + b), 1);
+            mbar_init(bar(kTBarPFull + b), 4);    // the four warps of group b
+            mbar_init(bar(kTBarPVDone + b), 1);
+        }
+        mbar_init(bar(kTBarMReady + 0), 2);       // the two warps of a query block's lane quarters
+        mbar_init(bar(kTBarMReady + 1), 2);
+        mbar_init(bar(kTBarEpi), 12);
+        mbar_init(bar(kTBarOFree), 12);
+        mbar_init(bar(kTBarDrain + 0), 1);
+        mbar_init(bar(kTBarDrain + 1), 1);
+        fence_mbar_init();
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    if (warp == kTSWarp) {
+        tmem_alloc(base + kTOffMisc, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    constexpr uint32_t kBytesQ = 2u * 64u * D * 2u;   // one tile's Q
+    constexpr uint32_t kBytesKV = 2u * 64u * D * 2u;  // one step's two K (or V) blocks
+    auto drain_wait = [&](uint32_t b, uint32_t par) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(b, par) && globaltimer() - t0 < kDrainLimitNs) {
+        }
+    };
+
+    if (warp == kTTmaWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t q_issued = 0, k_issued[kTKStages] = {}, v_issued[kTVStages] = {};
+            RingPos kp{0, 0}, vp{0, 0};
+            int n_item = 0;
+            bool ok = true;
+            for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
+                const Item item = decode_item(it, p);
+                auto load_pair = [&](const CUtensorMap* m, uint32_t dst, int ja, int jb, uint32_t b) {
+                    load_block<LM, D>(m, dst, ja, 0, b, item, p);
+                    load_block<LM, D>(m, dst + 8192, jb, 0, b, item, p);
+                    if (D == 128) {
+                        load_block<LM, D>(m, dst + 16384, ja, 64, b, item, p);
+                        load_block<LM, D>(m, dst + 24576, jb, 64, b, item, p);
+                    }
+                };
+                if (!(ok = bw.wait(bar(kTBarQEmpty), (n_item & 1) ^ 1))) break;
+                mbar_arrive_expect_tx(bar(kTBarQFull), kBytesQ);
+                ++q_issued;
+                load_pair(&tm_q, base + kTOffQ, item.blk[0], item.blk[1], bar(kTBarQFull));
+                for (int s = 0;; ++s) {
+                    const StepRec r = tile_step(p, it, s, item.present);
+                    if (!(ok = bw.wait(bar(kTBarKEmpty + kp.slot), kp.phase ^ 1u))) break;
+                    mbar_arrive_expect_tx(bar(kTBarKFull + kp.slot), kBytesKV);
+                    ++k_issued[kp.slot];
+                    load_pair(&tm_k, base + kTOffK + kp.slot * kKVBytes, r.ca, r.cb, bar(kTBarKFull + kp.slot));
+                    kp.advance<kTKStages>();
+                    if (!(ok = bw.wait(bar(kTBarVEmpty + vp.slot), vp.phase ^ 1u))) break;
+                    mbar_arrive_expect_tx(bar(kTBarVFull + vp.slot), kBytesKV);
+                    ++v_issued[vp.slot];
+                    load_pair(&tm_v, base + kTOffV + vp.slot * kKVBytes, r.ca, r.cb, bar(kTBarVFull + vp.slot));
+                    vp.advance<kTVStages>();
+                    if (r.last) break;
+                }
+            }
+            if (!ok) {
+                // wait for this CTA's own copies still in flight before exiting
+                if (q_issued) drain_wait(bar(kTBarQFull), (q_issued - 1u) & 1u);
+                for (int s = 0; s < kTKStages; ++s)
+                    if (k_issued[s]) drain_wait(bar(kTBarKFull + s), (k_issued[s] - 1u) & 1u);
+                for (int s = 0; s < kTVStages; ++s)
+                    if (v_issued[s]) drain_wait(bar(kTBarVFull + s), (v_issued[s] - 1u) & 1u);
+            }
+        }
+    } else if (warp == kTSWarp) {
+        // ------------------------------------------------------------ S = Q K^T issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);   // Q (K-major) x K^T (K-major)
+            const uint64_t fix_k = smem_desc_sw128(0, 16u, 1024u);         // K-major, 8-row groups 1 KB apart
+            RingPos kp{0, 0};
+            uint32_t uses[kTBufs] = {0u, 0u, 0u};   // S issued into each buffer so far
+            int n_item = 0;
+            bool ok = true, issued_any = false;
+            for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
+                const uint32_t present = decode_item(it, p).present;
+                if (!(ok = bw.wait(bar(kTBarQFull), n_item & 1))) break;
+                for (int s = 0;; ++s) {
+                    const StepRec r = tile_step(p, it, s, present);
+                    const int b = s % kTBufs;
+                    // the buffer's previous P must have been read by its PV
+                    if (uses[b] > 0 && !(ok = bw.wait(bar(kTBarPVDone + b), (uses[b] - 1u) & 1u))) break;
+                    if (!(ok = bw.wait(bar(kTBarKFull + kp.slot), kp.phase))) break;
+                    tc_fence_after();
+                    const uint32_t qa = base + kTOffQ, kb = base + kTOffK + kp.slot * kKVBytes;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                        mma_bf16_ss(tmem + 128u * b, desc_at(fix_k, qa + off), desc_at(fix_k, kb + off), idesc_s,
+                                    kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(kTBarSFull + b));
+                    mma_commit(bar(kTBarKEmpty + kp.slot));
+                    issued_any = true;
+                    ++uses[b];
+                    kp.advance<kTKStages>();
+                    if (r.last) break;
+                }
+                if (!ok) break;
+                mma_commit(bar(kTBarQEmpty));
+            }
+            if (issued_any) {
+                mma_commit(bar(kTBarDrain + 0));
+                drain_wait(bar(kTBarDrain + 0), 0u);
+            }
+        }
+    } else if (warp == kTPVWarp) {
+        // ------------------------------------------------------------ O += P V issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, 0, 1);     // P (TMEM, K-major) x V (MN-major)
+            const uint64_t fix_v = smem_desc_sw128(0, 16384u, 1024u);      // MN-major, d halves 16 KB apart
+            RingPos vp{0, 0};
+            uint32_t waits[kTBufs] = {0u, 0u, 0u};   // P-full phases consumed per buffer
+            int n_item = 0;
+            bool ok = true, issued_any = false;
+            for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
+                const uint32_t present = decode_item(it, p).present;
+                for (int s = 0;; ++s) {
+                    const StepRec r = tile_step(p, it, s, present);
+                    const int b = s % kTBufs;
+                    // the item's first PV overwrites O: the previous item's epilogue must have read it
+                    if (s == 0 && n_item > 0 && !(ok = bw.wait(bar(kTBarOFree), (n_item - 1) & 1))) break;
+                    if (!(ok = bw.wait(bar(kTBarPFull + b), waits[b] & 1u))) break;
+                    ++waits[b];
+                    if (!(ok = bw.wait(bar(kTBarVFull + vp.slot), vp.phase))) break;
+                    tc_fence_after();
+                    const uint32_t vb = base + kTOffV + vp.slot * kKVBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16_ts(tmem + kTColO, tmem + 128u * b + 8u * kk, desc_at(fix_v, vb + kk * 2048u), idesc_o,
+                                    (s > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(bar(kTBarPVDone + b));
+                    mma_commit(bar(kTBarVEmpty + vp.slot));
+                    issued_any = true;
+                    vp.advance<kTVStages>();
+                    if (r.last) break;
+                }
+                if (!ok) break;
+            }
+            if (issued_any) {
+                mma_commit(bar(kTBarDrain + 1));
+                drain_wait(bar(kTBarDrain + 1), 0u);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax groups + epilogue
+        const int g = warp >> 2;                 // group: score buffer g, steps s with s % 3 == g
+        const int q = warp & 3;                  // TMEM lane quarter
+        const int row = q * 32 + lane;           // query row of the tile, 0..127
+        const int slot = q >> 1;                 // query block of the row
+        const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
+        const uint32_t tS = tmem + 128u * g + lane_addr;
+        const uint32_t tO = tmem + kTColO + lane_addr;
+        const float c = p.c_log2;
+        uint32_t n_s = 0;                         // S-full phases consumed (buffer g)
+        uint32_t pvd[kTBufs] = {0u, 0u, 0u};      // PVs into each buffer so far, all steps of all items
+        bool ok = true;
+        auto wait_all = [&](uint32_t b, uint32_t par) -> bool {
+            const bool mine = bw.wait(b, par);
+            return __all_sync(0xffffffffu, mine);
+        };
+        int n_item = 0;
+        for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
+            const Item item = decode_item(it, p);
+            float m = 0.f, l = 0.f;
+            bool have_m = false;
+            int sfirst = -1;     // first step that selects this row's query block (the same in every warp)
+            int last_b = 0;
+            for (int s = 0;; ++s) {
+                const StepRec r = tile_step(p, it, s, item.present);
+                const bool sel_a = ((r.flags >> slot) & 1u) != 0u, sel_b = ((r.flags >> (4 + slot)) & 1u) != 0u;
+                if (sfirst < 0 && (sel_a || sel_b)) sfirst = s;
+                const int b = s % kTBufs;
+                ++pvd[b];
+                last_b = b;
+                if (b == g) {
+                    if (!(ok = wait_all(bar(kTBarSFull + g), n_s & 1u))) break;
+                    ++n_s;
+                    tc_fence_after();
+                    if (sel_a || sel_b) {
+                        // warp-uniform: this warp's rows belong to one query block
+                        const uint64_t vm_a = sel_a ? key_mask<LM>(r.ca, p) : 0ull;
+                        const uint64_t vm_b = sel_b ? key_mask<LM>(r.cb, p) : 0ull;
+                        if (s == sfirst) {
+                            // the row's first selected scores fix its maximum for the item
+                            float mx = -INFINITY;
+#pragma unroll 1
+                            for (int ch = 0; ch < 4; ++ch) {
+                                uint32_t sc[32];
+                                tmem_ld32_wait(tS + 32u * ch, sc);
+                                const uint64_t vm = ch < 2 ? vm_a : vm_b;
+                                mask32(sc, static_cast<uint32_t>(vm >> (32 * (ch & 1))));
+                                mx = fmaxf(mx, max32(sc));
+                            }
+                            m = mx == -INFINITY ? 0.f : mx * c;
+                            m_row[row] = m;
+                            have_m = true;
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar(kTBarMReady + slot));   // release: m_row visible
+                        } else if (!have_m) {
+                            if (!(ok = wait_all(bar(kTBarMReady + slot), n_item & 1))) break;
+                            m = m_row[row];
+                            have_m = true;
+                        }
+                        float sum = 0.f;
+#pragma unroll 1
+                        for (int ch = 0; ch < 4; ++ch) {
+                            uint32_t sc[32];
+                            tmem_ld32_wait(tS + 32u * ch, sc);
+                            const uint64_t vm = ch < 2 ? vm_a : vm_b;
+                            mask32(sc, static_cast<uint32_t>(vm >> (32 * (ch & 1))));
+                            uint32_t pk[16];
+                            sum += probs32(sc, c, m, pk);
+                            // P of keys 32ch.. over columns 16ch..: scores there were already read
+                            tmem_st16(tS + 16u * ch, pk);
+                        }
+                        if (!(sum <= kSumLimit) && p.overflow != nullptr) *p.overflow = 1;
+                        l += sum;
+                    } else {
+                        // neither key block is selected by this row's query block: P = 0
+                        uint32_t z[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) z[j] = 0u;
+                        tmem_st32(tS, z);
+                        tmem_st32(tS + 32u, z);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(kTBarPFull + g));
+                }
+                if (r.last) break;
+            }
+            if (!ok) break;
+            // one arrival per item and query block on its max-ready barrier: when no step selects
+            // the block, group 0's two warps of the block make it
+            if (sfirst < 0 && g == 0) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kTBarMReady + slot));
+            }
+            // ---------------- epilogue: all three groups' sums, the item's last PV complete
+            l_part[g * 128 + row] = l;
+            if (!(ok = wait_all(bar(kTBarPVDone + last_b), (pvd[last_b] - 1u) & 1u))) break;
+            tc_fence_after();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kTBarEpi));
+            if (!(ok = wait_all(bar(kTBarEpi), n_item & 1))) break;
+            const float l_tot = (l_part[row] + l_part[128 + row]) + l_part[256 + row];
+            const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
+            const int blk = item.blk[slot];
+            const int o_ = row & 63;
+            int64_t tok = -1;
+            int cube = 0;
+            if (blk >= 0) {
+                if (LM == kLoadTokens) {
+                    tok = 64ll * blk + o_;
+                    if (tok >= p.N) {
+                        tok = -1;
+                    } else if (p.o_coarse != nullptr) {
+                        const int64_t xy = static_cast<int64_t>(p.X) * p.Y;
+                        const int tt = static_cast<int>(tok / xy);
+                        const int rem = static_cast<int>(tok - tt * xy);
+                        const int xx = rem / p.Y, yy = rem - (rem / p.Y) * p.Y;
+                        cube = ((tt >> 2) * p.Cx + (xx >> 2)) * p.Cy + (yy >> 2);
+                    }
+                } else {
+                    const uint32_t qd = div_magic(static_cast<uint32_t>(blk), p.magic_cy);
+                    const uint32_t ct = div_magic(qd, p.magic_cx);
+                    const int cy = blk - static_cast<int>(qd) * p.Cy;
+                    const int cx = static_cast<int>(qd) - static_cast<int>(ct) * p.Cx;
+                    const int tt = 4 * static_cast<int>(ct) + (o_ >> 4);
+                    const int xx = 4 * cx + ((o_ >> 2) & 3), yy = 4 * cy + (o_ & 3);
+                    if (tt < p.T && xx < p.X && yy < p.Y) tok = (static_cast<int64_t>(tt) * p.X + xx) * p.Y + yy;
+                    cube = blk;
+                }
+            }
+            const bool store = tok >= 0;
+            float gc = 0.f, gf = 1.f;
+            const float* ocr = nullptr;
+            const int64_t grow = (static_cast<int64_t>(item.b) * p.N + (store ? tok : 0)) * p.H + item.h;
+            if (store) {
+                if (p.g_coarse) gc = __uint_as_float(static_cast<uint32_t>(__ldg(p.g_coarse + grow)) << 16);
+                if (p.g_fine) gf = __uint_as_float(static_cast<uint32_t>(__ldg(p.g_fine + grow)) << 16);
+                if (p.o_coarse) ocr = p.o_coarse + (item.bh * p.C + cube) * D;
+            }
+            const float sf = gf * inv_l;
+            // channel chunks of 32: D = 128 -> group 0 takes 0 and 1, group 1 takes 2, group 2 takes 3;
+            // D = 64 -> groups 0 and 1 take one each
+            const int ch0 = D == 128 ? (g == 0 ? 0 : g + 1) : g;
+            const int ch1 = D == 128 ? (g == 0 ? 2 : g + 2) : (g < 2 ? g + 1 : g);
+#pragma unroll 1
+            for (int ch = ch0; ch < ch1; ++ch) {
+                uint32_t o[32];
+                tmem_ld32_wait(tO + 32u * ch, o);
+                if (store) {
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(o[j]) * sf;
+                    if (ocr != nullptr) {
+                        const float4* oc4 = reinterpret_cast<const float4*>(ocr + 32 * ch);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 cv = __ldg(oc4 + j);
+                            v[4 * j] = fmaf(gc, cv.x, v[4 * j]);
+                            v[4 * j + 1] = fmaf(gc, cv.y, v[4 * j + 1]);
+                            v[4 * j + 2] = fmaf(gc, cv.z, v[4 * j + 2]);
+                            v[4 * j + 3] = fmaf(gc, cv.w, v[4 * j + 3]);
+                        }
+                    }
+                    uint32_t w16[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) w16[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                    uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + 32 * ch);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        dst[v4] = make_uint4(w16[4 * v4], w16[4 * v4 + 1], w16[4 * v4 + 2], w16[4 * v4 + 3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kTBarOFree));   // O may be overwritten by the next item
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kTSWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
 // Steps of one work item by the serial three-pass walk (TileWalk), written by
 // one thread: the general case, which also visits repeated entries of a list
 // as often as they appear.
@@ -953,7 +1406,7 @@ __host__ __device__ __forceinline__ int schedule_words(int C) { return (C + 8) >
 __global__ void __launch_bounds__(kScheduleWarps * 32) schedule_kernel(const FineParams p, uint2* __restrict__ steps) {
     extern __shared__ uint32_t sched_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int W = schedule_words(p.C), E = 4 * p.k;
+    const int W = schedule_words(p.C), E = p.group * p.k;
     uint32_t* nib = sched_smem + static_cast<int64_t>(warp) * (W + E);
     uint32_t* ent = nib + W;
     const int64_t it = static_cast<int64_t>(blockIdx.x) * kScheduleWarps + warp;
@@ -1124,6 +1577,22 @@ cudaError_t launch_instance(const CUtensorMap& tq, const CUtensorMap& tk, const 
     return cudaGetLastError();
 }
 
+template <int D, int LM>
+cudaError_t launch_tile_instance(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                 const FineParams& p, int grid, cudaStream_t s) {
+    static int done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!(dev >= 0 && dev < 64 && done[dev])) {
+        cudaError_t e = cudaFuncSetAttribute(fine_tile_kernel<D, LM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kTSmemBytes));
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) done[dev] = 1;
+    }
+    fine_tile_kernel<D, LM><<<grid, kTThreads, kTSmemBytes, s>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
 uint64_t magic48(uint32_t d) { return ((uint64_t{1} << 48) / d) + 1; }
 
 // Real offsets o = (t%4)*16 + (x%4)*4 + y%4 of a cube whose extent along one
@@ -1153,9 +1622,23 @@ int* status_word() {
     return ptrs[dev];
 }
 
+int* overflow_word() {
+    static std::mutex mu;
+    static int* ptrs[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_vsa_overflow) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<int*>(a);
+    }
+    return ptrs[dev];
+}
+
 namespace {
 
-FineParams make_params(const Dims& d, const FineArgs& a) {
+FineParams make_params(const Dims& d, const FineArgs& a, int group) {
     const int mode = a.mode;
     FineParams p{};
     p.idx = a.idx;
@@ -1179,7 +1662,8 @@ FineParams make_params(const Dims& d, const FineArgs& a) {
     p.X = d.X;
     p.Y = d.Y;
     p.N = d.N;
-    p.ngroups = (p.nblk + 3) / 4;
+    p.group = group;
+    p.ngroups = (p.nblk + group - 1) / group;
     p.magic_cxcy = magic48(static_cast<uint32_t>(d.Cx * d.Cy));
     p.magic_cy = magic48(static_cast<uint32_t>(d.Cy));
     p.magic_cx = magic48(static_cast<uint32_t>(d.Cx));
@@ -1198,13 +1682,13 @@ FineParams make_params(const Dims& d, const FineArgs& a) {
 }  // namespace
 
 size_t schedule_bytes(const Dims& d, int k) {
-    const int64_t items = static_cast<int64_t>(d.B) * d.H * ((d.C + 3) / 4);
+    const int64_t items = static_cast<int64_t>(d.B) * d.H * ((d.C + kTileGroup - 1) / kTileGroup);
     return static_cast<size_t>(items) * static_cast<size_t>(schedule_stride(k)) * sizeof(uint2);
 }
 
 namespace {
 size_t schedule_smem(const Dims& d, int k) {
-    return static_cast<size_t>(kScheduleWarps) * (static_cast<size_t>(schedule_words(d.C)) + 4ull * k) * 4u;
+    return static_cast<size_t>(kScheduleWarps) * (static_cast<size_t>(schedule_words(d.C)) + kTileGroup * k) * 4u;
 }
 }  // namespace
 
@@ -1220,7 +1704,7 @@ cudaError_t launch_schedule(const Dims& d, const int32_t* idx, int k, const int3
     a.idx = idx;
     a.k_sel = k;
     a.order = order;
-    const FineParams p = make_params(d, a);
+    const FineParams p = make_params(d, a, kTileGroup);
     const int64_t blocks = (p.items + kScheduleWarps - 1) / kScheduleWarps;
     if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidValue;
     if (blocks == 0) return cudaSuccess;
@@ -1247,7 +1731,40 @@ cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const 
         if (why) *why = "cuTensorMapEncodeTiled failed for a Q/K/V tensor";
         return cudaErrorInvalidValue;
     }
-    FineParams p = make_params(d, a);
+    // sparse selections with precomputed steps run on the one-tile kernel (shorter items, no
+    // four-list union); dense attention stays on fine_kernel, whose two tiles share each K/V step
+    const bool tile = mode == kFineCubesFused && a.steps != nullptr;
+    if (tile) {
+        // the one-tile kernel, then fine_kernel over the whole stage only if its fixed maxima overflowed
+        int* ovf = a.overflow ? a.overflow : overflow_word();
+        if (!ovf) {
+            if (why) *why = "overflow word unavailable";
+            return cudaErrorInvalidValue;
+        }
+        FineParams pt = make_params(d, a, kTileGroup);
+        if (!pt.status) {
+            if (why) *why = "watchdog word unavailable";
+            return cudaErrorInvalidValue;
+        }
+        pt.overflow = ovf;
+        cudaError_t e = cudaMemsetAsync(ovf, 0, sizeof(int), s);
+        if (e != cudaSuccess) return e;
+        const int gt = static_cast<int>(pt.items < sm_count() ? pt.items : sm_count());
+        if (gt > 0) {
+            e = d.D == 128 ? launch_tile_instance<128, kLoadCubes>(tq, tk, tv, pt, gt, s)
+                           : launch_tile_instance<64, kLoadCubes>(tq, tk, tv, pt, gt, s);
+            if (e != cudaSuccess) return e;
+        }
+        FineArgs ar = a;
+        ar.steps = nullptr;   // the re-run walks the selection itself
+        FineParams pr = make_params(d, ar, 4);
+        pr.run_if = ovf;
+        const int gr = static_cast<int>(pr.items < sm_count() ? pr.items : sm_count());
+        if (gr <= 0) return cudaSuccess;
+        return d.D == 128 ? launch_instance<128, kLoadCubes, true>(tq, tk, tv, pr, gr, s)
+                          : launch_instance<64, kLoadCubes, true>(tq, tk, tv, pr, gr, s);
+    }
+    FineParams p = make_params(d, a, 4);
     if (!p.status) {
         if (why) *why = "watchdog word unavailable";
         return cudaErrorInvalidValue;

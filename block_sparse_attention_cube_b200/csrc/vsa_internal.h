@@ -31,6 +31,10 @@ int sm_count();
 // Watchdog word of the current device (device address, cached per device).
 int* status_word();
 
+// Overflow word of the current device for fused fine-stage calls made without
+// a workspace (device address, cached per device).
+int* overflow_word();
+
 // Upper bound on any device-side wait, in nanoseconds.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
@@ -80,6 +84,7 @@ struct FineArgs {
     int k_sel;
     const int32_t* order;   // [B, H, C] or null
     const void* steps;      // precomputed steps (launch_schedule) or null: the kernel walks the selection
+    int* overflow;          // device word the one-tile kernel raises on overflow (null: a per-device word)
     float scale;
     uint16_t* out;
     float* lse;             // kFineTiled only
@@ -91,12 +96,14 @@ struct FineArgs {
 cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const char** why);
 
 // Precomputed steps of the fine stage's work items for a sparse selection
-// (idx [B, H, C, k], order [B, H, C] or null): 8 bytes per step, at most
-// 2k steps per item of four query cubes.  Cube indices travel in 16 bits, so
-// the fine kernel takes steps for C <= kScheduleMaxC; launch_schedule also
-// needs its shared memory (four warps x (C/8 + 1 + 4k) words) within 48 KB.
+// (idx [B, H, C, k], order [B, H, C] or null): a work item is a pair of query
+// cubes (consecutive entries of the order), one 128-row tile; 8 bytes per
+// step, at most k steps per item.  Cube indices travel in 16 bits, so the
+// fine kernel takes steps for C <= kScheduleMaxC; launch_schedule also needs
+// its shared memory (four warps x (C/8 + 1 + 2k) words) within 48 KB.
+constexpr int kTileGroup = 2;
 constexpr int kScheduleMaxC = 65534;
-inline int64_t schedule_stride(int k) { return 2ll * k; }
+inline int64_t schedule_stride(int k) { return k; }
 size_t schedule_bytes(const Dims& d, int k);
 bool schedule_supported(const Dims& d, int k);
 cudaError_t launch_schedule(const Dims& d, const int32_t* idx, int k, const int32_t* order, void* steps,

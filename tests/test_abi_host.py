@@ -111,16 +111,18 @@ def test_workspace_checks():
 def test_workspace_size_480p_matches_layout():
     # Q, K, V are read in place, so the workspace holds only the pooled q,k,v and o_coarse
     # (4 x 624*40*128*4 B), the scores (624*624*40*4 B), idx (624*40*32*4 B) and the work order
-    # (624*40*4 B) with its signatures (624*40*8 B) and the fine stage's steps, each rounded up to 256 B
+    # (624*40*4 B) with its signatures (624*40*8 B), the fine stage's steps and its overflow word, each
+    # rounded up to 256 B
     s = vsa.Shape(1, 40, 128, (21, 30, 52)).c()
     up = lambda n: (n + 255) // 256 * 256
     expect = 4 * up(624 * 40 * 128 * 4) + up(624 * 624 * 40 * 4) + up(624 * 40 * 32 * 4) + up(624 * 40 * 4) \
         + up(624 * 40 * 8) \
-        + up(156 * 40 * 64 * 8)   # work-order signatures; fine-stage steps: 156 groups x 2k steps x 8 B
+        + up(312 * 40 * 32 * 8) \
+        + up(4)   # work-order signatures; steps: 312 pairs of query cubes x k steps x 8 B; overflow word
     assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 32) == expect
     # every cube selected: dense attention; the coarse buffers are for a coarse gate only
     assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 624) == 4 * up(624 * 40 * 128 * 4) + \
-        up(624 * 624 * 40 * 4)
+        up(624 * 624 * 40 * 4) + up(4)
 
 
 def test_probe_limit_checked_before_device():

@@ -280,6 +280,35 @@ def test_overflow_scores_stay_finite():
     assert np.abs(from_dev(lse)[:, :, valid] - r_lse[:, :, valid]).max() <= LSE_ABS
 
 
+@pytest.mark.parametrize("dense", [False, True])
+def test_overflow_scores_through_the_forward_call(dense):
+    """The fused call on the same scaled inputs: its fixed per-row maxima overflow, so the call
+    re-runs the fine stage with the online rescaling kernel; the result must match the oracle."""
+    w = synth.WORKLOADS["padded_7x15x16"]
+    x = synth.make_inputs(w)
+    for n in ("q", "k"):
+        x[n] = synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(x[n]) * 16.0)
+    f64 = {k: O.bf16_to_f64(v) for k, v in x.items()}
+    dev = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).cuda() for k, v in x.items()}
+    s = _shape(w)
+    _, C = vsa.shape_info(s)
+    k = C if dense else w.topk
+    scale = 1 / math.sqrt(w.head_dim)
+    got = from_dev(vsa.forward(dev["q"], dev["k"], dev["v"], s, k, scale, None if dense else dev["g_coarse"],
+                               None if dense else dev["g_fine"]))
+    assert np.isfinite(got).all()
+    if dense:
+        ref, lse = O.dense(f64["q"], f64["k"], f64["v"], w.grid, scale)
+        assert lse.max() > 100
+    else:
+        ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, k, scale, f64["g_coarse"], f64["g_fine"])
+        ref = ora["out"]
+    for b in range(w.batch):
+        for h in range(w.heads):
+            check_close(got[b, :, h], ref[b, :, h], f"forward(overflow)[b={b},h={h}]")
+    vsa.device_status()
+
+
 def test_padded_key_rows_are_masked():
     """Large finite values written into the padded rows of the tiled K do not change the result."""
     w = synth.WORKLOADS["padded_7x15x16"]
@@ -481,10 +510,10 @@ def _decode_steps(raw: np.ndarray, items: int, stride: int):
 
 
 def test_schedule_covers_every_selection_once(case):
-    """Bit-exact check of the precomputed steps: each item's steps visit every (query cube,
-    selected key cube) entry of its four lists exactly as often as the lists hold it, two key
-    cubes at most per step, tile-A-only cubes before tile-B-only cubes before shared ones,
-    ascending within each class, and the last flag only on the final step."""
+    """Bit-exact check of the precomputed steps: each item (a pair of query cubes) visits every
+    (query cube, selected key cube) entry of its two lists exactly as often as the lists hold it,
+    two key cubes at most per step, in ascending cube order, and the last flag only on the final
+    step."""
     w, _, dev, _ = case
     s = _shape(w)
     scale = 1 / math.sqrt(w.head_dim)
@@ -499,13 +528,13 @@ def test_schedule_covers_every_selection_once(case):
     dup[..., -1] = np.where(rng.random(dup.shape[:-1]) < 0.2, C + 3, dup[..., -1])   # out of range: empty cube
     for sel in (idx.cpu().numpy(), dup):
         steps = vsa.schedule(torch.from_numpy(sel).cuda(), s, order).cpu().numpy()
-        groups = (C + 3) // 4
-        items, stride = w.batch * w.heads * groups, 2 * k
+        groups = (C + 1) // 2   # a work item is a pair of query cubes (one 128-row tile)
+        items, stride = w.batch * w.heads * groups, k
         a, b, fl, last = _decode_steps(steps, items, stride)
         o = order.cpu().numpy().reshape(-1, C)
         for it in range(items):
             bh, g = divmod(it, groups)
-            cubes = [o[bh, 4 * g + j] if 4 * g + j < C else -1 for j in range(4)]
+            cubes = [o[bh, 2 * g + j] if 2 * g + j < C else -1 for j in range(2)]
             want = {}
             for j, c in enumerate(cubes):
                 if c < 0:
