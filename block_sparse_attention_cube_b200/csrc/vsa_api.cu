@@ -245,6 +245,8 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
             }
         }
     }
+    if (sparse && order != nullptr && pair_order_supported(d, topk))
+        VSA_CUDA(launch_pair_order(d, c.idx, topk, c.order, s), "pair launch");
     const void* steps = nullptr;
     if (sparse && c.steps != nullptr) {
         VSA_CUDA(launch_schedule(d, c.idx, topk, order, c.steps, s), "schedule launch");
@@ -451,6 +453,21 @@ vsa_status vsa_topk_order(const vsa_shape* shape, const float* scores, int32_t k
     VSA_TRY(check_device());
     VSA_CUDA(launch_topk_sig(d, scores, k, idx, sig_scratch, as_stream(stream)), "topk launch");
     VSA_CUDA(launch_group_sort(d, sig_scratch, order, as_stream(stream)), "group launch");
+    return VSA_OK;
+}
+
+vsa_status vsa_pair_order(const vsa_shape* shape, const int32_t* idx, int32_t topk, int32_t* order,
+                          vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(check_k(d, topk));
+    VSA_TRY(need_ptr(idx, "idx"));
+    VSA_TRY(need_ptr(order, "order"));
+    if (!pair_order_supported(d, topk))
+        return fail(VSA_ERR_UNSUPPORTED, "vsa_pair_order supports C <= 1120 (got C=%d)", d.C);
+    VSA_TRY(check_disjoint({{idx, idx_bytes(d, topk), "idx"}}, {{order, order_bytes(d), "order"}}));
+    VSA_TRY(check_device());
+    VSA_CUDA(launch_pair_order(d, idx, topk, order, as_stream(stream)), "pair launch");
     return VSA_OK;
 }
 

@@ -480,4 +480,203 @@ cudaError_t launch_group_sort(const Dims& d, const uint64_t* sig, int32_t* order
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- pairing
+// The fine stage takes consecutive pairs of the work order as its 128-row
+// tiles, and a tile's steps are the union of its two selections.  After the
+// signature sort, pair_order_kernel re-pairs the order: it counts, for every
+// position p and each of the kPairWin positions after it, how many selected
+// key cubes the two query cubes share (popcounts of per-cube selection
+// bitmaps in shared memory, so C is bounded by that memory: C <= 1120); then,
+// for kPairRounds rounds, every unpaired position proposes to its best
+// unpaired neighbour within kPairWin positions (more shared cubes first, then
+// the nearer, then the earlier), and mutual proposals pair up.  The pairs are
+// written in the order of their first member, leftovers paired in order of
+// position (an odd one out last), if they share more key cubes in total than
+// the input's consecutive pairs, leftover pairs more than kPairWin apart
+// counting as sharing none (otherwise the input order stays).  One block per
+// (b, h).  A cube listed twice in a row counts once; any input gives a
+// permutation.
+constexpr int kPairWin = 16;
+constexpr int kPairMaxC = 1120;   // selection bitmaps and scan arrays within 220 KB of shared memory
+constexpr int kPairRounds = 8;
+constexpr int kPairThreads = 512;
+
+__global__ void __launch_bounds__(kPairThreads) pair_order_kernel(int C, int k, const int32_t* __restrict__ idx,
+                                                                  int32_t* __restrict__ order) {
+    extern __shared__ __align__(16) uint8_t pair_smem[];
+    const int nw = (C + 31) / 32;                                  // bitmap words per cube
+    uint32_t* bits = reinterpret_cast<uint32_t*>(pair_smem);       // [C][nw] selections of the cube at position p
+    int32_t* ord = reinterpret_cast<int32_t*>(bits + static_cast<size_t>(C) * nw);   // [C] cube at position p
+    int16_t* partner = reinterpret_cast<int16_t*>(ord + C);        // [C] partner position or -1
+    int16_t* best = partner + C;                                   // [C] this round's proposal
+    uint8_t* ov = reinterpret_cast<uint8_t*>(best + C);            // [C][2 kPairWin] shared-cube counts
+    int* urank = reinterpret_cast<int*>(ov + static_cast<size_t>(C) * 2 * kPairWin);   // [C] rank among the unmatched
+    int* upos = urank + C;                                         // [C] position of the u-th unmatched
+    int* scan = upos + C;                                          // [C] pair slot of a pair's first position
+    const int64_t bh = blockIdx.x;
+    const int32_t* I = idx + bh * static_cast<int64_t>(C) * k;
+    int32_t* O = order + bh * static_cast<int64_t>(C);
+    for (int p = threadIdx.x; p < C; p += blockDim.x) {
+        ord[p] = O[p];
+        partner[p] = -1;
+    }
+    for (int i = threadIdx.x; i < C * nw; i += blockDim.x) bits[i] = 0u;
+    for (int i = threadIdx.x; i < C * 2 * kPairWin; i += blockDim.x) ov[i] = 0;
+    __syncthreads();
+    for (int t = threadIdx.x; t < C * k; t += blockDim.x) {
+        const int p = t / k, i = t - p * k;
+        const int cp = ord[p];
+        if (cp < 0 || cp >= C) continue;
+        const int v = __ldg(I + static_cast<int64_t>(cp) * k + i);
+        if (v >= 0 && v < C) atomicOr(bits + static_cast<size_t>(p) * nw + (v >> 5), 1u << (v & 31));
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < C * kPairWin; t += blockDim.x) {
+        const int p = t / kPairWin, dd = t - p * kPairWin + 1;
+        if (p + dd >= C) continue;
+        const uint32_t* ra = bits + static_cast<size_t>(p) * nw;
+        const uint32_t* rb = bits + static_cast<size_t>(p + dd) * nw;
+        int o = 0;
+        for (int w = 0; w < nw; ++w) o += __popc(ra[w] & rb[w]);
+        const uint8_t o8 = static_cast<uint8_t>(o < 255 ? o : 255);
+        ov[p * 2 * kPairWin + kPairWin + dd - 1] = o8;             // neighbour p + dd
+        ov[(p + dd) * 2 * kPairWin + kPairWin - dd] = o8;          // neighbour (p + dd) - dd
+    }
+    for (int r = 0; r < kPairRounds; ++r) {
+        __syncthreads();
+        for (int p = threadIdx.x; p < C; p += blockDim.x) {
+            int bq = -1, bs = -1;
+            if (partner[p] < 0) {
+                for (int dd = 1; dd <= kPairWin; ++dd) {
+#pragma unroll
+                    for (int side = 0; side < 2; ++side) {
+                        const int q = side ? p + dd : p - dd;
+                        if (q < 0 || q >= C || partner[q] >= 0) continue;
+                        const int slot = side ? kPairWin + dd - 1 : kPairWin - dd;
+                        const int score = static_cast<int>(ov[p * 2 * kPairWin + slot]) * 64 + (kPairWin - dd);
+                        if (score > bs) {
+                            bs = score;
+                            bq = q;
+                        }
+                    }
+                }
+            }
+            best[p] = static_cast<int16_t>(bq);
+        }
+        __syncthreads();
+        for (int p = threadIdx.x; p < C; p += blockDim.x) {
+            const int q = best[p];
+            if (q >= 0 && best[q] == p) partner[p] = static_cast<int16_t>(q);
+        }
+    }
+    __syncthreads();
+    // Output.  A position starts a pair when it is matched to a later position, or when it is the
+    // 2u-th unmatched position (paired with the (2u+1)-th); a block-wide scan of those flags gives
+    // each pair its slot.  The pairs are kept if they share more key cubes in total than the
+    // input's consecutive pairs (leftover pairs more than kPairWin apart count as sharing none).
+    __shared__ int warp_sum[kPairThreads / 32];
+    __shared__ int totals[2];
+    // exclusive block-wide scan of a[0, C) in place; returns the total
+    auto scan_in_place = [&](int* a) -> int {
+        int carry = 0;
+        for (int base0 = 0; base0 < C; base0 += blockDim.x) {
+            const int p = base0 + threadIdx.x;
+            const int f = p < C ? a[p] : 0;
+            int incl = f;
+            const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (lane == 31) warp_sum[wid] = incl;
+            __syncthreads();
+            if (wid == 0) {
+                const int v = lane < static_cast<int>(blockDim.x >> 5) ? warp_sum[lane] : 0;
+                int vi = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, vi, o);
+                    if (lane >= o) vi += y;
+                }
+                if (lane < static_cast<int>(blockDim.x >> 5)) warp_sum[lane] = vi - v;   // exclusive warp offsets
+                if (lane == 31) totals[1] = vi;
+            }
+            __syncthreads();
+            if (p < C) a[p] = carry + warp_sum[wid] + incl - f;
+            carry += totals[1];
+            __syncthreads();
+        }
+        return carry;
+    };
+    // unmatched positions: their rank u among the unmatched, and the position of each rank
+    for (int p = threadIdx.x; p < C; p += blockDim.x) urank[p] = partner[p] < 0 ? 1 : 0;
+    __syncthreads();
+    const int n_unm = scan_in_place(urank);
+    for (int p = threadIdx.x; p < C; p += blockDim.x)
+        if (partner[p] < 0) upos[urank[p]] = p;
+    // pair starts and their slots; with an odd number of unmatched positions the last of them is
+    // left alone and goes to the end of the order
+    for (int p = threadIdx.x; p < C; p += blockDim.x)
+        scan[p] = (partner[p] > p || (partner[p] < 0 && (urank[p] & 1) == 0 && urank[p] + 1 < n_unm)) ? 1 : 0;
+    __syncthreads();
+    scan_in_place(scan);
+    if (threadIdx.x == 0) totals[0] = 0;
+    __syncthreads();
+    int my_new = 0, my_old = 0;
+    for (int p = threadIdx.x; p < C; p += blockDim.x) {
+        const int q = partner[p];
+        int mate = -1;
+        if (q > p) mate = q;
+        else if (q < 0 && (urank[p] & 1) == 0 && urank[p] + 1 < n_unm) mate = upos[urank[p] + 1];
+        if (mate > p && mate - p <= kPairWin) my_new += ov[p * 2 * kPairWin + kPairWin + (mate - p) - 1];
+        if ((p & 1) == 0 && p + 1 < C) my_old += ov[p * 2 * kPairWin + kPairWin];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        my_new += __shfl_xor_sync(0xffffffffu, my_new, o);
+        my_old += __shfl_xor_sync(0xffffffffu, my_old, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        atomicAdd(&totals[0], my_new - my_old);
+    }
+    __syncthreads();
+    if (totals[0] > 0) {
+        for (int p = threadIdx.x; p < C; p += blockDim.x) {
+            const int q = partner[p];
+            const bool unm_start = q < 0 && (urank[p] & 1) == 0 && urank[p] + 1 < n_unm;
+            if (q > p || unm_start) {
+                const int slot = 2 * scan[p];   // < C - 1: every pair before it fills two entries
+                O[slot] = ord[p];
+                O[slot + 1] = q > p ? ord[q] : ord[upos[urank[p] + 1]];
+            } else if (q < 0 && urank[p] == n_unm - 1 && (n_unm & 1)) {
+                O[C - 1] = ord[p];              // the lone leftover
+            }
+        }
+    }
+}
+
+size_t pair_smem_bytes(int C) {
+    return static_cast<size_t>(C) * ((C + 31) / 32) * 4 + static_cast<size_t>(C) * (4 + 2 + 2 + 2 * kPairWin + 12);
+}
+
+cudaError_t launch_pair_order(const Dims& d, const int32_t* idx, int k, int32_t* order, cudaStream_t s) {
+    if (!pair_order_supported(d, k)) return cudaErrorInvalidValue;
+    const size_t smem = pair_smem_bytes(d.C);
+    static int done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!(dev >= 0 && dev < 64 && done[dev])) {
+        cudaError_t e = cudaFuncSetAttribute(pair_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) done[dev] = 1;
+    }
+    pair_order_kernel<<<d.B * d.H, kPairThreads, smem, s>>>(d.C, k, idx, order);
+    return cudaGetLastError();
+}
+
+bool pair_order_supported(const Dims& d, int k) {
+    return k >= 1 && d.C <= kPairMaxC && pair_smem_bytes(d.C) <= 220 * 1024;
+}
+
 }  // namespace vsa

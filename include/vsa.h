@@ -264,6 +264,28 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
                           const float* o_coarse, const vsa_bf16* g_coarse, const vsa_bf16* g_fine,
                           vsa_bf16* out, vsa_stream_t stream);
 
+/*
+ * vsa_pair_order — re-pairs a work order for the fine stage, whose 128-row
+ * tiles are consecutive pairs of order entries and whose steps are the union
+ * of a pair's two selections (a schedule, not a step of the method).  For
+ * every position p and each of the 16 positions after it, the kernel counts
+ * the key cubes the two query cubes both selected; then, for 8 rounds, each
+ * unpaired position proposes to its best unpaired neighbour within 16
+ * positions (more shared cubes, then nearer, then earlier) and mutual
+ * proposals pair up.  Pairs are written in the order of their first member,
+ * the leftovers paired in order of position (an odd one out last), if they
+ * share more key cubes in total than the input's consecutive pairs (leftover
+ * pairs more than 16 positions apart counted as sharing none); otherwise the
+ * order is left as is.
+ *   idx    [B, H, C, k] int32 (read): a cube listed twice in a row counts
+ *          once; entries outside [0, C) are ignored.
+ *   order  [B, H, C] int32 (read and rewritten in place): a work order.
+ * Supported for C <= 1120 (its selections are held as bitmaps in shared
+ * memory; VSA_ERR_UNSUPPORTED otherwise).
+ */
+vsa_status vsa_pair_order(const vsa_shape* shape, const int32_t* idx, int32_t topk, int32_t* order,
+                          vsa_stream_t stream);
+
 /* Bytes of the step list vsa_schedule writes for this shape and top-k. */
 size_t vsa_schedule_bytes(const vsa_shape* shape, int32_t topk);
 
@@ -290,10 +312,11 @@ vsa_status vsa_schedule(const vsa_shape* shape, const int32_t* idx, int32_t topk
 size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
 
 /*
- * vsa_forward — the whole attention call on one stream, as seven launches:
- *   vsa_pool_qkv -> vsa_coarse (2) -> vsa_topk_order (2) -> vsa_schedule -> vsa_fine_fused
+ * vsa_forward — the whole attention call on one stream, as nine launches:
+ *   vsa_pool_qkv -> vsa_coarse (2) -> vsa_topk_order (2) -> vsa_pair_order -> vsa_schedule
+ *   -> vsa_fine_fused (the one-tile kernel and its re-run guard)
  * (vsa_topk -> vsa_group instead when C > 2048; the grouping step is skipped
- * when C > 4096).  The result equals
+ * when C > 4096, the pairing when C > 1120).  The result equals
  *   tile -> pool -> coarse -> topk -> group -> fine -> combine -> untile
  * up to the bf16 rounding of O_fine that the staged path makes.
  * When topk == C every cube is selected and the fine stage is dense attention
