@@ -290,11 +290,11 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     dense_ms_max = reduce_max(dense_ms, world)
 
     # ---- per-stage breakdown: the launches of vsa_forward, one by one through the entry points
-    names = ["pool", "coarse", "topk_order", "pair", "schedule", "fine"]
+    names = ["pool", "coarse", "topk_order", "schedule", "fine"]
     acc = {n: [] for n in names}
     acc["fine_dense"] = []
     for it in range(args.warmup + args.steps):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(9)]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
         e[0].record(stream)
         bars = vsa.pool_qkv(d["q"], d["k"], d["v"], s)
         e[1].record(stream)
@@ -302,20 +302,18 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         e[2].record(stream)
         idx, order = vsa.topk_order(scores, s, w.topk)
         e[3].record(stream)
-        vsa.pair_order(idx, s, order)
-        e[4].record(stream)
         steps = vsa.schedule(idx, s, order)
-        e[5].record(stream)
+        e[4].record(stream)
         vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, order, oc, d["g_coarse"], d["g_fine"], out=out,
                        steps=steps)
-        e[6].record(stream)
+        e[5].record(stream)
         vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out_d)
-        e[7].record(stream)
+        e[6].record(stream)
         torch.cuda.synchronize()
         if it >= args.warmup:
             for j, n in enumerate(names):
                 acc[n].append(e[j].elapsed_time(e[j + 1]))
-            acc["fine_dense"].append(e[6].elapsed_time(e[7]))
+            acc["fine_dense"].append(e[5].elapsed_time(e[6]))
         del bars, scores, oc, idx, order, steps
     stage_ms = {n: round(statistics.mean(v), 4) for n, v in acc.items()}
 
@@ -404,9 +402,9 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                           "per_launch": "Q and K read once and written once: 4*B*N*H*D*2 bytes"},
         "e2e": {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "vsa_forward_host (pinned host q/k/v/gates in, host out)"},
-        # VSA: pool, coarse (2), top-k, order sort, pairing, schedule, fine (one-tile kernel) and the re-run
-        # guard (fine_kernel, which returns at once unless the one-tile kernel overflowed); dense: fine
-        "gpu_launches": 11 * args.steps,
+        # VSA: pool, coarse (2), top-k, order sort, schedule, fine (one-tile kernel) and the re-run guard
+        # (fine_kernel, which returns at once unless the one-tile kernel overflowed); dense: fine
+        "gpu_launches": 10 * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
         "context": {"pages_dense_call_ms_b200": 17.0, "pages_vsa_kernel_ms_b200_k78": 4.719,

@@ -245,8 +245,6 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
             }
         }
     }
-    if (sparse && order != nullptr && pair_order_supported(d, topk))
-        VSA_CUDA(launch_pair_order(d, c.idx, topk, c.order, s), "pair launch");
     const void* steps = nullptr;
     if (sparse && c.steps != nullptr) {
         VSA_CUDA(launch_schedule(d, c.idx, topk, order, c.steps, s), "schedule launch");

@@ -239,9 +239,12 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(int64_t rows, int C, int
 // j % 32, slot j / 32), for C <= 32 * KPL.  The k-th largest key T is built
 // bit by bit from the top with warp sums (redux) of per-lane counts; the row
 // is then scanned in index order exactly as topk_kernel does, so both give
-// the same selection.  When `sig` is non-null the row's work-order signature
-// (its three best key cubes, see group_kernel) is written as well, from the
-// same registers.
+// the same selection.  When `sig` is non-null the row's work-order key is
+// written as well: its four smallest selected cubes (12 bits each, C <= 4096)
+// above the cube's own index, so that sorting the keys puts query cubes whose
+// selections start alike next to each other (the fine stage's tiles are pairs
+// of consecutive cubes, and a tile's steps are the union of its two
+// selections).
 template <int KPL>
 __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C, int k, const float* __restrict__ scores,
                                                             int32_t* __restrict__ idx, uint64_t* __restrict__ sig) {
@@ -285,6 +288,8 @@ __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C,
         const int need_eq = k - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
         int out = 0, eq_seen = 0;
         int32_t* dst = idx + row * k;
+        uint64_t lex = 0ull;   // the row's four smallest selected cubes, 12 bits each from bit 52 down
+        int nlex = 0;
 #pragma unroll
         for (int i = 0; i < KPL; ++i) {
             const int j = lane + 32 * i;
@@ -298,24 +303,11 @@ __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C,
             if (take) dst[out + __popc(take_mask & lt_mask)] = j;
             out += __popc(take_mask);
             eq_seen += __popc(eq_mask);
+            // warp-uniform: the selection is written in ascending order, so its first entries are these
+            for (uint32_t mk = take_mask; nlex < 4 && mk != 0u; mk &= mk - 1u, ++nlex)
+                lex |= static_cast<uint64_t>(32 * i + __ffs(mk) - 1) << (52 - 12 * nlex);
         }
-        if (sig != nullptr) {
-            uint64_t t[3] = {0ull, 0ull, 0ull};
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) {
-                const int j = lane + 32 * i;
-                if (j < C) top3_insert(t, (static_cast<uint64_t>(key[i]) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(j)));
-            }
-#pragma unroll
-            for (int off = 16; off; off >>= 1) {
-                uint64_t o[3];
-#pragma unroll
-                for (int e = 0; e < 3; ++e) o[e] = __shfl_xor_sync(0xffffffffu, t[e], off);
-#pragma unroll
-                for (int e = 0; e < 3; ++e) top3_insert(t, o[e]);
-            }
-            if (lane == 0) sig[row] = group_signature(t, static_cast<uint32_t>(row % C));
-        }
+        if (sig != nullptr && lane == 0) sig[row] = lex | static_cast<uint64_t>(row % C);
     }
 }
 
@@ -487,9 +479,10 @@ cudaError_t launch_group_sort(const Dims& d, const uint64_t* sig, int32_t* order
 // position p and each of the kPairWin positions after it, how many selected
 // key cubes the two query cubes share (popcounts of per-cube selection
 // bitmaps in shared memory, so C is bounded by that memory: C <= 1120); then,
-// for kPairRounds rounds, every unpaired position proposes to its best
-// unpaired neighbour within kPairWin positions (more shared cubes first, then
-// the nearer, then the earlier), and mutual proposals pair up.  The pairs are
+// for up to kPairRounds rounds (until one pairs nobody), every unpaired
+// position proposes to its best unpaired neighbour within kPairWin positions
+// (more shared cubes first, then the nearer, then the earlier), and mutual
+// proposals pair up.  The pairs are
 // written in the order of their first member, leftovers paired in order of
 // position (an odd one out last), if they share more key cubes in total than
 // the input's consecutive pairs, leftover pairs more than kPairWin apart
@@ -542,7 +535,10 @@ __global__ void __launch_bounds__(kPairThreads) pair_order_kernel(int C, int k, 
         ov[p * 2 * kPairWin + kPairWin + dd - 1] = o8;             // neighbour p + dd
         ov[(p + dd) * 2 * kPairWin + kPairWin - dd] = o8;          // neighbour (p + dd) - dd
     }
+    __syncthreads();
+    __shared__ int any_match;
     for (int r = 0; r < kPairRounds; ++r) {
+        if (threadIdx.x == 0) any_match = 0;
         __syncthreads();
         for (int p = threadIdx.x; p < C; p += blockDim.x) {
             int bq = -1, bs = -1;
@@ -566,8 +562,15 @@ __global__ void __launch_bounds__(kPairThreads) pair_order_kernel(int C, int k, 
         __syncthreads();
         for (int p = threadIdx.x; p < C; p += blockDim.x) {
             const int q = best[p];
-            if (q >= 0 && best[q] == p) partner[p] = static_cast<int16_t>(q);
+            if (q >= 0 && best[q] == p) {
+                partner[p] = static_cast<int16_t>(q);
+                any_match = 1;
+            }
         }
+        __syncthreads();
+        const bool again = any_match != 0;
+        __syncthreads();         // every thread has read the flag before the next round resets it
+        if (!again) break;       // nothing changed: every later round would propose the same
     }
     __syncthreads();
     // Output.  A position starts a pair when it is matched to a later position, or when it is the

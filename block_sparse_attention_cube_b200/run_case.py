@@ -3,7 +3,7 @@
     python -m block_sparse_attention_cube_b200.run_case --workload wan480p_vsa_k32 --iters 3
 
 Each iteration runs the launches of vsa_forward one by one through the C ABI,
-pool_qkv -> coarse -> topk_order -> pair_order -> schedule -> fine_fused (fine_fused alone, dense,
+pool_qkv -> coarse -> topk_order -> schedule -> fine_fused (fine_fused alone, dense,
 when top-k covers every cube), with CUDA events between the stages.
 `--dense-too` adds a dense fine_fused launch on the same inputs.  `--staged`
 runs the unfused per-step path instead (tile -> pool -> coarse -> top-k ->
@@ -49,7 +49,7 @@ def main(argv=None) -> int:
         names = ["tile", "fine", "untile"] if dense else ["tile", "pool", "coarse", "topk+group", "fine", "combine",
                                                            "untile"]
     else:
-        names = ["fine"] if dense else ["pool", "coarse", "topk_order", "pair", "schedule", "fine"]
+        names = ["fine"] if dense else ["pool", "coarse", "topk_order", "schedule", "fine"]
     if a.dense_too:
         names.append("fine_dense")
     times = {n: [] for n in names}
@@ -99,8 +99,6 @@ def main(argv=None) -> int:
                 scores, oc = vsa.coarse(*bars, s, scale)
                 mark()
                 idx, order = vsa.topk_order(scores, s, w.topk)
-                mark()
-                vsa.pair_order(idx, s, order)
                 mark()
                 steps = vsa.schedule(idx, s, order)
                 mark()

@@ -188,11 +188,14 @@ vsa_status vsa_combine(const vsa_shape* shape, const float* o_coarse, const vsa_
                        vsa_stream_t stream);
 
 /*
- * vsa_topk_order — vsa_topk and vsa_group from one pass over the scores: the
- * k best key cubes of every query cube (as vsa_topk) and the per-head work
- * order (as vsa_group), identical to the two calls.  Two launches: the
- * selection, which also writes each row's work-order key to sig_scratch,
- * then a per-head sort of those keys.
+ * vsa_topk_order — the selection and a work order from one pass over the
+ * scores: the k best key cubes of every query cube (identical to vsa_topk)
+ * and, per (b, h), the query cubes sorted by their four smallest selected key
+ * cubes, then by their own index (a schedule, not a step of the method: the
+ * fine stage's tiles are pairs of consecutive cubes, and cubes whose
+ * selections start alike share more of them than cubes with the same three
+ * best cubes, which vsa_group sorts by).  Two launches: the selection, which
+ * also writes each row's key to sig_scratch, then a per-head sort of the keys.
  *   scores       [B, H, C, C] float32 (read).
  *   idx          [B, H, C, k] int32 (written).
  *   order        [B, H, C] int32 (written).
@@ -269,10 +272,10 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
  * tiles are consecutive pairs of order entries and whose steps are the union
  * of a pair's two selections (a schedule, not a step of the method).  For
  * every position p and each of the 16 positions after it, the kernel counts
- * the key cubes the two query cubes both selected; then, for 8 rounds, each
- * unpaired position proposes to its best unpaired neighbour within 16
- * positions (more shared cubes, then nearer, then earlier) and mutual
- * proposals pair up.  Pairs are written in the order of their first member,
+ * the key cubes the two query cubes both selected; then, for up to 8 rounds
+ * (until one pairs nobody), each unpaired position proposes to its best
+ * unpaired neighbour within 16 positions (more shared cubes, then nearer,
+ * then earlier) and mutual proposals pair up.  Pairs are written in the order of their first member,
  * the leftovers paired in order of position (an odd one out last), if they
  * share more key cubes in total than the input's consecutive pairs (leftover
  * pairs more than 16 positions apart counted as sharing none); otherwise the
@@ -312,11 +315,13 @@ vsa_status vsa_schedule(const vsa_shape* shape, const int32_t* idx, int32_t topk
 size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
 
 /*
- * vsa_forward — the whole attention call on one stream, as nine launches:
- *   vsa_pool_qkv -> vsa_coarse (2) -> vsa_topk_order (2) -> vsa_pair_order -> vsa_schedule
+ * vsa_forward — the whole attention call on one stream, as eight launches:
+ *   vsa_pool_qkv -> vsa_coarse (2) -> vsa_topk_order (2) -> vsa_schedule
  *   -> vsa_fine_fused (the one-tile kernel and its re-run guard)
  * (vsa_topk -> vsa_group instead when C > 2048; the grouping step is skipped
- * when C > 4096, the pairing when C > 1120).  The result equals
+ * when C > 4096).  vsa_pair_order is not part of it: on the 480p workload its
+ * better pairs save about as much fine-stage time as the pass costs.  The
+ * result equals
  *   tile -> pool -> coarse -> topk -> group -> fine -> combine -> untile
  * up to the bf16 rounding of O_fine that the staged path makes.
  * When topk == C every cube is selected and the fine stage is dense attention
