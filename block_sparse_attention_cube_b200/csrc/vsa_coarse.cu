@@ -492,20 +492,24 @@ cudaError_t launch_group_sort(const Dims& d, const uint64_t* sig, int32_t* order
 constexpr int kPairWin = 16;
 constexpr int kPairMaxC = 1120;   // selection bitmaps and scan arrays within 220 KB of shared memory
 constexpr int kPairRounds = 8;
+__host__ __device__ inline int pair_row_words(int C) { return ((C + 31) / 32) | 1; }
 constexpr int kPairThreads = 512;
 
 __global__ void __launch_bounds__(kPairThreads) pair_order_kernel(int C, int k, const int32_t* __restrict__ idx,
                                                                   int32_t* __restrict__ order) {
     extern __shared__ __align__(16) uint8_t pair_smem[];
-    const int nw = (C + 31) / 32;                                  // bitmap words per cube
-    uint32_t* bits = reinterpret_cast<uint32_t*>(pair_smem);       // [C][nw] selections of the cube at position p
-    int32_t* ord = reinterpret_cast<int32_t*>(bits + static_cast<size_t>(C) * nw);   // [C] cube at position p
+    const int nws = pair_row_words(C);                             // bitmap row stride (odd: no bank conflicts)
+    const int nw = (C + 31) / 32;                                  // bitmap words in use per row
+    uint32_t* bits = reinterpret_cast<uint32_t*>(pair_smem);       // [C][nws] selections of the cube at position p
+    int32_t* ord = reinterpret_cast<int32_t*>(bits + static_cast<size_t>(C) * nws);   // [C] cube at position p
     int16_t* partner = reinterpret_cast<int16_t*>(ord + C);        // [C] partner position or -1
     int16_t* best = partner + C;                                   // [C] this round's proposal
     uint8_t* ov = reinterpret_cast<uint8_t*>(best + C);            // [C][2 kPairWin] shared-cube counts
     int* urank = reinterpret_cast<int*>(ov + static_cast<size_t>(C) * 2 * kPairWin);   // [C] rank among the unmatched
     int* upos = urank + C;                                         // [C] position of the u-th unmatched
     int* scan = upos + C;                                          // [C] pair slot of a pair's first position
+    uint32_t* taken = reinterpret_cast<uint32_t*>(scan + C);       // bit 32 + p: position p is paired (or absent)
+    const int ntw = (C + 64 + 31) / 32;
     const int64_t bh = blockIdx.x;
     const int32_t* I = idx + bh * static_cast<int64_t>(C) * k;
     int32_t* O = order + bh * static_cast<int64_t>(C);
@@ -513,27 +517,56 @@ __global__ void __launch_bounds__(kPairThreads) pair_order_kernel(int C, int k, 
         ord[p] = O[p];
         partner[p] = -1;
     }
-    for (int i = threadIdx.x; i < C * nw; i += blockDim.x) bits[i] = 0u;
+    for (int i = threadIdx.x; i < C * nws; i += blockDim.x) bits[i] = 0u;
     for (int i = threadIdx.x; i < C * 2 * kPairWin; i += blockDim.x) ov[i] = 0;
-    __syncthreads();
-    for (int t = threadIdx.x; t < C * k; t += blockDim.x) {
-        const int p = t / k, i = t - p * k;
-        const int cp = ord[p];
-        if (cp < 0 || cp >= C) continue;
-        const int v = __ldg(I + static_cast<int64_t>(cp) * k + i);
-        if (v >= 0 && v < C) atomicOr(bits + static_cast<size_t>(p) * nw + (v >> 5), 1u << (v & 31));
+    for (int wdx = threadIdx.x; wdx < ntw; wdx += blockDim.x) {
+        // positions below 0 and from C on count as taken
+        uint32_t m = 0u;
+        for (int b2 = 0; b2 < 32; ++b2) {
+            const int pos = 32 * wdx + b2 - 32;
+            if (pos < 0 || pos >= C) m |= 1u << b2;
+        }
+        taken[wdx] = m;
     }
     __syncthreads();
-    for (int t = threadIdx.x; t < C * kPairWin; t += blockDim.x) {
-        const int p = t / kPairWin, dd = t - p * kPairWin + 1;
-        if (p + dd >= C) continue;
-        const uint32_t* ra = bits + static_cast<size_t>(p) * nw;
-        const uint32_t* rb = bits + static_cast<size_t>(p + dd) * nw;
-        int o = 0;
-        for (int w = 0; w < nw; ++w) o += __popc(ra[w] & rb[w]);
-        const uint8_t o8 = static_cast<uint8_t>(o < 255 ? o : 255);
-        ov[p * 2 * kPairWin + kPairWin + dd - 1] = o8;             // neighbour p + dd
-        ov[(p + dd) * 2 * kPairWin + kPairWin - dd] = o8;          // neighbour (p + dd) - dd
+    // selection bitmaps: loads batched so that several are in flight per thread
+    constexpr int kBatch = 8;
+    for (int t0 = threadIdx.x; t0 < C * k; t0 += blockDim.x * kBatch) {
+        int v[kBatch], pp[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int t = t0 + u * static_cast<int>(blockDim.x);
+            v[u] = -1;
+            pp[u] = 0;
+            if (t < C * k) {
+                const int p = t / k, i = t - p * k;
+                const int cp = ord[p];
+                pp[u] = p;
+                if (cp >= 0 && cp < C) v[u] = __ldg(I + static_cast<int64_t>(cp) * k + i);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u)
+            if (v[u] >= 0 && v[u] < C) atomicOr(bits + static_cast<size_t>(pp[u]) * nws + (v[u] >> 5), 1u << (v[u] & 31));
+    }
+    __syncthreads();
+    // shared-cube counts: a thread per position holds its row and walks the next kPairWin rows
+    constexpr int kMaxWords = (kPairMaxC + 31) / 32;
+    for (int p = threadIdx.x; p < C; p += blockDim.x) {
+        uint32_t ra[kMaxWords];
+        const uint32_t* rp = bits + static_cast<size_t>(p) * nws;
+#pragma unroll
+        for (int w = 0; w < kMaxWords; ++w) ra[w] = w < nw ? rp[w] : 0u;
+        for (int dd = 1; dd <= kPairWin && p + dd < C; ++dd) {
+            const uint32_t* rb = bits + static_cast<size_t>(p + dd) * nws;
+            int o = 0;
+#pragma unroll
+            for (int w = 0; w < kMaxWords; ++w)
+                if (w < nw) o += __popc(ra[w] & rb[w]);
+            const uint8_t o8 = static_cast<uint8_t>(o < 255 ? o : 255);
+            ov[p * 2 * kPairWin + kPairWin + dd - 1] = o8;         // neighbour p + dd
+            ov[(p + dd) * 2 * kPairWin + kPairWin - dd] = o8;      // neighbour (p + dd) - dd
+        }
     }
     __syncthreads();
     __shared__ int any_match;
@@ -541,18 +574,29 @@ __global__ void __launch_bounds__(kPairThreads) pair_order_kernel(int C, int k, 
         if (threadIdx.x == 0) any_match = 0;
         __syncthreads();
         for (int p = threadIdx.x; p < C; p += blockDim.x) {
-            int bq = -1, bs = -1;
+            int bq = -1;
             if (partner[p] < 0) {
-                for (int dd = 1; dd <= kPairWin; ++dd) {
+                // bit j of win: position p - kPairWin + j is taken (j = 0 .. 2 kPairWin)
+                const int s0 = p - kPairWin + 32;
+                const uint64_t w2 = (static_cast<uint64_t>(taken[(s0 >> 5) + 1]) << 32) | taken[s0 >> 5];
+                const uint64_t win = w2 >> (s0 & 31);
+                const uint32_t* ovw = reinterpret_cast<const uint32_t*>(ov + p * 2 * kPairWin);
+                int bkey = -1;
 #pragma unroll
-                    for (int side = 0; side < 2; ++side) {
-                        const int q = side ? p + dd : p - dd;
-                        if (q < 0 || q >= C || partner[q] >= 0) continue;
-                        const int slot = side ? kPairWin + dd - 1 : kPairWin - dd;
-                        const int score = static_cast<int>(ov[p * 2 * kPairWin + slot]) * 64 + (kPairWin - dd);
-                        if (score > bs) {
-                            bs = score;
-                            bq = q;
+                for (int wq = 0; wq < 2 * kPairWin / 4; ++wq) {
+                    const uint32_t four = ovw[wq];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int sl = 4 * wq + e;                      // slot: p - kPairWin + sl, or p + sl - kPairWin + 1
+                        const int j = sl < kPairWin ? sl : sl + 1;      // window bit of that neighbour
+                        const int near = sl < kPairWin ? sl : 2 * kPairWin - 1 - sl;   // kPairWin - distance
+                        // more shared, then nearer, then the earlier of two equally near
+                        const int key = ((static_cast<int>((four >> (8 * e)) & 0xFFu) * 64 + near) * 2) +
+                                        (sl < kPairWin ? 1 : 0);
+                        const bool free_q = ((win >> j) & 1ull) == 0ull;
+                        if (free_q && key > bkey) {
+                            bkey = key;
+                            bq = p - kPairWin + j;
                         }
                     }
                 }
@@ -564,6 +608,7 @@ __global__ void __launch_bounds__(kPairThreads) pair_order_kernel(int C, int k, 
             const int q = best[p];
             if (q >= 0 && best[q] == p) {
                 partner[p] = static_cast<int16_t>(q);
+                atomicOr(taken + ((p + 32) >> 5), 1u << ((p + 32) & 31));
                 any_match = 1;
             }
         }
@@ -660,7 +705,8 @@ __global__ void __launch_bounds__(kPairThreads) pair_order_kernel(int C, int k, 
 }
 
 size_t pair_smem_bytes(int C) {
-    return static_cast<size_t>(C) * ((C + 31) / 32) * 4 + static_cast<size_t>(C) * (4 + 2 + 2 + 2 * kPairWin + 12);
+    return static_cast<size_t>(C) * pair_row_words(C) * 4 + static_cast<size_t>(C) * (4 + 2 + 2 + 2 * kPairWin + 12) +
+           static_cast<size_t>((C + 64 + 31) / 32) * 4;
 }
 
 cudaError_t launch_pair_order(const Dims& d, const int32_t* idx, int k, int32_t* order, cudaStream_t s) {
