@@ -13,66 +13,116 @@
 namespace vsa {
 namespace {
 
-constexpr int kTile = 64;   // output tile edge
 constexpr int kBK = 16;     // reduction slice
 constexpr int kThreads = 256;
+constexpr int kSTI = 128;   // score tile rows (query cubes)
+constexpr int kSTJ = 64;    // score tile columns (key cubes)
+constexpr int kSRI = 8;     // rows per thread
+constexpr int kSRJ = 4;     // columns per thread
+static_assert((kSTI / kSRI) * (kSTJ / kSRJ) == kThreads, "one output block per thread");
 
 // scores[bh][i][j] = scale * sum_d qbar[bh][i][d] * kbar[bh][j][d]
-// A 64x64 output tile per block; thread (ty, tx) owns rows 4ty..4ty+3 and
-// columns 4tx..4tx+3, reading four operands at a time from shared memory.
-// Each output is one sequential float32 fma chain over the channels.
+// A 128x64 output tile per block; thread (ty, tx) owns rows 8ty..8ty+7 and
+// columns 4tx..4tx+3 (32 accumulators, 12 operands read from shared memory
+// per 32 fma).  Each output is one sequential float32 fma chain over the
+// channels, so the tile shape does not change a single bit of the result.
 __global__ void __launch_bounds__(kThreads) coarse_scores_kernel(int C, int D, const float* __restrict__ qbar,
                                                                  const float* __restrict__ kbar, float scale,
                                                                  float* __restrict__ scores) {
-    __shared__ __align__(16) float As[kBK][kTile + 4];
-    __shared__ __align__(16) float Bs[kBK][kTile + 4];
+    __shared__ __align__(16) float As[kBK][kSTI + 4];
+    __shared__ __align__(16) float Bs[kBK][kSTJ + 4];
     const int bh = blockIdx.z;
-    const int i0 = blockIdx.y * kTile, j0 = blockIdx.x * kTile;
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int i0 = blockIdx.y * kSTI, j0 = blockIdx.x * kSTJ;
+    constexpr int NTX = kSTJ / kSRJ;
+    const int tx = threadIdx.x % NTX, ty = threadIdx.x / NTX;
     const float* Q = qbar + static_cast<int64_t>(bh) * C * D;
     const float* K = kbar + static_cast<int64_t>(bh) * C * D;
-    float acc[4][4] = {};
+    float acc[kSRI][kSRJ] = {};
     for (int d0 = 0; d0 < D; d0 += kBK) {
-        // 64 rows x 16 channels of each operand, stored channel-major; 4 elements per thread each
+        // the tile's rows x 16 channels of each operand, stored channel-major
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int e = 0; e < kSTI * kBK / kThreads; ++e) {
             const int idx = threadIdx.x + e * kThreads;
             const int r = idx / kBK, cc = idx % kBK;
-            const int gi = i0 + r, gj = j0 + r;
+            const int gi = i0 + r;
             As[cc][r] = gi < C ? Q[static_cast<int64_t>(gi) * D + d0 + cc] : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < kSTJ * kBK / kThreads; ++e) {
+            const int idx = threadIdx.x + e * kThreads;
+            const int r = idx / kBK, cc = idx % kBK;
+            const int gj = j0 + r;
             Bs[cc][r] = gj < C ? K[static_cast<int64_t>(gj) * D + d0 + cc] : 0.f;
         }
         __syncthreads();
 #pragma unroll
         for (int kk = 0; kk < kBK; ++kk) {
-            const float4 a = *reinterpret_cast<const float4*>(&As[kk][4 * ty]);
-            const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][4 * tx]);
-            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+            float av[kSRI], bv[kSRJ];
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
+            for (int q4 = 0; q4 < kSRI / 4; ++q4) {
+                const float4 a = *reinterpret_cast<const float4*>(&As[kk][kSRI * ty + 4 * q4]);
+                av[4 * q4] = a.x;
+                av[4 * q4 + 1] = a.y;
+                av[4 * q4 + 2] = a.z;
+                av[4 * q4 + 3] = a.w;
+            }
+            const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][kSRJ * tx]);
+            bv[0] = b.x;
+            bv[1] = b.y;
+            bv[2] = b.z;
+            bv[3] = b.w;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+            for (int r = 0; r < kSRI; ++r)
+#pragma unroll
+                for (int c = 0; c < kSRJ; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
         }
         __syncthreads();
     }
     float* S = scores + static_cast<int64_t>(bh) * C * C;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int gi = i0 + 4 * ty + r;
+    for (int r = 0; r < kSRI; ++r) {
+        const int gi = i0 + kSRI * ty + r;
         if (gi >= C) continue;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int gj = j0 + 4 * tx + c;
+        for (int c = 0; c < kSRJ; ++c) {
+            const int gj = j0 + kSRJ * tx + c;
             if (gj < C) S[static_cast<int64_t>(gi) * C + gj] = scale * acc[r][c];
         }
     }
 }
 
 // o_coarse[bh][i] = sum_j softmax(scores[bh][i][:])_j * vbar[bh][j]
-// A block owns kPvRows query rows: it reduces their row maxima and
-// denominators (a warp per row), then accumulates exp(S - max) * Vbar over
-// key slices of 16; thread (ty, tx) owns RPT rows and 4 output channels.
+// One pass over each score row (online maximum): a block owns kPvRows query
+// rows and walks the keys in slices of 16.  Half a warp holds a row's 16
+// scores of the slice: it takes their maximum by shuffles, raises the row's
+// running maximum m, and writes p = exp(s - m) to shared memory together with
+// the factor exp(m_old - m) by which the row's accumulators are rescaled; each
+// lane keeps a partial denominator, summed over the half warp at the end.
+// Thread (ty, tx) owns RPT rows and 4 output channels.  The next slice's
+// scores and V rows are loaded into registers while this slice accumulates.
 constexpr int kPvRows = 32;
+
+// n consecutive floats of shared memory (16-byte aligned for n % 4 == 0, else 8-byte) into registers
+template <int n>
+__device__ __forceinline__ void read_rows(const float* src, float* dst) {
+    if constexpr (n % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < n / 4; ++i) {
+            const float4 a = reinterpret_cast<const float4*>(src)[i];
+            dst[4 * i] = a.x;
+            dst[4 * i + 1] = a.y;
+            dst[4 * i + 2] = a.z;
+            dst[4 * i + 3] = a.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float2 a = reinterpret_cast<const float2*>(src)[i];
+            dst[2 * i] = a.x;
+            dst[2 * i + 1] = a.y;
+        }
+    }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) coarse_pv_kernel(int C, const float* __restrict__ scores,
@@ -80,62 +130,94 @@ __global__ void __launch_bounds__(kThreads) coarse_pv_kernel(int C, const float*
                                                              float* __restrict__ o_coarse) {
     constexpr int TX = D / 4;                     // threads across the channels
     constexpr int RPT = kPvRows * TX / kThreads;  // rows per thread
-    __shared__ float row_max[kPvRows], row_inv[kPvRows];
+    constexpr int SPT = kPvRows * kBK / kThreads; // scores per thread per slice
+    constexpr int VPT = kBK * D / 4 / kThreads;   // V float4 per thread per slice
+    static_assert(RPT % 2 == 0 && SPT >= 1 && VPT >= 1, "tile shape");
     __shared__ __align__(16) float Ps[kBK][kPvRows + 4];
     __shared__ __align__(16) float Vs[kBK][D];
+    __shared__ __align__(16) float alpha_s[kPvRows];
+    __shared__ float row_inv[kPvRows];
     const int bh = blockIdx.y;
     const int i0 = blockIdx.x * kPvRows;
     const float* S = scores + static_cast<int64_t>(bh) * C * C;
     const float* V = vbar + static_cast<int64_t>(bh) * C * D;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int r = warp; r < kPvRows; r += kThreads / 32) {
-        const int gi = i0 + r;
-        float m = -FLT_MAX, l = 0.f;
-        if (gi < C) {
-            const float* row = S + static_cast<int64_t>(gi) * C;
-            for (int j = lane; j < C; j += 32) m = fmaxf(m, row[j]);
+    const int cc = threadIdx.x % kBK, rbase = threadIdx.x / kBK;   // score role: key cc of rows rbase + 16e
+    const int tx = threadIdx.x % TX, ty = threadIdx.x / TX;        // accumulate role
+    float m[SPT], l[SPT], s_next[SPT];
+    float4 v_next[VPT];
+    auto load_slice = [&](int j0) {
+        const int gj = j0 + cc;
 #pragma unroll
-            for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            for (int j = lane; j < C; j += 32) l += expf(row[j] - m);
+        for (int e = 0; e < SPT; ++e) {
+            const int gi = i0 + rbase + e * (kThreads / kBK);
+            s_next[e] = gi >= C ? 0.f : gj < C ? __ldg(S + static_cast<int64_t>(gi) * C + gj) : -FLT_MAX;
+        }
 #pragma unroll
-            for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-        }
-        if (lane == 0) {
-            row_max[r] = m;
-            row_inv[r] = l > 0.f ? 1.0f / l : 0.f;
-        }
-    }
-    __syncthreads();
-    const int tx = threadIdx.x % TX, ty = threadIdx.x / TX;
-    float acc[RPT][4] = {};
-    for (int j0 = 0; j0 < C; j0 += kBK) {
-        for (int idx = threadIdx.x; idx < kPvRows * kBK; idx += kThreads) {   // kPvRows rows x 16 keys
-            const int r = idx / kBK, cc = idx % kBK;
-            const int gi = i0 + r, gj = j0 + cc;
-            Ps[cc][r] = (gi < C && gj < C) ? expf(S[static_cast<int64_t>(gi) * C + gj] - row_max[r]) : 0.f;
-        }
-        for (int idx = threadIdx.x; idx < kBK * D / 4; idx += kThreads) {      // 16 keys x D channels
+        for (int e = 0; e < VPT; ++e) {
+            const int idx = threadIdx.x + e * kThreads;
             const int kk = idx / (D / 4), c4 = idx % (D / 4);
-            const int gj = j0 + kk;
-            *reinterpret_cast<float4*>(&Vs[kk][4 * c4]) =
-                gj < C ? *reinterpret_cast<const float4*>(V + static_cast<int64_t>(gj) * D + 4 * c4)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+            v_next[e] = j0 + kk < C ? __ldg(reinterpret_cast<const float4*>(V + static_cast<int64_t>(j0 + kk) * D) + c4)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+#pragma unroll
+    for (int e = 0; e < SPT; ++e) {
+        m[e] = -FLT_MAX;
+        l[e] = 0.f;
+    }
+    float acc[RPT][4] = {};
+    load_slice(0);
+    for (int j0 = 0; j0 < C; j0 += kBK) {
+#pragma unroll
+        for (int e = 0; e < SPT; ++e) {
+            const int r = rbase + e * (kThreads / kBK);
+            float mx = s_next[e];
+#pragma unroll
+            for (int off = kBK / 2; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float mn = fmaxf(m[e], mx);
+            const float a = expf(m[e] - mn);
+            const float pv = expf(s_next[e] - mn);
+            m[e] = mn;
+            l[e] = l[e] * a + pv;
+            Ps[cc][r] = pv;
+            if (cc == 0) alpha_s[r] = a;
+        }
+#pragma unroll
+        for (int e = 0; e < VPT; ++e) {
+            const int idx = threadIdx.x + e * kThreads;
+            *reinterpret_cast<float4*>(&Vs[idx / (D / 4)][4 * (idx % (D / 4))]) = v_next[e];
         }
         __syncthreads();
+        if (j0 + kBK < C) load_slice(j0 + kBK);
+        {
+            float av[RPT];
+            read_rows<RPT>(&alpha_s[RPT * ty], av);
+#pragma unroll
+            for (int r = 0; r < RPT; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[r][c] *= av[r];
+        }
 #pragma unroll
         for (int kk = 0; kk < kBK; ++kk) {
-            float a[RPT];
-#pragma unroll
-            for (int r = 0; r < RPT; ++r) a[r] = Ps[kk][RPT * ty + r];
+            float pr[RPT];
+            read_rows<RPT>(&Ps[kk][RPT * ty], pr);
             const float4 b = *reinterpret_cast<const float4*>(&Vs[kk][4 * tx]);
             const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
             for (int r = 0; r < RPT; ++r)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], bv[c], acc[r][c]);
+                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(pr[r], bv[c], acc[r][c]);
         }
         __syncthreads();
     }
+#pragma unroll
+    for (int e = 0; e < SPT; ++e) {
+        float t = l[e];
+#pragma unroll
+        for (int off = kBK / 2; off; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+        if (cc == 0) row_inv[rbase + e * (kThreads / kBK)] = t > 0.f ? 1.0f / t : 0.f;
+    }
+    __syncthreads();
     float* O = o_coarse + static_cast<int64_t>(bh) * C * D;
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
@@ -391,8 +473,8 @@ cudaError_t launch_group(const Dims& d, const float* scores, int32_t* order, cud
 cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
                           float* scores, float* o_coarse, cudaStream_t s) {
     const int bh = d.B * d.H;
-    const int tiles = (d.C + kTile - 1) / kTile;
-    coarse_scores_kernel<<<dim3(tiles, tiles, bh), kThreads, 0, s>>>(d.C, d.D, qbar, kbar, scale, scores);
+    const dim3 grid((d.C + kSTJ - 1) / kSTJ, (d.C + kSTI - 1) / kSTI, bh);
+    coarse_scores_kernel<<<grid, kThreads, 0, s>>>(d.C, d.D, qbar, kbar, scale, scores);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int pv_blocks = (d.C + kPvRows - 1) / kPvRows;

@@ -914,13 +914,20 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // one thread issues an M128N128K16 MMA only every ~95 cycles, against ~68 for
 // the tensor core to run it.
 //
-// Roles (480 threads): warps 0-11 are three softmax groups of four warps
+// Roles (512 threads): warps 0-11 are three softmax groups of four warps
 // (group g owns score buffer g and takes the steps s with s % 3 == g; warp
-// 4g + q reads TMEM lane quarter q); warp 12 issues TMA (the tile's Q, then
-// per step two K blocks through a 3-deep ring and two V blocks through a
-// 2-deep ring); warp 13 allocates tensor memory and issues S(s) into buffer
-// s % 3 once PV(s - 3) has drained it; warp 14 issues PV(s) into the output
-// accumulator once group s % 3 has stored P(s).
+// 4g + q reads TMEM lane quarter q); warp 12 loads the tile's Q and per step
+// two K blocks through a 3-deep ring; warp 15 loads per step two V blocks
+// through a 2-deep ring; warp 13 allocates tensor memory and issues S(s) into
+// buffer s % 3 once PV(s - 3) has drained it; warp 14 issues PV(s) into the
+// output accumulator once group s % 3 has stored P(s).
+//
+// Loads: a thread that issues TMA copies is held for roughly as long as the
+// copies take to land (about 1,300 cycles for a step's 32 KB of K, measured
+// with clock stamps), so one thread issuing K and V in turn paced the whole
+// pipeline: V(s) waits for PV(s - 2), and K(s + 1) queued behind it.  K and V
+// therefore have producers of their own, and the four 8 KB boxes of a load
+// (two blocks x two 64-channel halves) are issued by four lanes at once.
 //
 // Tensor memory: buffers at columns 0, 128 and 256 (128 fp32 scores for a
 // step's 128 keys; P, as bf16 pairs, over the first 64 columns), the output
@@ -934,7 +941,8 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // maximum) or a non-finite sum raises the overflow word, and the caller then
 // runs fine_kernel, whose online maximum is rescaled per step, over the whole
 // stage again: the teardown's guard that re-runs a tile with online rescaling.
-constexpr int kTThreads = 480;
+constexpr int kTThreads = 512;
+constexpr int kTVWarp = 15;
 constexpr int kTTmaWarp = 12;
 constexpr int kTSWarp = 13;
 constexpr int kTPVWarp = 14;
@@ -1039,49 +1047,44 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
     };
 
+    constexpr int kBoxes = D == 128 ? 4 : 2;
+    constexpr unsigned kBoxMask = (1u << kBoxes) - 1u;
     if (warp == kTTmaWarp) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            uint32_t q_issued = 0, k_issued[kTKStages] = {}, v_issued[kTVStages] = {};
-            RingPos kp{0, 0}, vp{0, 0};
+        // ------------------------------------------------------------ Q and K producer (lane i: box i)
+        if (lane < kBoxes) {
+            uint32_t q_issued = 0, k_issued[kTKStages] = {};
+            RingPos kp{0, 0};
             int n_item = 0;
             bool ok = true;
             for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
                 const Item item = decode_item(it, p);
                 auto load_pair = [&](const CUtensorMap* m, uint32_t dst, int ja, int jb, uint32_t b) {
-                    load_block<LM, D>(m, dst, ja, 0, b, item, p);
-                    load_block<LM, D>(m, dst + 8192, jb, 0, b, item, p);
-                    if (D == 128) {
-                        load_block<LM, D>(m, dst + 16384, ja, 64, b, item, p);
-                        load_block<LM, D>(m, dst + 24576, jb, 64, b, item, p);
-                    }
+                    __syncwarp(kBoxMask);   // lane 0's expect_tx first
+                    load_block<LM, D>(m, dst + 8192u * lane, (lane & 1) ? jb : ja, 64 * (lane >> 1), b, item, p);
                 };
-                if (!(ok = bw.wait(bar(kTBarQEmpty), (n_item & 1) ^ 1))) break;
-                mbar_arrive_expect_tx(bar(kTBarQFull), kBytesQ);
-                ++q_issued;
+                if (!(ok = __all_sync(kBoxMask, bw.wait(bar(kTBarQEmpty), (n_item & 1) ^ 1)))) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(kTBarQFull), kBytesQ);
+                    ++q_issued;
+                }
                 load_pair(&tm_q, base + kTOffQ, item.blk[0], item.blk[1], bar(kTBarQFull));
                 for (int s = 0;; ++s) {
                     const StepRec r = tile_step(p, it, s, item.present);
-                    if (!(ok = bw.wait(bar(kTBarKEmpty + kp.slot), kp.phase ^ 1u))) break;
-                    mbar_arrive_expect_tx(bar(kTBarKFull + kp.slot), kBytesKV);
-                    ++k_issued[kp.slot];
+                    if (!(ok = __all_sync(kBoxMask, bw.wait(bar(kTBarKEmpty + kp.slot), kp.phase ^ 1u)))) break;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(kTBarKFull + kp.slot), kBytesKV);
+                        ++k_issued[kp.slot];
+                    }
                     load_pair(&tm_k, base + kTOffK + kp.slot * kKVBytes, r.ca, r.cb, bar(kTBarKFull + kp.slot));
                     kp.advance<kTKStages>();
-                    if (!(ok = bw.wait(bar(kTBarVEmpty + vp.slot), vp.phase ^ 1u))) break;
-                    mbar_arrive_expect_tx(bar(kTBarVFull + vp.slot), kBytesKV);
-                    ++v_issued[vp.slot];
-                    load_pair(&tm_v, base + kTOffV + vp.slot * kKVBytes, r.ca, r.cb, bar(kTBarVFull + vp.slot));
-                    vp.advance<kTVStages>();
                     if (r.last) break;
                 }
             }
-            if (!ok) {
+            if (!ok && lane == 0) {
                 // wait for this CTA's own copies still in flight before exiting
                 if (q_issued) drain_wait(bar(kTBarQFull), (q_issued - 1u) & 1u);
                 for (int s = 0; s < kTKStages; ++s)
                     if (k_issued[s]) drain_wait(bar(kTBarKFull + s), (k_issued[s] - 1u) & 1u);
-                for (int s = 0; s < kTVStages; ++s)
-                    if (v_issued[s]) drain_wait(bar(kTBarVFull + s), (v_issued[s] - 1u) & 1u);
             }
         }
     } else if (warp == kTSWarp) {
@@ -1161,6 +1164,34 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (issued_any) {
                 mma_commit(bar(kTBarDrain + 1));
                 drain_wait(bar(kTBarDrain + 1), 0u);
+            }
+        }
+    } else if (warp == kTVWarp) {
+        // ------------------------------------------------------------ V producer (lane i: box i)
+        if (lane < kBoxes) {
+            uint32_t v_issued[kTVStages] = {};
+            RingPos vp{0, 0};
+            bool ok = true;
+            for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x) {
+                const Item item = decode_item(it, p);
+                for (int s = 0;; ++s) {
+                    const StepRec r = tile_step(p, it, s, item.present);
+                    if (!(ok = __all_sync(kBoxMask, bw.wait(bar(kTBarVEmpty + vp.slot), vp.phase ^ 1u)))) break;
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(bar(kTBarVFull + vp.slot), kBytesKV);
+                        ++v_issued[vp.slot];
+                    }
+                    __syncwarp(kBoxMask);
+                    const uint32_t dst = base + kTOffV + vp.slot * kKVBytes;
+                    load_block<LM, D>(&tm_v, dst + 8192u * lane, (lane & 1) ? r.cb : r.ca, 64 * (lane >> 1),
+                                      bar(kTBarVFull + vp.slot), item, p);
+                    vp.advance<kTVStages>();
+                    if (r.last) break;
+                }
+            }
+            if (!ok && lane == 0) {
+                for (int s = 0; s < kTVStages; ++s)
+                    if (v_issued[s]) drain_wait(bar(kTBarVFull + s), (v_issued[s] - 1u) & 1u);
             }
         }
     } else {
