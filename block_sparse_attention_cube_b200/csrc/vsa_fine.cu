@@ -172,12 +172,16 @@ struct Item {
     uint32_t present;   // bit j set when slot j holds a query block
 };
 
+// Item counts fit in 31 bits (make_params' callers check), so the divisions are 32-bit ones.
 __device__ __forceinline__ Item decode_item(int64_t it, const FineParams& p) {
     Item r;
-    const int g = static_cast<int>(it % p.ngroups);
-    r.bh = it / p.ngroups;
-    r.b = static_cast<int>(r.bh / p.H);
-    r.h = static_cast<int>(r.bh - static_cast<int64_t>(r.b) * p.H);
+    const uint32_t itu = static_cast<uint32_t>(it), ng = static_cast<uint32_t>(p.ngroups);
+    const uint32_t bh = itu / ng, nh = static_cast<uint32_t>(p.H);
+    const int g = static_cast<int>(itu - bh * ng);
+    const uint32_t b = bh / nh;
+    r.bh = bh;
+    r.b = static_cast<int>(b);
+    r.h = static_cast<int>(bh - b * nh);
     r.present = 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -914,13 +918,14 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // one thread issues an M128N128K16 MMA only every ~95 cycles, against ~68 for
 // the tensor core to run it.
 //
-// Roles (512 threads): warps 0-11 are three softmax groups of four warps
+// Roles (640 threads): warps 0-11 are three softmax groups of four warps
 // (group g owns score buffer g and takes the steps s with s % 3 == g; warp
 // 4g + q reads TMEM lane quarter q); warp 12 loads the tile's Q and per step
 // two K blocks through a 3-deep ring; warp 15 loads per step two V blocks
 // through a 2-deep ring; warp 13 allocates tensor memory and issues S(s) into
 // buffer s % 3 once PV(s - 3) has drained it; warp 14 issues PV(s) into the
-// output accumulator once group s % 3 has stored P(s).
+// output accumulator once group s % 3 has stored P(s); warps 16-19 write the
+// output (warp 16 + q: lane quarter q).
 //
 // Loads: a thread that issues TMA copies is held for roughly as long as the
 // copies take to land (about 1,300 cycles for a step's 32 KB of K, measured
@@ -937,12 +942,29 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // "Fixed-max softmax is a numerical contract"): the maximum of a row's first
 // selected scores is kept for the whole item, so the three groups need no
 // exchange per step; each keeps its own partial row sum and the epilogue adds
-// the three.  A probability above 2^64 (a later score far above the first
+// the three.
+//
+// Epilogue: warps 16-19 merge and store the item's output while the three
+// softmax groups go on to the next item, which they start as soon as their
+// steps of this one are done; the first PV of the next item waits only until
+// the epilogue warps have read O out of tensor memory.  The epilogue fetches
+// its inputs (gates, the coarse outputs of the tile's query cubes) while the
+// item's steps run.  Because the groups run one item ahead of the epilogue,
+// the per-item maxima, row sums and their barriers come in two sets, used by
+// even and odd items; a group cannot get two items ahead, since its next
+// item's PVs queue behind the release of O.  The epilogue waits for the
+// item's last PV on a barrier committed once per item: a wait by parity on
+// the last step's PV-done barrier would pass early whenever that buffer's
+// previous PV were still pending (a parity wait returns at once when the
+// barrier is one phase behind).
+//
+// A probability above 2^64 (a later score far above the first
 // maximum) or a non-finite sum raises the overflow word, and the caller then
 // runs fine_kernel, whose online maximum is rescaled per step, over the whole
 // stage again: the teardown's guard that re-runs a tile with online rescaling.
-constexpr int kTThreads = 512;
+constexpr int kTThreads = 640;
 constexpr int kTVWarp = 15;
+constexpr int kTEpiWarp = 16;                                     // warps 16-19: the epilogue
 constexpr int kTTmaWarp = 12;
 constexpr int kTSWarp = 13;
 constexpr int kTPVWarp = 14;
@@ -952,9 +974,10 @@ constexpr int kTVStages = 2;
 constexpr uint32_t kTOffQ = 0;                                   // one tile: 128 rows x 256 B
 constexpr uint32_t kTOffK = kTOffQ + kQTileBytes;                // [kTKStages]
 constexpr uint32_t kTOffV = kTOffK + kTKStages * kKVBytes;       // [kTVStages]
-constexpr uint32_t kTOffM = kTOffV + kTVStages * kKVBytes;       // [128] each row's fixed maximum
-constexpr uint32_t kTOffL = kTOffM + 128 * 4;                    // [kTBufs][128] each group's row sums
-constexpr uint32_t kTOffBar = kTOffL + kTBufs * 128 * 4;
+constexpr uint32_t kTOffM = kTOffV + kTVStages * kKVBytes;       // [2 items][128] each row's fixed maximum
+constexpr uint32_t kTOffL = kTOffM + 2 * 128 * 4;                // [2 items][kTBufs][128] each group's row sums
+constexpr uint32_t kTOffOC = kTOffL + 2 * kTBufs * 128 * 4;      // [4 epilogue warps][128] coarse outputs
+constexpr uint32_t kTOffBar = kTOffOC + 4 * 128 * 4;
 constexpr int kTBarQFull = 0;
 constexpr int kTBarQEmpty = 1;
 constexpr int kTBarKFull = 2;                                    // [kTKStages]
@@ -964,10 +987,11 @@ constexpr int kTBarVEmpty = kTBarVFull + kTVStages;
 constexpr int kTBarSFull = kTBarVEmpty + kTVStages;             // [kTBufs]
 constexpr int kTBarPFull = kTBarSFull + kTBufs;                  // [kTBufs], four arrivals
 constexpr int kTBarPVDone = kTBarPFull + kTBufs;                 // [kTBufs]
-constexpr int kTBarMReady = kTBarPVDone + kTBufs;                // [2 query blocks], two arrivals
-constexpr int kTBarEpi = kTBarMReady + 2;                        // twelve arrivals
-constexpr int kTBarOFree = kTBarEpi + 1;                         // twelve arrivals
-constexpr int kTBarDrain = kTBarOFree + 1;                       // [2 issuers]
+constexpr int kTBarMReady = kTBarPVDone + kTBufs;                // [2 items][2 query blocks], two arrivals
+constexpr int kTBarEpi = kTBarMReady + 4;                        // [2 items], twelve arrivals
+constexpr int kTBarOFree = kTBarEpi + 2;                         // four arrivals (the epilogue warps)
+constexpr int kTBarODone = kTBarOFree + 1;                       // the item's last PV complete (one commit per item)
+constexpr int kTBarDrain = kTBarODone + 1;                       // [2 issuers]
 constexpr int kTNumBars = kTBarDrain + 2;
 constexpr uint32_t kTOffMisc = kTOffBar + kTNumBars * 8;         // tmem slot (4 B) + abort flag (4 B)
 constexpr uint32_t kTSmemBytes = kTOffMisc + 16 + 1024;
@@ -1000,6 +1024,7 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kTOffMisc + 4);
     float* m_row = reinterpret_cast<float*>(smem + kTOffM);
     float* l_part = reinterpret_cast<float*>(smem + kTOffL);
+    float* oc_s = reinterpret_cast<float*>(smem + kTOffOC);
     const BoundedWait bw{abort_flag, p.status, p.limit_ns};
 
     if (threadIdx.x == 0) {
@@ -1019,10 +1044,11 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_init(bar(kTBarPFull + b), 4);    // the four warps of group b
             mbar_init(bar(kTBarPVDone + b), 1);
         }
-        mbar_init(bar(kTBarMReady + 0), 2);       // the two warps of a query block's lane quarters
-        mbar_init(bar(kTBarMReady + 1), 2);
-        mbar_init(bar(kTBarEpi), 12);
-        mbar_init(bar(kTBarOFree), 12);
+        for (int i = 0; i < 4; ++i) mbar_init(bar(kTBarMReady + i), 2);   // the two warps of a query block
+        mbar_init(bar(kTBarEpi + 0), 12);
+        mbar_init(bar(kTBarEpi + 1), 12);
+        mbar_init(bar(kTBarOFree), 4);
+        mbar_init(bar(kTBarODone), 1);
         mbar_init(bar(kTBarDrain + 0), 1);
         mbar_init(bar(kTBarDrain + 1), 1);
         fence_mbar_init();
@@ -1157,7 +1183,10 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mma_commit(bar(kTBarVEmpty + vp.slot));
                     issued_any = true;
                     vp.advance<kTVStages>();
-                    if (r.last) break;
+                    if (r.last) {
+                        mma_commit(bar(kTBarODone));   // O of the item is complete
+                        break;
+                    }
                 }
                 if (!ok) break;
             }
@@ -1194,18 +1223,152 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (v_issued[s]) drain_wait(bar(kTBarVFull + s), (v_issued[s] - 1u) & 1u);
             }
         }
+    } else if (warp >= kTEpiWarp) {
+        // ------------------------------------------------------------ epilogue warpgroup
+        const int q = warp & 3;                  // TMEM lane quarter
+        const int row = q * 32 + lane;           // query row of the tile, 0..127
+        const int slot = q >> 1;                 // query block of the row
+        const uint32_t tO = tmem + kTColO + (static_cast<uint32_t>(q * 32) << 16);
+        float* oc_w = oc_s + (warp - kTEpiWarp) * 128;   // this warp's query cube's coarse output
+        bool ok = true;
+        auto wait_all = [&](uint32_t b, uint32_t par) -> bool {
+            const bool mine = bw.wait(b, par);
+            return __all_sync(0xffffffffu, mine);
+        };
+        // token of this row (-1: none) and, for the token layout, its cube
+        auto row_token = [&](const Item& item, int& cube) -> int64_t {
+            const int blk = item.blk[slot];
+            const int o_ = row & 63;
+            int64_t tok = -1;
+            cube = 0;
+            if (blk >= 0) {
+                if (LM == kLoadTokens) {
+                    tok = 64ll * blk + o_;
+                    if (tok >= p.N) {
+                        tok = -1;
+                    } else if (p.o_coarse != nullptr) {
+                        const int64_t xy = static_cast<int64_t>(p.X) * p.Y;
+                        const int tt = static_cast<int>(tok / xy);
+                        const int rem = static_cast<int>(tok - tt * xy);
+                        const int xx = rem / p.Y, yy = rem - (rem / p.Y) * p.Y;
+                        cube = ((tt >> 2) * p.Cx + (xx >> 2)) * p.Cy + (yy >> 2);
+                    }
+                } else {
+                    const uint32_t qd = div_magic(static_cast<uint32_t>(blk), p.magic_cy);
+                    const uint32_t ct = div_magic(qd, p.magic_cx);
+                    const int cy = blk - static_cast<int>(qd) * p.Cy;
+                    const int cx = static_cast<int>(qd) - static_cast<int>(ct) * p.Cx;
+                    const int tt = 4 * static_cast<int>(ct) + (o_ >> 4);
+                    const int xx = 4 * cx + ((o_ >> 2) & 3), yy = 4 * cy + (o_ & 3);
+                    if (tt < p.T && xx < p.X && yy < p.Y) tok = (static_cast<int64_t>(tt) * p.X + xx) * p.Y + yy;
+                    cube = blk;
+                }
+            }
+            return tok;
+        };
+        int n_item = 0;
+        for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
+            const Item item = decode_item(it, p);
+            const int ip = n_item & 1;
+            const uint32_t ipar = static_cast<uint32_t>(n_item >> 1) & 1u;
+            const float* l_it = l_part + ip * (kTBufs * 128);
+            // inputs fetched while the item's steps run: this row's gates and (cube layout) the
+            // coarse output of the warp's query cube; and the next item's records, towards L1
+            int cube;
+            const int64_t tok = row_token(item, cube);
+            const bool store = tok >= 0;
+            const int64_t grow = (static_cast<int64_t>(item.b) * p.N + (store ? tok : 0)) * p.H + item.h;
+            float gc = 0.f, gf = 1.f;
+            if (store) {
+                if (p.g_coarse) gc = __uint_as_float(static_cast<uint32_t>(__ldg(p.g_coarse + grow)) << 16);
+                if (p.g_fine) gf = __uint_as_float(static_cast<uint32_t>(__ldg(p.g_fine + grow)) << 16);
+            }
+            const float* ocr = nullptr;
+            if (p.o_coarse != nullptr) {
+                if (LM == kLoadTokens) {
+                    ocr = p.o_coarse + (item.bh * p.C + cube) * D;
+                } else {
+                    const int cb = item.blk[slot];
+                    if (lane < D / 4) {
+                        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (cb >= 0) v = __ldg(reinterpret_cast<const float4*>(p.o_coarse + (item.bh * p.C + cb) * D) + lane);
+                        reinterpret_cast<float4*>(oc_w)[lane] = v;
+                    }
+                    __syncwarp();
+                    ocr = oc_w;
+                }
+            }
+            const int64_t nxt = it + gridDim.x;
+            if (nxt < p.items && q == 0 && lane < 3) {
+                if (lane < 2 && p.steps != nullptr && 128 * lane < 8 * p.steps_stride)
+                    prefetch_l1(reinterpret_cast<const uint8_t*>(p.steps + nxt * p.steps_stride) + 128 * lane);
+                if (lane == 2 && p.order != nullptr) {
+                    const int64_t nbh = nxt / p.ngroups, pos = p.group * (nxt - nbh * p.ngroups);
+                    if (pos < p.nblk) prefetch_l1(p.order + nbh * p.C + pos);
+                }
+            }
+            // the item's output accumulator is complete and the three groups' row sums are in
+            if (!(ok = wait_all(bar(kTBarODone), static_cast<uint32_t>(n_item) & 1u))) break;
+            if (!(ok = wait_all(bar(kTBarEpi + ip), ipar))) break;
+            tc_fence_after();
+            const float l_tot = (l_it[row] + l_it[128 + row]) + l_it[256 + row];
+            const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
+            const float sf = gf * inv_l;
+            // 32-column chunk ch of O (in registers) -> gated merge -> bf16 row segment
+            auto emit = [&](int ch, const uint32_t* o) {
+                float v[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(o[j]) * sf;
+                if (ocr != nullptr) {
+                    const float4* oc4 = reinterpret_cast<const float4*>(ocr + 32 * ch);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 cv = oc4[j];
+                        v[4 * j] = fmaf(gc, cv.x, v[4 * j]);
+                        v[4 * j + 1] = fmaf(gc, cv.y, v[4 * j + 1]);
+                        v[4 * j + 2] = fmaf(gc, cv.z, v[4 * j + 2]);
+                        v[4 * j + 3] = fmaf(gc, cv.w, v[4 * j + 3]);
+                    }
+                }
+                uint32_t w16[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) w16[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + 32 * ch);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                    dst[v4] = make_uint4(w16[4 * v4], w16[4 * v4 + 1], w16[4 * v4 + 2], w16[4 * v4 + 3]);
+            };
+            // O in two halves of 64 columns (D = 128) or one (D = 64); O is released after the
+            // last read, so the next item's first PV does not wait for the last stores
+            uint32_t o[64];
+            if constexpr (D == 128) {
+                tmem_ld64_wait(tO, o);
+                if (store) {
+                    emit(0, o);
+                    emit(1, o + 32);
+                }
+                tmem_ld64_wait(tO + 64u, o);
+            } else {
+                tmem_ld64_wait(tO, o);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kTBarOFree));   // O may be overwritten by the next item
+            if (store) {
+                emit(D / 32 - 2, o);
+                emit(D / 32 - 1, o + 32);
+            }
+        }
     } else {
-        // ------------------------------------------------------------ softmax groups + epilogue
+        // ------------------------------------------------------------ softmax groups
         const int g = warp >> 2;                 // group: score buffer g, steps s with s % 3 == g
         const int q = warp & 3;                  // TMEM lane quarter
         const int row = q * 32 + lane;           // query row of the tile, 0..127
         const int slot = q >> 1;                 // query block of the row
         const uint32_t lane_addr = static_cast<uint32_t>(q * 32) << 16;
         const uint32_t tS = tmem + 128u * g + lane_addr;
-        const uint32_t tO = tmem + kTColO + lane_addr;
         const float c = p.c_log2;
         uint32_t n_s = 0;                         // S-full phases consumed (buffer g)
-        uint32_t pvd[kTBufs] = {0u, 0u, 0u};      // PVs into each buffer so far, all steps of all items
         bool ok = true;
         auto wait_all = [&](uint32_t b, uint32_t par) -> bool {
             const bool mine = bw.wait(b, par);
@@ -1214,17 +1377,21 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         int n_item = 0;
         for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
             const Item item = decode_item(it, p);
+            // The groups go on to the next item while the epilogue warps write this one, so the
+            // maxima, the row sums and their barriers alternate between two sets by item parity.
+            const int ip = n_item & 1;
+            const uint32_t ipar = static_cast<uint32_t>(n_item >> 1) & 1u;
+            float* m_it = m_row + ip * 128;
+            float* l_it = l_part + ip * (kTBufs * 128);
+            const uint32_t mready = bar(kTBarMReady + 2 * ip + slot);
             float m = 0.f, l = 0.f;
             bool have_m = false;
             int sfirst = -1;     // first step that selects this row's query block (the same in every warp)
-            int last_b = 0;
             for (int s = 0;; ++s) {
                 const StepRec r = tile_step(p, it, s, item.present);
                 const bool sel_a = ((r.flags >> slot) & 1u) != 0u, sel_b = ((r.flags >> (4 + slot)) & 1u) != 0u;
                 if (sfirst < 0 && (sel_a || sel_b)) sfirst = s;
                 const int b = s % kTBufs;
-                ++pvd[b];
-                last_b = b;
                 if (b == g) {
                     if (!(ok = wait_all(bar(kTBarSFull + g), n_s & 1u))) break;
                     ++n_s;
@@ -1245,13 +1412,13 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                 mx = fmaxf(mx, max32(sc));
                             }
                             m = mx == -INFINITY ? 0.f : mx * c;
-                            m_row[row] = m;
+                            m_it[row] = m;
                             have_m = true;
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(bar(kTBarMReady + slot));   // release: m_row visible
+                            if (lane == 0) mbar_arrive(mready);   // release: the maximum is visible
                         } else if (!have_m) {
-                            if (!(ok = wait_all(bar(kTBarMReady + slot), n_item & 1))) break;
-                            m = m_row[row];
+                            if (!(ok = wait_all(mready, ipar))) break;
+                            m = m_it[row];
                             have_m = true;
                         }
                         float sum = 0.f;
@@ -1288,89 +1455,12 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // the block, group 0's two warps of the block make it
             if (sfirst < 0 && g == 0) {
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kTBarMReady + slot));
+                if (lane == 0) mbar_arrive(mready);
             }
-            // ---------------- epilogue: all three groups' sums, the item's last PV complete
-            l_part[g * 128 + row] = l;
-            if (!(ok = wait_all(bar(kTBarPVDone + last_b), (pvd[last_b] - 1u) & 1u))) break;
-            tc_fence_after();
+            // hand the row sums to the epilogue warps and go on
+            l_it[g * 128 + row] = l;
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kTBarEpi));
-            if (!(ok = wait_all(bar(kTBarEpi), n_item & 1))) break;
-            const float l_tot = (l_part[row] + l_part[128 + row]) + l_part[256 + row];
-            const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
-            const int blk = item.blk[slot];
-            const int o_ = row & 63;
-            int64_t tok = -1;
-            int cube = 0;
-            if (blk >= 0) {
-                if (LM == kLoadTokens) {
-                    tok = 64ll * blk + o_;
-                    if (tok >= p.N) {
-                        tok = -1;
-                    } else if (p.o_coarse != nullptr) {
-                        const int64_t xy = static_cast<int64_t>(p.X) * p.Y;
-                        const int tt = static_cast<int>(tok / xy);
-                        const int rem = static_cast<int>(tok - tt * xy);
-                        const int xx = rem / p.Y, yy = rem - (rem / p.Y) * p.Y;
-                        cube = ((tt >> 2) * p.Cx + (xx >> 2)) * p.Cy + (yy >> 2);
-                    }
-                } else {
-                    const uint32_t qd = div_magic(static_cast<uint32_t>(blk), p.magic_cy);
-                    const uint32_t ct = div_magic(qd, p.magic_cx);
-                    const int cy = blk - static_cast<int>(qd) * p.Cy;
-                    const int cx = static_cast<int>(qd) - static_cast<int>(ct) * p.Cx;
-                    const int tt = 4 * static_cast<int>(ct) + (o_ >> 4);
-                    const int xx = 4 * cx + ((o_ >> 2) & 3), yy = 4 * cy + (o_ & 3);
-                    if (tt < p.T && xx < p.X && yy < p.Y) tok = (static_cast<int64_t>(tt) * p.X + xx) * p.Y + yy;
-                    cube = blk;
-                }
-            }
-            const bool store = tok >= 0;
-            float gc = 0.f, gf = 1.f;
-            const float* ocr = nullptr;
-            const int64_t grow = (static_cast<int64_t>(item.b) * p.N + (store ? tok : 0)) * p.H + item.h;
-            if (store) {
-                if (p.g_coarse) gc = __uint_as_float(static_cast<uint32_t>(__ldg(p.g_coarse + grow)) << 16);
-                if (p.g_fine) gf = __uint_as_float(static_cast<uint32_t>(__ldg(p.g_fine + grow)) << 16);
-                if (p.o_coarse) ocr = p.o_coarse + (item.bh * p.C + cube) * D;
-            }
-            const float sf = gf * inv_l;
-            // channel chunks of 32: D = 128 -> group 0 takes 0 and 1, group 1 takes 2, group 2 takes 3;
-            // D = 64 -> groups 0 and 1 take one each
-            const int ch0 = D == 128 ? (g == 0 ? 0 : g + 1) : g;
-            const int ch1 = D == 128 ? (g == 0 ? 2 : g + 2) : (g < 2 ? g + 1 : g);
-#pragma unroll 1
-            for (int ch = ch0; ch < ch1; ++ch) {
-                uint32_t o[32];
-                tmem_ld32_wait(tO + 32u * ch, o);
-                if (store) {
-                    float v[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(o[j]) * sf;
-                    if (ocr != nullptr) {
-                        const float4* oc4 = reinterpret_cast<const float4*>(ocr + 32 * ch);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float4 cv = __ldg(oc4 + j);
-                            v[4 * j] = fmaf(gc, cv.x, v[4 * j]);
-                            v[4 * j + 1] = fmaf(gc, cv.y, v[4 * j + 1]);
-                            v[4 * j + 2] = fmaf(gc, cv.z, v[4 * j + 2]);
-                            v[4 * j + 3] = fmaf(gc, cv.w, v[4 * j + 3]);
-                        }
-                    }
-                    uint32_t w16[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) w16[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-                    uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + 32 * ch);
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        dst[v4] = make_uint4(w16[4 * v4], w16[4 * v4 + 1], w16[4 * v4 + 2], w16[4 * v4 + 3]);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kTBarOFree));   // O may be overwritten by the next item
+            if (lane == 0) mbar_arrive(bar(kTBarEpi + ip));   // release: the sums are visible
         }
     }
 
@@ -1736,8 +1826,8 @@ cudaError_t launch_schedule(const Dims& d, const int32_t* idx, int k, const int3
     a.k_sel = k;
     a.order = order;
     const FineParams p = make_params(d, a, kTileGroup);
+    if (p.items > 0x7FFFFFFFll) return cudaErrorInvalidValue;   // decode_item's 32-bit arithmetic
     const int64_t blocks = (p.items + kScheduleWarps - 1) / kScheduleWarps;
-    if (blocks > 0x7FFFFFFFll) return cudaErrorInvalidValue;
     if (blocks == 0) return cudaSuccess;
     schedule_kernel<<<static_cast<unsigned>(blocks), kScheduleWarps * 32, schedule_smem(d, k), s>>>(
         p, static_cast<uint2*>(steps));
@@ -1773,6 +1863,10 @@ cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const 
             return cudaErrorInvalidValue;
         }
         FineParams pt = make_params(d, a, kTileGroup);
+        if (pt.items > 0x7FFFFFFFll) {   // decode_item's 32-bit arithmetic
+            if (why) *why = "too many work items";
+            return cudaErrorInvalidValue;
+        }
         if (!pt.status) {
             if (why) *why = "watchdog word unavailable";
             return cudaErrorInvalidValue;
@@ -1796,6 +1890,10 @@ cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const 
                           : launch_instance<64, kLoadCubes, true>(tq, tk, tv, pr, gr, s);
     }
     FineParams p = make_params(d, a, 4);
+    if (p.items > 0x7FFFFFFFll) {   // decode_item's 32-bit arithmetic
+        if (why) *why = "too many work items";
+        return cudaErrorInvalidValue;
+    }
     if (!p.status) {
         if (why) *why = "watchdog word unavailable";
         return cudaErrorInvalidValue;
