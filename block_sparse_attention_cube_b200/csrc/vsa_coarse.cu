@@ -24,8 +24,9 @@ static_assert((kSTI / kSRI) * (kSTJ / kSRJ) == kThreads, "one output block per t
 // scores[bh][i][j] = scale * sum_d qbar[bh][i][d] * kbar[bh][j][d]
 // A 128x64 output tile per block; thread (ty, tx) owns rows 8ty..8ty+7 and
 // columns 4tx..4tx+3 (32 accumulators, 12 operands read from shared memory
-// per 32 fma).  Each output is one sequential float32 fma chain over the
-// channels, so the tile shape does not change a single bit of the result.
+// per 32 fma); the next 16-channel slice is loaded into registers while the
+// current one is multiplied.  Each output is one sequential float32 fma chain
+// over the channels, so the tiling does not change a single bit of the result.
 __global__ void __launch_bounds__(kThreads) coarse_scores_kernel(int C, int D, const float* __restrict__ qbar,
                                                                  const float* __restrict__ kbar, float scale,
                                                                  float* __restrict__ scores) {
@@ -38,23 +39,38 @@ __global__ void __launch_bounds__(kThreads) coarse_scores_kernel(int C, int D, c
     const float* Q = qbar + static_cast<int64_t>(bh) * C * D;
     const float* K = kbar + static_cast<int64_t>(bh) * C * D;
     float acc[kSRI][kSRJ] = {};
-    for (int d0 = 0; d0 < D; d0 += kBK) {
-        // the tile's rows x 16 channels of each operand, stored channel-major
+    // the tile's rows x 16 channels of each operand: this thread's share, loaded one slice ahead
+    constexpr int kLA = kSTI * kBK / kThreads, kLB = kSTJ * kBK / kThreads;
+    float ra[kLA], rb[kLB];
+    auto load_slice = [&](int d0) {
 #pragma unroll
-        for (int e = 0; e < kSTI * kBK / kThreads; ++e) {
+        for (int e = 0; e < kLA; ++e) {
             const int idx = threadIdx.x + e * kThreads;
-            const int r = idx / kBK, cc = idx % kBK;
-            const int gi = i0 + r;
-            As[cc][r] = gi < C ? Q[static_cast<int64_t>(gi) * D + d0 + cc] : 0.f;
+            const int gi = i0 + idx / kBK;
+            ra[e] = gi < C ? __ldg(Q + static_cast<int64_t>(gi) * D + d0 + idx % kBK) : 0.f;
         }
 #pragma unroll
-        for (int e = 0; e < kSTJ * kBK / kThreads; ++e) {
+        for (int e = 0; e < kLB; ++e) {
             const int idx = threadIdx.x + e * kThreads;
-            const int r = idx / kBK, cc = idx % kBK;
-            const int gj = j0 + r;
-            Bs[cc][r] = gj < C ? K[static_cast<int64_t>(gj) * D + d0 + cc] : 0.f;
+            const int gj = j0 + idx / kBK;
+            rb[e] = gj < C ? __ldg(K + static_cast<int64_t>(gj) * D + d0 + idx % kBK) : 0.f;
+        }
+    };
+    load_slice(0);
+    for (int d0 = 0; d0 < D; d0 += kBK) {
+        // stored channel-major; the next slice's loads are in flight while this one is multiplied
+#pragma unroll
+        for (int e = 0; e < kLA; ++e) {
+            const int idx = threadIdx.x + e * kThreads;
+            As[idx % kBK][idx / kBK] = ra[e];
+        }
+#pragma unroll
+        for (int e = 0; e < kLB; ++e) {
+            const int idx = threadIdx.x + e * kThreads;
+            Bs[idx % kBK][idx / kBK] = rb[e];
         }
         __syncthreads();
+        if (d0 + kBK < D) load_slice(d0 + kBK);
 #pragma unroll
         for (int kk = 0; kk < kBK; ++kk) {
             float av[kSRI], bv[kSRJ];

@@ -951,12 +951,14 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // its inputs (gates, the coarse outputs of the tile's query cubes) while the
 // item's steps run.  Because the groups run one item ahead of the epilogue,
 // the per-item maxima, row sums and their barriers come in two sets, used by
-// even and odd items; a group cannot get two items ahead, since its next
-// item's PVs queue behind the release of O.  The epilogue waits for the
+// even and odd items.  The epilogue waits for the
 // item's last PV on a barrier committed once per item: a wait by parity on
 // the last step's PV-done barrier would pass early whenever that buffer's
 // previous PV were still pending (a parity wait returns at once when the
-// barrier is one phase behind).
+// barrier is one phase behind).  A group that has no step in an item (items
+// of one or two steps) depends on nothing in it, so each group also waits,
+// before item n, until the epilogue has read item n - 2's row sums (SetFree):
+// no group runs more than one item ahead of the epilogue.
 //
 // A probability above 2^64 (a later score far above the first
 // maximum) or a non-finite sum raises the overflow word, and the caller then
@@ -991,7 +993,8 @@ constexpr int kTBarMReady = kTBarPVDone + kTBufs;                // [2 items][2 
 constexpr int kTBarEpi = kTBarMReady + 4;                        // [2 items], twelve arrivals
 constexpr int kTBarOFree = kTBarEpi + 2;                         // four arrivals (the epilogue warps)
 constexpr int kTBarODone = kTBarOFree + 1;                       // the item's last PV complete (one commit per item)
-constexpr int kTBarDrain = kTBarODone + 1;                       // [2 issuers]
+constexpr int kTBarSetFree = kTBarODone + 1;                     // [2 items], four arrivals: the set is read
+constexpr int kTBarDrain = kTBarSetFree + 2;                     // [2 issuers]
 constexpr int kTNumBars = kTBarDrain + 2;
 constexpr uint32_t kTOffMisc = kTOffBar + kTNumBars * 8;         // tmem slot (4 B) + abort flag (4 B)
 constexpr uint32_t kTSmemBytes = kTOffMisc + 16 + 1024;
@@ -1049,6 +1052,8 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_init(bar(kTBarEpi + 1), 12);
         mbar_init(bar(kTBarOFree), 4);
         mbar_init(bar(kTBarODone), 1);
+        mbar_init(bar(kTBarSetFree + 0), 4);
+        mbar_init(bar(kTBarSetFree + 1), 4);
         mbar_init(bar(kTBarDrain + 0), 1);
         mbar_init(bar(kTBarDrain + 1), 1);
         fence_mbar_init();
@@ -1312,6 +1317,8 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (!(ok = wait_all(bar(kTBarEpi + ip), ipar))) break;
             tc_fence_after();
             const float l_tot = (l_it[row] + l_it[128 + row]) + l_it[256 + row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kTBarSetFree + ip));   // this item's set may be reused
             const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
             const float sf = gf * inv_l;
             // 32-column chunk ch of O (in registers) -> gated merge -> bf16 row segment
@@ -1384,6 +1391,11 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             float* m_it = m_row + ip * 128;
             float* l_it = l_part + ip * (kTBufs * 128);
             const uint32_t mready = bar(kTBarMReady + 2 * ip + slot);
+            // The set was last used by item n - 2: its row sums must have been read.  A group with no
+            // step in an item depends on nothing else, so without this wait it could run two items
+            // ahead and arrive on a barrier phase that belongs to the earlier item.
+            if (n_item >= 2 && !(ok = wait_all(bar(kTBarSetFree + ip), static_cast<uint32_t>((n_item - 2) >> 1) & 1u)))
+                break;
             float m = 0.f, l = 0.f;
             bool have_m = false;
             int sfirst = -1;     // first step that selects this row's query block (the same in every warp)

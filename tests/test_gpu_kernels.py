@@ -365,6 +365,35 @@ def test_repeated_calls_are_deterministic():
     assert torch.equal(a, b)
 
 
+def test_one_tile_kernel_with_many_items_per_cta():
+    """160 heads of an 8x8x8 grid at top-k 2: 640 work items of one or two steps over at most one CTA per
+    SM, so every CTA carries several items and the per-item hand-overs between the softmax groups, the
+    epilogue warps and the next item's first steps happen many times.  The fused fine stage with
+    precomputed steps (the one-tile kernel) must match the oracle on every head and give the same bits
+    on every one of 20 repeated launches; the whole forward call must repeat bit for bit too."""
+    w = synth.custom_workload("many_items_8x8x8", 1, 160, 64, (8, 8, 8), 2, field=True, wid=97)
+    x = synth.make_inputs(w)
+    d = {k: to_dev(v) for k, v in x.items()}
+    f64 = {k: O.bf16_to_f64(v) for k, v in x.items()}
+    s = _shape(w)
+    scale = 1 / math.sqrt(w.head_dim)
+    ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, w.topk, scale, f64["g_coarse"], f64["g_fine"])
+    idx = torch.from_numpy(ora["idx"]).cuda()
+    steps = vsa.schedule(idx, s)
+    first = vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, steps=steps)
+    ref = O.untile(ora["o_fine"], w.grid)
+    got = from_dev(first)
+    for h in range(w.heads):
+        check_close(got[0, :, h], ref[0, :, h], f"many items fine_fused h={h}")
+    for rep in range(20):
+        again = vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, steps=steps)
+        assert torch.equal(again.view(torch.int16), first.view(torch.int16)), f"launch {rep} differs"
+    a = vsa.forward(d["q"], d["k"], d["v"], s, w.topk, scale, d["g_coarse"], d["g_fine"])
+    for rep in range(5):
+        b = vsa.forward(d["q"], d["k"], d["v"], s, w.topk, scale, d["g_coarse"], d["g_fine"])
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"forward call {rep} differs"
+
+
 def test_forward_host_matches_device_forward():
     w = synth.WORKLOADS["padded_7x15x16"]
     x = synth.make_inputs(w)
