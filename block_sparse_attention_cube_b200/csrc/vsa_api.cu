@@ -110,6 +110,49 @@ vsa_status check_device() {
 
 cudaStream_t as_stream(vsa_stream_t s) { return static_cast<cudaStream_t>(s); }
 
+// vsa_forward_host's two copy streams (host->device, device->host) of the current device, created
+// on first use and kept for the life of the process.
+vsa_status copy_streams(cudaStream_t* up_s, cudaStream_t* down_s) {
+    static std::mutex mu;
+    static cudaStream_t streams[64][2] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(VSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < 2; ++i) {
+        if (streams[dev][i] != nullptr) continue;
+        if ((e = cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking)) != cudaSuccess) {
+            streams[dev][i] = nullptr;
+            return cuda_fail(e, "cudaStreamCreateWithFlags");
+        }
+    }
+    *up_s = streams[dev][0];
+    *down_s = streams[dev][1];
+    return VSA_OK;
+}
+
+// vsa_forward_host: head groups per call (the copies of one overlap the compute of another)
+constexpr int kHostGroups = 8;
+
+// Events of one vsa_forward_host call, destroyed when it returns (CUDA keeps a recorded event
+// alive until the work it marks is done).
+struct EventSet {
+    cudaEvent_t e[2 * kHostGroups + 2] = {};
+    int n = 0;
+    cudaError_t create(int count) {
+        for (; n < count; ++n) {
+            const cudaError_t r = cudaEventCreateWithFlags(&e[n], cudaEventDisableTiming);
+            if (r != cudaSuccess) return r;
+        }
+        return cudaSuccess;
+    }
+    cudaEvent_t operator[](int i) const { return e[i]; }
+    ~EventSet() {
+        for (int i = 0; i < n; ++i) cudaEventDestroy(e[i]);
+    }
+};
+
 size_t tiled_bytes(const Dims& d) { return static_cast<size_t>(d.rows) * d.D * 2; }
 size_t token_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.N * d.H * d.D * 2; }
 size_t gate_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.N * d.H * 2; }
@@ -656,13 +699,77 @@ vsa_status vsa_forward_host(const vsa_shape* shape, const vsa_bf16* q, const vsa
     uint16_t* dgc = g_coarse ? reinterpret_cast<uint16_t*>(w + fwd + 4 * up(tb)) : nullptr;
     uint16_t* dgf = g_fine ? reinterpret_cast<uint16_t*>(w + fwd + 4 * up(tb) + up(gb)) : nullptr;
     cudaStream_t s = as_stream(stream);
-    VSA_CUDA(cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, s), "copy q to device");
-    VSA_CUDA(cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, s), "copy k to device");
-    VSA_CUDA(cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, s), "copy v to device");
-    if (dgc) VSA_CUDA(cudaMemcpyAsync(dgc, g_coarse, gb, cudaMemcpyHostToDevice, s), "copy g_coarse to device");
-    if (dgf) VSA_CUDA(cudaMemcpyAsync(dgf, g_fine, gb, cudaMemcpyHostToDevice, s), "copy g_fine to device");
-    VSA_TRY(run_forward(d, dq, dk, dv, dgc, dgf, topk, scale, workspace, dout, s));
-    VSA_CUDA(cudaMemcpyAsync(out, dout, tb, cudaMemcpyDeviceToHost, s), "copy out to host");
+
+    // Head groups: the heads never mix, so the call runs group by group, and the host->device copies of
+    // group g+1 and the device->host copy of group g-1 overlap the compute of group g (two copy streams
+    // of the library's, ordered against `stream` by events).  A group's q, k, v and output live compact,
+    // [B, N, hn, D], one after the other in the staging buffers; its gates are gathered on the device
+    // from the whole arrays into the part of the forward workspace that the smaller call leaves free.
+    const int64_t rows = static_cast<int64_t>(d.B) * d.N;
+    int hg = d.H >= 2 ? (d.H + kHostGroups - 1) / kHostGroups : d.H;
+    Dims dg{};
+    vsa_shape sg = *shape;
+    sg.heads = hg;
+    size_t gate_g = 0, fwd_g = 0;
+    if (hg < d.H && make_dims(&sg, &dg) == VSA_OK) {
+        fwd_g = carve(dg, topk, true, nullptr).bytes;
+        gate_g = up(static_cast<size_t>(rows) * hg * 2);
+        if (fwd_g + 2 * gate_g > fwd) hg = d.H;   // no room for the gathered gates: one group
+    } else {
+        hg = d.H;
+    }
+    if (hg == d.H) {
+        VSA_CUDA(cudaMemcpyAsync(dq, q, tb, cudaMemcpyHostToDevice, s), "copy q to device");
+        VSA_CUDA(cudaMemcpyAsync(dk, k, tb, cudaMemcpyHostToDevice, s), "copy k to device");
+        VSA_CUDA(cudaMemcpyAsync(dv, v, tb, cudaMemcpyHostToDevice, s), "copy v to device");
+        if (dgc) VSA_CUDA(cudaMemcpyAsync(dgc, g_coarse, gb, cudaMemcpyHostToDevice, s), "copy g_coarse to device");
+        if (dgf) VSA_CUDA(cudaMemcpyAsync(dgf, g_fine, gb, cudaMemcpyHostToDevice, s), "copy g_fine to device");
+        VSA_TRY(run_forward(d, dq, dk, dv, dgc, dgf, topk, scale, workspace, dout, s));
+        VSA_CUDA(cudaMemcpyAsync(out, dout, tb, cudaMemcpyDeviceToHost, s), "copy out to host");
+        return VSA_OK;
+    }
+    cudaStream_t up_s = nullptr, down_s = nullptr;
+    VSA_TRY(copy_streams(&up_s, &down_s));
+    const int groups = (d.H + hg - 1) / hg;
+    EventSet ev;
+    VSA_CUDA(ev.create(2 * groups + 2), "create events");
+    uint16_t* cgc = dgc ? reinterpret_cast<uint16_t*>(w + fwd_g) : nullptr;
+    uint16_t* cgf = dgf ? reinterpret_cast<uint16_t*>(w + fwd_g + gate_g) : nullptr;
+    // everything already on `stream` (earlier users of the workspace) comes first
+    VSA_CUDA(cudaEventRecord(ev[0], s), "record start");
+    VSA_CUDA(cudaStreamWaitEvent(up_s, ev[0], 0), "order copies");
+    VSA_CUDA(cudaStreamWaitEvent(down_s, ev[0], 0), "order copies");
+    if (dgc) VSA_CUDA(cudaMemcpyAsync(dgc, g_coarse, gb, cudaMemcpyHostToDevice, up_s), "copy g_coarse to device");
+    if (dgf) VSA_CUDA(cudaMemcpyAsync(dgf, g_fine, gb, cudaMemcpyHostToDevice, up_s), "copy g_fine to device");
+    const size_t row_all = static_cast<size_t>(d.H) * d.D * 2;
+    for (int gi = 0; gi < groups; ++gi) {
+        const int h0 = gi * hg, hn = d.H - h0 < hg ? d.H - h0 : hg;
+        const size_t off = static_cast<size_t>(rows) * h0 * d.D;   // elements before this group's block
+        const size_t row_g = static_cast<size_t>(hn) * d.D * 2;
+        const size_t src_off = static_cast<size_t>(h0) * d.D;
+        VSA_CUDA(cudaMemcpy2DAsync(dq + off, row_g, q + src_off, row_all, row_g, rows, cudaMemcpyHostToDevice, up_s),
+                 "copy q to device");
+        VSA_CUDA(cudaMemcpy2DAsync(dk + off, row_g, k + src_off, row_all, row_g, rows, cudaMemcpyHostToDevice, up_s),
+                 "copy k to device");
+        VSA_CUDA(cudaMemcpy2DAsync(dv + off, row_g, v + src_off, row_all, row_g, rows, cudaMemcpyHostToDevice, up_s),
+                 "copy v to device");
+        VSA_CUDA(cudaEventRecord(ev[1 + gi], up_s), "record upload");
+        VSA_CUDA(cudaStreamWaitEvent(s, ev[1 + gi], 0), "wait upload");
+        sg.heads = hn;
+        Dims dh{};
+        VSA_TRY(make_dims(&sg, &dh));
+        if (cgc) VSA_CUDA(launch_gather_heads(dgc, rows, d.H, h0, hn, cgc, s), "gate gather launch");
+        if (cgf) VSA_CUDA(launch_gather_heads(dgf, rows, d.H, h0, hn, cgf, s), "gate gather launch");
+        VSA_TRY(run_forward(dh, dq + off, dk + off, dv + off, cgc, cgf, topk, scale, workspace, dout + off, s));
+        VSA_CUDA(cudaEventRecord(ev[1 + groups + gi], s), "record compute");
+        VSA_CUDA(cudaStreamWaitEvent(down_s, ev[1 + groups + gi], 0), "wait compute");
+        VSA_CUDA(cudaMemcpy2DAsync(out + src_off, row_all, dout + off, row_g, row_g, rows, cudaMemcpyDeviceToHost,
+                                   down_s),
+                 "copy out to host");
+    }
+    // the call is complete on `stream` once the last output copy is
+    VSA_CUDA(cudaEventRecord(ev[1 + 2 * groups], down_s), "record end");
+    VSA_CUDA(cudaStreamWaitEvent(s, ev[1 + 2 * groups], 0), "wait end");
     return VSA_OK;
 }
 

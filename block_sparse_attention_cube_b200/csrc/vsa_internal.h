@@ -131,6 +131,11 @@ cudaError_t launch_norm_rope(const Dims& d, const NormRopeArgs& a, cudaStream_t 
 
 // Cube mean-pool read straight from the projection layout [B, N, H, D]
 // (same fp32 summation order as launch_pool on the tiled tensor).
+// dst[r][j] = src[r][h0 + j] for r < rows, j < hg: a head range of per-(token, head) values [rows, H]
+// (the gates) gathered into [rows, hg].
+cudaError_t launch_gather_heads(const uint16_t* src, int64_t rows, int H, int h0, int hg, uint16_t* dst,
+                                cudaStream_t s);
+
 cudaError_t launch_pool_tokens(const Dims& d, const uint16_t* const* x, float* const* xbar, int count,
                                cudaStream_t s);
 

@@ -300,6 +300,26 @@ cudaError_t launch_pool_tokens(const Dims& d, const uint16_t* const* x, float* c
     return cudaGetLastError();
 }
 
+namespace {
+__global__ void gather_heads_kernel(const uint16_t* __restrict__ src, int64_t rows, int H, int h0, int hg,
+                                    uint16_t* __restrict__ dst) {
+    const int64_t total = rows * hg;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t r = i / hg;
+        dst[i] = src[r * H + h0 + (i - r * hg)];
+    }
+}
+}  // namespace
+
+cudaError_t launch_gather_heads(const uint16_t* src, int64_t rows, int H, int h0, int hg, uint16_t* dst,
+                                cudaStream_t s) {
+    if (rows <= 0 || hg <= 0) return cudaSuccess;
+    const int grid = grid_for((rows * hg + kBlock - 1) / kBlock, 8);
+    gather_heads_kernel<<<grid, kBlock, 0, s>>>(src, rows, H, h0, hg, dst);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const Dims& d, const float* o_coarse, const uint16_t* o_fine, const uint16_t* g_coarse,
                            const uint16_t* g_fine, uint16_t* o_tiled, cudaStream_t s) {
     const int grid = grid_for(static_cast<int64_t>(d.B) * d.H * d.C, 8);

@@ -30,7 +30,8 @@
  *  * Every pointer argument is a DEVICE pointer owned by the caller, except in
  *    vsa_forward_host where the tensors are HOST pointers.  The library never
  *    allocates or frees memory and keeps no device state other than one
- *    watchdog status word per device.
+ *    watchdog status word per device (and, once vsa_forward_host has run on a
+ *    device, that function's two copy streams).
  *  * Every device pointer must be 16-byte aligned; input and output ranges of
  *    one call must not overlap.
  *  * `stream` is a cudaStream_t passed as an opaque pointer (NULL = the
@@ -345,11 +346,21 @@ vsa_status vsa_forward(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16
 size_t vsa_workspace_bytes_host(const vsa_shape* shape, int32_t topk);
 
 /*
- * vsa_forward_host — vsa_forward on HOST tensors: copies q, k, v and the
- * gates host->device (one cudaMemcpyAsync each), runs the call, copies the
- * output device->host, all on `stream`.  Host buffers should be pinned for
- * the copies to be asynchronous; the call returns once the work is enqueued
- * and `out` is valid after the stream is synchronized.
+ * vsa_forward_host — vsa_forward on HOST tensors.  The heads are independent
+ * (Wan2.2 teardown, zharfai.com, section "Video sparse attention selects
+ * cubes": attention per head), so with two or more heads the call runs in up
+ * to eight groups of heads: each group's q, k and v are copied host->device
+ * (2-D copies of its head range into compact staging), its call runs on
+ * `stream`, and its output is copied back into its head range of `out`; the
+ * copies run on two copy streams of the library's, ordered against `stream`
+ * by events, so the uploads of one group and the download of another overlap
+ * the compute of a third.  The gates are copied whole and gathered per group
+ * on the device.  The result is bit-identical to vsa_forward on the same
+ * inputs.  Everything already enqueued on `stream` happens before the copies,
+ * and the call's last copy is complete when `stream` reaches the point after
+ * the call.  Host buffers must be pinned for the copies to be asynchronous
+ * (pageable buffers work, without overlap); the call returns once the work
+ * is enqueued and `out` is valid after the stream is synchronized.
  *   q, k, v, g_coarse, g_fine, out: HOST pointers (gates may be NULL).
  *   workspace: DEVICE buffer of vsa_workspace_bytes_host(shape, topk) bytes.
  */

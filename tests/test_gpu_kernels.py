@@ -394,18 +394,37 @@ def test_one_tile_kernel_with_many_items_per_cta():
         assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"forward call {rep} differs"
 
 
-def test_forward_host_matches_device_forward():
-    w = synth.WORKLOADS["padded_7x15x16"]
+HOST_CASES = {
+    # name: (workload, gates): 4 heads -> four groups of one head; 1 head -> one group (no pipeline);
+    # 11 heads -> groups of two heads with a last group of one, no gates; B = 2, d = 64
+    "padded_4_heads": ("padded_7x15x16", True),
+    "one_head": (("one_head_7x15x16", 1, 1, 128, (7, 15, 16), 8), True),
+    "eleven_heads_no_gates": (("eleven_heads_9x6x5", 2, 11, 64, (9, 6, 5), 4), False),
+}
+
+
+@pytest.mark.parametrize("name", list(HOST_CASES))
+def test_forward_host_matches_device_forward(name):
+    """vsa_forward_host (head groups, copy streams, gathered gates) gives the bits of vsa_forward, twice in a
+    row on the same workspace (the second call's copies must wait for the first call's work)."""
+    spec, gates = HOST_CASES[name]
+    w = synth.WORKLOADS[spec] if isinstance(spec, str) else synth.custom_workload(*spec[:5], spec[5], wid=98)
     x = synth.make_inputs(w)
     d = {k: to_dev(v) for k, v in x.items()}
     h = {k: d[k].cpu().pin_memory() for k in d}
     s = _shape(w)
-    ref = vsa.forward(d["q"], d["k"], d["v"], s, w.topk, None, d["g_coarse"], d["g_fine"])
+    gc, gf = (d["g_coarse"], d["g_fine"]) if gates else (None, None)
+    hgc, hgf = (h["g_coarse"], h["g_fine"]) if gates else (None, None)
+    ref = vsa.forward(d["q"], d["k"], d["v"], s, w.topk, None, gc, gf)
     ws = vsa.alloc_workspace(s, w.topk, host_io=True)
-    out = torch.empty_like(h["q"]).pin_memory()
-    vsa.forward_host(h["q"], h["k"], h["v"], s, w.topk, ws, out, None, h["g_coarse"], h["g_fine"])
+    out1 = torch.empty_like(h["q"]).pin_memory()
+    out2 = torch.empty_like(h["q"]).pin_memory()
+    vsa.forward_host(h["q"], h["k"], h["v"], s, w.topk, ws, out1, None, hgc, hgf)
+    vsa.forward_host(h["q"], h["k"], h["v"], s, w.topk, ws, out2, None, hgc, hgf)
     torch.cuda.current_stream().synchronize()
-    assert torch.equal(out, ref.cpu())
+    r = ref.cpu()
+    assert torch.equal(out1, r)
+    assert torch.equal(out2, r)
 
 
 def test_group_is_a_permutation_and_does_not_change_the_output(case):
