@@ -402,9 +402,10 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                           "per_launch": "Q and K read once and written once: 4*B*N*H*D*2 bytes"},
         "e2e": {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "vsa_forward_host (pinned host q/k/v/gates in, host out)"},
-        # VSA: pool, coarse (2), top-k, order sort, schedule, fine (one-tile kernel) and the re-run guard
-        # (fine_kernel, which returns at once unless the one-tile kernel overflowed); dense: fine
-        "gpu_launches": 10 * args.steps,
+        # per step, VSA call: pool, coarse scores, coarse softmax x V, top-k, order sort, schedule, fine
+        # (one-tile kernel) and the re-run guard (fine_kernel, which returns at once unless the one-tile
+        # kernel overflowed) = 8; dense call: fine = 1
+        "gpu_launches": 9 * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
         "context": {"pages_dense_call_ms_b200": 17.0, "pages_vsa_kernel_ms_b200_k78": 4.719,

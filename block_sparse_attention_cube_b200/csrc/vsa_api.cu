@@ -110,9 +110,9 @@ vsa_status check_device() {
 
 cudaStream_t as_stream(vsa_stream_t s) { return static_cast<cudaStream_t>(s); }
 
-// vsa_forward_host's two copy streams (host->device, device->host) of the current device, created
+// vsa_forward_host's copy streams on the current device (0: host->device, 1: device->host), created
 // on first use and kept for the life of the process.
-vsa_status copy_streams(cudaStream_t* up_s, cudaStream_t* down_s) {
+vsa_status lib_stream(int which, cudaStream_t* out) {
     static std::mutex mu;
     static cudaStream_t streams[64][2] = {};
     int dev = 0;
@@ -120,15 +120,13 @@ vsa_status copy_streams(cudaStream_t* up_s, cudaStream_t* down_s) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= 64) return fail(VSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
     std::lock_guard<std::mutex> lock(mu);
-    for (int i = 0; i < 2; ++i) {
-        if (streams[dev][i] != nullptr) continue;
-        if ((e = cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking)) != cudaSuccess) {
-            streams[dev][i] = nullptr;
+    if (streams[dev][which] == nullptr) {
+        if ((e = cudaStreamCreateWithFlags(&streams[dev][which], cudaStreamNonBlocking)) != cudaSuccess) {
+            streams[dev][which] = nullptr;
             return cuda_fail(e, "cudaStreamCreateWithFlags");
         }
     }
-    *up_s = streams[dev][0];
-    *down_s = streams[dev][1];
+    *out = streams[dev][which];
     return VSA_OK;
 }
 
@@ -271,8 +269,10 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
         const uint16_t* pin[3] = {q, k, v};
         float* pout[3] = {c.qbar, c.kbar, c.vbar};
         VSA_CUDA(launch_pool_tokens(d, pin, pout, 3, s), "pool launch");
-        VSA_CUDA(launch_coarse(d, c.qbar, c.kbar, c.vbar, scale, c.scores, c.oc, s), "coarse launch");
+        VSA_CUDA(launch_coarse_scores(d, c.qbar, c.kbar, scale, c.scores, s), "coarse launch");
     }
+    // the coarse output (softmax(scores) x V-bar) is used only by the merge, and only with a coarse gate
+    if (gc != nullptr) VSA_CUDA(launch_coarse_pv(d, c.scores, c.vbar, c.oc, s), "coarse launch");
     const int32_t* order = nullptr;
     if (sparse) {
         if (d.C <= kTopkRegMaxC && d.C <= kGroupMaxC) {
@@ -729,7 +729,8 @@ vsa_status vsa_forward_host(const vsa_shape* shape, const vsa_bf16* q, const vsa
         return VSA_OK;
     }
     cudaStream_t up_s = nullptr, down_s = nullptr;
-    VSA_TRY(copy_streams(&up_s, &down_s));
+    VSA_TRY(lib_stream(0, &up_s));
+    VSA_TRY(lib_stream(1, &down_s));
     const int groups = (d.H + hg - 1) / hg;
     EventSet ev;
     VSA_CUDA(ev.create(2 * groups + 2), "create events");

@@ -486,17 +486,27 @@ cudaError_t launch_group(const Dims& d, const float* scores, int32_t* order, cud
     return cudaGetLastError();
 }
 
-cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
-                          float* scores, float* o_coarse, cudaStream_t s) {
+cudaError_t launch_coarse_scores(const Dims& d, const float* qbar, const float* kbar, float scale, float* scores,
+                                 cudaStream_t s) {
     const int bh = d.B * d.H;
     const dim3 grid((d.C + kSTJ - 1) / kSTJ, (d.C + kSTI - 1) / kSTI, bh);
     coarse_scores_kernel<<<grid, kThreads, 0, s>>>(d.C, d.D, qbar, kbar, scale, scores);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_coarse_pv(const Dims& d, const float* scores, const float* vbar, float* o_coarse, cudaStream_t s) {
+    const int bh = d.B * d.H;
     const int pv_blocks = (d.C + kPvRows - 1) / kPvRows;
     if (d.D == 128) coarse_pv_kernel<128><<<dim3(pv_blocks, bh), kThreads, 0, s>>>(d.C, scores, vbar, o_coarse);
     else coarse_pv_kernel<64><<<dim3(pv_blocks, bh), kThreads, 0, s>>>(d.C, scores, vbar, o_coarse);
     return cudaGetLastError();
+}
+
+cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
+                          float* scores, float* o_coarse, cudaStream_t s) {
+    const cudaError_t e = launch_coarse_scores(d, qbar, kbar, scale, scores, s);
+    if (e != cudaSuccess) return e;
+    return launch_coarse_pv(d, scores, vbar, o_coarse, s);
 }
 
 // Largest C the selection kernel keeps in shared memory (one row per warp).

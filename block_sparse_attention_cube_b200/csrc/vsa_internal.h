@@ -50,6 +50,10 @@ cudaError_t launch_untile(const Dims& d, const uint16_t* xt, uint16_t* x, cudaSt
 cudaError_t launch_pool(const Dims& d, const uint16_t* const* xt, float* const* xbar, int count, cudaStream_t s);
 cudaError_t launch_combine(const Dims& d, const float* o_coarse, const uint16_t* o_fine, const uint16_t* g_coarse,
                            const uint16_t* g_fine, uint16_t* o_tiled, cudaStream_t s);
+// The two halves of launch_coarse: the scores, and softmax(scores) x vbar.
+cudaError_t launch_coarse_scores(const Dims& d, const float* qbar, const float* kbar, float scale, float* scores,
+                                 cudaStream_t s);
+cudaError_t launch_coarse_pv(const Dims& d, const float* scores, const float* vbar, float* o_coarse, cudaStream_t s);
 cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
                           float* scores, float* o_coarse, cudaStream_t s);
 cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx, cudaStream_t s);

@@ -319,6 +319,8 @@ size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
  * vsa_forward — the whole attention call on one stream, as eight launches:
  *   vsa_pool_qkv -> vsa_coarse (2) -> vsa_topk_order (2) -> vsa_schedule
  *   -> vsa_fine_fused (the one-tile kernel and its re-run guard)
+ * (the second vsa_coarse launch, the coarse output softmax(scores) x V-bar,
+ * is skipped when g_coarse is NULL, since only the merge uses it)
  * (vsa_topk -> vsa_group instead when C > 2048; the grouping step is skipped
  * when C > 4096).  vsa_pair_order is not part of it: on the 480p workload its
  * better pairs save about as much fine-stage time as the pass costs.  The
