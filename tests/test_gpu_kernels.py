@@ -214,6 +214,12 @@ def test_forward_matches_oracle(case):
     _compare_call(w, dev, f64, w.topk, 1 / math.sqrt(w.head_dim))
 
 
+def test_forward_without_gates_matches_oracle(case):
+    """Both gates NULL (g_c = 0, g_f = 1): the call skips the coarse output, which only the merge uses."""
+    w, _, dev, f64 = case
+    _compare_call(w, dev, f64, w.topk, 1 / math.sqrt(w.head_dim), gates=False)
+
+
 def test_combine_matches_oracle(case):
     w, _, dev, f64 = case
     s = _shape(w)
