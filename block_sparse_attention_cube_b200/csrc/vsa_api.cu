@@ -297,6 +297,61 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
                           gf, out, c.overflow, s);
 }
 
+// vsa_forward_host's pipeline over head groups of hg heads (see vsa_forward_host): uploads on up_s,
+// compute on s, downloads on down_s, ordered by events; `stream` waits for the last download.
+vsa_status forward_host_groups(const Dims& d, const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k,
+                               const vsa_bf16* v, const vsa_bf16* g_coarse, const vsa_bf16* g_fine, int32_t topk,
+                               float scale, void* workspace, int hg, size_t fwd_g, size_t gate_g,
+                               uint16_t* dq, uint16_t* dk, uint16_t* dv, uint16_t* dout, uint16_t* dgc,
+                               uint16_t* dgf, vsa_bf16* out, cudaStream_t s, cudaStream_t up_s,
+                               cudaStream_t down_s) {
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    const int64_t rows = static_cast<int64_t>(d.B) * d.N;
+    const size_t gb = gate_bytes(d);
+    vsa_shape sg = *shape;
+    const int groups = (d.H + hg - 1) / hg;
+    EventSet ev;
+    VSA_CUDA(ev.create(2 * groups + 2), "create events");
+    uint16_t* cgc = dgc ? reinterpret_cast<uint16_t*>(w + fwd_g) : nullptr;
+    uint16_t* cgf = dgf ? reinterpret_cast<uint16_t*>(w + fwd_g + gate_g) : nullptr;
+    // everything already on `stream` (earlier users of the workspace) comes first
+    VSA_CUDA(cudaEventRecord(ev[0], s), "record start");
+    VSA_CUDA(cudaStreamWaitEvent(up_s, ev[0], 0), "order copies");
+    VSA_CUDA(cudaStreamWaitEvent(down_s, ev[0], 0), "order copies");
+    if (dgc) VSA_CUDA(cudaMemcpyAsync(dgc, g_coarse, gb, cudaMemcpyHostToDevice, up_s), "copy g_coarse to device");
+    if (dgf) VSA_CUDA(cudaMemcpyAsync(dgf, g_fine, gb, cudaMemcpyHostToDevice, up_s), "copy g_fine to device");
+    const size_t row_all = static_cast<size_t>(d.H) * d.D * 2;
+    for (int gi = 0; gi < groups; ++gi) {
+        const int h0 = gi * hg, hn = d.H - h0 < hg ? d.H - h0 : hg;
+        const size_t off = static_cast<size_t>(rows) * h0 * d.D;   // elements before this group's block
+        const size_t row_g = static_cast<size_t>(hn) * d.D * 2;
+        const size_t src_off = static_cast<size_t>(h0) * d.D;
+        VSA_CUDA(cudaMemcpy2DAsync(dq + off, row_g, q + src_off, row_all, row_g, rows, cudaMemcpyHostToDevice, up_s),
+                 "copy q to device");
+        VSA_CUDA(cudaMemcpy2DAsync(dk + off, row_g, k + src_off, row_all, row_g, rows, cudaMemcpyHostToDevice, up_s),
+                 "copy k to device");
+        VSA_CUDA(cudaMemcpy2DAsync(dv + off, row_g, v + src_off, row_all, row_g, rows, cudaMemcpyHostToDevice, up_s),
+                 "copy v to device");
+        VSA_CUDA(cudaEventRecord(ev[1 + gi], up_s), "record upload");
+        VSA_CUDA(cudaStreamWaitEvent(s, ev[1 + gi], 0), "wait upload");
+        sg.heads = hn;
+        Dims dh{};
+        VSA_TRY(make_dims(&sg, &dh));
+        if (cgc) VSA_CUDA(launch_gather_heads(dgc, rows, d.H, h0, hn, cgc, s), "gate gather launch");
+        if (cgf) VSA_CUDA(launch_gather_heads(dgf, rows, d.H, h0, hn, cgf, s), "gate gather launch");
+        VSA_TRY(run_forward(dh, dq + off, dk + off, dv + off, cgc, cgf, topk, scale, workspace, dout + off, s));
+        VSA_CUDA(cudaEventRecord(ev[1 + groups + gi], s), "record compute");
+        VSA_CUDA(cudaStreamWaitEvent(down_s, ev[1 + groups + gi], 0), "wait compute");
+        VSA_CUDA(cudaMemcpy2DAsync(out + src_off, row_all, dout + off, row_g, row_g, rows, cudaMemcpyDeviceToHost,
+                                   down_s),
+                 "copy out to host");
+    }
+    // the call is complete on `stream` once the last output copy is
+    VSA_CUDA(cudaEventRecord(ev[1 + 2 * groups], down_s), "record end");
+    VSA_CUDA(cudaStreamWaitEvent(s, ev[1 + 2 * groups], 0), "wait end");
+    return VSA_OK;
+}
+
 }  // namespace
 
 int sm_count() {
@@ -731,47 +786,21 @@ vsa_status vsa_forward_host(const vsa_shape* shape, const vsa_bf16* q, const vsa
     cudaStream_t up_s = nullptr, down_s = nullptr;
     VSA_TRY(lib_stream(0, &up_s));
     VSA_TRY(lib_stream(1, &down_s));
-    const int groups = (d.H + hg - 1) / hg;
-    EventSet ev;
-    VSA_CUDA(ev.create(2 * groups + 2), "create events");
-    uint16_t* cgc = dgc ? reinterpret_cast<uint16_t*>(w + fwd_g) : nullptr;
-    uint16_t* cgf = dgf ? reinterpret_cast<uint16_t*>(w + fwd_g + gate_g) : nullptr;
-    // everything already on `stream` (earlier users of the workspace) comes first
-    VSA_CUDA(cudaEventRecord(ev[0], s), "record start");
-    VSA_CUDA(cudaStreamWaitEvent(up_s, ev[0], 0), "order copies");
-    VSA_CUDA(cudaStreamWaitEvent(down_s, ev[0], 0), "order copies");
-    if (dgc) VSA_CUDA(cudaMemcpyAsync(dgc, g_coarse, gb, cudaMemcpyHostToDevice, up_s), "copy g_coarse to device");
-    if (dgf) VSA_CUDA(cudaMemcpyAsync(dgf, g_fine, gb, cudaMemcpyHostToDevice, up_s), "copy g_fine to device");
-    const size_t row_all = static_cast<size_t>(d.H) * d.D * 2;
-    for (int gi = 0; gi < groups; ++gi) {
-        const int h0 = gi * hg, hn = d.H - h0 < hg ? d.H - h0 : hg;
-        const size_t off = static_cast<size_t>(rows) * h0 * d.D;   // elements before this group's block
-        const size_t row_g = static_cast<size_t>(hn) * d.D * 2;
-        const size_t src_off = static_cast<size_t>(h0) * d.D;
-        VSA_CUDA(cudaMemcpy2DAsync(dq + off, row_g, q + src_off, row_all, row_g, rows, cudaMemcpyHostToDevice, up_s),
-                 "copy q to device");
-        VSA_CUDA(cudaMemcpy2DAsync(dk + off, row_g, k + src_off, row_all, row_g, rows, cudaMemcpyHostToDevice, up_s),
-                 "copy k to device");
-        VSA_CUDA(cudaMemcpy2DAsync(dv + off, row_g, v + src_off, row_all, row_g, rows, cudaMemcpyHostToDevice, up_s),
-                 "copy v to device");
-        VSA_CUDA(cudaEventRecord(ev[1 + gi], up_s), "record upload");
-        VSA_CUDA(cudaStreamWaitEvent(s, ev[1 + gi], 0), "wait upload");
-        sg.heads = hn;
-        Dims dh{};
-        VSA_TRY(make_dims(&sg, &dh));
-        if (cgc) VSA_CUDA(launch_gather_heads(dgc, rows, d.H, h0, hn, cgc, s), "gate gather launch");
-        if (cgf) VSA_CUDA(launch_gather_heads(dgf, rows, d.H, h0, hn, cgf, s), "gate gather launch");
-        VSA_TRY(run_forward(dh, dq + off, dk + off, dv + off, cgc, cgf, topk, scale, workspace, dout + off, s));
-        VSA_CUDA(cudaEventRecord(ev[1 + groups + gi], s), "record compute");
-        VSA_CUDA(cudaStreamWaitEvent(down_s, ev[1 + groups + gi], 0), "wait compute");
-        VSA_CUDA(cudaMemcpy2DAsync(out + src_off, row_all, dout + off, row_g, row_g, rows, cudaMemcpyDeviceToHost,
-                                   down_s),
-                 "copy out to host");
+    const vsa_status st = forward_host_groups(d, shape, q, k, v, g_coarse, g_fine, topk, scale, workspace, hg, fwd_g,
+                                              gate_g, dq, dk, dv, dout, dgc, dgf, out, s, up_s, down_s);
+    if (st != VSA_OK) {
+        // best effort: whatever the copy streams still hold comes before anything later on `stream`
+        cudaEvent_t e1 = nullptr, e2 = nullptr;
+        if (cudaEventCreateWithFlags(&e1, cudaEventDisableTiming) == cudaSuccess) {
+            if (cudaEventRecord(e1, up_s) == cudaSuccess) cudaStreamWaitEvent(s, e1, 0);
+            cudaEventDestroy(e1);
+        }
+        if (cudaEventCreateWithFlags(&e2, cudaEventDisableTiming) == cudaSuccess) {
+            if (cudaEventRecord(e2, down_s) == cudaSuccess) cudaStreamWaitEvent(s, e2, 0);
+            cudaEventDestroy(e2);
+        }
     }
-    // the call is complete on `stream` once the last output copy is
-    VSA_CUDA(cudaEventRecord(ev[1 + 2 * groups], down_s), "record end");
-    VSA_CUDA(cudaStreamWaitEvent(s, ev[1 + 2 * groups], 0), "wait end");
-    return VSA_OK;
+    return st;
 }
 
 vsa_status vsa_device_status(vsa_stream_t stream) {
