@@ -401,7 +401,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                           "frac": round(pre_bytes / (pre_ms * 1e-3) / 1e9 / hbm_peak, 4),
                           "per_launch": "Q and K read once and written once: 4*B*N*H*D*2 bytes"},
         "e2e": {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": "vsa_forward_host (pinned host q/k/v/gates in, host out)"},
+                "api": "vsa_forward_host (pinned host q/k/v/gates in, host out; copies pipelined by head groups)"},
         # per step, VSA call: pool, coarse scores, coarse softmax x V, top-k, order sort, schedule, fine
         # (one-tile kernel) and the re-run guard (fine_kernel, which returns at once unless the one-tile
         # kernel overflowed) = 8; dense call: fine = 1

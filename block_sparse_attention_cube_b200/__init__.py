@@ -312,7 +312,9 @@ def _host_ptr(t: Optional[torch.Tensor], name: str) -> Optional[int]:
 def forward_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, shape: Shape, topk_k: int,
                  workspace: torch.Tensor, out: torch.Tensor, scale: Optional[float] = None,
                  g_coarse: Optional[torch.Tensor] = None, g_fine: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """vsa_forward_host: host tensors in and out, copies enqueued on the current stream."""
+    """vsa_forward_host: host tensors in and out. With two or more heads the copies run by head groups on
+    the library's two copy streams, overlapping the compute on the current stream, which waits for the
+    last copy; `out` is valid once the current stream is synchronized. Pin the host tensors for overlap."""
     scale = default_scale(shape) if scale is None else scale
     _check(_L.vsa_forward_host(ctypes.byref(shape.c()), _host_ptr(q, "q"), _host_ptr(k, "k"), _host_ptr(v, "v"),
                                _host_ptr(g_coarse, "g_coarse"), _host_ptr(g_fine, "g_fine"), topk_k, scale,
