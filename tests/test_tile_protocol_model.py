@@ -1,6 +1,7 @@
 """A model of the one-tile fine kernel's per-item synchronization, checked under random schedules (CPU).
 
-fine_tile_kernel (block_sparse_attention_cube_b200/csrc/vsa_fine.cu) coordinates a QK^T issuer, a PV issuer,
+fine_tile_kernel (block_sparse_attention_cube_b200/csrc/vsa_fine.cu) coordinates a Q/K producer (one Q
+buffer, a 3-deep K ring), a V producer (a 2-deep V ring), a QK^T issuer, a PV issuer,
 three softmax groups (here six half-groups: group g x query slot, each standing for the two warps of that
 slot), and an epilogue warpgroup through mbarriers.  This file restates that protocol: the same barriers, the
 same arrival counts (in half-group units) and the same parity waits.  An mbarrier wait by parity P succeeds
@@ -8,7 +9,8 @@ when the barrier's phase parity differs from P, so a waiter that falls a phase b
 tensor core completes MMAs in issue order.  Random interleavings, some with one role starved, run item
 sequences of one to seven steps with random selections, and every cross-role read is checked: a row's maximum
 must come from the same item, the epilogue must see the row sums of its item and an accumulator holding
-exactly that item's PVs, and nothing may deadlock.
+exactly that item's PVs, every MMA must find its own item's Q and its own step's K or V in the buffer it
+reads (copies land in any order), and nothing may deadlock.
 
 Without the SetFree wait (a group with no step in an item can run two items ahead) or without the
 once-per-item ODone barrier, the same schedules find violations; the kernel has both.  This checks the
@@ -16,6 +18,8 @@ protocol as designed, not the CUDA code; the GPU tests check the code (test_gpu_
 test_one_tile_kernel_with_many_items_per_cta).
 """
 import random
+
+import pytest
 
 class Bar:
     def __init__(self, name, count):
@@ -29,9 +33,10 @@ class Bar:
         return (self.phase & 1) != parity
 
 class Model:
-    def __init__(self, items, seed, setfree=True, odone=True, slow=None):
+    def __init__(self, items, seed, setfree=True, odone=True, slow=None, drop=()):
         self.rng = random.Random(seed)
         self.slow = slow
+        self.drop = set(drop)          # waits left out (to show that the checks catch their absence)
         self.items = items            # list of (steps, sel) where sel[s][slot] bool
         self.setfree, self.odone = setfree, odone
         B = {}
@@ -46,13 +51,21 @@ class Model:
             B[f"SetFree{ip}"] = Bar(f"SetFree{ip}", 1)
         B["OFree"] = Bar("OFree", 1)
         B["ODone"] = Bar("ODone", 1)
+        B["QFull"], B["QEmpty"] = Bar("QFull", 1), Bar("QEmpty", 1)
+        for i in range(3):
+            B[f"KFull{i}"], B[f"KEmpty{i}"] = Bar(f"KFull{i}", 1), Bar(f"KEmpty{i}", 1)
+        for i in range(2):
+            B[f"VFull{i}"], B[f"VEmpty{i}"] = Bar(f"VFull{i}", 1), Bar(f"VEmpty{i}", 1)
         self.B = B
+        self.loads = []                # copies in flight: (buffer, content, barrier), landing in any order
+        self.qbuf, self.kbuf, self.vbuf = None, [None] * 3, [None] * 2
         self.fifo = []                 # tensor pipe: (kind, item, step, buf)
         self.m = {(ip, sl): None for ip in range(2) for sl in range(2)}   # value: item index
         self.l = {(ip, g, sl): None for ip in range(2) for g in range(3) for sl in range(2)}
         self.O = []                    # list of (item, step) PVs accumulated since the last release
         self.errors = []
-        self.procs = {"S": self.s_issuer(), "PV": self.pv_issuer(), "EW": self.epilogue()}
+        self.procs = {"S": self.s_issuer(), "PV": self.pv_issuer(), "EW": self.epilogue(),
+                      "LQK": self.qk_producer(), "LV": self.v_producer(), "TMA": self.copies()}
         for g in range(3):
             for sl in range(2):
                 self.procs[f"G{g}{sl}"] = self.half_group(g, sl)
@@ -63,19 +76,70 @@ class Model:
         b = self.B[bar]
         return lambda: b.ready(parity)
 
+    def qk_producer(self):
+        kslot, kph = 0, 0
+        for n, (steps, sel) in enumerate(self.items):
+            if "QEmpty" not in self.drop:
+                yield self.wait("QEmpty", (n & 1) ^ 1)
+            self.loads.append(("Q", None, n, "QFull"))
+            yield None
+            for s in range(steps):
+                yield self.wait(f"KEmpty{kslot}", kph ^ 1)
+                self.loads.append(("K", kslot, (n, s), f"KFull{kslot}"))
+                kslot += 1
+                if kslot == 3:
+                    kslot, kph = 0, kph ^ 1
+                yield None
+
+    def v_producer(self):
+        vslot, vph = 0, 0
+        for n, (steps, sel) in enumerate(self.items):
+            for s in range(steps):
+                yield self.wait(f"VEmpty{vslot}", vph ^ 1)
+                self.loads.append(("V", vslot, (n, s), f"VFull{vslot}"))
+                vslot += 1
+                if vslot == 2:
+                    vslot, vph = 0, vph ^ 1
+                yield None
+
+    def copies(self):
+        while True:
+            while not self.loads:
+                yield lambda: bool(self.loads) or self.done_all()
+                if self.done_all() and not self.loads:
+                    return
+            kind, slot, content, bar = self.loads.pop(self.rng.randrange(len(self.loads)))
+            if kind == "Q":
+                self.qbuf = content
+            elif kind == "K":
+                self.kbuf[slot] = content
+            else:
+                self.vbuf[slot] = content
+            self.B[bar].arrive()
+            yield None
+
     def s_issuer(self):
         uses = [0, 0, 0]
+        kslot, kph = 0, 0
         for n, (steps, sel) in enumerate(self.items):
+            yield self.wait("QFull", n & 1)
             for s in range(steps):
                 b = s % 3
                 if uses[b] > 0:
                     yield self.wait(f"PVDone{b}", (uses[b] - 1) & 1)
-                self.fifo.append(("S", n, s, b))
+                if "KFull" not in self.drop:
+                    yield self.wait(f"KFull{kslot}", kph)
+                self.fifo.append(("S", n, s, (b, kslot)))
                 uses[b] += 1
+                kslot += 1
+                if kslot == 3:
+                    kslot, kph = 0, kph ^ 1
                 yield None
+            self.fifo.append(("QEMPTY", n, 0, None))
 
     def pv_issuer(self):
         waits = [0, 0, 0]
+        vslot, vph = 0, 0
         for n, (steps, sel) in enumerate(self.items):
             for s in range(steps):
                 b = s % 3
@@ -83,7 +147,12 @@ class Model:
                     yield self.wait("OFree", (n - 1) & 1)
                 yield self.wait(f"PFull{b}", waits[b] & 1)
                 waits[b] += 1
-                self.fifo.append(("PV", n, s, b))
+                if "VFull" not in self.drop:
+                    yield self.wait(f"VFull{vslot}", vph)
+                self.fifo.append(("PV", n, s, (b, vslot)))
+                vslot += 1
+                if vslot == 2:
+                    vslot, vph = 0, vph ^ 1
                 if s == steps - 1:
                     self.fifo.append(("ODONE", n, s, b))
                 yield None
@@ -96,10 +165,20 @@ class Model:
                     return
             kind, n, s, b = self.fifo.pop(0)
             if kind == "S":
+                b, ks = b
+                if self.qbuf != n or self.kbuf[ks] != (n, s):
+                    self.errors.append(f"S({n},{s}) read Q of item {self.qbuf} and K {self.kbuf[ks]}")
                 self.B[f"SFull{b}"].arrive()
+                self.B[f"KEmpty{ks}"].arrive()
             elif kind == "PV":
+                b, vs = b
+                if self.vbuf[vs] != (n, s):
+                    self.errors.append(f"PV({n},{s}) read V {self.vbuf[vs]}")
                 self.O.append((n, s))
                 self.B[f"PVDone{b}"].arrive()
+                self.B[f"VEmpty{vs}"].arrive()
+            elif kind == "QEMPTY":
+                self.B["QEmpty"].arrive()
             else:
                 self.B["ODone"].arrive()
             yield None
@@ -158,7 +237,7 @@ class Model:
             yield None
 
     def done_all(self):
-        return all(k == "T" or self.finished.get(k) for k in self.procs)
+        return all(k in ("T", "TMA") or self.finished.get(k) for k in self.procs)
 
     def run(self, max_steps=200000):
         self.finished = {}
@@ -173,7 +252,7 @@ class Model:
                     runnable.append(k)
             if not runnable:
                 live = [k for k in self.procs if not self.finished.get(k)]
-                if live == ["T"] or not live:
+                if set(live) <= {"T", "TMA"}:
                     return
                 self.errors.append("deadlock: " + ", ".join(live))
                 return
@@ -186,7 +265,8 @@ class Model:
             except StopIteration:
                 self.finished[k] = True
                 blocked_on.pop(k, None)
-            if all(self.finished.get(x) for x in self.procs if x != "T") and not self.fifo:
+            if all(self.finished.get(x) for x in self.procs if x not in ("T", "TMA")) and not self.fifo \
+                    and not self.loads:
                 return
         self.errors.append("step limit")
 
@@ -209,15 +289,15 @@ def random_items(rng, n_items):
     return items
 
 
-ROLES = ["S", "PV", "EW", "T"] + [f"G{g}{sl}" for g in range(3) for sl in range(2)] + [None]
+ROLES = ["S", "PV", "EW", "T", "LQK", "LV", "TMA"] + [f"G{g}{sl}" for g in range(3) for sl in range(2)] + [None]
 
 
-def _violations(trials, setfree=True, odone=True):
+def _violations(trials, setfree=True, odone=True, drop=()):
     bad = []
     for t in range(trials):
         rng = random.Random(t)
         m = Model(random_items(rng, rng.randint(1, 12)), seed=t, setfree=setfree, odone=odone,
-                  slow=rng.choice(ROLES))
+                  slow=rng.choice(ROLES), drop=drop)
         m.run()
         if m.errors:
             bad.append((t, m.errors[:2]))
@@ -235,3 +315,8 @@ def test_the_model_finds_the_run_ahead_race_without_setfree():
 
 def test_the_model_finds_an_early_output_read_without_the_once_per_item_barrier():
     assert _violations(200, odone=False)
+
+
+@pytest.mark.parametrize("wait", ["QEmpty", "KFull", "VFull"])
+def test_the_model_finds_stale_operands_without_each_load_wait(wait):
+    assert _violations(200, drop=(wait,))
