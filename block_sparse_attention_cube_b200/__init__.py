@@ -230,20 +230,33 @@ def fine_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, shape: Shape, 
                scale: Optional[float] = None, order: Optional[torch.Tensor] = None,
                o_coarse: Optional[torch.Tensor] = None, g_coarse: Optional[torch.Tensor] = None,
                g_fine: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-               steps: Optional[torch.Tensor] = None) -> torch.Tensor:
+               steps: Optional[torch.Tensor] = None, overflow: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Fine attention + gated merge on the token layout, written as [B,N,H,D] (idx None: dense attention).
 
-    `steps` (from schedule()) replaces the kernel's own walk of the selection."""
+    `steps` (from schedule()) replaces the kernel's own walk of the selection; the fixed-maximum
+    kernel that then runs reports an overflow (and the re-run it caused) in `overflow`, one int32
+    on the device (allocated here when omitted)."""
     scale = default_scale(shape) if scale is None else scale
     kk = int(idx.shape[-1]) if idx is not None else 0
     if out is None:
         out = torch.empty_like(q)
+    if steps is not None and overflow is None:
+        overflow = torch.empty(4, dtype=torch.int32, device=q.device)
     _check(_L.vsa_fine_fused(ctypes.byref(shape.c()), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
                              _ptr(v, torch.bfloat16, "v"), _ptr(idx, torch.int32, "idx"), kk,
                              _ptr(order, torch.int32, "order"), _ptr(steps, torch.uint8, "steps"), scale,
                              _ptr(o_coarse, torch.float32, "o_coarse"), _ptr(g_coarse, torch.bfloat16, "g_coarse"),
-                             _ptr(g_fine, torch.bfloat16, "g_fine"), _ptr(out, torch.bfloat16, "out"), _stream()))
+                             _ptr(g_fine, torch.bfloat16, "g_fine"), _ptr(out, torch.bfloat16, "out"),
+                             _ptr(overflow, torch.int32, "overflow"), _stream()))
     return out
+
+
+def forward_rerun(shape: Shape, topk_k: int, workspace: torch.Tensor, has_g_coarse: bool) -> bool:
+    """After forward() on `workspace`: did its fixed-maximum fine stage overflow and re-run (synchronizes)?"""
+    r = ctypes.c_int32(-1)
+    _check(_L.vsa_forward_rerun(ctypes.byref(shape.c()), topk_k, int(bool(has_g_coarse)),
+                                _ptr(workspace, torch.uint8, "workspace"), ctypes.byref(r), _stream()))
+    return bool(r.value)
 
 
 def workspace_bytes(shape: Shape, k: int) -> int:

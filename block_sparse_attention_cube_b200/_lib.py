@@ -46,13 +46,14 @@ SIGNATURES = {
     "vsa_combine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P]),
     "vsa_pool_qkv": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P]),
     "vsa_topk_order": (ctypes.c_int, [_SP, _P, _I32, _P, _P, _P, _P]),
-    "vsa_fine_fused": (ctypes.c_int, [_SP, _P, _P, _P, _P, _I32, _P, _P, _F32, _P, _P, _P, _P, _P]),
+    "vsa_fine_fused": (ctypes.c_int, [_SP, _P, _P, _P, _P, _I32, _P, _P, _F32, _P, _P, _P, _P, _P, _P]),
     "vsa_schedule_bytes": (_SZ, [_SP, _I32]),
     "vsa_schedule": (ctypes.c_int, [_SP, _P, _I32, _P, _P, _P]),
     "vsa_pair_order": (ctypes.c_int, [_SP, _P, _I32, _P, _P]),
     "vsa_qk_norm_rope": (ctypes.c_int, [_SP, _P, _P, _P, _P, _F32, _F32, _I64, _I64, _P, _P, _P]),
     "vsa_workspace_bytes": (_SZ, [_SP, _I32]),
     "vsa_forward": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _I32, _F32, _P, _SZ, _P, _P]),
+    "vsa_forward_rerun": (ctypes.c_int, [_SP, _I32, _I32, _P, ctypes.POINTER(ctypes.c_int32), _P]),
     "vsa_workspace_bytes_host": (_SZ, [_SP, _I32]),
     "vsa_forward_host": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _I32, _F32, _P, _SZ, _P, _P]),
     "vsa_forward_noalloc": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _I32, _F32, _P, _P]),

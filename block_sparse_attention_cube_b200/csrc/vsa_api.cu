@@ -658,7 +658,7 @@ vsa_status vsa_pool_qkv(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf1
 vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
                           const int32_t* idx, int32_t topk, const int32_t* order, const void* steps, float scale,
                           const float* o_coarse, const vsa_bf16* g_coarse, const vsa_bf16* g_fine, vsa_bf16* out,
-                          vsa_stream_t stream) {
+                          int32_t* overflow, vsa_stream_t stream) {
     Dims d{};
     VSA_TRY(make_dims(shape, &d));
     if (idx) VSA_TRY(check_k(d, topk));
@@ -669,6 +669,8 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
     VSA_TRY(opt_ptr(order, "order"));
     VSA_TRY(opt_ptr(steps, "steps"));
     if (steps && !idx) return fail(VSA_ERR_INVALID_ARGUMENT, "steps given without idx");
+    VSA_TRY(opt_ptr(overflow, "overflow"));
+    if (steps && !overflow) return fail(VSA_ERR_INVALID_ARGUMENT, "steps given without an overflow word");
     if (steps && d.C > kScheduleMaxC)
         return fail(VSA_ERR_UNSUPPORTED, "precomputed steps support at most %d cubes (got %d)", kScheduleMaxC, d.C);
     VSA_TRY(opt_ptr(o_coarse, "o_coarse"));
@@ -682,10 +684,10 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
                             {steps, steps ? schedule_bytes(d, topk) : 0, "steps"},
                             {o_coarse, o_coarse ? pooled_bytes(d) : 0, "o_coarse"},
                             {g_coarse, g_coarse ? gb : 0, "g_coarse"}, {g_fine, g_fine ? gb : 0, "g_fine"}},
-                           {{out, tb, "out"}}));
+                           {{out, tb, "out"}, {overflow, steps ? sizeof(int32_t) : 0, "overflow"}}));
     VSA_TRY(check_device());
-    return run_fine_fused(d, q, k, v, idx, topk, order, steps, scale, o_coarse, g_coarse, g_fine, out, nullptr,
-                          as_stream(stream));
+    return run_fine_fused(d, q, k, v, idx, topk, order, steps, scale, o_coarse, g_coarse, g_fine, out,
+                          steps ? overflow : nullptr, as_stream(stream));
 }
 
 size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk) {
@@ -720,6 +722,25 @@ vsa_status vsa_forward(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16
                            {{out, tb, "out"}, {workspace, need, "workspace"}}));
     VSA_TRY(check_device());
     return run_forward(d, q, k, v, g_coarse, g_fine, topk, scale, workspace, out, as_stream(stream));
+}
+
+vsa_status vsa_forward_rerun(const vsa_shape* shape, int32_t topk, int32_t has_g_coarse, const void* workspace,
+                             int32_t* rerun, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(check_k(d, topk));
+    if (!rerun) return fail(VSA_ERR_INVALID_ARGUMENT, "rerun is NULL");
+    VSA_TRY(need_ptr(workspace, "workspace"));
+    *rerun = 0;
+    const Carve c = carve(d, topk, has_g_coarse != 0, const_cast<void*>(workspace));
+    if (topk == d.C || c.steps == nullptr) return VSA_OK;   // no fixed-maximum stage ran
+    cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int value = 0;
+    if ((e = cudaMemcpy(&value, c.overflow, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "read overflow word");
+    *rerun = value != 0 ? 1 : 0;
+    return VSA_OK;
 }
 
 size_t vsa_workspace_bytes_host(const vsa_shape* shape, int32_t topk) {

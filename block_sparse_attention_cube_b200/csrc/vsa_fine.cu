@@ -82,7 +82,6 @@
 namespace vsa {
 
 __device__ int g_vsa_status;   // watchdog word (VSA_OK or VSA_ERR_TIMEOUT)
-__device__ int g_vsa_overflow;   // fine_tile_kernel's overflow word for callers without a workspace
 
 namespace {
 
@@ -1755,20 +1754,6 @@ int* status_word() {
     return ptrs[dev];
 }
 
-int* overflow_word() {
-    static std::mutex mu;
-    static int* ptrs[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!ptrs[dev]) {
-        void* a = nullptr;
-        if (cudaGetSymbolAddress(&a, g_vsa_overflow) != cudaSuccess) return nullptr;
-        ptrs[dev] = static_cast<int*>(a);
-    }
-    return ptrs[dev];
-}
-
 namespace {
 
 FineParams make_params(const Dims& d, const FineArgs& a, int group) {
@@ -1869,9 +1854,9 @@ cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const 
     const bool tile = mode == kFineCubesFused && a.steps != nullptr;
     if (tile) {
         // the one-tile kernel, then fine_kernel over the whole stage only if its fixed maxima overflowed
-        int* ovf = a.overflow ? a.overflow : overflow_word();
+        int* ovf = a.overflow;   // the caller's word: calls on other streams never share it
         if (!ovf) {
-            if (why) *why = "overflow word unavailable";
+            if (why) *why = "precomputed steps need an overflow word";
             return cudaErrorInvalidValue;
         }
         FineParams pt = make_params(d, a, kTileGroup);

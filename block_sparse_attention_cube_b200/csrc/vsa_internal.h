@@ -31,10 +31,6 @@ int sm_count();
 // Watchdog word of the current device (device address, cached per device).
 int* status_word();
 
-// Overflow word of the current device for fused fine-stage calls made without
-// a workspace (device address, cached per device).
-int* overflow_word();
-
 // Upper bound on any device-side wait, in nanoseconds.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
@@ -93,7 +89,8 @@ struct FineArgs {
     int k_sel;
     const int32_t* order;   // [B, H, C] or null
     const void* steps;      // precomputed steps (launch_schedule) or null: the kernel walks the selection
-    int* overflow;          // device word the one-tile kernel raises on overflow (null: a per-device word)
+    int* overflow;          // caller's device word: cleared, raised by the one-tile kernel on overflow,
+                            // read by the re-run (required with steps)
     float scale;
     uint16_t* out;
     float* lse;             // kFineTiled only

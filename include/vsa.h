@@ -29,9 +29,13 @@
  *  * bf16 values are passed as uint16_t bit patterns (vsa_bf16).
  *  * Every pointer argument is a DEVICE pointer owned by the caller, except in
  *    vsa_forward_host where the tensors are HOST pointers.  The library never
- *    allocates or frees memory and keeps no device state other than one
- *    watchdog status word per device (and, once vsa_forward_host has run on a
- *    device, that function's two copy streams).
+ *    allocates or frees memory.  Its only device state is one watchdog status
+ *    word per device, the static workspace of vsa_forward_noalloc, and, once
+ *    vsa_forward_host has run on a device, that function's two copy streams.
+ *    The device addresses of the two static words are looked up once per
+ *    device and kept for the life of the process, so the library must not be
+ *    used across a cudaDeviceReset (or any other teardown of the device's
+ *    primary context): the module is then loaded again at other addresses.
  *  * Every device pointer must be 16-byte aligned; input and output ranges of
  *    one call must not overlap.
  *  * `stream` is a cudaStream_t passed as an opaque pointer (NULL = the
@@ -53,7 +57,7 @@
 extern "C" {
 #endif
 
-#define VSA_ABI_VERSION 1
+#define VSA_ABI_VERSION 2
 
 typedef uint16_t vsa_bf16;
 typedef void* vsa_stream_t;
@@ -262,11 +266,22 @@ vsa_status vsa_pool_qkv(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf1
  *   o_coarse   [B, H, C, D] float32, or NULL (no coarse term; g_coarse ignored).
  *   g_coarse, g_fine  [B, N, H] bf16 or NULL (g_coarse = 0, g_fine = 1).
  *   out        [B, N, H, D] bf16 (written at every real token).
+ *   overflow   one int32 of caller-owned device memory; required with
+ *              `steps` (VSA_ERR_INVALID_ARGUMENT otherwise), ignored without.
+ *              With steps the stage runs on the one-tile kernel, which keeps
+ *              each query row's first selected maximum fixed for the whole row
+ *              (teardown section "Fixed-max softmax is a numerical contract"):
+ *              the call clears the word, the kernel sets it to 1 when a
+ *              probability would exceed 2^64 or a row sum is not finite, and a
+ *              second launch then re-runs the whole stage with online
+ *              rescaling (it returns at once when the word is 0).  When the
+ *              stream has passed the call the word tells whether the re-run
+ *              happened.  Calls running at the same time need distinct words.
  */
 vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
                           const int32_t* idx, int32_t topk, const int32_t* order, const void* steps, float scale,
                           const float* o_coarse, const vsa_bf16* g_coarse, const vsa_bf16* g_fine,
-                          vsa_bf16* out, vsa_stream_t stream);
+                          vsa_bf16* out, int32_t* overflow, vsa_stream_t stream);
 
 /*
  * vsa_pair_order — re-pairs a work order for the fine stage, whose 128-row
@@ -342,6 +357,19 @@ size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
 vsa_status vsa_forward(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k, const vsa_bf16* v,
                        const vsa_bf16* g_coarse, const vsa_bf16* g_fine, int32_t topk, float scale,
                        void* workspace, size_t workspace_bytes, vsa_bf16* out, vsa_stream_t stream);
+
+/*
+ * vsa_forward_rerun — whether the last vsa_forward call on `workspace` (with
+ * this shape, top-k and coarse gate given or not: has_g_coarse 0 or 1) had to
+ * re-run its fine stage with online rescaling because the fixed per-row
+ * maxima overflowed (see the `overflow` argument of vsa_fine_fused; the
+ * forward call keeps that word in its workspace).  Synchronizes `stream`,
+ * then sets *rerun to 1 or 0.  A dense call (topk == C), which rescales
+ * online from the start, and a call whose fine stage walked the selection
+ * itself (no precomputed steps) always give 0 without touching the device.
+ */
+vsa_status vsa_forward_rerun(const vsa_shape* shape, int32_t topk, int32_t has_g_coarse, const void* workspace,
+                             int32_t* rerun, vsa_stream_t stream);
 
 /* Bytes of device workspace vsa_forward_host needs: vsa_workspace_bytes plus
  * device staging for the inputs and the output. */

@@ -41,3 +41,23 @@ def _no_device_timeout(request):
         return
     import block_sparse_attention_cube_b200 as vsa
     vsa.device_status()
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """How many selection rows the near-tie rule excused in each comparison of the session."""
+    try:
+        from tests._util import NEAR_TIE_LOG
+    except Exception:  # pragma: no cover
+        return
+    if not NEAR_TIE_LOG:
+        return
+    tr = terminalreporter
+    tr.section("near-tie rows (GPU selection differs from the oracle's)")
+    rows = sum(r for _, r, _, _ in NEAR_TIE_LOG)
+    excused = sum(e for _, _, e, _ in NEAR_TIE_LOG)
+    failed = sum(f for _, _, _, f in NEAR_TIE_LOG)
+    tr.write_line(f"total: {excused} of {rows} rows excused as near-ties, {failed} failed, "
+                  f"{len(NEAR_TIE_LOG)} comparisons")
+    for label, r, e, f in NEAR_TIE_LOG:
+        if e or f or "wan" in label:
+            tr.write_line(f"  {label}: {e} of {r} rows excused, {f} failed")

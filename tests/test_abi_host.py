@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert vsa.abi_version() == 1
+    assert vsa.abi_version() == 2
     for code, name in _lib.STATUS_NAMES.items():
         assert _lib.load().vsa_status_string(code).decode() == name
 
@@ -70,6 +70,31 @@ def test_null_and_misaligned_pointers():
     assert "x is NULL" in vsa.last_error()
     assert vsa.raw_call("vsa_tile", ctypes.byref(s), ctypes.c_void_p(4104), ctypes.c_void_p(1 << 40), None) == MISALIGNED
     assert vsa.raw_call("vsa_shape_info", None, None, None) == INVALID
+
+
+def test_fine_fused_steps_need_an_overflow_word():
+    """With precomputed steps the fixed-maximum kernel reports overflow in a caller word: no word, no call."""
+    s = _shape()
+    p = [ctypes.c_void_p((1 << 40) + i * (1 << 32)) for i in range(8)]
+    st = vsa.raw_call("vsa_fine_fused", ctypes.byref(s), p[0], p[1], p[2], p[3], 2, None, p[4], 0.125,
+                      None, None, None, p[5], None, None)
+    assert st == INVALID and "overflow word" in vsa.last_error()
+    st = vsa.raw_call("vsa_fine_fused", ctypes.byref(s), p[0], p[1], p[2], p[3], 2, None, p[4], 0.125,
+                      None, None, None, p[5], ctypes.c_void_p(p[6].value + 4), None)
+    assert st == MISALIGNED and "overflow" in vsa.last_error()
+
+
+def test_forward_rerun_argument_checks():
+    s = _shape()
+    r = ctypes.c_int32(-5)
+    ws = ctypes.c_void_p(1 << 40)
+    assert vsa.raw_call("vsa_forward_rerun", ctypes.byref(s), 2, 1, ws, None, None) == INVALID
+    assert vsa.raw_call("vsa_forward_rerun", ctypes.byref(s), 0, 1, ws, ctypes.byref(r), None) == INVALID
+    assert vsa.raw_call("vsa_forward_rerun", ctypes.byref(s), 2, 1, None, ctypes.byref(r), None) == INVALID
+    # dense call (top-k = C): no fixed-maximum stage, answered without touching the device
+    _, c = vsa.shape_info(vsa.Shape(s.batch, s.heads, s.head_dim, (s.grid_t, s.grid_h, s.grid_w)))
+    assert vsa.raw_call("vsa_forward_rerun", ctypes.byref(s), c, 0, ws, ctypes.byref(r), None) == 0
+    assert r.value == 0
 
 
 def test_overlapping_input_and_output_rejected():

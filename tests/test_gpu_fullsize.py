@@ -11,7 +11,7 @@ import torch
 import block_sparse_attention_cube_b200 as vsa
 import synth
 from oracle import vsa_oracle as O
-from tests._util import (COARSE_REL_L2, LSE_ABS, bf16_bits, check_close, from_dev, near_tie_ok, to_dev)
+from tests._util import (COARSE_REL_L2, LSE_ABS, assert_selection, bf16_bits, check_close, from_dev, to_dev)
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -125,17 +125,17 @@ def test_selection_sampled_heads(run):
         np.testing.assert_allclose(g_scores, r_scores, rtol=0, atol=1e-5 * np.abs(r_scores).max())
         g_oc = run["oc"][b, h].numpy().astype(np.float64)
         assert np.linalg.norm(g_oc - r_oc) / np.linalg.norm(r_oc) <= COARSE_REL_L2
-        ok = near_tie_ok(run["idx"][b, h], r_idx, r_scores, k)
-        assert ok.all(), f"b={b} h={h}: {(~ok).sum()} rows differ beyond the near-tie rule"
+        assert_selection(run["idx"][b, h], r_idx, r_scores, k, f"{w.name} b={b} h={h}")
 
 
 def test_fine_and_output_sampled_cubes(run):
-    """Sampled query cubes against the oracle with its own selection; a cube whose
-    GPU selection differs (a documented near-tie) is left out of the comparison."""
+    """Sampled query cubes against the oracle's fine step and merge.  The oracle runs each cube
+    over the GPU's own selection, so a documented near-tie swap (checked and counted by
+    test_selection_sampled_heads) is compared like any other cube instead of being left out."""
     w, x, C = run["w"], run["x"], run["C"]
     kv = O.key_valid_mask(w.grid)
     src = O.tile_source_index(w.grid)
-    compared = 0
+    compared = swapped = 0
     for b, h in _sample_heads(w):
         if run["dense"]:
             qt, kt, vt = (_head_f64(x, b, h, n, w.grid) for n in ("q", "k", "v"))
@@ -145,9 +145,8 @@ def test_fine_and_output_sampled_cubes(run):
             if run["dense"]:
                 sel = range(C)
             else:
-                sel = r_idx[i]
-                if not np.array_equal(sel, run["idx"][b, h, i]):
-                    continue
+                sel = run["idx"][b, h, i]
+                swapped += int(not np.array_equal(sel, r_idx[i]))
             r = slice(i * 64, (i + 1) * 64)
             ro, rl = O.fine_cube(qt[r], kt, vt, sel, kv, run["scale"])
             valid = kv[r]
@@ -165,4 +164,5 @@ def test_fine_and_output_sampled_cubes(run):
             got_out = O.bf16_to_f64(bf16_bits(run["out"][b, torch.from_numpy(toks), h]))
             check_close(got_out, ref_out, f"out b={b} h={h} cube={i}")
             compared += 1
-    assert compared >= 3 * len(_sample_heads(w))
+    assert swapped <= max(1, 0.02 * compared), f"{swapped} of {compared} sampled cubes carry a near-tie swap"
+    print(f"{w.name}: {compared} sampled query cubes compared, {swapped} with a near-tie swap")

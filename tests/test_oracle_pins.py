@@ -186,6 +186,94 @@ def test_topk_brute_force_tuples():
         assert O.topk(row, k).tolist() == sorted(ranked[:k])
 
 
+def test_kth_value_is_the_smallest_selected_and_next_the_largest_left_out():
+    """kth_gap agrees with topk's own selection: the k-th largest score is the
+    smallest selected one and the (k+1)-th the largest left out (-inf at k = C)."""
+    rng = np.random.default_rng(5)
+    scores = rng.integers(-4, 5, size=(3, 2, 9)).astype(float) + rng.normal(size=(3, 2, 9)) * (rng.random((3, 2, 9)) < 0.5)
+    for k in range(1, 10):
+        kth, nxt = O.kth_gap(scores, k)
+        sel = O.topk(scores, k)
+        for pos in np.ndindex(*scores.shape[:-1]):
+            row = scores[pos]
+            chosen = row[sel[pos]]
+            rest = np.delete(row, sel[pos])
+            assert kth[pos] == chosen.min()
+            assert nxt[pos] == (rest.max() if rest.size else -np.inf)
+
+
+# ---------------------------------------------------------------- near-tie rule inputs
+@pytest.mark.parametrize("row,k,expect", [
+    ([3.0, 1.0, 3.0, 2.0, 3.0], 1, (3.0, 3.0)),
+    ([3.0, 1.0, 3.0, 2.0, 3.0], 2, (3.0, 3.0)),
+    ([3.0, 1.0, 3.0, 2.0, 3.0], 3, (3.0, 2.0)),
+    ([3.0, 1.0, 3.0, 2.0, 3.0], 4, (2.0, 1.0)),
+    ([3.0, 1.0, 3.0, 2.0, 3.0], 5, (1.0, -math.inf)),    # k = C: nothing is left out
+    ([0.5, -1.0, 2.0, 7.0], 1, (7.0, 2.0)),
+    ([0.5, -1.0, 2.0, 7.0], 2, (2.0, 0.5)),
+    ([-4.0, -2.5, -3.0], 2, (-3.0, -4.0)),
+    ([1.0, 1.0 + 1e-9, 0.0], 1, (1.0 + 1e-9, 1.0)),
+])
+def test_kth_gap_hand_rows(row, k, expect):
+    """k-th and (k+1)-th largest entries of hand rows (counted with repeats)."""
+    kth, nxt = O.kth_gap(np.array(row), k)
+    assert (float(kth), float(nxt)) == expect
+
+
+def test_kth_gap_brute_force_tuples():
+    """Random tie-heavy rows, several leading axes: Python's sorted() gives the two values."""
+    rng = np.random.default_rng(2)
+    for _ in range(100):
+        C = int(rng.integers(1, 10))
+        k = int(rng.integers(1, C + 1))
+        a = rng.integers(-3, 4, size=(2, 3, C)).astype(float)
+        kth, nxt = O.kth_gap(a, k)
+        for pos in np.ndindex(2, 3):
+            desc = sorted(a[pos].tolist(), reverse=True)
+            assert kth[pos] == desc[k - 1]
+            assert nxt[pos] == (desc[k] if k < C else -math.inf)
+
+
+# ---------------------------------------------------------------- bf16 decoding
+# bit pattern -> exact value (sign bit, 8 exponent bits with bias 127, 7 fraction bits)
+BF16_TABLE = [
+    (0x0000, 0.0), (0x3F80, 1.0), (0xBF80, -1.0), (0xC040, -3.0), (0x3F00, 0.5), (0x4120, 10.0),
+    (0x4049, 3.140625), (0x3C00, 2.0 ** -7), (0x0080, 2.0 ** -126), (0x0001, 2.0 ** -133),
+    (0x007F, 127 * 2.0 ** -133), (0x8001, -(2.0 ** -133)), (0x7F7F, (2 - 2 ** -7) * 2.0 ** 127),
+    (0xFF7F, -(2 - 2 ** -7) * 2.0 ** 127), (0x7F80, math.inf), (0xFF80, -math.inf), (0x3FC0, 1.5),
+    (0x4B00, 2.0 ** 23), (0x4B01, 2.0 ** 23 + 2.0 ** 16),
+]
+
+
+def test_bf16_decode_table():
+    got = O.bf16_to_f64(np.array([b for b, _ in BF16_TABLE], dtype=np.uint16))
+    assert got.dtype == np.float64
+    assert got.tolist() == [v for _, v in BF16_TABLE]
+    z = O.bf16_to_f64(np.array([0x0000, 0x8000], dtype=np.uint16))
+    assert z.tolist() == [0.0, 0.0] and not np.signbit(z[0]) and np.signbit(z[1])
+    assert np.isnan(O.bf16_to_f64(np.array([0x7FC0, 0xFFC1, 0x7F81], dtype=np.uint16))).all()
+
+
+def _bf16_by_fields(u: int) -> float:
+    sign = -1.0 if u >> 15 else 1.0
+    e, f = (u >> 7) & 0xFF, u & 0x7F
+    if e == 0xFF:
+        return sign * math.inf if f == 0 else math.nan
+    if e == 0:
+        return sign * math.ldexp(f, -133)                 # subnormal: f / 128 * 2^-126
+    return sign * math.ldexp(128 + f, e - 134)            # (1 + f/128) * 2^(e - 127)
+
+
+def test_bf16_decode_every_pattern_by_fields():
+    u = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = O.bf16_to_f64(u)
+    ref = np.array([_bf16_by_fields(int(b)) for b in range(1 << 16)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
 # ---------------------------------------------------------------- fine / dense
 @pytest.mark.parametrize("name", ["tiny_8x8x8", "padded_7x15x16"])
 def test_dense_equals_library_sdpa(name):
@@ -315,6 +403,10 @@ def _pins_pass():
         test_dense_equals_library_sdpa("padded_7x15x16")
         test_zero_query_closed_form()
         test_combine_hand_value()
+        test_kth_gap_hand_rows([3.0, 1.0, 3.0, 2.0, 3.0], 3, (3.0, 2.0))
+        test_kth_gap_hand_rows([3.0, 1.0, 3.0, 2.0, 3.0], 5, (1.0, -math.inf))
+        test_kth_gap_hand_rows([0.5, -1.0, 2.0, 7.0], 2, (2.0, 0.5))
+        test_bf16_decode_table()
     except AssertionError:
         return False
     return True
@@ -325,9 +417,12 @@ def test_pins_pass_on_the_oracle():
 
 
 @pytest.mark.parametrize("mutation", ["swap_xy", "pool_all64", "transpose_coarse",
-                                      "topk_smallest", "no_scale", "swap_gates", "keep_padded_keys"])
+                                      "topk_smallest", "no_scale", "swap_gates", "keep_padded_keys",
+                                      "kth_off_by_one", "kth_unsorted", "kth_ascending",
+                                      "bf16_shift15", "bf16_no_sign"])
 def test_planted_mistake_is_caught(monkeypatch, mutation):
-    good = {n: getattr(O, n) for n in ("tile_source_index", "pool", "coarse", "topk", "fine_cube", "combine")}
+    good = {n: getattr(O, n) for n in ("tile_source_index", "pool", "coarse", "topk", "fine_cube", "combine",
+                                       "kth_gap", "bf16_to_f64")}
     if mutation == "swap_xy":
         def bad(grid):
             T, X, Y = grid
@@ -349,4 +444,23 @@ def test_planted_mistake_is_caught(monkeypatch, mutation):
     elif mutation == "keep_padded_keys":
         monkeypatch.setattr(O, "fine_cube",
                             lambda q, k, v, sel, kv, s: good["fine_cube"](q, k, v, sel, np.ones_like(kv), s))
+    elif mutation == "kth_off_by_one":
+        # the (k+1)-th and (k+2)-th instead of the k-th and (k+1)-th
+        monkeypatch.setattr(O, "kth_gap", lambda s, k: good["kth_gap"](s, min(k + 1, s.shape[-1])))
+    elif mutation == "kth_unsorted":
+        def bad(scores, k):
+            kth = scores[..., k - 1]
+            return kth, (scores[..., k] if k < scores.shape[-1] else np.full(kth.shape, -np.inf))
+        monkeypatch.setattr(O, "kth_gap", bad)
+    elif mutation == "kth_ascending":
+        def bad(scores, k):
+            s = np.sort(scores, axis=-1)
+            kth = s[..., k - 1]
+            return kth, (s[..., k] if k < scores.shape[-1] else np.full(kth.shape, -np.inf))
+        monkeypatch.setattr(O, "kth_gap", bad)
+    elif mutation == "bf16_shift15":
+        monkeypatch.setattr(O, "bf16_to_f64", lambda u: (np.ascontiguousarray(u, dtype=np.uint16).astype(np.uint32)
+                                                         << np.uint32(15)).view(np.float32).astype(np.float64))
+    elif mutation == "bf16_no_sign":
+        monkeypatch.setattr(O, "bf16_to_f64", lambda u: np.abs(good["bf16_to_f64"](u)))
     assert not _pins_pass()

@@ -5,8 +5,8 @@ whose pool owns the device, real-time code that must not allocate after
 start-up) get the same result as vsa_forward with a caller workspace; the
 workspace lives in the library's static device array instead.  The test
 goes through the C ABI (ctypes) and compares two calls in a row, of different
-shapes, with the existing entry point.  The file name makes pytest collect it
-last.
+shapes and in both orders, with the existing entry point, bit for bit.  The
+file name makes pytest collect it last.
 """
 import ctypes
 
@@ -17,7 +17,7 @@ import torch
 import block_sparse_attention_cube_b200 as vsa
 import synth
 from block_sparse_attention_cube_b200 import _lib
-from tests._util import check_close, from_dev, to_dev
+from tests._util import to_dev
 
 WORKSPACE = 4   # VSA_ERR_WORKSPACE
 
@@ -32,25 +32,40 @@ def _c_call(w, d, out):
     assert st == 0, lib.vsa_last_error().decode()
 
 
+def _two_calls_in_a_row(names, device):
+    """Each shape through the static workspace and through vsa_forward with a caller workspace: the same
+    kernels on the same inputs, so the bits must agree exactly."""
+    with torch.cuda.device(device):
+        results = []
+        for name in names:
+            w = synth.WORKLOADS[name]
+            assert vsa.workspace_bytes(vsa.Shape(w.batch, w.heads, w.head_dim, w.grid), w.topk) \
+                <= vsa.NOALLOC_WORKSPACE_BYTES
+            d = {k: to_dev(v).to(device) for k, v in synth.make_inputs(w).items()}
+            out = torch.empty_like(d["q"])
+            _c_call(w, d, out)
+            ref = vsa.forward(d["q"], d["k"], d["v"], vsa.Shape(w.batch, w.heads, w.head_dim, w.grid), w.topk,
+                              1.0 / np.sqrt(w.head_dim), d["g_coarse"], d["g_fine"])
+            torch.cuda.synchronize()
+            results.append((name, out, ref))
+        vsa.device_status()
+        for name, got, ref in results:
+            assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), f"{name}: noalloc differs from forward"
+
+
 @pytest.mark.gpu
-def test_noalloc_matches_forward_on_two_calls_in_a_row():
-    results = []
-    for name in ("padded_7x15x16", "tiny_8x8x8"):
-        w = synth.WORKLOADS[name]
-        assert vsa.workspace_bytes(vsa.Shape(w.batch, w.heads, w.head_dim, w.grid), w.topk) \
-            <= vsa.NOALLOC_WORKSPACE_BYTES
-        d = {k: to_dev(v) for k, v in synth.make_inputs(w).items()}
-        out = torch.empty_like(d["q"])
-        _c_call(w, d, out)
-        ref = vsa.forward(d["q"], d["k"], d["v"], vsa.Shape(w.batch, w.heads, w.head_dim, w.grid), w.topk,
-                          1.0 / np.sqrt(w.head_dim), d["g_coarse"], d["g_fine"])
-        torch.cuda.synchronize()
-        results.append((name, from_dev(out), from_dev(ref)))
-    vsa.device_status()
-    for name, got, ref in results:
-        for b in range(got.shape[0]):
-            for h in range(got.shape[2]):
-                check_close(got[b, :, h], ref[b, :, h], f"{name} noalloc vs forward b={b} h={h}")
+@pytest.mark.parametrize("names", [("padded_7x15x16", "tiny_8x8x8"), ("tiny_8x8x8", "padded_7x15x16")],
+                         ids=["large_then_small", "small_then_large"])
+def test_noalloc_matches_forward_on_two_calls_in_a_row(names):
+    _two_calls_in_a_row(names, torch.device("cuda", 0))
+
+
+@pytest.mark.gpu
+def test_noalloc_on_a_second_device():
+    """The static array's address is looked up per device: a call on the second GPU uses that GPU's copy."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("one GPU visible")
+    _two_calls_in_a_row(("tiny_8x8x8", "padded_7x15x16"), torch.device("cuda", 1))
 
 
 def test_noalloc_rejects_shapes_beyond_the_static_workspace():
