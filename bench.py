@@ -5,17 +5,25 @@ One step = one VSA call (grid 21x30x52 -> 39,936 padded tokens, 624 cubes,
 dense attention call on the same Q/K/V (every cube selected, no gates), both
 through the library's C ABI on one stream with inputs resident in HBM.
 
-Prints one JSON line.  `value` is milliseconds per VSA call (whole job: with
-N GPUs, N independent calls complete per step, so value = step time / N for
-the VSA part); the dense call is reported beside it.  Timing: CUDA events on
-the launching stream after warm-up, synchronize + barrier around the timed
-region, max over ranks.  Inputs (1.0 GB of Q/K/V per call) exceed the 126 MB
-L2, so L2 is not flushed between steps.
+Prints one JSON line.  `value` is the median milliseconds per VSA call (whole
+job: with N GPUs, N independent calls complete per step, so value = step
+time / N for the VSA part); the dense call is reported beside it.  Timing:
+CUDA events on the launching stream after warm-up, synchronize + barrier
+around the timed region, max over ranks, medians over the timed calls.
+Inputs (1.0 GB of Q/K/V per call) exceed the 126 MB L2, so L2 is not flushed
+between steps.  After the timed region, on the same process: the per-stage
+breakdown of the call, the Wan 720p CFG batch (2 x 21x45x80 tokens, top-k
+64), the memory-bound entry points one by one (HBM GB/s), the pre-attention
+pass, the end-to-end call on host buffers, and (rank 0, one GPU) the oracle
+on the host cores.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py --stages [--workload NAME] [--iters I] [--dense-too] [--staged]
 
-`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
-workload (extrapolated to one whole call) on rank 0 only.
+`--impl reference` times the fp64 CPU oracle, one whole head per step, on
+rank 0 only.  `--stages` runs the launches of one call stage by stage on a
+named workload and prints their median times (a small fixed case to put
+under a profiler).
 """
 from __future__ import annotations
 
@@ -41,7 +49,12 @@ import synth  # noqa: E402
 METRIC = "ms per VSA/dense attention call at 480p (40 heads, d=128); fine-kernel % BF16 peak"
 WORKLOAD = "wan480p_vsa_k32"
 DENSE_WORKLOAD = "wan480p_dense"
+CFG_WORKLOAD = "wan720p_cfg_k64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# oracle sample: step s runs the whole call (tile .. untile) on head (ORACLE_STRIDE * s) mod H
+# of batch element 0; the per-call figure is the median head time times B * H
+ORACLE_STRIDE = 7
+ORACLE_BASELINE_HEADS = 12
 
 
 # ---------------------------------------------------------------- shared helpers
@@ -79,6 +92,23 @@ def reduce_max(value: float, world: int) -> float:
 def whole_job_ms_per_call(max_step_ms: float, calls_per_step_per_rank: int, world: int) -> float:
     """Weak scaling: every rank runs its own calls; the job completes world*calls per step."""
     return max_step_ms / (calls_per_step_per_rank * world)
+
+
+def memory_bytes(w, npad: int, c: int) -> dict:
+    """Algorithmic HBM bytes per launch of the memory-bound entry points (each input read once, each
+    output written once; padded rows are neither read nor needed where the kernel skips them)."""
+    tok = w.batch * w.tokens * w.heads * w.head_dim * 2          # one [B, N, H, D] bf16 tensor
+    til = w.batch * w.heads * npad * w.head_dim * 2             # one [B, H, Npad, D] bf16 tensor
+    bar = w.batch * w.heads * c * w.head_dim * 4                # one [B, H, C, D] fp32 tensor
+    gate = w.batch * w.tokens * w.heads * 2
+    return {
+        "tile": tok + til,                                      # real rows read, every row written (zeros)
+        "untile": 2 * tok,                                      # real rows read and written
+        "pool": tok + bar,                                      # real rows of one tiled tensor read
+        "pool_qkv": 3 * (tok + bar),
+        "combine": tok + 2 * gate + bar + til,                  # O_f real rows, gates, O_c; every row written
+        "topk": w.batch * w.heads * c * c * 4 + w.batch * w.heads * c * w.topk * 4,
+    }
 
 
 def traffic_for(kernel_src: str, key: str):
@@ -148,45 +178,30 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-# ---------------------------------------------------------------- the oracle arm
-def oracle_sample(w, x, heads, cubes_per_head, seed=0):
-    """Time the fp64 oracle on a bounded sample of workload `w` and extrapolate to one call.
-
-    For each sampled head: tiling, pooling, coarse attention and top-k of the
-    whole head, then the fine step for `cubes_per_head` query cubes and the
-    merge / untiling of the head.  Returns (ms per call, seconds spent, sample text).
-    """
+# ---------------------------------------------------------------- the oracle
+def oracle_head_seconds(w, x, h: int) -> float:
+    """Seconds the fp64 oracle takes for the whole call (tile, pool, coarse, top-k, fine, merge,
+    untile) on head h of batch element 0; decoding the bf16 inputs is not timed."""
     from oracle import vsa_oracle as O
-    C = O.num_cubes(w.grid)
     scale = 1.0 / math.sqrt(w.head_dim)
-    rng = np.random.default_rng(seed)
-    cubes = sorted(rng.choice(C, size=min(cubes_per_head, C), replace=False).tolist())
-    t_head = t_fine = 0.0
-    for h in heads:
-        f = {n: O.bf16_to_f64(x[n][:1, :, h:h + 1]) for n in x}
-        t0 = time.perf_counter()
-        qt, kt, vt = (O.tile(f[n], w.grid) for n in ("q", "k", "v"))
-        if w.topk < C:
-            bars = [O.pool(t, w.grid) for t in (qt, kt, vt)]
-            scores, oc = O.coarse(*bars, scale)
-            idx = O.topk(scores, w.topk)
-        else:
-            idx, oc = None, None
-        t1 = time.perf_counter()
-        o, _ = O.fine(qt, kt, vt, idx, scale, w.grid, items=[(0, 0, i) for i in cubes])
-        t2 = time.perf_counter()
-        o = np.nan_to_num(o)
-        if oc is not None:
-            o = O.combine(oc, o, f["g_coarse"], f["g_fine"], w.grid)
-        O.untile(o, w.grid)
-        t3 = time.perf_counter()
-        t_head += (t1 - t0) + (t3 - t2)
-        t_fine += t2 - t1
-    nh = len(heads)
-    per_call_s = w.batch * w.heads * (t_head / nh + (t_fine / nh) * C / len(cubes))
-    sample = (f"{w.name}: heads {list(heads)} of {w.heads} (tile/pool/coarse/top-k/merge of each), fine step for "
-              f"{len(cubes)} of {C} query cubes per head; extrapolated to {w.batch}x{w.heads} heads x {C} cubes")
-    return per_call_s * 1e3, t_head + t_fine, sample
+    f = {n: O.bf16_to_f64(x[n][:1, :, h:h + 1]) for n in x}
+    t0 = time.perf_counter()
+    O.forward(f["q"], f["k"], f["v"], w.grid, w.topk, scale, f["g_coarse"], f["g_fine"])
+    return time.perf_counter() - t0
+
+
+def oracle_sample_heads(w, steps: range):
+    return [(ORACLE_STRIDE * s) % w.heads for s in steps]
+
+
+def oracle_rule_text(w) -> str:
+    return (f"{w.name}: whole oracle call (tile, pool, coarse, top-k, fine over all {synth_cubes(w)} query cubes, "
+            f"merge, untile) on one head per step, head (7*step) mod {w.heads} of batch element 0; "
+            f"per-call figure = median head time x B*H = {w.batch * w.heads} heads")
+
+
+def synth_cubes(w) -> int:
+    return math.prod((a + 3) // 4 for a in w.grid)
 
 
 def blas_threads() -> int:
@@ -205,30 +220,179 @@ def run_reference(args, rank: int):
         return
     w = synth.WORKLOADS[WORKLOAD]
     x = synth.make_inputs(w)
-    # each step: one head, 32 query cubes (about a second of fp64 work)
-    for _ in range(args.warmup):
-        oracle_sample(w, x, heads=(0,), cubes_per_head=32, seed=0)
-    vals, spent, sample = [], 0.0, ""
-    for s in range(args.steps):
-        ms, sec, sample = oracle_sample(w, x, heads=(s % w.heads,), cubes_per_head=32, seed=s)
-        vals.append(ms)
-        spent += sec
-    value = statistics.mean(vals)
+    for h in oracle_sample_heads(w, range(args.warmup)):
+        oracle_head_seconds(w, x, h)
+    secs = []
+    t0 = time.perf_counter()
+    for h in oracle_sample_heads(w, range(args.warmup, args.warmup + args.steps)):
+        secs.append(oracle_head_seconds(w, x, h))
+    wall_ms_per_step = (time.perf_counter() - t0) * 1e3 / args.steps
+    per_call_ms = statistics.median(secs) * w.batch * w.heads * 1e3
     cores = blas_threads()
+    sample = oracle_rule_text(w) + f"; {args.steps} timed steps, {sum(secs):.1f} s of CPU work"
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "ms", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value, 3), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded Philox, Wan 480p field inputs)",
+        "impl": "reference", "metric": METRIC, "value": round(per_call_ms, 2), "unit": "ms", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(wall_ms_per_step, 2),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Philox, Wan 480p field inputs)",
         "config": {"workload": WORKLOAD, "batch": w.batch, "grid": "x".join(map(str, w.grid)), "heads": w.heads,
                    "head_dim": w.head_dim, "topk": w.topk},
-        "cpu_baseline": {"value": round(value, 3), "unit": "ms", "cores": cores, "kind": "oracle",
-                         "sample": sample + f" (one sampled head per step; {spent:.1f} s of CPU work in total)"},
-        "e2e": {"value": round(value, 3), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "extrapolated": {"ms_per_call": round(per_call_ms, 2), "from": "median head time x B*H",
+                         "step": "one whole head of the call per step (ms_per_step is its measured wall time)"},
+        "cpu_baseline": {"value": round(per_call_ms, 2), "unit": "ms", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(per_call_ms, 2), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------------- the CUDA arm
+def _events(torch, n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def stage_times(vsa, torch, d, w, iters: int, warmup: int, dense_too: bool = False, staged: bool = False):
+    """Median ms of each launch group of one call, run stage by stage through the entry points."""
+    s = vsa.Shape(w.batch, w.heads, w.head_dim, w.grid)
+    _, C = vsa.shape_info(s)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    dense = w.topk == C
+    stream = torch.cuda.current_stream()
+    out = torch.empty_like(d["q"])
+    word = torch.zeros(4, dtype=torch.int32, device=d["q"].device)
+    acc = {}
+    for it in range(warmup + iters):
+        marks = []
+
+        def mark(name=None):
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            marks.append((name, e))
+
+        mark()
+        if staged:
+            qt, kt, vt = (vsa.tile(d[n], s) for n in ("q", "k", "v"))
+            mark("tile")
+            if dense:
+                of, _ = vsa.fine(qt, kt, vt, s, None, scale, want_lse=False)
+                mark("fine")
+                vsa.untile(of, s)
+                mark("untile")
+            else:
+                bars = [vsa.pool(t, s) for t in (qt, kt, vt)]
+                mark("pool")
+                scores, oc = vsa.coarse(*bars, s, scale)
+                mark("coarse")
+                idx = vsa.topk(scores, s, w.topk)
+                order = vsa.group(scores, s)
+                mark("topk+group")
+                of, _ = vsa.fine(qt, kt, vt, s, idx, scale, want_lse=False, order=order)
+                mark("fine")
+                ot = vsa.combine(oc, of, s, d["g_coarse"], d["g_fine"])
+                mark("combine")
+                vsa.untile(ot, s)
+                mark("untile")
+            if dense_too:
+                vsa.fine(qt, kt, vt, s, None, scale, want_lse=False)
+                mark("fine_dense")
+        else:
+            if dense:
+                vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out)
+                mark("fine")
+            else:
+                bars = vsa.pool_qkv(d["q"], d["k"], d["v"], s)
+                mark("pool")
+                scores, oc = vsa.coarse(*bars, s, scale)
+                mark("coarse")
+                idx, order = vsa.topk_order(scores, s, w.topk)
+                mark("topk_order")
+                steps = vsa.schedule(idx, s, order)
+                mark("schedule")
+                vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, order, oc, d["g_coarse"], d["g_fine"],
+                               out=out, steps=steps, overflow=word)
+                mark("fine")
+            if dense_too:
+                vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out)
+                mark("fine_dense")
+        torch.cuda.synchronize()
+        if it >= warmup:
+            for (_, e0), (name, e1) in zip(marks, marks[1:]):
+                acc.setdefault(name, []).append(e0.elapsed_time(e1))
+    return {n: round(statistics.median(v), 4) for n, v in acc.items()}
+
+
+def time_launches(torch, fn, iters: int, warmup: int = 3) -> float:
+    """Median ms of fn() over `iters` launches, each bracketed by events on the current stream."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    ev = [_events(torch, 2) for _ in range(iters)]
+    for e in ev:
+        e[0].record(stream)
+        fn()
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+
+
+def memory_kernels(vsa, torch, d, w, hbm_peak: float, iters: int) -> dict:
+    """The memory-bound entry points one launch at a time on the 480p tensors: median ms, GB/s of
+    algorithmic bytes, fraction of the measured HBM copy bandwidth."""
+    s = vsa.Shape(w.batch, w.heads, w.head_dim, w.grid)
+    npad, C = vsa.shape_info(s)
+    nbytes = memory_bytes(w, npad, C)
+    qt = vsa.tile(d["q"], s)
+    back = torch.empty_like(d["q"])
+    qbar = vsa.pool(qt, s)
+    kbar, vbar = vsa.pool(vsa.tile(d["k"], s), s), vsa.pool(vsa.tile(d["v"], s), s)
+    scores, oc = vsa.coarse(qbar, kbar, vbar, s)
+    of = qt   # any finite tiled tensor stands in for O_f: the merge's traffic does not depend on values
+    fns = {
+        "tile": lambda: vsa.tile(d["q"], s, out=qt),
+        "untile": lambda: vsa.untile(qt, s, out=back),
+        "pool": lambda: vsa.pool(qt, s),
+        "pool_qkv": lambda: vsa.pool_qkv(d["q"], d["k"], d["v"], s),
+        "combine": lambda: vsa.combine(oc, of, s, d["g_coarse"], d["g_fine"]),
+        "topk": lambda: vsa.topk(scores, s, w.topk),
+    }
+    rec = {}
+    for name, fn in fns.items():
+        ms = time_launches(torch, fn, iters)
+        gbs = nbytes[name] / (ms * 1e-3) / 1e9
+        rec[name] = {"ms": round(ms, 4), "bytes": nbytes[name], "gbps": round(gbs, 1),
+                     "frac_hbm": round(gbs / hbm_peak, 4)}
+    del qt, back, scores
+    return rec
+
+
+def cfg720_record(vsa, torch, dev, bf16_peak: float, iters: int, warmup: int) -> dict:
+    """The Wan 720p CFG batch (2 x 21x45x80 tokens, 1,440 cubes, top-k 64) through vsa_forward."""
+    w = synth.WORKLOADS[CFG_WORKLOAD]
+    x = synth.make_inputs(w)
+    d = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).to(dev) for k, v in x.items()}
+    del x
+    s = vsa.Shape(w.batch, w.heads, w.head_dim, w.grid)
+    npad, C = vsa.shape_info(s)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    ws = vsa.alloc_workspace(s, w.topk, device=dev)
+    out = torch.empty_like(d["q"])
+    ms = time_launches(torch, lambda: vsa.forward(d["q"], d["k"], d["v"], s, w.topk, scale, d["g_coarse"],
+                                                  d["g_fine"], workspace=ws, out=out), iters, warmup)
+    stages = stage_times(vsa, torch, d, w, iters, warmup)
+    vsa.device_status()
+    flops = executed_fine_flops(w.batch, w.heads, npad, w.topk, w.head_dim)
+    tf = flops / (stages["fine"] * 1e-3) / 1e12
+    del d, ws, out
+    torch.cuda.empty_cache()
+    return {"workload": CFG_WORKLOAD, "batch": w.batch, "grid": "x".join(map(str, w.grid)), "padded_tokens": npad,
+            "cubes": C, "heads": w.heads, "head_dim": w.head_dim, "topk": w.topk,
+            "ms_per_call": round(ms, 4), "stage_ms": stages,
+            "fine": {"executed_tflop": round(flops / 1e12, 3), "tflops": round(tf, 1),
+                     "frac_bf16_peak": round(tf / bf16_peak, 4),
+                     "dense_equivalent_tflops": round(dense_equivalent_flops(w.batch, w.heads, w.tokens, w.head_dim)
+                                                      / (stages["fine"] * 1e-3) / 1e12, 1)}}
+
+
 def run_cuda(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -264,8 +428,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     for _ in range(args.warmup):
         step()
     vsa.device_status()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [_events(torch, 3) for _ in range(args.steps)]
+    t_start, t_end = _events(torch, 2)
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
     if world > 1:
@@ -283,80 +447,49 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         dist.barrier()
     vsa.device_status()
     step_ms = t_start.elapsed_time(t_end) / args.steps
-    vsa_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    dense_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    vsa_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    dense_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
     step_ms_max = reduce_max(step_ms, world)
     vsa_ms_max = reduce_max(vsa_ms, world)
     dense_ms_max = reduce_max(dense_ms, world)
+    rerun = vsa.forward_rerun(s, w.topk, ws, has_g_coarse=True)
+
+    peaks, peaks_src = load_peaks()
+    bf16_peak = float(peaks["bf16_tflops"])
+    hbm_peak = float(peaks["hbm_gbs"])
 
     # ---- per-stage breakdown: the launches of vsa_forward, one by one through the entry points
-    names = ["pool", "coarse", "topk_order", "schedule", "fine"]
-    acc = {n: [] for n in names}
-    acc["fine_dense"] = []
-    for it in range(args.warmup + args.steps):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
-        e[0].record(stream)
-        bars = vsa.pool_qkv(d["q"], d["k"], d["v"], s)
-        e[1].record(stream)
-        scores, oc = vsa.coarse(*bars, s, scale)
-        e[2].record(stream)
-        idx, order = vsa.topk_order(scores, s, w.topk)
-        e[3].record(stream)
-        steps = vsa.schedule(idx, s, order)
-        e[4].record(stream)
-        vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, order, oc, d["g_coarse"], d["g_fine"], out=out,
-                       steps=steps)
-        e[5].record(stream)
-        vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out_d)
-        e[6].record(stream)
-        torch.cuda.synchronize()
-        if it >= args.warmup:
-            for j, n in enumerate(names):
-                acc[n].append(e[j].elapsed_time(e[j + 1]))
-            acc["fine_dense"].append(e[5].elapsed_time(e[6]))
-        del bars, scores, oc, idx, order, steps
-    stage_ms = {n: round(statistics.mean(v), 4) for n, v in acc.items()}
+    stage_ms = stage_times(vsa, torch, d, w, args.steps, args.warmup, dense_too=True)
+
+    # ---- the memory-bound entry points one launch at a time
+    mem = memory_kernels(vsa, torch, d, w, hbm_peak, max(10, args.steps))
 
     # ---- the pre-attention pass (Q/K RMSNorm + 3D RoPE) on the same Q/K, timed on its own
     wts = synth.make_projection_inputs(synth.custom_workload("weights", 1, w.heads, w.head_dim, (1, 1, 1), 1))
     w_q, w_k = (torch.from_numpy(wts[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("w_q", "w_k"))
     q_n, k_n = torch.empty_like(d["q"]), torch.empty_like(d["k"])
-    pre = []
-    for it in range(args.warmup + args.steps):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-        e[0].record(stream)
-        vsa.qk_norm_rope(d["q"], d["k"], s, w_q, w_k, out=(q_n, k_n))
-        e[1].record(stream)
-        torch.cuda.synchronize()
-        if it >= args.warmup:
-            pre.append(e[0].elapsed_time(e[1]))
-    pre_ms = reduce_max(statistics.mean(pre), world)
+    pre_ms = reduce_max(time_launches(torch, lambda: vsa.qk_norm_rope(d["q"], d["k"], s, w_q, w_k, out=(q_n, k_n)),
+                                      max(10, args.steps), args.warmup), world)
     del q_n, k_n
 
     # ---- end to end through vsa_forward_host (pinned host buffers, copies inside the timed region)
     h = {k: v.cpu().pin_memory() for k, v in d.items()}
     h_out = torch.empty_like(h["q"]).pin_memory()
     ws_host = vsa.alloc_workspace(s, w.topk, host_io=True, device=dev)
-    for _ in range(max(1, args.warmup // 2)):
-        vsa.forward_host(h["q"], h["k"], h["v"], s, w.topk, ws_host, h_out, scale, h["g_coarse"], h["g_fine"])
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(3, args.steps // 2)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        vsa.forward_host(h["q"], h["k"], h["v"], s, w.topk, ws_host, h_out, scale, h["g_coarse"], h["g_fine"])
-    e1.record(stream)
-    torch.cuda.synchronize()
+    e2e_ms = reduce_max(time_launches(
+        torch, lambda: vsa.forward_host(h["q"], h["k"], h["v"], s, w.topk, ws_host, h_out, scale, h["g_coarse"],
+                                        h["g_fine"]), max(5, args.steps // 2), max(1, args.warmup // 2)), world)
     vsa.device_status()
-    e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, world)
     h2d = sum(h[k].numel() * 2 for k in ("q", "k", "v", "g_coarse", "g_fine"))
     d2h = h_out.numel() * 2
+    del h, h_out, ws_host, ws, ws_dense, out, out_d, d
+    torch.cuda.empty_cache()
+
+    # ---- the 720p CFG batch
+    cfg = cfg720_record(vsa, torch, dev, bf16_peak, max(5, args.steps // 2), args.warmup)
 
     if rank != 0:
         return
-    peaks, peaks_src = load_peaks()
-    bf16_peak = float(peaks["bf16_tflops"])
-    hbm_peak = float(peaks["hbm_gbs"])
     pre_bytes = 4 * w.batch * w.tokens * w.heads * w.head_dim * 2
     fine_flops = executed_fine_flops(w.batch, w.heads, npad, w.topk, w.head_dim)
     nblk = (w.tokens + 63) // 64   # dense attention walks blocks of 64 consecutive real tokens
@@ -367,9 +500,12 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     traffic = traffic_for(fine_src, "fine_kernel_wan480p_vsa_k32")
     cpu = None
     if world == 1:
-        ms_cpu, spent, sample = oracle_sample(w, x, heads=tuple(range(0, w.heads, 5)), cubes_per_head=320)
-        cpu = {"value": round(ms_cpu, 1), "unit": "ms", "cores": blas_threads(), "kind": "oracle",
-               "sample": sample + f" ({spent:.1f} s of CPU work)"}
+        heads = oracle_sample_heads(w, range(ORACLE_BASELINE_HEADS))
+        secs = [oracle_head_seconds(w, x, hh) for hh in heads]
+        cpu = {"value": round(statistics.median(secs) * w.batch * w.heads * 1e3, 1), "unit": "ms",
+               "cores": blas_threads(), "kind": "oracle",
+               "sample": oracle_rule_text(w) + f"; steps 0..{len(heads) - 1}, heads {heads}, "
+                                               f"{sum(secs):.1f} s of CPU work"}
     line = {
         "metric": METRIC, "value": round(whole_job_ms_per_call(vsa_ms_max, 1, world), 4), "unit": "ms",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 4),
@@ -379,9 +515,11 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                    "padded_tokens": npad, "cubes": C, "heads": w.heads, "head_dim": w.head_dim, "topk": w.topk,
                    "dense_call": {"workload": DENSE_WORKLOAD, "topk": C},
                    "l2": "no flush: 1.0 GB of Q/K/V per call exceeds the 126 MB L2",
+                   "timing": "median of the timed calls (CUDA events on the launching stream)",
                    "parallelism": f"{world} independent replicas (weak scaling)"},
         "dense_ms_per_call": round(whole_job_ms_per_call(dense_ms_max, 1, world), 4),
         "stage_ms": stage_ms,
+        "fixed_max_rerun": rerun,
         "fine": {"executed_tflop": round(fine_flops / 1e12, 4), "tflops": round(fine_tflops, 1),
                  "frac_bf16_peak": round(fine_tflops / bf16_peak, 4),
                  "dense_equivalent_tflops": round(dense_equivalent_flops(w.batch, w.heads, w.tokens, w.head_dim)
@@ -395,6 +533,9 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                      "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)" if peaks_src == "measured"
                      else "fallback 1.59 PFLOP/s", "traffic": traffic,
                      "per_launch": "4*B*H*Npad*k*64*D executed flops (64x64 cube tiles of the k selected cubes)"},
+        "wan720p_cfg_k64": cfg,
+        "memory_kernels": {"workload": WORKLOAD, "peak_gbps": hbm_peak,
+                           "peak_source": f"{peaks_src} HBM copy (MEASURED_PEAKS.json)", "kernels": mem},
         "pre_attention": {"api": "vsa_qk_norm_rope (Q/K RMSNorm over H*D + 3D RoPE), timed on its own, not in value",
                           "ms": round(pre_ms, 4), "bytes": pre_bytes, "bound": "hbm",
                           "achieved_gbps": round(pre_bytes / (pre_ms * 1e-3) / 1e9, 1), "peak_gbps": hbm_peak,
@@ -414,13 +555,34 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     print(json.dumps(line), flush=True)
 
 
+def run_stages(args):
+    """Stage-by-stage times of one call on a named workload (rank 0 only, no process group)."""
+    import torch
+
+    import block_sparse_attention_cube_b200 as vsa
+    w = synth.WORKLOADS[args.workload]
+    x = synth.make_inputs(w)
+    d = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).cuda() for k, v in x.items()}
+    ms = stage_times(vsa, torch, d, w, args.iters, 0, dense_too=args.dense_too, staged=args.staged)
+    vsa.device_status()
+    print(json.dumps({"workload": w.name, "iters": args.iters, "staged": args.staged, "ms": ms}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--stages", action="store_true", help="stage-by-stage times of one call (profiling case)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS), help="with --stages")
+    ap.add_argument("--iters", type=int, default=3, help="with --stages")
+    ap.add_argument("--dense-too", action="store_true", help="with --stages: add a dense fine-stage launch")
+    ap.add_argument("--staged", action="store_true", help="with --stages: the unfused per-step entry points")
     args = ap.parse_args(argv)
+    if args.stages:
+        run_stages(args)
+        return 0
     if args.warmup < 3 and args.impl == "cuda":
         ap.error("at least 3 warm-up steps")
     world = int(os.environ.get("WORLD_SIZE", "1"))

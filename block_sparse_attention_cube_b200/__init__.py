@@ -208,14 +208,6 @@ def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, shape: Shape, w_q: Optional[t
     return qo, ko
 
 
-def pair_order(idx: torch.Tensor, shape: Shape, order: torch.Tensor) -> torch.Tensor:
-    """Re-pairs the work order in place so that consecutive pairs share many selected key cubes; returns it."""
-    k = int(idx.shape[-1])
-    _check(_L.vsa_pair_order(ctypes.byref(shape.c()), _ptr(idx, torch.int32, "idx"), k,
-                             _ptr(order, torch.int32, "order"), _stream()))
-    return order
-
-
 def schedule(idx: torch.Tensor, shape: Shape, order: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Precomputed steps of the fine stage for the selection idx [B,H,C,k] (and work order)."""
     k = int(idx.shape[-1])

@@ -49,7 +49,6 @@ SIGNATURES = {
     "vsa_fine_fused": (ctypes.c_int, [_SP, _P, _P, _P, _P, _I32, _P, _P, _F32, _P, _P, _P, _P, _P, _P]),
     "vsa_schedule_bytes": (_SZ, [_SP, _I32]),
     "vsa_schedule": (ctypes.c_int, [_SP, _P, _I32, _P, _P, _P]),
-    "vsa_pair_order": (ctypes.c_int, [_SP, _P, _I32, _P, _P]),
     "vsa_qk_norm_rope": (ctypes.c_int, [_SP, _P, _P, _P, _P, _F32, _F32, _I64, _I64, _P, _P, _P]),
     "vsa_workspace_bytes": (_SZ, [_SP, _I32]),
     "vsa_forward": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _I32, _F32, _P, _SZ, _P, _P]),

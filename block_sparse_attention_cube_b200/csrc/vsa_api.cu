@@ -552,21 +552,6 @@ vsa_status vsa_topk_order(const vsa_shape* shape, const float* scores, int32_t k
     return VSA_OK;
 }
 
-vsa_status vsa_pair_order(const vsa_shape* shape, const int32_t* idx, int32_t topk, int32_t* order,
-                          vsa_stream_t stream) {
-    Dims d{};
-    VSA_TRY(make_dims(shape, &d));
-    VSA_TRY(check_k(d, topk));
-    VSA_TRY(need_ptr(idx, "idx"));
-    VSA_TRY(need_ptr(order, "order"));
-    if (!pair_order_supported(d, topk))
-        return fail(VSA_ERR_UNSUPPORTED, "vsa_pair_order supports C <= 1120 (got C=%d)", d.C);
-    VSA_TRY(check_disjoint({{idx, idx_bytes(d, topk), "idx"}}, {{order, order_bytes(d), "order"}}));
-    VSA_TRY(check_device());
-    VSA_CUDA(launch_pair_order(d, idx, topk, order, as_stream(stream)), "pair launch");
-    return VSA_OK;
-}
-
 size_t vsa_schedule_bytes(const vsa_shape* shape, int32_t topk) {
     Dims d{};
     if (make_dims(shape, &d) != VSA_OK || topk < 1 || topk > d.C) return 0;

@@ -580,260 +580,5 @@ cudaError_t launch_group_sort(const Dims& d, const uint64_t* sig, int32_t* order
     return cudaGetLastError();
 }
 
-// ---------------------------------------------------------------- pairing
-// The fine stage takes consecutive pairs of the work order as its 128-row
-// tiles, and a tile's steps are the union of its two selections.  After the
-// signature sort, pair_order_kernel re-pairs the order: it counts, for every
-// position p and each of the kPairWin positions after it, how many selected
-// key cubes the two query cubes share (popcounts of per-cube selection
-// bitmaps in shared memory, so C is bounded by that memory: C <= 1120); then,
-// for up to kPairRounds rounds (until one pairs nobody), every unpaired
-// position proposes to its best unpaired neighbour within kPairWin positions
-// (more shared cubes first, then the nearer, then the earlier), and mutual
-// proposals pair up.  The pairs are
-// written in the order of their first member, leftovers paired in order of
-// position (an odd one out last), if they share more key cubes in total than
-// the input's consecutive pairs, leftover pairs more than kPairWin apart
-// counting as sharing none (otherwise the input order stays).  One block per
-// (b, h).  A cube listed twice in a row counts once; any input gives a
-// permutation.
-constexpr int kPairWin = 16;
-constexpr int kPairMaxC = 1120;   // selection bitmaps and scan arrays within 220 KB of shared memory
-constexpr int kPairRounds = 8;
-__host__ __device__ inline int pair_row_words(int C) { return ((C + 31) / 32) | 1; }
-constexpr int kPairThreads = 512;
-
-__global__ void __launch_bounds__(kPairThreads) pair_order_kernel(int C, int k, const int32_t* __restrict__ idx,
-                                                                  int32_t* __restrict__ order) {
-    extern __shared__ __align__(16) uint8_t pair_smem[];
-    const int nws = pair_row_words(C);                             // bitmap row stride (odd: no bank conflicts)
-    const int nw = (C + 31) / 32;                                  // bitmap words in use per row
-    uint32_t* bits = reinterpret_cast<uint32_t*>(pair_smem);       // [C][nws] selections of the cube at position p
-    int32_t* ord = reinterpret_cast<int32_t*>(bits + static_cast<size_t>(C) * nws);   // [C] cube at position p
-    int16_t* partner = reinterpret_cast<int16_t*>(ord + C);        // [C] partner position or -1
-    int16_t* best = partner + C;                                   // [C] this round's proposal
-    uint8_t* ov = reinterpret_cast<uint8_t*>(best + C);            // [C][2 kPairWin] shared-cube counts
-    int* urank = reinterpret_cast<int*>(ov + static_cast<size_t>(C) * 2 * kPairWin);   // [C] rank among the unmatched
-    int* upos = urank + C;                                         // [C] position of the u-th unmatched
-    int* scan = upos + C;                                          // [C] pair slot of a pair's first position
-    uint32_t* taken = reinterpret_cast<uint32_t*>(scan + C);       // bit 32 + p: position p is paired (or absent)
-    const int ntw = (C + 64 + 31) / 32;
-    const int64_t bh = blockIdx.x;
-    const int32_t* I = idx + bh * static_cast<int64_t>(C) * k;
-    int32_t* O = order + bh * static_cast<int64_t>(C);
-    for (int p = threadIdx.x; p < C; p += blockDim.x) {
-        ord[p] = O[p];
-        partner[p] = -1;
-    }
-    for (int i = threadIdx.x; i < C * nws; i += blockDim.x) bits[i] = 0u;
-    for (int i = threadIdx.x; i < C * 2 * kPairWin; i += blockDim.x) ov[i] = 0;
-    for (int wdx = threadIdx.x; wdx < ntw; wdx += blockDim.x) {
-        // positions below 0 and from C on count as taken
-        uint32_t m = 0u;
-        for (int b2 = 0; b2 < 32; ++b2) {
-            const int pos = 32 * wdx + b2 - 32;
-            if (pos < 0 || pos >= C) m |= 1u << b2;
-        }
-        taken[wdx] = m;
-    }
-    __syncthreads();
-    // selection bitmaps: loads batched so that several are in flight per thread
-    constexpr int kBatch = 8;
-    for (int t0 = threadIdx.x; t0 < C * k; t0 += blockDim.x * kBatch) {
-        int v[kBatch], pp[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int t = t0 + u * static_cast<int>(blockDim.x);
-            v[u] = -1;
-            pp[u] = 0;
-            if (t < C * k) {
-                const int p = t / k, i = t - p * k;
-                const int cp = ord[p];
-                pp[u] = p;
-                if (cp >= 0 && cp < C) v[u] = __ldg(I + static_cast<int64_t>(cp) * k + i);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-            if (v[u] >= 0 && v[u] < C) atomicOr(bits + static_cast<size_t>(pp[u]) * nws + (v[u] >> 5), 1u << (v[u] & 31));
-    }
-    __syncthreads();
-    // shared-cube counts: a thread per position holds its row and walks the next kPairWin rows
-    constexpr int kMaxWords = (kPairMaxC + 31) / 32;
-    for (int p = threadIdx.x; p < C; p += blockDim.x) {
-        uint32_t ra[kMaxWords];
-        const uint32_t* rp = bits + static_cast<size_t>(p) * nws;
-#pragma unroll
-        for (int w = 0; w < kMaxWords; ++w) ra[w] = w < nw ? rp[w] : 0u;
-        for (int dd = 1; dd <= kPairWin && p + dd < C; ++dd) {
-            const uint32_t* rb = bits + static_cast<size_t>(p + dd) * nws;
-            int o = 0;
-#pragma unroll
-            for (int w = 0; w < kMaxWords; ++w)
-                if (w < nw) o += __popc(ra[w] & rb[w]);
-            const uint8_t o8 = static_cast<uint8_t>(o < 255 ? o : 255);
-            ov[p * 2 * kPairWin + kPairWin + dd - 1] = o8;         // neighbour p + dd
-            ov[(p + dd) * 2 * kPairWin + kPairWin - dd] = o8;      // neighbour (p + dd) - dd
-        }
-    }
-    __syncthreads();
-    __shared__ int any_match;
-    for (int r = 0; r < kPairRounds; ++r) {
-        if (threadIdx.x == 0) any_match = 0;
-        __syncthreads();
-        for (int p = threadIdx.x; p < C; p += blockDim.x) {
-            int bq = -1;
-            if (partner[p] < 0) {
-                // bit j of win: position p - kPairWin + j is taken (j = 0 .. 2 kPairWin)
-                const int s0 = p - kPairWin + 32;
-                const uint64_t w2 = (static_cast<uint64_t>(taken[(s0 >> 5) + 1]) << 32) | taken[s0 >> 5];
-                const uint64_t win = w2 >> (s0 & 31);
-                const uint32_t* ovw = reinterpret_cast<const uint32_t*>(ov + p * 2 * kPairWin);
-                int bkey = -1;
-#pragma unroll
-                for (int wq = 0; wq < 2 * kPairWin / 4; ++wq) {
-                    const uint32_t four = ovw[wq];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int sl = 4 * wq + e;                      // slot: p - kPairWin + sl, or p + sl - kPairWin + 1
-                        const int j = sl < kPairWin ? sl : sl + 1;      // window bit of that neighbour
-                        const int near = sl < kPairWin ? sl : 2 * kPairWin - 1 - sl;   // kPairWin - distance
-                        // more shared, then nearer, then the earlier of two equally near
-                        const int key = ((static_cast<int>((four >> (8 * e)) & 0xFFu) * 64 + near) * 2) +
-                                        (sl < kPairWin ? 1 : 0);
-                        const bool free_q = ((win >> j) & 1ull) == 0ull;
-                        if (free_q && key > bkey) {
-                            bkey = key;
-                            bq = p - kPairWin + j;
-                        }
-                    }
-                }
-            }
-            best[p] = static_cast<int16_t>(bq);
-        }
-        __syncthreads();
-        for (int p = threadIdx.x; p < C; p += blockDim.x) {
-            const int q = best[p];
-            if (q >= 0 && best[q] == p) {
-                partner[p] = static_cast<int16_t>(q);
-                atomicOr(taken + ((p + 32) >> 5), 1u << ((p + 32) & 31));
-                any_match = 1;
-            }
-        }
-        __syncthreads();
-        const bool again = any_match != 0;
-        __syncthreads();         // every thread has read the flag before the next round resets it
-        if (!again) break;       // nothing changed: every later round would propose the same
-    }
-    __syncthreads();
-    // Output.  A position starts a pair when it is matched to a later position, or when it is the
-    // 2u-th unmatched position (paired with the (2u+1)-th); a block-wide scan of those flags gives
-    // each pair its slot.  The pairs are kept if they share more key cubes in total than the
-    // input's consecutive pairs (leftover pairs more than kPairWin apart count as sharing none).
-    __shared__ int warp_sum[kPairThreads / 32];
-    __shared__ int totals[2];
-    // exclusive block-wide scan of a[0, C) in place; returns the total
-    auto scan_in_place = [&](int* a) -> int {
-        int carry = 0;
-        for (int base0 = 0; base0 < C; base0 += blockDim.x) {
-            const int p = base0 + threadIdx.x;
-            const int f = p < C ? a[p] : 0;
-            int incl = f;
-            const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            if (lane == 31) warp_sum[wid] = incl;
-            __syncthreads();
-            if (wid == 0) {
-                const int v = lane < static_cast<int>(blockDim.x >> 5) ? warp_sum[lane] : 0;
-                int vi = v;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int y = __shfl_up_sync(0xffffffffu, vi, o);
-                    if (lane >= o) vi += y;
-                }
-                if (lane < static_cast<int>(blockDim.x >> 5)) warp_sum[lane] = vi - v;   // exclusive warp offsets
-                if (lane == 31) totals[1] = vi;
-            }
-            __syncthreads();
-            if (p < C) a[p] = carry + warp_sum[wid] + incl - f;
-            carry += totals[1];
-            __syncthreads();
-        }
-        return carry;
-    };
-    // unmatched positions: their rank u among the unmatched, and the position of each rank
-    for (int p = threadIdx.x; p < C; p += blockDim.x) urank[p] = partner[p] < 0 ? 1 : 0;
-    __syncthreads();
-    const int n_unm = scan_in_place(urank);
-    for (int p = threadIdx.x; p < C; p += blockDim.x)
-        if (partner[p] < 0) upos[urank[p]] = p;
-    // pair starts and their slots; with an odd number of unmatched positions the last of them is
-    // left alone and goes to the end of the order
-    for (int p = threadIdx.x; p < C; p += blockDim.x)
-        scan[p] = (partner[p] > p || (partner[p] < 0 && (urank[p] & 1) == 0 && urank[p] + 1 < n_unm)) ? 1 : 0;
-    __syncthreads();
-    scan_in_place(scan);
-    if (threadIdx.x == 0) totals[0] = 0;
-    __syncthreads();
-    int my_new = 0, my_old = 0;
-    for (int p = threadIdx.x; p < C; p += blockDim.x) {
-        const int q = partner[p];
-        int mate = -1;
-        if (q > p) mate = q;
-        else if (q < 0 && (urank[p] & 1) == 0 && urank[p] + 1 < n_unm) mate = upos[urank[p] + 1];
-        if (mate > p && mate - p <= kPairWin) my_new += ov[p * 2 * kPairWin + kPairWin + (mate - p) - 1];
-        if ((p & 1) == 0 && p + 1 < C) my_old += ov[p * 2 * kPairWin + kPairWin];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        my_new += __shfl_xor_sync(0xffffffffu, my_new, o);
-        my_old += __shfl_xor_sync(0xffffffffu, my_old, o);
-    }
-    if ((threadIdx.x & 31) == 0) {
-        atomicAdd(&totals[0], my_new - my_old);
-    }
-    __syncthreads();
-    if (totals[0] > 0) {
-        for (int p = threadIdx.x; p < C; p += blockDim.x) {
-            const int q = partner[p];
-            const bool unm_start = q < 0 && (urank[p] & 1) == 0 && urank[p] + 1 < n_unm;
-            if (q > p || unm_start) {
-                const int slot = 2 * scan[p];   // < C - 1: every pair before it fills two entries
-                O[slot] = ord[p];
-                O[slot + 1] = q > p ? ord[q] : ord[upos[urank[p] + 1]];
-            } else if (q < 0 && urank[p] == n_unm - 1 && (n_unm & 1)) {
-                O[C - 1] = ord[p];              // the lone leftover
-            }
-        }
-    }
-}
-
-size_t pair_smem_bytes(int C) {
-    return static_cast<size_t>(C) * pair_row_words(C) * 4 + static_cast<size_t>(C) * (4 + 2 + 2 + 2 * kPairWin + 12) +
-           static_cast<size_t>((C + 64 + 31) / 32) * 4;
-}
-
-cudaError_t launch_pair_order(const Dims& d, const int32_t* idx, int k, int32_t* order, cudaStream_t s) {
-    if (!pair_order_supported(d, k)) return cudaErrorInvalidValue;
-    const size_t smem = pair_smem_bytes(d.C);
-    static int done[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (!(dev >= 0 && dev < 64 && done[dev])) {
-        cudaError_t e = cudaFuncSetAttribute(pair_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) done[dev] = 1;
-    }
-    pair_order_kernel<<<d.B * d.H, kPairThreads, smem, s>>>(d.C, k, idx, order);
-    return cudaGetLastError();
-}
-
-bool pair_order_supported(const Dims& d, int k) {
-    return k >= 1 && d.C <= kPairMaxC && pair_smem_bytes(d.C) <= 220 * 1024;
-}
 
 }  // namespace vsa

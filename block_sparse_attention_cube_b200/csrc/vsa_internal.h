@@ -64,11 +64,6 @@ cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* 
 constexpr int kGroupMaxC = 4096;
 cudaError_t launch_group(const Dims& d, const float* scores, int32_t* order, cudaStream_t s);
 cudaError_t launch_group_sort(const Dims& d, const uint64_t* sig, int32_t* order, cudaStream_t s);
-// Re-pairs a work order (order [B, H, C], in place) so that each pair of
-// consecutive entries shares many selected key cubes (idx [B, H, C, k], rows
-// ascending); supported while its selection bitmaps fit in shared memory (C <= 1120).
-bool pair_order_supported(const Dims& d, int k);
-cudaError_t launch_pair_order(const Dims& d, const int32_t* idx, int k, int32_t* order, cudaStream_t s);
 
 // Fine stage.  Modes:
 //  kFineTiled       - q/k/v tiled [B, H, Npad, D]; out = tiled O_f (+ lse when non-null);

@@ -645,76 +645,3 @@ def test_schedule_covers_every_selection_once(case):
                             got[(j, int(blk))] = got.get((j, int(blk)), 0) + 1
             assert got == want, it
             assert pats == sorted(pats), it
-
-
-def _pair_reference(order, idx, win=16, rounds=8):
-    """The documented pairing rule of vsa_pair_order, restated on the host for one head."""
-    C = len(order)
-    sets = [set(idx[c].tolist()) if 0 <= c < C else set() for c in order]
-    ov = {}
-    for p in range(C):
-        for dd in range(1, win + 1):
-            if p + dd < C:
-                ov[(p, p + dd)] = ov[(p + dd, p)] = min(len(sets[p] & sets[p + dd]), 255)
-    partner = [-1] * C
-    for _ in range(rounds):
-        best = [-1] * C
-        for p in range(C):
-            if partner[p] >= 0:
-                continue
-            bs, bq = -1, -1
-            for dd in range(1, win + 1):
-                for q in (p - dd, p + dd):
-                    if 0 <= q < C and partner[q] < 0:
-                        sc = ov[(p, q)] * 64 + (win - dd)
-                        if sc > bs:
-                            bs, bq = sc, q
-            best[p] = bq
-        matched = False
-        for p in range(C):
-            q = best[p]
-            if q >= 0 and best[q] == p:
-                partner[p] = q
-                matched = True
-        if not matched:
-            break
-    # pairs in the order of their first position; unmatched positions paired in order of position,
-    # an odd one out last
-    unmatched = [p for p in range(C) if partner[p] < 0]
-    starts = [(p, [order[p], order[partner[p]]]) for p in range(C) if partner[p] > p]
-    starts += [(unmatched[i], [order[unmatched[i]], order[unmatched[i + 1]]])
-               for i in range(0, len(unmatched) - 1, 2)]
-    out = [c for _, pr in sorted(starts) for c in pr]
-    if len(unmatched) % 2:
-        out.append(order[unmatched[-1]])
-    pos = {c: p for p, c in enumerate(order)}
-    def total(seq):
-        t = 0
-        for i in range(0, C - 1, 2):
-            a, b = sorted((pos[seq[i]], pos[seq[i + 1]]))
-            t += ov[(a, b)] if b - a <= win else 0
-        return t
-    return out if total(out) > total(order) else list(order)
-
-
-def test_pair_order_follows_its_rule_and_pairs_better(case):
-    """vsa_pair_order is a permutation that follows its documented rule exactly (restated on the
-    host): its pairs share more selected cubes in total than the signature order's, or the order
-    is left as it was."""
-    w, _, dev, _ = case
-    s = _shape(w)
-    _, C = vsa.shape_info(s)
-    scale = 1 / math.sqrt(w.head_dim)
-    scores, _ = vsa.coarse(*vsa.pool_qkv(dev["q"], dev["k"], dev["v"], s), s, scale)
-    for k in sorted({1, min(w.topk, 64), min(C, 64)}):
-        idx, order = vsa.topk_order(scores, s, k)
-        base = order.clone()
-        vsa.pair_order(idx, s, order)
-        o, b0, ix = order.cpu().numpy(), base.cpu().numpy(), idx.cpu().numpy()
-        for bh in range(w.batch * w.heads):
-            got, start = o.reshape(-1, C)[bh], b0.reshape(-1, C)[bh]
-            sel = ix.reshape(-1, C, k)[bh]
-            assert sorted(got.tolist()) == list(range(C))
-            assert got.tolist() == _pair_reference(start.tolist(), sel), (bh, k)
-            shared = lambda seq: sum(len(set(sel[seq[i]]) & set(sel[seq[i + 1]])) for i in range(0, C - 1, 2))
-            assert shared(got.tolist()) >= shared(start.tolist()), (bh, k)
