@@ -46,6 +46,7 @@ SIGNATURES = {
     "vsa_combine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P]),
     "vsa_pool_qkv": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P]),
     "vsa_topk_order": (ctypes.c_int, [_SP, _P, _I32, _P, _P, _P, _P]),
+    "vsa_coarse_topk": (ctypes.c_int, [_SP, _P, _P, _P, _F32, _I32, _P, _P, _P, _P, _P, _P]),
     "vsa_fine_fused": (ctypes.c_int, [_SP, _P, _P, _P, _P, _I32, _P, _P, _F32, _P, _P, _P, _P, _P, _P]),
     "vsa_schedule_bytes": (_SZ, [_SP, _I32]),
     "vsa_schedule": (ctypes.c_int, [_SP, _P, _I32, _P, _P, _P]),

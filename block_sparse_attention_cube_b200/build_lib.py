@@ -25,7 +25,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libvsa_b200.so")
 
-SOURCES = ["vsa_api.cu", "vsa_layout.cu", "vsa_coarse.cu", "vsa_fine.cu", "vsa_prenorm.cu", "vsa_noalloc.cu"]
+SOURCES = sorted(f for f in os.listdir(CSRC) if f.endswith(".cu"))
 HEADERS = ["ptx_sm100.cuh", "vsa_internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -76,7 +76,9 @@ def build(force: bool = False, ptxas_v: bool = False, verbose: bool = False) -> 
                 logs.append((futs[f], f.result()))
     if jobs or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
         tmp = LIB + ".tmp"
-        cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
+        # every symbol must resolve inside the library (a source left out fails here, not at load time)
+        cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-Xlinker", "--no-undefined", "-o", tmp, *objs,
+               "-lpthread", "-ldl", "-lrt"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")

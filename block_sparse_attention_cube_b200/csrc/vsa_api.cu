@@ -162,6 +162,12 @@ size_t order_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C 
 constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+// Whether the forward call runs its selection as the one fused launch (coarse scores, top-k,
+// work-order keys and the coarse output; vsa_coarse_topk).  Measured on B200 it is no faster than the
+// two-launch path at 480p (0.41 against 0.40 ms) and slower at 720p (5.4 against 4.5 ms: a block's
+// 32 score rows take 184 KB of shared memory there, one block of 8 warps per SM), so it is off.
+bool fused_selection(const Dims&) { return false; }
+
 // Workspace of vsa_forward: qbar | kbar | vbar | o_coarse | scores | idx | order | sig | steps | overflow.
 // Q, K and V are read in the caller's [B, N, H, D] layout (the fine stage
 // gathers cubes with TMA), so no tiled copies are kept.  With every cube
@@ -192,7 +198,9 @@ Carve carve(const Dims& d, int k, bool coarse_gate, void* ws) {
         c.kbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
         c.vbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
         c.oc = reinterpret_cast<float*>(take(pooled_bytes(d)));
-        c.scores = reinterpret_cast<float*>(take(score_bytes(d)));
+        // the fused selection keeps the scores in shared memory; the scores buffer serves the
+        // two-launch path (and a coarse gate at top-k == C, whose output still needs the scores)
+        if (!(sparse && fused_selection(d))) c.scores = reinterpret_cast<float*>(take(score_bytes(d)));
     }
     if (sparse) {
         c.idx = reinterpret_cast<int32_t*>(take(idx_bytes(d, k)));
@@ -265,16 +273,23 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
                        const uint16_t* gf, int topk, float scale, void* ws, uint16_t* out, cudaStream_t s) {
     const bool sparse = topk < d.C;
     const Carve c = carve(d, topk, gc != nullptr, ws);
+    const bool fused = sparse && fused_selection(d);
     if (sparse || gc != nullptr) {
         const uint16_t* pin[3] = {q, k, v};
         float* pout[3] = {c.qbar, c.kbar, c.vbar};
         VSA_CUDA(launch_pool_tokens(d, pin, pout, 3, s), "pool launch");
-        VSA_CUDA(launch_coarse_scores(d, c.qbar, c.kbar, scale, c.scores, s), "coarse launch");
+        if (!fused) VSA_CUDA(launch_coarse_scores(d, c.qbar, c.kbar, scale, c.scores, s), "coarse launch");
     }
     // the coarse output (softmax(scores) x V-bar) is used only by the merge, and only with a coarse gate
-    if (gc != nullptr) VSA_CUDA(launch_coarse_pv(d, c.scores, c.vbar, c.oc, s), "coarse launch");
+    if (gc != nullptr && !fused) VSA_CUDA(launch_coarse_pv(d, c.scores, c.vbar, c.oc, s), "coarse launch");
     const int32_t* order = nullptr;
-    if (sparse) {
+    if (fused) {
+        // scores, selection, work-order keys and the coarse output in one launch, then the key sort
+        VSA_CUDA(launch_coarse_select(d, c.qbar, c.kbar, c.vbar, scale, topk, c.idx, c.sig, gc ? c.oc : nullptr,
+                                      nullptr, s), "coarse select launch");
+        VSA_CUDA(launch_group_sort(d, c.sig, c.order, s), "group launch");
+        order = c.order;
+    } else if (sparse) {
         if (d.C <= kTopkRegMaxC && d.C <= kGroupMaxC) {
             // one pass over the scores gives the selection and the work-order keys
             VSA_CUDA(launch_topk_sig(d, c.scores, topk, c.idx, c.sig, s), "topk launch");
@@ -549,6 +564,40 @@ vsa_status vsa_topk_order(const vsa_shape* shape, const float* scores, int32_t k
     VSA_TRY(check_device());
     VSA_CUDA(launch_topk_sig(d, scores, k, idx, sig_scratch, as_stream(stream)), "topk launch");
     VSA_CUDA(launch_group_sort(d, sig_scratch, order, as_stream(stream)), "group launch");
+    return VSA_OK;
+}
+
+vsa_status vsa_coarse_topk(const vsa_shape* shape, const float* qbar, const float* kbar, const float* vbar,
+                           float scale, int32_t k, int32_t* idx, int32_t* order, uint64_t* sig_scratch,
+                           float* o_coarse, float* scores, vsa_stream_t stream) {
+    Dims d{};
+    VSA_TRY(make_dims(shape, &d));
+    VSA_TRY(check_k(d, k));
+    VSA_TRY(check_scale(scale));
+    VSA_TRY(need_ptr(qbar, "qbar"));
+    VSA_TRY(need_ptr(kbar, "kbar"));
+    VSA_TRY(need_ptr(idx, "idx"));
+    VSA_TRY(opt_ptr(vbar, "vbar"));
+    VSA_TRY(opt_ptr(o_coarse, "o_coarse"));
+    VSA_TRY(opt_ptr(order, "order"));
+    VSA_TRY(opt_ptr(sig_scratch, "sig_scratch"));
+    VSA_TRY(opt_ptr(scores, "scores"));
+    if ((vbar == nullptr) != (o_coarse == nullptr))
+        return fail(VSA_ERR_INVALID_ARGUMENT, "vbar and o_coarse must both be given or both be NULL");
+    if ((order == nullptr) != (sig_scratch == nullptr))
+        return fail(VSA_ERR_INVALID_ARGUMENT, "order and sig_scratch must both be given or both be NULL");
+    if (!coarse_select_supported(d))
+        return fail(VSA_ERR_UNSUPPORTED, "vsa_coarse_topk keeps a block's score rows in shared memory: C <= 1536 "
+                    "(got %d)", d.C);
+    const size_t pb = pooled_bytes(d);
+    VSA_TRY(check_disjoint({{qbar, pb, "qbar"}, {kbar, pb, "kbar"}, {vbar, vbar ? pb : 0, "vbar"}},
+                           {{idx, idx_bytes(d, k), "idx"}, {order, order ? order_bytes(d) : 0, "order"},
+                            {sig_scratch, sig_scratch ? 2 * order_bytes(d) : 0, "sig_scratch"},
+                            {o_coarse, o_coarse ? pb : 0, "o_coarse"}, {scores, scores ? score_bytes(d) : 0, "scores"}}));
+    VSA_TRY(check_device());
+    VSA_CUDA(launch_coarse_select(d, qbar, kbar, vbar, scale, k, idx, sig_scratch, o_coarse, scores,
+                                  as_stream(stream)), "coarse select launch");
+    if (order) VSA_CUDA(launch_group_sort(d, sig_scratch, order, as_stream(stream)), "group launch");
     return VSA_OK;
 }
 

@@ -60,6 +60,14 @@ cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx,
 constexpr int kTopkRegMaxC = 2048;
 cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s);
 
+// The coarse scores, the top-k selection (and each row's work-order key) and, with o_coarse, the
+// coarse output in one launch; the scores stay in shared memory (copied to scores_out when given).
+// Bit-identical scores and selection to launch_coarse_scores + launch_topk_sig.
+bool coarse_select_supported(const Dims& d);
+cudaError_t launch_coarse_select(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
+                                 int k, int32_t* idx, uint64_t* sig, float* o_coarse, float* scores_out,
+                                 cudaStream_t s);
+
 // Work order of the fine stage from the coarse scores (C <= kGroupMaxC).
 constexpr int kGroupMaxC = 4096;
 cudaError_t launch_group(const Dims& d, const float* scores, int32_t* order, cudaStream_t s);

@@ -212,6 +212,34 @@ vsa_status vsa_topk_order(const vsa_shape* shape, const float* scores, int32_t k
                           uint64_t* sig_scratch, vsa_stream_t stream);
 
 /*
+ * vsa_coarse_topk — the coarse stage and the selection in one pass over the
+ * pooled cubes (same section, part 1), so the [B, H, C, C] scores never reach
+ * global memory (teardown section "Fusion targets launch overhead and
+ * memory").  One block per 32 query cubes of one (b, h) computes their rows of
+ * scale * qbar kbar^T in shared memory, each score the same float32 sum as
+ * vsa_coarse's (identical bits), keeps each row's k best key cubes (identical
+ * to vsa_topk on those scores: ties to the lower index, rows ascending) and
+ * each row's work-order key (as vsa_topk_order), and, when vbar and o_coarse
+ * are given, turns the rows into softmax(scores) in place and writes
+ * o_coarse = softmax(scores) vbar (the same values as vsa_coarse's up to
+ * float32 rounding order).  With `order`, a second launch sorts the keys into
+ * the work order of vsa_topk_order.
+ *   qbar, kbar   [B, H, C, D] float32 (read).
+ *   vbar         [B, H, C, D] float32 (read), or NULL together with o_coarse.
+ *   idx          [B, H, C, k] int32 (written).
+ *   order        [B, H, C] int32 (written), or NULL together with sig_scratch.
+ *   sig_scratch  [B, H, C] uint64 caller scratch (overwritten), or NULL.
+ *   o_coarse     [B, H, C, D] float32 (written), or NULL.
+ *   scores       [B, H, C, C] float32, or NULL: a copy of the scores the
+ *                kernel ranked (a check of the fusion; it costs the write).
+ * Supported for C <= 1536 (a block's 32 score rows must fit in shared memory;
+ * VSA_ERR_UNSUPPORTED otherwise: use vsa_coarse and vsa_topk_order).
+ */
+vsa_status vsa_coarse_topk(const vsa_shape* shape, const float* qbar, const float* kbar, const float* vbar,
+                           float scale, int32_t k, int32_t* idx, int32_t* order, uint64_t* sig_scratch,
+                           float* o_coarse, float* scores, vsa_stream_t stream);
+
+/*
  * vsa_qk_norm_rope — the pre-attention pass of a Wan DiT block: RMSNorm of each
  * token's query and key over all H*D channels, then the 3D rotary position
  * embedding, in one read and one write of Q and K (WorldFoundry inference guide,
@@ -309,7 +337,8 @@ vsa_status vsa_schedule(const vsa_shape* shape, const int32_t* idx, int32_t topk
 size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
 
 /*
- * vsa_forward — the whole attention call on one stream, as eight launches:
+ * vsa_forward — the whole attention call on one stream, as eight launches for
+ * top-k < C:
  *   vsa_pool_qkv -> vsa_coarse (2) -> vsa_topk_order (2) -> vsa_schedule
  *   -> vsa_fine_fused (the one-tile kernel and its re-run guard)
  * (the second vsa_coarse launch, the coarse output softmax(scores) x V-bar,

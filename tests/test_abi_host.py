@@ -97,6 +97,18 @@ def test_forward_rerun_argument_checks():
     assert r.value == 0
 
 
+def test_coarse_topk_argument_checks():
+    s = _shape()
+    p = [ctypes.c_void_p((1 << 40) + i * (1 << 32)) for i in range(8)]
+    call = lambda vbar, order, sig, oc, sh=s: vsa.raw_call("vsa_coarse_topk", ctypes.byref(sh), p[0], p[1], vbar,
+                                                          0.125, 2, p[2], order, sig, oc, None, None)
+    assert call(p[3], None, None, None) == INVALID and "vbar and o_coarse" in vsa.last_error()
+    assert call(None, p[4], None, None) == INVALID and "order and sig_scratch" in vsa.last_error()
+    # C = 6*8*33 = 1584 cubes: the score rows of a block no longer fit in shared memory
+    big = _lib.VsaShape(1, 1, 64, 24, 32, 132)
+    assert call(None, None, None, None, big) == UNSUPPORTED and "1536" in vsa.last_error()
+
+
 def test_overlapping_input_and_output_rejected():
     s = _shape()
     base = 1 << 40
@@ -145,6 +157,7 @@ def test_workspace_size_480p_matches_layout():
         + up(312 * 40 * 32 * 8) \
         + up(4)   # work-order signatures; steps: 312 pairs of query cubes x k steps x 8 B; overflow word
     assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 32) == expect
+
     # every cube selected: dense attention; the coarse buffers are for a coarse gate only
     assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 624) == 4 * up(624 * 40 * 128 * 4) + \
         up(624 * 624 * 40 * 4) + up(4)

@@ -592,6 +592,61 @@ def test_topk_order_selection_and_order(case):
                 assert o[bh].tolist() == want, (k, bh)
 
 
+def _check_coarse_topk(s, bars, scale, ks, label):
+    """vsa_coarse_topk against the two-launch path on the same pooled inputs: identical scores (the
+    copy of what it ranked), identical selection and work order, coarse output within float32 rounding."""
+    scores, oc = vsa.coarse(*bars, s, scale)
+    for k in ks:
+        idx, order, oc2, sc2 = vsa.coarse_topk(*bars, s, k, scale, want_scores=True)
+        assert torch.equal(sc2, scores), f"{label}: fused scores differ (k={k})"
+        ref_idx, ref_order = vsa.topk_order(scores, s, k)
+        assert torch.equal(idx, ref_idx), f"{label}: fused selection differs (k={k})"
+        assert torch.equal(order, ref_order), f"{label}: fused work order differs (k={k})"
+        rel = float((oc2 - oc).norm() / oc.norm())
+        assert rel <= 1e-6, f"{label}: coarse output rel L2 {rel:.2e} (k={k})"
+        # without the coarse output, the order or the score copy: the same selection
+        idx2, none_order, none_oc, none_sc = vsa.coarse_topk(bars[0], bars[1], None, s, k, scale, order=False)
+        assert none_order is None and none_oc is None and none_sc is None
+        assert torch.equal(idx2, idx), f"{label}: selection without the coarse output differs (k={k})"
+    return scores, oc
+
+
+def test_coarse_topk_equals_the_two_launch_path(case):
+    """The fused coarse stage + selection on every small and edge case, against vsa_coarse +
+    vsa_topk_order bit for bit, and its coarse output against the oracle's."""
+    w, _, dev, f64 = case
+    s = _shape(w)
+    _, C = vsa.shape_info(s)
+    scale = 1 / math.sqrt(w.head_dim)
+    bars = vsa.pool_qkv(dev["q"], dev["k"], dev["v"], s)
+    ks = sorted({1, min(w.topk, C), min(33, C), C})
+    _check_coarse_topk(s, bars, scale, ks, w.name)
+    ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, w.topk, scale)
+    _, _, oc, _ = vsa.coarse_topk(*bars, s, w.topk, scale)
+    rel = np.linalg.norm(from_dev(oc) - ora["o_coarse"]) / np.linalg.norm(ora["o_coarse"])
+    assert rel <= COARSE_REL_L2, rel
+
+
+@pytest.mark.parametrize("grid,heads", [((8, 16, 16), 3), ((12, 32, 64), 2), ((24, 32, 128), 1)],
+                         ids=["C32", "C384", "C1536"])
+def test_coarse_topk_tie_heavy_pooled_vectors(grid, heads):
+    """Small-integer pooled vectors make many scores exactly equal (integer dot products are exact in
+    float32): the fused selection must break every tie like vsa_topk, for k on the compacted-candidate
+    path (k <= 128) and beyond it, up to C = 1536 (the largest the fused kernel takes)."""
+    s = vsa.Shape(1, heads, 64, grid)
+    _, C = vsa.shape_info(s)
+    rng = np.random.default_rng(C)
+    mk = lambda: torch.from_numpy(rng.integers(-2, 3, size=(1, heads, C, 64)).astype(np.float32)).cuda()
+    bars = (mk(), mk(), torch.from_numpy(rng.standard_normal((1, heads, C, 64)).astype(np.float32)).cuda())
+    ks = sorted({k for k in (1, 2, 31, 32, 33, 64, 65, 96, 128, 129, 200, C - 1, C) if 1 <= k <= C})
+    _check_coarse_topk(s, bars, 0.125, ks, f"ties C={C}")
+    # every query vector zero: all scores 0, so cubes 0..k-1 for every row
+    zero = torch.zeros_like(bars[0])
+    for k in (k for k in (1, 32, 65) if k <= C):
+        idx, _, _, _ = vsa.coarse_topk(zero, bars[1], None, s, k, 0.125, order=False)
+        assert torch.equal(idx, torch.arange(k, dtype=torch.int32, device="cuda").expand_as(idx)), k
+
+
 def _decode_steps(raw: np.ndarray, items: int, stride: int):
     e = raw.view(np.uint32).reshape(items, stride, 2)
     a, b = (e[..., 0] & 0xFFFF).astype(np.int64), (e[..., 0] >> 16).astype(np.int64)
