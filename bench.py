@@ -251,10 +251,8 @@ def _events(torch, n):
     return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
 
 
-def stage_times(vsa, torch, d, w, iters: int, warmup: int, dense_too: bool = False, staged: bool = False,
-                fused_selection: bool = False):
-    """Median ms of each launch group of one call, run stage by stage through the entry points
-    (fused_selection: vsa_coarse_topk in place of vsa_coarse + vsa_topk_order)."""
+def stage_times(vsa, torch, d, w, iters: int, warmup: int, dense_too: bool = False, staged: bool = False):
+    """Median ms of each launch group of one call, run stage by stage through the entry points."""
     s = vsa.Shape(w.batch, w.heads, w.head_dim, w.grid)
     _, C = vsa.shape_info(s)
     scale = 1.0 / math.sqrt(w.head_dim)
@@ -304,14 +302,10 @@ def stage_times(vsa, torch, d, w, iters: int, warmup: int, dense_too: bool = Fal
             else:
                 bars = vsa.pool_qkv(d["q"], d["k"], d["v"], s)
                 mark("pool")
-                if fused_selection:
-                    idx, order, oc, _ = vsa.coarse_topk(*bars, s, w.topk, scale)
-                    mark("coarse_topk")
-                else:
-                    scores, oc = vsa.coarse(*bars, s, scale)
-                    mark("coarse")
-                    idx, order = vsa.topk_order(scores, s, w.topk)
-                    mark("topk_order")
+                scores, oc = vsa.coarse(*bars, s, scale)
+                mark("coarse")
+                idx, order = vsa.topk_order(scores, s, w.topk)
+                mark("topk_order")
                 steps = vsa.schedule(idx, s, order)
                 mark("schedule")
                 vsa.fine_fused(d["q"], d["k"], d["v"], s, idx, scale, order, oc, d["g_coarse"], d["g_fine"],
@@ -569,8 +563,7 @@ def run_stages(args):
     w = synth.WORKLOADS[args.workload]
     x = synth.make_inputs(w)
     d = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).cuda() for k, v in x.items()}
-    ms = stage_times(vsa, torch, d, w, args.iters, 2, dense_too=args.dense_too, staged=args.staged,
-                     fused_selection=args.fused_selection)
+    ms = stage_times(vsa, torch, d, w, args.iters, 2, dense_too=args.dense_too, staged=args.staged)
     vsa.device_status()
     print(json.dumps({"workload": w.name, "iters": args.iters, "staged": args.staged, "ms": ms}), flush=True)
 
@@ -586,8 +579,6 @@ def main(argv=None):
     ap.add_argument("--iters", type=int, default=3, help="with --stages")
     ap.add_argument("--dense-too", action="store_true", help="with --stages: add a dense fine-stage launch")
     ap.add_argument("--staged", action="store_true", help="with --stages: the unfused per-step entry points")
-    ap.add_argument("--fused-selection", action="store_true",
-                    help="with --stages: the selection as vsa_coarse_topk (one fused launch)")
     args = ap.parse_args(argv)
     if args.stages:
         run_stages(args)

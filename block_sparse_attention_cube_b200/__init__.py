@@ -113,9 +113,12 @@ def coarse(qbar: torch.Tensor, kbar: torch.Tensor, vbar: torch.Tensor, shape: Sh
     scale = default_scale(shape) if scale is None else scale
     scores = torch.empty((shape.batch, shape.heads, c, c), dtype=torch.float32, device=qbar.device)
     oc = torch.empty_like(qbar)
+    n = int(_L.vsa_coarse_workspace_bytes(ctypes.byref(shape.c())))
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=qbar.device)
     _check(_L.vsa_coarse(ctypes.byref(shape.c()), _ptr(qbar, torch.float32, "qbar"), _ptr(kbar, torch.float32, "kbar"),
                          _ptr(vbar, torch.float32, "vbar"), scale, _ptr(scores, torch.float32, "scores"),
-                         _ptr(oc, torch.float32, "o_coarse"), _stream()))
+                         _ptr(oc, torch.float32, "o_coarse"), _ptr(ws, torch.uint8, "workspace"), ws.numel(),
+                         _stream()))
     return scores, oc
 
 
@@ -173,27 +176,6 @@ def topk_order(scores: torch.Tensor, shape: Shape, k: int) -> Tuple[torch.Tensor
                              _ptr(idx, torch.int32, "idx"), _ptr(order, torch.int32, "order"),
                              _ptr(sig, torch.int64, "sig_scratch"), _stream()))
     return idx, order
-
-
-def coarse_topk(qbar: torch.Tensor, kbar: torch.Tensor, vbar: Optional[torch.Tensor], shape: Shape, k: int,
-                scale: Optional[float] = None, order: bool = True, want_scores: bool = False):
-    """Coarse scores, top-k selection, work order and (with vbar) coarse output in one fused launch
-    (plus the order sort).  Returns (idx [B,H,C,k], order [B,H,C] or None, o_coarse [B,H,C,D] or None,
-    scores [B,H,C,C] or None: the ranked scores, copied out only when want_scores)."""
-    _, c = shape_info(shape)
-    scale = default_scale(shape) if scale is None else scale
-    dev = qbar.device
-    idx = torch.empty((shape.batch, shape.heads, c, k), dtype=torch.int32, device=dev)
-    od = torch.empty((shape.batch, shape.heads, c), dtype=torch.int32, device=dev) if order else None
-    sig = torch.empty((shape.batch, shape.heads, c), dtype=torch.int64, device=dev) if order else None
-    oc = torch.empty_like(qbar) if vbar is not None else None
-    scores = torch.empty((shape.batch, shape.heads, c, c), dtype=torch.float32, device=dev) if want_scores else None
-    _check(_L.vsa_coarse_topk(ctypes.byref(shape.c()), _ptr(qbar, torch.float32, "qbar"),
-                              _ptr(kbar, torch.float32, "kbar"), _ptr(vbar, torch.float32, "vbar"), scale, k,
-                              _ptr(idx, torch.int32, "idx"), _ptr(od, torch.int32, "order"),
-                              _ptr(sig, torch.int64, "sig_scratch"), _ptr(oc, torch.float32, "o_coarse"),
-                              _ptr(scores, torch.float32, "scores"), _stream()))
-    return idx, od, oc, scores
 
 
 def pool_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -291,7 +273,7 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, shape: Shape, top
             scale: Optional[float] = None, g_coarse: Optional[torch.Tensor] = None,
             g_fine: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
             out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """The whole VSA call: pool_qkv -> coarse_topk -> schedule -> fine_fused (topk_k == C: dense fine stage)."""
+    """The whole VSA call: pool_qkv -> coarse -> topk_order -> schedule -> fine_fused (topk_k == C: dense fine stage)."""
     scale = default_scale(shape) if scale is None else scale
     if workspace is None:
         workspace = alloc_workspace(shape, topk_k, device=q.device)

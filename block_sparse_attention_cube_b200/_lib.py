@@ -39,14 +39,14 @@ SIGNATURES = {
     "vsa_tile": (ctypes.c_int, [_SP, _P, _P, _P]),
     "vsa_untile": (ctypes.c_int, [_SP, _P, _P, _P]),
     "vsa_pool": (ctypes.c_int, [_SP, _P, _P, _P]),
-    "vsa_coarse": (ctypes.c_int, [_SP, _P, _P, _P, _F32, _P, _P, _P]),
+    "vsa_coarse_workspace_bytes": (_SZ, [_SP]),
+    "vsa_coarse": (ctypes.c_int, [_SP, _P, _P, _P, _F32, _P, _P, _P, _SZ, _P]),
     "vsa_topk": (ctypes.c_int, [_SP, _P, _I32, _P, _P]),
     "vsa_group": (ctypes.c_int, [_SP, _P, _P, _P]),
     "vsa_fine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _I32, _P, _F32, _P, _P, _P]),
     "vsa_combine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P]),
     "vsa_pool_qkv": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P]),
     "vsa_topk_order": (ctypes.c_int, [_SP, _P, _I32, _P, _P, _P, _P]),
-    "vsa_coarse_topk": (ctypes.c_int, [_SP, _P, _P, _P, _F32, _I32, _P, _P, _P, _P, _P, _P]),
     "vsa_fine_fused": (ctypes.c_int, [_SP, _P, _P, _P, _P, _I32, _P, _P, _F32, _P, _P, _P, _P, _P, _P]),
     "vsa_schedule_bytes": (_SZ, [_SP, _I32]),
     "vsa_schedule": (ctypes.c_int, [_SP, _P, _I32, _P, _P, _P]),

@@ -162,19 +162,15 @@ size_t order_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C 
 constexpr size_t kAlign = 256;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Whether the forward call runs its selection as the one fused launch (coarse scores, top-k,
-// work-order keys and the coarse output; vsa_coarse_topk).  Measured on B200 it is no faster than the
-// two-launch path at 480p (0.41 against 0.40 ms) and slower at 720p (5.4 against 4.5 ms: a block's
-// 32 score rows take 184 KB of shared memory there, one block of 8 warps per SM), so it is off.
-bool fused_selection(const Dims&) { return false; }
-
-// Workspace of vsa_forward: qbar | kbar | vbar | o_coarse | scores | idx | order | sig | steps | overflow.
-// Q, K and V are read in the caller's [B, N, H, D] layout (the fine stage
-// gathers cubes with TMA), so no tiled copies are kept.  With every cube
-// selected the fine stage is dense attention and needs none of it; the
-// coarse buffers are then used only when a coarse gate is given.
+// Workspace of vsa_forward: q/k/v parts | row stats | o_coarse | scores | idx | order | sig | steps |
+// overflow.  Q, K and V are read in the caller's [B, N, H, D] layout (the fine stage gathers cubes with
+// TMA), so no tiled copies are kept; the pooled vectors are kept only as their three bf16 parts (the
+// coarse stage's tensor-core operands).  With every cube selected the fine stage is dense attention
+// and needs none of it; the coarse buffers are then used only when a coarse gate is given.
 struct Carve {
-    float *qbar, *kbar, *vbar, *oc, *scores;
+    uint16_t *qp, *kp, *vp;   // the pooled q, k, v as three bf16 parts each
+    float* stats;             // per score row: maximum and 1 / sum of exp
+    float *oc, *scores;
     int32_t* idx;
     int32_t* order;
     uint64_t* sig;   // work-order signatures, when top-k computes them (C <= kTopkRegMaxC)
@@ -182,6 +178,9 @@ struct Carve {
     int* overflow;   // the fine stage's overflow word
     size_t bytes;
 };
+
+size_t parts_bytes(const Dims& d) { return split_parts_elems(d) * 2u; }
+size_t stats_bytes(const Dims& d) { return static_cast<size_t>(d.B) * d.H * d.C * 8u; }
 
 Carve carve(const Dims& d, int k, bool coarse_gate, void* ws) {
     Carve c{};
@@ -194,13 +193,12 @@ Carve carve(const Dims& d, int k, bool coarse_gate, void* ws) {
     };
     const bool sparse = k < d.C;
     if (sparse || coarse_gate) {
-        c.qbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
-        c.kbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
-        c.vbar = reinterpret_cast<float*>(take(pooled_bytes(d)));
+        c.qp = reinterpret_cast<uint16_t*>(take(parts_bytes(d)));
+        c.kp = reinterpret_cast<uint16_t*>(take(parts_bytes(d)));
+        c.vp = reinterpret_cast<uint16_t*>(take(parts_bytes(d)));
+        c.stats = reinterpret_cast<float*>(take(stats_bytes(d)));
         c.oc = reinterpret_cast<float*>(take(pooled_bytes(d)));
-        // the fused selection keeps the scores in shared memory; the scores buffer serves the
-        // two-launch path (and a coarse gate at top-k == C, whose output still needs the scores)
-        if (!(sparse && fused_selection(d))) c.scores = reinterpret_cast<float*>(take(score_bytes(d)));
+        c.scores = reinterpret_cast<float*>(take(score_bytes(d)));
     }
     if (sparse) {
         c.idx = reinterpret_cast<int32_t*>(take(idx_bytes(d, k)));
@@ -273,26 +271,22 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
                        const uint16_t* gf, int topk, float scale, void* ws, uint16_t* out, cudaStream_t s) {
     const bool sparse = topk < d.C;
     const Carve c = carve(d, topk, gc != nullptr, ws);
-    const bool fused = sparse && fused_selection(d);
+    const char* why = nullptr;
+    bool have_stats = false;
     if (sparse || gc != nullptr) {
+        // pooled q, k, v straight into their bf16 parts, then the scores on the tensor cores
         const uint16_t* pin[3] = {q, k, v};
-        float* pout[3] = {c.qbar, c.kbar, c.vbar};
-        VSA_CUDA(launch_pool_tokens(d, pin, pout, 3, s), "pool launch");
-        if (!fused) VSA_CUDA(launch_coarse_scores(d, c.qbar, c.kbar, scale, c.scores, s), "coarse launch");
+        uint16_t* parts[3] = {c.qp, c.kp, c.vp};
+        VSA_CUDA(launch_pool_tokens(d, pin, nullptr, 3, s, parts), "pool launch");
+        const cudaError_t e = launch_coarse_scores_mma(d, c.qp, c.kp, scale, c.scores, s, &why);
+        if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "coarse launch");
     }
-    // the coarse output (softmax(scores) x V-bar) is used only by the merge, and only with a coarse gate
-    if (gc != nullptr && !fused) VSA_CUDA(launch_coarse_pv(d, c.scores, c.vbar, c.oc, s), "coarse launch");
     const int32_t* order = nullptr;
-    if (fused) {
-        // scores, selection, work-order keys and the coarse output in one launch, then the key sort
-        VSA_CUDA(launch_coarse_select(d, c.qbar, c.kbar, c.vbar, scale, topk, c.idx, c.sig, gc ? c.oc : nullptr,
-                                      nullptr, s), "coarse select launch");
-        VSA_CUDA(launch_group_sort(d, c.sig, c.order, s), "group launch");
-        order = c.order;
-    } else if (sparse) {
+    if (sparse) {
         if (d.C <= kTopkRegMaxC && d.C <= kGroupMaxC) {
-            // one pass over the scores gives the selection and the work-order keys
-            VSA_CUDA(launch_topk_sig(d, c.scores, topk, c.idx, c.sig, s), "topk launch");
+            // one pass over the scores gives the selection, the work-order keys and the softmax statistics
+            VSA_CUDA(launch_topk_sig(d, c.scores, topk, c.idx, c.sig, s, c.stats), "topk launch");
+            have_stats = true;
             VSA_CUDA(launch_group_sort(d, c.sig, c.order, s), "group launch");
             order = c.order;
         } else {
@@ -302,6 +296,12 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
                 order = c.order;
             }
         }
+    }
+    // the coarse output (softmax(scores) x V-bar) is used only by the merge, and only with a coarse gate
+    if (gc != nullptr) {
+        if (!have_stats) VSA_CUDA(launch_row_stats(d, c.scores, c.stats, s), "row stats launch");
+        const cudaError_t e = launch_coarse_pv_mma(d, c.scores, c.stats, c.vp, c.oc, s, &why);
+        if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "coarse launch");
     }
     const void* steps = nullptr;
     if (sparse && c.steps != nullptr) {
@@ -450,8 +450,14 @@ vsa_status vsa_pool(const vsa_shape* shape, const vsa_bf16* xt, float* xbar, vsa
     return VSA_OK;
 }
 
+size_t vsa_coarse_workspace_bytes(const vsa_shape* shape) {
+    Dims d{};
+    if (make_dims(shape, &d) != VSA_OK) return 0;
+    return 3 * up(parts_bytes(d)) + up(stats_bytes(d));
+}
+
 vsa_status vsa_coarse(const vsa_shape* shape, const float* qbar, const float* kbar, const float* vbar, float scale,
-                      float* scores, float* o_coarse, vsa_stream_t stream) {
+                      float* scores, float* o_coarse, void* workspace, size_t workspace_bytes, vsa_stream_t stream) {
     Dims d{};
     VSA_TRY(make_dims(shape, &d));
     VSA_TRY(need_ptr(qbar, "qbar"));
@@ -460,11 +466,30 @@ vsa_status vsa_coarse(const vsa_shape* shape, const float* qbar, const float* kb
     VSA_TRY(need_ptr(scores, "scores"));
     VSA_TRY(need_ptr(o_coarse, "o_coarse"));
     VSA_TRY(check_scale(scale));
+    const size_t need = 3 * up(parts_bytes(d)) + up(stats_bytes(d));
+    if (!workspace) return fail(VSA_ERR_WORKSPACE, "workspace is NULL (%zu bytes needed)", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign != 0)
+        return fail(VSA_ERR_MISALIGNED, "workspace is not 256-byte aligned");
+    if (workspace_bytes < need) return fail(VSA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, need);
     const size_t pb = pooled_bytes(d);
     VSA_TRY(check_disjoint({{qbar, pb, "qbar"}, {kbar, pb, "kbar"}, {vbar, pb, "vbar"}},
-                           {{scores, score_bytes(d), "scores"}, {o_coarse, pb, "o_coarse"}}));
+                           {{scores, score_bytes(d), "scores"}, {o_coarse, pb, "o_coarse"}, {workspace, need, "workspace"}}));
     VSA_TRY(check_device());
-    VSA_CUDA(launch_coarse(d, qbar, kbar, vbar, scale, scores, o_coarse, as_stream(stream)), "coarse launch");
+    cudaStream_t s = as_stream(stream);
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    uint16_t* qp = reinterpret_cast<uint16_t*>(w);
+    uint16_t* kp = reinterpret_cast<uint16_t*>(w + up(parts_bytes(d)));
+    uint16_t* vp = reinterpret_cast<uint16_t*>(w + 2 * up(parts_bytes(d)));
+    float* stats = reinterpret_cast<float*>(w + 3 * up(parts_bytes(d)));
+    VSA_CUDA(launch_split_parts(d, qbar, qp, s), "split launch");
+    VSA_CUDA(launch_split_parts(d, kbar, kp, s), "split launch");
+    VSA_CUDA(launch_split_parts(d, vbar, vp, s), "split launch");
+    const char* why = nullptr;
+    cudaError_t e = launch_coarse_scores_mma(d, qp, kp, scale, scores, s, &why);
+    if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "coarse launch");
+    VSA_CUDA(launch_row_stats(d, scores, stats, s), "row stats launch");
+    e = launch_coarse_pv_mma(d, scores, stats, vp, o_coarse, s, &why);
+    if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "coarse launch");
     return VSA_OK;
 }
 
@@ -564,40 +589,6 @@ vsa_status vsa_topk_order(const vsa_shape* shape, const float* scores, int32_t k
     VSA_TRY(check_device());
     VSA_CUDA(launch_topk_sig(d, scores, k, idx, sig_scratch, as_stream(stream)), "topk launch");
     VSA_CUDA(launch_group_sort(d, sig_scratch, order, as_stream(stream)), "group launch");
-    return VSA_OK;
-}
-
-vsa_status vsa_coarse_topk(const vsa_shape* shape, const float* qbar, const float* kbar, const float* vbar,
-                           float scale, int32_t k, int32_t* idx, int32_t* order, uint64_t* sig_scratch,
-                           float* o_coarse, float* scores, vsa_stream_t stream) {
-    Dims d{};
-    VSA_TRY(make_dims(shape, &d));
-    VSA_TRY(check_k(d, k));
-    VSA_TRY(check_scale(scale));
-    VSA_TRY(need_ptr(qbar, "qbar"));
-    VSA_TRY(need_ptr(kbar, "kbar"));
-    VSA_TRY(need_ptr(idx, "idx"));
-    VSA_TRY(opt_ptr(vbar, "vbar"));
-    VSA_TRY(opt_ptr(o_coarse, "o_coarse"));
-    VSA_TRY(opt_ptr(order, "order"));
-    VSA_TRY(opt_ptr(sig_scratch, "sig_scratch"));
-    VSA_TRY(opt_ptr(scores, "scores"));
-    if ((vbar == nullptr) != (o_coarse == nullptr))
-        return fail(VSA_ERR_INVALID_ARGUMENT, "vbar and o_coarse must both be given or both be NULL");
-    if ((order == nullptr) != (sig_scratch == nullptr))
-        return fail(VSA_ERR_INVALID_ARGUMENT, "order and sig_scratch must both be given or both be NULL");
-    if (!coarse_select_supported(d))
-        return fail(VSA_ERR_UNSUPPORTED, "vsa_coarse_topk keeps a block's score rows in shared memory: C <= 1536 "
-                    "(got %d)", d.C);
-    const size_t pb = pooled_bytes(d);
-    VSA_TRY(check_disjoint({{qbar, pb, "qbar"}, {kbar, pb, "kbar"}, {vbar, vbar ? pb : 0, "vbar"}},
-                           {{idx, idx_bytes(d, k), "idx"}, {order, order ? order_bytes(d) : 0, "order"},
-                            {sig_scratch, sig_scratch ? 2 * order_bytes(d) : 0, "sig_scratch"},
-                            {o_coarse, o_coarse ? pb : 0, "o_coarse"}, {scores, scores ? score_bytes(d) : 0, "scores"}}));
-    VSA_TRY(check_device());
-    VSA_CUDA(launch_coarse_select(d, qbar, kbar, vbar, scale, k, idx, sig_scratch, o_coarse, scores,
-                                  as_stream(stream)), "coarse select launch");
-    if (order) VSA_CUDA(launch_group_sort(d, sig_scratch, order, as_stream(stream)), "group launch");
     return VSA_OK;
 }
 

@@ -1,11 +1,7 @@
-// Coarse stage and cube selection (Wan2.2 teardown, zharfai.com, section
-// "Video sparse attention selects cubes", part 1: cheap block-level attention
-// over the mean-pooled cubes that ranks the candidate key cubes, of which
-// each query cube keeps the top-k).
-//
-// The coarse scores decide the selection, so they are computed in float32 on
-// the CUDA cores (a deterministic sequential sum over the channels), not on
-// the bf16/tf32 tensor paths whose rounding would reorder near-equal cubes.
+// Cube selection (Wan2.2 teardown, zharfai.com, section "Video sparse
+// attention selects cubes", part 1: the coarse scores rank the candidate key
+// cubes, of which each query cube keeps the top-k) and the fine stage's work
+// order.  The scores themselves come from vsa_coarse_mma.cu.
 #include <cfloat>
 
 #include "vsa_internal.h"
@@ -13,237 +9,7 @@
 namespace vsa {
 namespace {
 
-constexpr int kBK = 16;     // reduction slice
 constexpr int kThreads = 256;
-constexpr int kSTI = 128;   // score tile rows (query cubes)
-constexpr int kSTJ = 64;    // score tile columns (key cubes)
-constexpr int kSRI = 8;     // rows per thread
-constexpr int kSRJ = 4;     // columns per thread
-static_assert((kSTI / kSRI) * (kSTJ / kSRJ) == kThreads, "one output block per thread");
-
-// scores[bh][i][j] = scale * sum_d qbar[bh][i][d] * kbar[bh][j][d]
-// A 128x64 output tile per block; thread (ty, tx) owns rows 8ty..8ty+7 and
-// columns 4tx..4tx+3 (32 accumulators, 12 operands read from shared memory
-// per 32 fma); the next 16-channel slice is loaded into registers while the
-// current one is multiplied.  Each output is one sequential float32 fma chain
-// over the channels, so the tiling does not change a single bit of the result.
-__global__ void __launch_bounds__(kThreads) coarse_scores_kernel(int C, int D, const float* __restrict__ qbar,
-                                                                 const float* __restrict__ kbar, float scale,
-                                                                 float* __restrict__ scores) {
-    __shared__ __align__(16) float As[kBK][kSTI + 4];
-    __shared__ __align__(16) float Bs[kBK][kSTJ + 4];
-    const int bh = blockIdx.z;
-    const int i0 = blockIdx.y * kSTI, j0 = blockIdx.x * kSTJ;
-    constexpr int NTX = kSTJ / kSRJ;
-    const int tx = threadIdx.x % NTX, ty = threadIdx.x / NTX;
-    const float* Q = qbar + static_cast<int64_t>(bh) * C * D;
-    const float* K = kbar + static_cast<int64_t>(bh) * C * D;
-    float acc[kSRI][kSRJ] = {};
-    // the tile's rows x 16 channels of each operand: this thread's share, loaded one slice ahead
-    constexpr int kLA = kSTI * kBK / kThreads, kLB = kSTJ * kBK / kThreads;
-    float ra[kLA], rb[kLB];
-    auto load_slice = [&](int d0) {
-#pragma unroll
-        for (int e = 0; e < kLA; ++e) {
-            const int idx = threadIdx.x + e * kThreads;
-            const int gi = i0 + idx / kBK;
-            ra[e] = gi < C ? __ldg(Q + static_cast<int64_t>(gi) * D + d0 + idx % kBK) : 0.f;
-        }
-#pragma unroll
-        for (int e = 0; e < kLB; ++e) {
-            const int idx = threadIdx.x + e * kThreads;
-            const int gj = j0 + idx / kBK;
-            rb[e] = gj < C ? __ldg(K + static_cast<int64_t>(gj) * D + d0 + idx % kBK) : 0.f;
-        }
-    };
-    load_slice(0);
-    for (int d0 = 0; d0 < D; d0 += kBK) {
-        // stored channel-major; the next slice's loads are in flight while this one is multiplied
-#pragma unroll
-        for (int e = 0; e < kLA; ++e) {
-            const int idx = threadIdx.x + e * kThreads;
-            As[idx % kBK][idx / kBK] = ra[e];
-        }
-#pragma unroll
-        for (int e = 0; e < kLB; ++e) {
-            const int idx = threadIdx.x + e * kThreads;
-            Bs[idx % kBK][idx / kBK] = rb[e];
-        }
-        __syncthreads();
-        if (d0 + kBK < D) load_slice(d0 + kBK);
-#pragma unroll
-        for (int kk = 0; kk < kBK; ++kk) {
-            float av[kSRI], bv[kSRJ];
-#pragma unroll
-            for (int q4 = 0; q4 < kSRI / 4; ++q4) {
-                const float4 a = *reinterpret_cast<const float4*>(&As[kk][kSRI * ty + 4 * q4]);
-                av[4 * q4] = a.x;
-                av[4 * q4 + 1] = a.y;
-                av[4 * q4 + 2] = a.z;
-                av[4 * q4 + 3] = a.w;
-            }
-            const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][kSRJ * tx]);
-            bv[0] = b.x;
-            bv[1] = b.y;
-            bv[2] = b.z;
-            bv[3] = b.w;
-#pragma unroll
-            for (int r = 0; r < kSRI; ++r)
-#pragma unroll
-                for (int c = 0; c < kSRJ; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-        }
-        __syncthreads();
-    }
-    float* S = scores + static_cast<int64_t>(bh) * C * C;
-#pragma unroll
-    for (int r = 0; r < kSRI; ++r) {
-        const int gi = i0 + kSRI * ty + r;
-        if (gi >= C) continue;
-#pragma unroll
-        for (int c = 0; c < kSRJ; ++c) {
-            const int gj = j0 + kSRJ * tx + c;
-            if (gj < C) S[static_cast<int64_t>(gi) * C + gj] = scale * acc[r][c];
-        }
-    }
-}
-
-// o_coarse[bh][i] = sum_j softmax(scores[bh][i][:])_j * vbar[bh][j]
-// One pass over each score row (online maximum): a block owns kPvRows query
-// rows and walks the keys in slices of 16.  Half a warp holds a row's 16
-// scores of the slice: it takes their maximum by shuffles, raises the row's
-// running maximum m, and writes p = exp(s - m) to shared memory together with
-// the factor exp(m_old - m) by which the row's accumulators are rescaled; each
-// lane keeps a partial denominator, summed over the half warp at the end.
-// Thread (ty, tx) owns RPT rows and 4 output channels.  The next slice's
-// scores and V rows are loaded into registers while this slice accumulates.
-constexpr int kPvRows = 32;
-
-// n consecutive floats of shared memory (16-byte aligned for n % 4 == 0, else 8-byte) into registers
-template <int n>
-__device__ __forceinline__ void read_rows(const float* src, float* dst) {
-    if constexpr (n % 4 == 0) {
-#pragma unroll
-        for (int i = 0; i < n / 4; ++i) {
-            const float4 a = reinterpret_cast<const float4*>(src)[i];
-            dst[4 * i] = a.x;
-            dst[4 * i + 1] = a.y;
-            dst[4 * i + 2] = a.z;
-            dst[4 * i + 3] = a.w;
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < n / 2; ++i) {
-            const float2 a = reinterpret_cast<const float2*>(src)[i];
-            dst[2 * i] = a.x;
-            dst[2 * i + 1] = a.y;
-        }
-    }
-}
-
-template <int D>
-__global__ void __launch_bounds__(kThreads) coarse_pv_kernel(int C, const float* __restrict__ scores,
-                                                             const float* __restrict__ vbar,
-                                                             float* __restrict__ o_coarse) {
-    constexpr int TX = D / 4;                     // threads across the channels
-    constexpr int RPT = kPvRows * TX / kThreads;  // rows per thread
-    constexpr int SPT = kPvRows * kBK / kThreads; // scores per thread per slice
-    constexpr int VPT = kBK * D / 4 / kThreads;   // V float4 per thread per slice
-    static_assert(RPT % 2 == 0 && SPT >= 1 && VPT >= 1, "tile shape");
-    __shared__ __align__(16) float Ps[kBK][kPvRows + 4];
-    __shared__ __align__(16) float Vs[kBK][D];
-    __shared__ __align__(16) float alpha_s[kPvRows];
-    __shared__ float row_inv[kPvRows];
-    const int bh = blockIdx.y;
-    const int i0 = blockIdx.x * kPvRows;
-    const float* S = scores + static_cast<int64_t>(bh) * C * C;
-    const float* V = vbar + static_cast<int64_t>(bh) * C * D;
-    const int cc = threadIdx.x % kBK, rbase = threadIdx.x / kBK;   // score role: key cc of rows rbase + 16e
-    const int tx = threadIdx.x % TX, ty = threadIdx.x / TX;        // accumulate role
-    float m[SPT], l[SPT], s_next[SPT];
-    float4 v_next[VPT];
-    auto load_slice = [&](int j0) {
-        const int gj = j0 + cc;
-#pragma unroll
-        for (int e = 0; e < SPT; ++e) {
-            const int gi = i0 + rbase + e * (kThreads / kBK);
-            s_next[e] = gi >= C ? 0.f : gj < C ? __ldg(S + static_cast<int64_t>(gi) * C + gj) : -FLT_MAX;
-        }
-#pragma unroll
-        for (int e = 0; e < VPT; ++e) {
-            const int idx = threadIdx.x + e * kThreads;
-            const int kk = idx / (D / 4), c4 = idx % (D / 4);
-            v_next[e] = j0 + kk < C ? __ldg(reinterpret_cast<const float4*>(V + static_cast<int64_t>(j0 + kk) * D) + c4)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    };
-#pragma unroll
-    for (int e = 0; e < SPT; ++e) {
-        m[e] = -FLT_MAX;
-        l[e] = 0.f;
-    }
-    float acc[RPT][4] = {};
-    load_slice(0);
-    for (int j0 = 0; j0 < C; j0 += kBK) {
-#pragma unroll
-        for (int e = 0; e < SPT; ++e) {
-            const int r = rbase + e * (kThreads / kBK);
-            float mx = s_next[e];
-#pragma unroll
-            for (int off = kBK / 2; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            const float mn = fmaxf(m[e], mx);
-            const float a = expf(m[e] - mn);
-            const float pv = expf(s_next[e] - mn);
-            m[e] = mn;
-            l[e] = l[e] * a + pv;
-            Ps[cc][r] = pv;
-            if (cc == 0) alpha_s[r] = a;
-        }
-#pragma unroll
-        for (int e = 0; e < VPT; ++e) {
-            const int idx = threadIdx.x + e * kThreads;
-            *reinterpret_cast<float4*>(&Vs[idx / (D / 4)][4 * (idx % (D / 4))]) = v_next[e];
-        }
-        __syncthreads();
-        if (j0 + kBK < C) load_slice(j0 + kBK);
-        {
-            float av[RPT];
-            read_rows<RPT>(&alpha_s[RPT * ty], av);
-#pragma unroll
-            for (int r = 0; r < RPT; ++r)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[r][c] *= av[r];
-        }
-#pragma unroll
-        for (int kk = 0; kk < kBK; ++kk) {
-            float pr[RPT];
-            read_rows<RPT>(&Ps[kk][RPT * ty], pr);
-            const float4 b = *reinterpret_cast<const float4*>(&Vs[kk][4 * tx]);
-            const float bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int r = 0; r < RPT; ++r)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(pr[r], bv[c], acc[r][c]);
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int e = 0; e < SPT; ++e) {
-        float t = l[e];
-#pragma unroll
-        for (int off = kBK / 2; off; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
-        if (cc == 0) row_inv[rbase + e * (kThreads / kBK)] = t > 0.f ? 1.0f / t : 0.f;
-    }
-    __syncthreads();
-    float* O = o_coarse + static_cast<int64_t>(bh) * C * D;
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-        const int li = RPT * ty + r, gi = i0 + li;
-        if (gi >= C) continue;
-        const float inv = row_inv[li];
-        *reinterpret_cast<float4*>(O + static_cast<int64_t>(gi) * D + 4 * tx) =
-            make_float4(acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv, acc[r][3] * inv);
-    }
-}
 
 // Order-preserving map float -> uint32 (larger float, larger key); -0 is
 // folded onto +0 so that equal scores compare equal.
@@ -333,79 +99,197 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(int64_t rows, int C, int
     }
 }
 
-// Top-k with the row held in registers (KPL keys per lane, key j in lane
-// j % 32, slot j / 32), for C <= 32 * KPL.  The k-th largest key T is built
-// bit by bit from the top with warp sums (redux) of per-lane counts; the row
-// is then scanned in index order exactly as topk_kernel does, so both give
-// the same selection.  When `sig` is non-null the row's work-order key is
-// written as well: its four smallest selected cubes (12 bits each, C <= 4096)
-// above the cube's own index, so that sorting the keys puts query cubes whose
-// selections start alike next to each other (the fine stage's tiles are pairs
-// of consecutive cubes, and a tile's steps are the union of its two
-// selections).
+// T = the k-th largest key of a row, built bit by bit from the top, searching only the bits below the
+// highest one in which hi and lo differ (lo <= T <= hi); keys are counted over n[] (N per lane).
+template <int N>
+__device__ __forceinline__ uint32_t kth_key(const uint32_t (&n)[N], uint32_t hi, uint32_t lo, int k) {
+    const uint32_t diff = hi ^ lo;
+    const int top = diff ? 31 - __clz(diff) : -1;
+    uint32_t T = top < 0 ? hi : (top >= 31 ? 0u : (hi & ~((2u << top) - 1u)));
+#pragma unroll 1
+    for (int bit = top; bit >= 0; --bit) {
+        const uint32_t cand = T | (1u << bit);
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int i = 0; i < N; ++i) cnt += n[i] >= cand ? 1u : 0u;
+        if (static_cast<int>(__reduce_add_sync(0xffffffffu, cnt)) >= k) T = cand;
+    }
+    return T;
+}
+
+__device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+constexpr int kTopM = 4;      // k <= 32 * kTopM: the k-th largest is searched in a compacted candidate list
+constexpr int kTopCand = 8;   // candidates per lane in that list (256 per row)
+
+// Hint: start moving `bytes` (a multiple of 16, 16-byte aligned) at `src` into L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+
+// Writes a row's selection (every key above T, then the lowest-index keys equal to T, ascending
+// index) from keys held key j in lane j % 32, slot j / 32 of n[] (idx_of gives j), and returns the
+// row's work-order key bits (its four smallest selected cubes, 12 bits each from bit 52 down).
+template <int N, typename IndexOf>
+__device__ __forceinline__ uint64_t write_selection(const uint32_t (&n)[N], int count, uint32_t T, int need_eq,
+                                                    int32_t* dst, IndexOf idx_of) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    int out = 0, eq_seen = 0, nlex = 0;
+    uint64_t lex = 0ull;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        if (32 * i >= count) break;                      // warp-uniform
+        const bool valid = lane + 32 * i < count;
+        const bool is_gt = valid && n[i] > T;
+        const bool is_eq = valid && n[i] == T;
+        const uint32_t eq_mask = __ballot_sync(0xffffffffu, is_eq);
+        const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
+        const bool take = is_gt || (is_eq && eq_rank < need_eq);
+        const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
+        const int j = idx_of(i);
+        if (take) dst[out + __popc(take_mask & lt_mask)] = j;
+        for (uint32_t mk = take_mask; nlex < 4 && mk != 0u; mk &= mk - 1u, ++nlex)   // warp-uniform
+            lex |= static_cast<uint64_t>(__shfl_sync(0xffffffffu, j, __ffs(mk) - 1)) << (52 - 12 * nlex);
+        out += __popc(take_mask);
+        eq_seen += __popc(eq_mask);
+    }
+    return lex;
+}
+
+// Top-k with the row held in registers (KPL keys per lane, key j in lane j % 32, slot j / 32), for
+// C <= 32 * KPL.  For k <= 128 each lane's m = ceil(k / 32) largest keys bound the k-th largest from
+// below (32 m >= k keys reach the smallest of them, lo); when at most 256 keys reach lo they are
+// compacted, with their cube indices and in index order, into a list whose count of keys >= t equals
+// the row's for every t > lo (and both reach k for t <= lo), so the k-th largest key T is built bit
+// by bit from the top over that short list, and the selection (every key above T, then the
+// lowest-index keys equal to T, ascending) is read off the same list; otherwise both run over the
+// whole row.  Either way the selection is topk_kernel's.  When `sig` is non-null the row's work-order
+// key is written as well: its four smallest selected cubes (12 bits each, C <= 4096) above the
+// cube's own index, so that sorting the keys puts query cubes whose selections start alike next to
+// each other (the fine stage's tiles are pairs of consecutive cubes, and a tile's steps are the
+// union of its two selections).  When `stats` is non-null, the row's maximum m and
+// 1 / sum(exp(s - m)) are written (the coarse output's softmax).  While a warp works on a row, the
+// next row it will take is prefetched into L2.
 template <int KPL>
 __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C, int k, const float* __restrict__ scores,
-                                                            int32_t* __restrict__ idx, uint64_t* __restrict__ sig) {
+                                                            int32_t* __restrict__ idx, uint64_t* __restrict__ sig,
+                                                            float2* __restrict__ stats) {
+    __shared__ uint32_t cand_key_all[kThreads / 32][32 * kTopCand];
+    __shared__ uint16_t cand_idx_all[kThreads / 32][32 * kTopCand];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lt_mask = (1u << lane) - 1u;
+    uint32_t* cand_key = cand_key_all[warp];
+    uint16_t* cand_idx = cand_idx_all[warp];
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
+    const int m = (k + 31) / 32;
+    const bool bulk_prefetch = (C & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
     for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + warp; row < rows; row += warps) {
         const float* s = scores + row * C;
+        if (bulk_prefetch && lane == 0 && row + warps < rows)
+            prefetch_l2_bulk(s + warps * C, static_cast<uint32_t>(C) * 4u);
         uint32_t key[KPL];
 #pragma unroll
         for (int i = 0; i < KPL; ++i) {
             const int j = lane + 32 * i;
             key[i] = j < C ? order_key(__ldcs(s + j)) : 0u;   // 0 ranks below every real score
         }
-        // T lies between a lower bound and the largest key, so it shares their
-        // leading bits: only the bits below the highest differing one are searched.
-        // Lower bound: the smallest lane maximum when k <= 32 (at least 32 keys
-        // reach it), else the smallest key.
-        uint32_t lane_max = 0u, lane_min = 0xFFFFFFFFu;
+        // the lane's largest key and its m-th largest (m <= kTopM), or its smallest real key
+        uint32_t lane_max = 0u, lane_m = 0u;
+        if (m == 1) {
 #pragma unroll
-        for (int i = 0; i < KPL; ++i) {
-            lane_max = max(lane_max, key[i]);
-            if (lane + 32 * i < C) lane_min = min(lane_min, key[i]);
+            for (int i = 0; i < KPL; ++i) lane_max = max(lane_max, key[i]);
+            lane_m = lane_max;
+        } else if (m == 2) {
+            uint32_t second = 0u;
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) {
+                second = max(second, min(lane_max, key[i]));
+                lane_max = max(lane_max, key[i]);
+            }
+            lane_m = second;
+        } else if (m <= kTopM) {
+            uint32_t top[kTopM] = {0u, 0u, 0u, 0u};   // descending
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) {
+                uint32_t v = key[i];
+#pragma unroll
+                for (int e = 0; e < kTopM; ++e) {
+                    const uint32_t hv = max(top[e], v);
+                    v = min(top[e], v);
+                    top[e] = hv;
+                }
+            }
+            lane_max = top[0];
+            lane_m = m == 3 ? top[2] : top[3];
+        } else {
+            lane_m = 0xFFFFFFFFu;
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) {
+                lane_max = max(lane_max, key[i]);
+                if (lane + 32 * i < C) lane_m = min(lane_m, key[i]);
+            }
         }
         const uint32_t hi = __reduce_max_sync(0xffffffffu, lane_max);
-        const uint32_t lo = k <= 32 ? __reduce_min_sync(0xffffffffu, lane_max) : __reduce_min_sync(0xffffffffu, lane_min);
-        const uint32_t diff = hi ^ lo;
-        const int top = diff ? 31 - __clz(diff) : -1;          // highest differing bit
-        uint32_t T = top < 0 ? hi : (top >= 31 ? 0u : (hi & ~((2u << top) - 1u)));
-#pragma unroll 1
-        for (int bit = top; bit >= 0; --bit) {
-            const uint32_t cand = T | (1u << bit);
-            uint32_t cnt = 0;
+        const uint32_t lo = __reduce_min_sync(0xffffffffu, lane_m);
+        int ncand = 0x7FFFFFFF;
+        if (m <= kTopM) {
+            uint32_t mine = 0;
 #pragma unroll
-            for (int i = 0; i < KPL; ++i) cnt += key[i] >= cand ? 1u : 0u;
-            if (static_cast<int>(__reduce_add_sync(0xffffffffu, cnt)) >= k) T = cand;
+            for (int i = 0; i < KPL; ++i) mine += (lane + 32 * i < C && key[i] >= lo) ? 1u : 0u;
+            ncand = static_cast<int>(__reduce_add_sync(0xffffffffu, mine));
         }
-        uint32_t gt = 0;
-#pragma unroll
-        for (int i = 0; i < KPL; ++i) gt += key[i] > T ? 1u : 0u;
-        const int need_eq = k - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
-        int out = 0, eq_seen = 0;
         int32_t* dst = idx + row * k;
-        uint64_t lex = 0ull;   // the row's four smallest selected cubes, 12 bits each from bit 52 down
-        int nlex = 0;
+        uint64_t lex;
+        if (ncand <= 32 * kTopCand) {
+            int base = 0;
 #pragma unroll
-        for (int i = 0; i < KPL; ++i) {
-            const int j = lane + 32 * i;
-            const bool valid = j < C;
-            const bool is_gt = valid && key[i] > T;
-            const bool is_eq = valid && key[i] == T;
-            const uint32_t eq_mask = __ballot_sync(0xffffffffu, is_eq);
-            const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
-            const bool take = is_gt || (is_eq && eq_rank < need_eq);
-            const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
-            if (take) dst[out + __popc(take_mask & lt_mask)] = j;
-            out += __popc(take_mask);
-            eq_seen += __popc(eq_mask);
-            // warp-uniform: the selection is written in ascending order, so its first entries are these
-            for (uint32_t mk = take_mask; nlex < 4 && mk != 0u; mk &= mk - 1u, ++nlex)
-                lex |= static_cast<uint64_t>(32 * i + __ffs(mk) - 1) << (52 - 12 * nlex);
+            for (int i = 0; i < KPL; ++i) {
+                const bool f = lane + 32 * i < C && key[i] >= lo;
+                const uint32_t bal = __ballot_sync(0xffffffffu, f);
+                if (f) {
+                    cand_key[base + __popc(bal & lt_mask)] = key[i];
+                    cand_idx[base + __popc(bal & lt_mask)] = static_cast<uint16_t>(lane + 32 * i);
+                }
+                base += __popc(bal);
+            }
+            __syncwarp();
+            uint32_t ck[kTopCand];
+#pragma unroll
+            for (int e = 0; e < kTopCand; ++e) ck[e] = lane + 32 * e < ncand ? cand_key[lane + 32 * e] : 0u;
+            const uint32_t T = ncand <= 32 * (kTopCand / 2)
+                                   ? kth_key<kTopCand / 2>(reinterpret_cast<const uint32_t(&)[kTopCand / 2]>(ck), hi, lo, k)
+                                   : kth_key<kTopCand>(ck, hi, lo, k);
+            uint32_t gt = 0;
+#pragma unroll
+            for (int e = 0; e < kTopCand; ++e) gt += ck[e] > T ? 1u : 0u;
+            const int need_eq = k - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+            lex = write_selection<kTopCand>(ck, ncand, T, need_eq, dst,
+                                            [&](int e) { return lane + 32 * e < ncand ? int(cand_idx[lane + 32 * e]) : 0; });
+            __syncwarp();
+        } else {
+            const uint32_t T = kth_key<KPL>(key, hi, lo, k);
+            uint32_t gt = 0;
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) gt += key[i] > T ? 1u : 0u;
+            const int need_eq = k - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+            lex = write_selection<KPL>(key, C, T, need_eq, dst, [&](int i) { return lane + 32 * i; });
         }
         if (sig != nullptr && lane == 0) sig[row] = lex | static_cast<uint64_t>(row % C);
+        if (stats != nullptr) {
+            // the keys decode back to the scores exactly (-0 as +0)
+            const float mx = key_value(hi);
+            float l = 0.f;
+#pragma unroll
+            for (int i = 0; i < KPL; ++i)
+                if (lane + 32 * i < C) l += __expf(key_value(key[i]) - mx);
+#pragma unroll
+            for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+            if (lane == 0) stats[row] = make_float2(mx, 1.0f / l);
+        }
     }
 }
 
@@ -486,29 +370,6 @@ cudaError_t launch_group(const Dims& d, const float* scores, int32_t* order, cud
     return cudaGetLastError();
 }
 
-cudaError_t launch_coarse_scores(const Dims& d, const float* qbar, const float* kbar, float scale, float* scores,
-                                 cudaStream_t s) {
-    const int bh = d.B * d.H;
-    const dim3 grid((d.C + kSTJ - 1) / kSTJ, (d.C + kSTI - 1) / kSTI, bh);
-    coarse_scores_kernel<<<grid, kThreads, 0, s>>>(d.C, d.D, qbar, kbar, scale, scores);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_coarse_pv(const Dims& d, const float* scores, const float* vbar, float* o_coarse, cudaStream_t s) {
-    const int bh = d.B * d.H;
-    const int pv_blocks = (d.C + kPvRows - 1) / kPvRows;
-    if (d.D == 128) coarse_pv_kernel<128><<<dim3(pv_blocks, bh), kThreads, 0, s>>>(d.C, scores, vbar, o_coarse);
-    else coarse_pv_kernel<64><<<dim3(pv_blocks, bh), kThreads, 0, s>>>(d.C, scores, vbar, o_coarse);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
-                          float* scores, float* o_coarse, cudaStream_t s) {
-    const cudaError_t e = launch_coarse_scores(d, qbar, kbar, scale, scores, s);
-    if (e != cudaSuccess) return e;
-    return launch_coarse_pv(d, scores, vbar, o_coarse, s);
-}
-
 // Largest C the selection kernel keeps in shared memory (one row per warp).
 constexpr int kTopkMaxC = 49152;
 
@@ -523,35 +384,35 @@ namespace {
 // Register-resident selection for C <= 2048 (a warp holds the row, KPL keys per lane).
 template <int KPL>
 cudaError_t launch_topk_reg(int64_t rows, int C, int k, const float* scores, int32_t* idx, uint64_t* sig,
-                            cudaStream_t s) {
+                            float* stats, cudaStream_t s) {
     const int64_t blocks_needed = (rows + kThreads / 32 - 1) / (kThreads / 32);
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-    topk_reg_kernel<KPL><<<grid, kThreads, 0, s>>>(rows, C, k, scores, idx, sig);
+    topk_reg_kernel<KPL><<<grid, kThreads, 0, s>>>(rows, C, k, scores, idx, sig, reinterpret_cast<float2*>(stats));
     return cudaGetLastError();
 }
 
-cudaError_t topk_reg_dispatch(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig,
+cudaError_t topk_reg_dispatch(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, float* stats,
                               cudaStream_t s) {
     const int64_t rows = static_cast<int64_t>(d.B) * d.H * d.C;
     const int kpl = (d.C + 31) / 32;
-    if (kpl <= 4) return launch_topk_reg<4>(rows, d.C, k, scores, idx, sig, s);
-    if (kpl <= 8) return launch_topk_reg<8>(rows, d.C, k, scores, idx, sig, s);
-    if (kpl <= 12) return launch_topk_reg<12>(rows, d.C, k, scores, idx, sig, s);
-    if (kpl <= 16) return launch_topk_reg<16>(rows, d.C, k, scores, idx, sig, s);
-    if (kpl <= 20) return launch_topk_reg<20>(rows, d.C, k, scores, idx, sig, s);
-    if (kpl <= 24) return launch_topk_reg<24>(rows, d.C, k, scores, idx, sig, s);
-    if (kpl <= 32) return launch_topk_reg<32>(rows, d.C, k, scores, idx, sig, s);
-    if (kpl <= 40) return launch_topk_reg<40>(rows, d.C, k, scores, idx, sig, s);
-    if (kpl <= 48) return launch_topk_reg<48>(rows, d.C, k, scores, idx, sig, s);
-    return launch_topk_reg<64>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 4) return launch_topk_reg<4>(rows, d.C, k, scores, idx, sig, stats, s);
+    if (kpl <= 8) return launch_topk_reg<8>(rows, d.C, k, scores, idx, sig, stats, s);
+    if (kpl <= 12) return launch_topk_reg<12>(rows, d.C, k, scores, idx, sig, stats, s);
+    if (kpl <= 16) return launch_topk_reg<16>(rows, d.C, k, scores, idx, sig, stats, s);
+    if (kpl <= 20) return launch_topk_reg<20>(rows, d.C, k, scores, idx, sig, stats, s);
+    if (kpl <= 24) return launch_topk_reg<24>(rows, d.C, k, scores, idx, sig, stats, s);
+    if (kpl <= 32) return launch_topk_reg<32>(rows, d.C, k, scores, idx, sig, stats, s);
+    if (kpl <= 40) return launch_topk_reg<40>(rows, d.C, k, scores, idx, sig, stats, s);
+    if (kpl <= 48) return launch_topk_reg<48>(rows, d.C, k, scores, idx, sig, stats, s);
+    return launch_topk_reg<64>(rows, d.C, k, scores, idx, sig, stats, s);
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx, cudaStream_t s) {
     if (d.C > kTopkMaxC) return cudaErrorInvalidValue;
-    if (d.C <= kTopkRegMaxC) return topk_reg_dispatch(d, scores, k, idx, nullptr, s);
+    if (d.C <= kTopkRegMaxC) return topk_reg_dispatch(d, scores, k, idx, nullptr, nullptr, s);
     const int64_t rows = static_cast<int64_t>(d.B) * d.H * d.C;
     const int wpb = topk_warps_per_block(d.C);
     const size_t smem = static_cast<size_t>(wpb) * d.C * 4;
@@ -567,9 +428,10 @@ cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx,
     return cudaGetLastError();
 }
 
-cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s) {
+cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s,
+                            float* stats) {
     if (d.C > kTopkRegMaxC) return cudaErrorInvalidValue;
-    return topk_reg_dispatch(d, scores, k, idx, sig, s);
+    return topk_reg_dispatch(d, scores, k, idx, sig, stats, s);
 }
 
 cudaError_t launch_group_sort(const Dims& d, const uint64_t* sig, int32_t* order, cudaStream_t s) {

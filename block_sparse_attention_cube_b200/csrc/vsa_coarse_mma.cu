@@ -1,0 +1,602 @@
+// The coarse stage's two contractions on the tensor cores (Wan2.2 teardown,
+// zharfai.com, section "Video sparse attention selects cubes", part 1: block-
+// level attention over the mean-pooled cubes; section "Blackwell changes the
+// optimisation problem": dense contractions belong on the fifth-generation
+// tensor cores).
+//
+// The pooled vectors are float32, and the scores decide the selection, so a
+// plain bf16 product (8-bit significands) would reorder near-equal cubes.
+// Each float32 value x is therefore carried as three bf16 parts
+//     hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid)
+// (x = hi + mid + lo to within 2^-24 |x|, each part rounded to nearest), and
+// a product a*b is formed from the six partial products whose size is at
+// least 2^-18 |a b|:
+//     hi*hi + hi*mid + mid*hi + hi*lo + lo*hi + mid*mid,
+// each exact in the float32 accumulator's input (8 x 8 significand bits).
+// The dropped terms are below 2^-26 |a b|, so a score carries about the error
+// of a float32 dot product.  Six tcgen05 MMAs per 16-channel step replace one;
+// on B200 that is still several times the float32 CUDA-core rate.
+//
+// Scores: one CTA per (b, h, 128 query cubes) loops over the head's key cubes
+// in tiles of 128: a TMA producer warp, an MMA issuer warp, and four epilogue
+// warps that move each 128 x 128 float32 tile from tensor memory to the
+// [B, H, C, C] scores (scaled), two tiles in flight.
+#include <cfloat>
+#include <mutex>
+
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include "ptx_sm100.cuh"
+#include "vsa_internal.h"
+
+namespace vsa {
+namespace {
+
+using namespace ptx;
+
+constexpr int kCmThreads = 192;                 // warps 0-3 epilogue (one TMEM lane quarter each), 4 TMA, 5 MMA
+constexpr int kCmTmaWarp = 4;
+constexpr int kCmMmaWarp = 5;
+constexpr uint32_t kCmHalf = 128u * 128u;       // 128 rows x 64 bf16 channels, 128-byte swizzled: 16 KB
+constexpr uint32_t kCmOffA = 0;                 // query cubes: [part][channel half], up to 6 x 16 KB
+constexpr uint32_t kCmOffB = 6u * kCmHalf;      // key cubes: 2 stages x [part] (one channel half), 3 x 16 KB
+constexpr uint32_t kCmStage = 3u * kCmHalf;
+constexpr int kCmStages = 2;
+constexpr uint32_t kCmOffBar = kCmOffB + kCmStages * kCmStage;
+enum CmBar : int { kCmBarA = 0, kCmBarBFull = 1, kCmBarBEmpty = 3, kCmBarSFull = 5, kCmBarSEmpty = 7, kCmBarDrain = 9,
+                   kCmBars = 10 };
+constexpr uint32_t kCmOffMisc = kCmOffBar + 8u * kCmBars;          // TMEM address, abort flag
+constexpr uint32_t kCmSmem = kCmOffMisc + 16u + 1024u;             // + slack for the 1 KB alignment
+constexpr uint32_t kCmTmemCols = 256;                              // two 128-column score buffers
+constexpr uint64_t kCmDrainNs = 200000000ull;
+
+// the six partial products (part of the query cube, part of the key cube), largest first:
+// (hi, hi), (hi, mid), (mid, hi), (hi, lo), (lo, hi), (mid, mid)
+__host__ __device__ constexpr int prod_a(int pr) { return pr == 2 || pr == 5 ? 1 : pr == 4 ? 2 : 0; }
+__host__ __device__ constexpr int prod_b(int pr) { return pr == 1 || pr == 5 ? 1 : pr == 3 ? 2 : 0; }
+
+struct CmParams {
+    int C, B, H;
+    int row_tiles;           // ceil(C / 128)
+    float scale;
+    float* scores;           // [B, H, C, C]
+    int* status;             // watchdog word
+    uint64_t limit_ns;
+};
+
+// x = hi + mid + lo, each part the bf16 nearest to what the larger parts leave (as the pooling pass
+// splits the pooled vectors)
+__device__ __forceinline__ void split3(float x, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    const __nv_bfloat16 l = __float2bfloat16_rn(r2);
+    hi = __bfloat16_as_ushort(h);
+    mid = __bfloat16_as_ushort(m);
+    lo = __bfloat16_as_ushort(l);
+}
+
+__device__ __forceinline__ uint64_t desc_at(uint64_t fixed, uint32_t saddr) {
+    return fixed | static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kCmThreads, 1)
+coarse_scores_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const CmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t base = (raw_u32 + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_u32);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto bar = [&](int i) -> uint32_t { return base + kCmOffBar + 8u * static_cast<uint32_t>(i); };
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kCmOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kCmOffMisc + 4);
+    const BoundedWait bw{abort_flag, p.status, p.limit_ns};
+
+    const int bh = blockIdx.x / p.row_tiles;
+    const int i0 = (blockIdx.x % p.row_tiles) * 128;
+    const int C = p.C;
+    const int tiles = (C + 127) / 128;
+    constexpr int kHalves = D / 64;   // 64-channel halves: one swizzled 128-byte row each
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        mbar_init(bar(kCmBarA), 1);
+        for (int s = 0; s < kCmStages; ++s) {
+            mbar_init(bar(kCmBarBFull + s), 1);
+            mbar_init(bar(kCmBarBEmpty + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(kCmBarSFull + b), 1);
+            mbar_init(bar(kCmBarSEmpty + b), 4);   // one arrival per epilogue warp
+        }
+        mbar_init(bar(kCmBarDrain), 1);
+        fence_mbar_init();
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+    }
+    if (warp == kCmMmaWarp) {
+        tmem_alloc(base + kCmOffMisc, kCmTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    auto drain_wait = [&](uint32_t b, uint32_t par) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(b, par) && globaltimer() - t0 < kCmDrainNs) {
+        }
+    };
+
+    if (warp == kCmTmaWarp) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            uint32_t issued[kCmStages] = {0u, 0u};
+            // the CTA's 128 query cubes: three parts x two channel halves (rows past C read as zeros)
+            mbar_arrive_expect_tx(bar(kCmBarA), 3u * kHalves * kCmHalf);
+            for (int part = 0; part < 3; ++part)
+                for (int h = 0; h < kHalves; ++h)
+                    tma_load_4d(base + kCmOffA + (kHalves * part + h) * kCmHalf, &tm_q, 64 * h, i0, bh, part,
+                                bar(kCmBarA));
+            int slot = 0;
+            uint32_t phase = 0;
+            for (int n = 0; ok && n < tiles; ++n) {
+                for (int h = 0; h < kHalves; ++h) {
+                    if (!(ok = bw.wait(bar(kCmBarBEmpty + slot), phase ^ 1u))) break;
+                    mbar_arrive_expect_tx(bar(kCmBarBFull + slot), kCmStage);
+                    ++issued[slot];
+                    for (int part = 0; part < 3; ++part)
+                        tma_load_4d(base + kCmOffB + slot * kCmStage + part * kCmHalf, &tm_k, 64 * h, 128 * n, bh,
+                                    part, bar(kCmBarBFull + slot));
+                    if (++slot == kCmStages) {
+                        slot = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // copies still in flight land before the CTA exits
+                drain_wait(bar(kCmBarA), 0u);
+                for (int s = 0; s < kCmStages; ++s)
+                    if (issued[s]) drain_wait(bar(kCmBarBFull + s), (issued[s] - 1u) & 1u);
+            }
+        }
+    } else if (warp == kCmMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);   // both operands K-major
+            const uint64_t fix = smem_desc_sw128(0, 16u, 1024u);         // 8-row groups 1 KB apart
+            bool ok = bw.wait(bar(kCmBarA), 0u);
+            bool issued_any = false;
+            int slot = 0;
+            uint32_t phase = 0;
+            for (int n = 0; ok && n < tiles; ++n) {
+                const int b = n & 1;
+                // the epilogue has read this buffer's previous tile
+                if (n >= 2 && !(ok = bw.wait(bar(kCmBarSEmpty + b), ((n >> 1) - 1) & 1))) break;
+                for (int h = 0; h < kHalves; ++h) {
+                    if (!(ok = bw.wait(bar(kCmBarBFull + slot), phase))) break;
+                    tc_fence_after();
+                    const uint32_t kb = base + kCmOffB + slot * kCmStage;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                        for (int pr = 0; pr < 6; ++pr) {
+                            const uint32_t qa = base + kCmOffA + (kHalves * prod_a(pr) + h) * kCmHalf + kk * 32u;
+                            const uint32_t ka = kb + prod_b(pr) * kCmHalf + kk * 32u;
+                            mma_bf16_ss(tmem + 128u * b, desc_at(fix, qa), desc_at(fix, ka), idesc,
+                                        (h | kk | pr) != 0 ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(bar(kCmBarBEmpty + slot));
+                    issued_any = true;
+                    if (++slot == kCmStages) {
+                        slot = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(bar(kCmBarSFull + b));
+            }
+            if (issued_any) {
+                mma_commit(bar(kCmBarDrain));
+                drain_wait(bar(kCmBarDrain), 0u);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue: TMEM -> scores
+        const int r = 32 * warp + lane;   // TMEM lane = query row of the tile
+        const int gi = i0 + r;
+        float* srow = p.scores + (static_cast<int64_t>(bh) * C + (gi < C ? gi : 0)) * C;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+        for (int n = 0; n < tiles; ++n) {
+            const int b = n & 1;
+            if (!__all_sync(0xffffffffu, bw.wait(bar(kCmBarSFull + b), (n >> 1) & 1))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t v[32];
+                tmem_ld32_wait(lane_base + 128u * b + 32u * cc, v);
+                const int j0 = 128 * n + 32 * cc;
+                if (gi < C) {
+                    if (j0 + 32 <= C && (C & 3) == 0) {
+                        float4* dst = reinterpret_cast<float4*>(srow + j0);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(p.scale * __uint_as_float(v[4 * e]), p.scale * __uint_as_float(v[4 * e + 1]),
+                                                 p.scale * __uint_as_float(v[4 * e + 2]),
+                                                 p.scale * __uint_as_float(v[4 * e + 3]));
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (j0 + e < C) srow[j0 + e] = p.scale * __uint_as_float(v[e]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kCmBarSEmpty + b));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kCmMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kCmTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- coarse output
+// o_coarse = softmax(scores) vbar, as exp(s - m) vbar / l with each row's maximum m and sum l from
+// row_stats.  One CTA per (b, h, 128 query cubes): four converter warps (one query row per thread,
+// also the TMEM lane quarters of the epilogue) turn each 64-key slice of the row into exp(s - m),
+// split it into three bf16 parts and store them K-major with the 128-byte swizzle (the A operand);
+// a TMA warp brings the same keys' vbar parts (the B operand, MN-major); an MMA warp issues the six
+// partial products per 16-key step into one 128 x D float32 accumulator.
+constexpr uint32_t kPvA = 3u * 128u * 128u;     // P parts of one 64-key slice: 3 x (128 rows x 128 B)
+constexpr uint32_t kPvB = 3u * 64u * 256u;      // vbar parts of 64 keys x D = 128: 3 x (2 halves x 8 KB)
+constexpr int kPvStages = 2;
+constexpr uint32_t kPvOffA = 0;
+constexpr uint32_t kPvOffB = kPvOffA + kPvStages * kPvA;
+constexpr uint32_t kPvOffBar = kPvOffB + kPvStages * kPvB;
+enum PvBar : int { kPvBarAFull = 0, kPvBarAEmpty = 2, kPvBarBFull = 4, kPvBarBEmpty = 6, kPvBarODone = 8,
+                   kPvBarDrain = 9, kPvBars = 10 };
+constexpr uint32_t kPvOffMisc = kPvOffBar + 8u * kPvBars;
+constexpr uint32_t kPvSmem = kPvOffMisc + 16u + 1024u;
+
+struct PvParams {
+    int C, row_tiles;
+    const float* scores;      // [B, H, C, C]
+    const float2* stats;      // [B, H, C]: (row maximum, 1 / sum of exp(s - maximum))
+    float* o_coarse;          // [B, H, C, D]
+    int* status;
+    uint64_t limit_ns;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kCmThreads, 1)
+coarse_pv_mma_kernel(const __grid_constant__ CUtensorMap tm_v, const PvParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_u32 = smem_u32(smem_raw);
+    const uint32_t base = (raw_u32 + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_u32);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto bar = [&](int i) -> uint32_t { return base + kPvOffBar + 8u * static_cast<uint32_t>(i); };
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kPvOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kPvOffMisc + 4);
+    const BoundedWait bw{abort_flag, p.status, p.limit_ns};
+    constexpr int kHalves = D / 64;
+    constexpr uint32_t kPartB = 64u * 128u * kHalves;   // one part of a 64-key vbar slice
+
+    const int bh = blockIdx.x / p.row_tiles;
+    const int i0 = (blockIdx.x % p.row_tiles) * 128;
+    const int C = p.C;
+    const int slices = (C + 63) / 64;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int s = 0; s < kPvStages; ++s) {
+            mbar_init(bar(kPvBarAFull + s), 4);   // one arrival per converter warp
+            mbar_init(bar(kPvBarAEmpty + s), 1);
+            mbar_init(bar(kPvBarBFull + s), 1);
+            mbar_init(bar(kPvBarBEmpty + s), 1);
+        }
+        mbar_init(bar(kPvBarODone), 1);
+        mbar_init(bar(kPvBarDrain), 1);
+        fence_mbar_init();
+        prefetch_tensormap(&tm_v);
+    }
+    if (warp == kCmMmaWarp) {
+        tmem_alloc(base + kPvOffMisc, 128u);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    auto drain_wait = [&](uint32_t b, uint32_t par) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(b, par) && globaltimer() - t0 < kCmDrainNs) {
+        }
+    };
+
+    if (warp == kCmTmaWarp) {
+        // ------------------------------------------------------------ vbar parts
+        if (lane == 0) {
+            bool ok = true;
+            uint32_t issued[kPvStages] = {0u, 0u};
+            for (int n = 0; n < slices; ++n) {
+                const int slot = n % kPvStages;
+                if (!(ok = bw.wait(bar(kPvBarBEmpty + slot), ((n / kPvStages) & 1) ^ 1))) break;
+                mbar_arrive_expect_tx(bar(kPvBarBFull + slot), 3u * kPartB);
+                ++issued[slot];
+                for (int part = 0; part < 3; ++part)
+                    for (int h = 0; h < kHalves; ++h)
+                        tma_load_4d(base + kPvOffB + slot * kPvB + part * kPartB + h * 8192u, &tm_v, 64 * h, 64 * n,
+                                    bh, part, bar(kPvBarBFull + slot));
+            }
+            if (!ok)
+                for (int s = 0; s < kPvStages; ++s)
+                    if (issued[s]) drain_wait(bar(kPvBarBFull + s), (issued[s] - 1u) & 1u);
+        }
+    } else if (warp == kCmMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);     // P K-major, vbar MN-major
+            const uint64_t fix_p = smem_desc_sw128(0, 16u, 1024u);       // K-major, 8-row groups 1 KB apart
+            const uint64_t fix_v = smem_desc_sw128(0, 8192u, 1024u);     // MN-major, channel halves 8 KB apart
+            bool ok = true, issued_any = false;
+            for (int n = 0; ok && n < slices; ++n) {
+                const int slot = n % kPvStages;
+                const uint32_t par = (n / kPvStages) & 1;
+                if (!(ok = bw.wait(bar(kPvBarAFull + slot), par))) break;
+                if (!(ok = bw.wait(bar(kPvBarBFull + slot), par))) break;
+                tc_fence_after();
+                const uint32_t pa = base + kPvOffA + slot * kPvA, vb = base + kPvOffB + slot * kPvB;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                    for (int pr = 0; pr < 6; ++pr) {
+                        mma_bf16_ss(tmem, desc_at(fix_p, pa + prod_a(pr) * 16384u + kk * 32u),
+                                    desc_at(fix_v, vb + prod_b(pr) * kPartB + kk * 2048u), idesc,
+                                    (n | kk | pr) != 0 ? 1u : 0u);
+                    }
+                }
+                mma_commit(bar(kPvBarAEmpty + slot));
+                mma_commit(bar(kPvBarBEmpty + slot));
+                issued_any = true;
+            }
+            if (ok) mma_commit(bar(kPvBarODone));
+            if (issued_any) {
+                mma_commit(bar(kPvBarDrain));
+                drain_wait(bar(kPvBarDrain), 0u);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ converters, then the epilogue
+        const int r = 32 * warp + lane;
+        const int gi = i0 + r;
+        const bool real = gi < C;
+        const float2 st = real ? p.stats[static_cast<int64_t>(bh) * C + gi] : make_float2(0.f, 0.f);
+        const float* srow = p.scores + (static_cast<int64_t>(bh) * C + (real ? gi : 0)) * C;
+        bool ok = true;
+        for (int n = 0; n < slices; ++n) {
+            const int slot = n % kPvStages;
+            if (!(ok = __all_sync(0xffffffffu, bw.wait(bar(kPvBarAEmpty + slot), ((n / kPvStages) & 1) ^ 1)))) break;
+            uint8_t* a = smem + kPvOffA + slot * kPvA + r * 128;
+            const int j0 = 64 * n;
+            const bool vec = real && (C & 3) == 0 && j0 + 64 <= C;   // whole slice in the row, 16-byte aligned
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {                 // 16-byte chunk c: keys j0 + 8c .. j0 + 8c + 7
+                float v[8];
+                if (vec) {
+                    const float4 x0 = *reinterpret_cast<const float4*>(srow + j0 + 8 * c);
+                    const float4 x1 = *reinterpret_cast<const float4*>(srow + j0 + 8 * c + 4);
+                    const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] = __expf(xs[e] - st.x);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = j0 + 8 * c + e;
+                        v[e] = (real && j < C) ? __expf(srow[j] - st.x) : 0.f;
+                    }
+                }
+                uint32_t hw[4], mw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    uint16_t h0, m0, l0, h1, m1, l1;
+                    split3(v[2 * e], h0, m0, l0);
+                    split3(v[2 * e + 1], h1, m1, l1);
+                    hw[e] = h0 | (uint32_t{h1} << 16);
+                    mw[e] = m0 | (uint32_t{m1} << 16);
+                    lw[e] = l0 | (uint32_t{l1} << 16);
+                }
+                const int sc = (c ^ (r & 7)) * 16;         // the 128-byte swizzle of row r
+                *reinterpret_cast<uint4*>(a + sc) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(a + 16384 + sc) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
+                *reinterpret_cast<uint4*>(a + 32768 + sc) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            fence_proxy_async_smem();   // the stores become visible to the tensor cores
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kPvBarAFull + slot));
+        }
+        if (ok && __all_sync(0xffffffffu, bw.wait(bar(kPvBarODone), 0u))) {
+            tc_fence_after();
+            const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+            float* orow = p.o_coarse + (static_cast<int64_t>(bh) * C + (real ? gi : 0)) * D;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld32_wait(lane_base + 32u * cc, v);
+                if (real) {
+                    float4* dst = reinterpret_cast<float4*>(orow + 32 * cc);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(__uint_as_float(v[4 * e]) * st.y, __uint_as_float(v[4 * e + 1]) * st.y,
+                                             __uint_as_float(v[4 * e + 2]) * st.y,
+                                             __uint_as_float(v[4 * e + 3]) * st.y);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kCmMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128u);
+    }
+}
+
+// Row maximum m and 1 / sum(exp(s - m)) of every score row, one warp per row (the coarse output's
+// softmax statistics when no selection pass computes them).
+__global__ void __launch_bounds__(256) row_stats_kernel(int64_t rows, int C, const float* __restrict__ scores,
+                                                        float2* __restrict__ stats) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = static_cast<int64_t>(gridDim.x) * 8;
+    for (int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); row < rows; row += warps) {
+        const float* s = scores + row * C;
+        float m = -FLT_MAX;
+        for (int j = lane; j < C; j += 32) m = fmaxf(m, s[j]);
+#pragma unroll
+        for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float l = 0.f;
+        for (int j = lane; j < C; j += 32) l += __expf(s[j] - m);
+#pragma unroll
+        for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+        if (lane == 0) stats[row] = make_float2(m, 1.0f / l);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 cm_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// Split parts [3][B*H][C][D] bf16 as (D, C, B*H, part): box 64 channels x `rows` cubes, 128-byte swizzle.
+bool encode_parts(CUtensorMap* m, const uint16_t* parts, const Dims& d, uint32_t rows) {
+    auto fn = cm_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t bh = static_cast<cuuint64_t>(d.B) * d.H;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d.D), static_cast<cuuint64_t>(d.C), bh, 3u};
+    const cuuint64_t row = static_cast<cuuint64_t>(d.D) * 2u;
+    const cuuint64_t strides[3] = {row, row * d.C, row * d.C * bh};
+    const cuuint32_t box[4] = {64u, rows, 1u, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t*>(parts), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+size_t split_parts_elems(const Dims& d) { return 3u * static_cast<size_t>(d.B) * d.H * d.C * d.D; }
+
+cudaError_t launch_coarse_scores_mma(const Dims& d, const uint16_t* q_parts, const uint16_t* k_parts, float scale,
+                                     float* scores, cudaStream_t s, const char** why) {
+    if (d.D != 128 && d.D != 64) return cudaErrorInvalidValue;
+    CUtensorMap tq, tk;
+    if (!encode_parts(&tq, q_parts, d, 128u) || !encode_parts(&tk, k_parts, d, 128u)) {
+        if (why) *why = "cuTensorMapEncodeTiled failed for the split pooled vectors";
+        return cudaErrorInvalidValue;
+    }
+    static int configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (!(dev >= 0 && dev < 64 && configured[dev])) {
+        e = cudaFuncSetAttribute(coarse_scores_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kCmSmem));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(coarse_scores_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(kCmSmem));
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = 1;
+    }
+    CmParams p{};
+    p.C = d.C;
+    p.B = d.B;
+    p.H = d.H;
+    p.row_tiles = (d.C + 127) / 128;
+    p.scale = scale;
+    p.scores = scores;
+    p.status = status_word();
+    p.limit_ns = kWaitLimitNs;
+    if (!p.status) {
+        if (why) *why = "watchdog word unavailable";
+        return cudaErrorInvalidValue;
+    }
+    const int64_t grid = static_cast<int64_t>(d.B) * d.H * p.row_tiles;
+    if (grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+    if (d.D == 128) coarse_scores_mma_kernel<128><<<static_cast<unsigned>(grid), kCmThreads, kCmSmem, s>>>(tq, tk, p);
+    else coarse_scores_mma_kernel<64><<<static_cast<unsigned>(grid), kCmThreads, kCmSmem, s>>>(tq, tk, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_row_stats(const Dims& d, const float* scores, float* stats, cudaStream_t s) {
+    const int64_t rows = static_cast<int64_t>(d.B) * d.H * d.C;
+    const int64_t blocks = (rows + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    row_stats_kernel<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(
+        rows, d.C, scores, reinterpret_cast<float2*>(stats));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_coarse_pv_mma(const Dims& d, const float* scores, const float* stats, const uint16_t* v_parts,
+                                 float* o_coarse, cudaStream_t s, const char** why) {
+    if (d.D != 128 && d.D != 64) return cudaErrorInvalidValue;
+    CUtensorMap tv;
+    if (!encode_parts(&tv, v_parts, d, 64u)) {
+        if (why) *why = "cuTensorMapEncodeTiled failed for the split pooled values";
+        return cudaErrorInvalidValue;
+    }
+    static int configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (!(dev >= 0 && dev < 64 && configured[dev])) {
+        e = cudaFuncSetAttribute(coarse_pv_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kPvSmem));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(coarse_pv_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(kPvSmem));
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = 1;
+    }
+    PvParams p{};
+    p.C = d.C;
+    p.row_tiles = (d.C + 127) / 128;
+    p.scores = scores;
+    p.stats = reinterpret_cast<const float2*>(stats);
+    p.o_coarse = o_coarse;
+    p.status = status_word();
+    p.limit_ns = kWaitLimitNs;
+    if (!p.status) {
+        if (why) *why = "watchdog word unavailable";
+        return cudaErrorInvalidValue;
+    }
+    const int64_t grid = static_cast<int64_t>(d.B) * d.H * p.row_tiles;
+    if (grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+    if (d.D == 128) coarse_pv_mma_kernel<128><<<static_cast<unsigned>(grid), kCmThreads, kPvSmem, s>>>(tv, p);
+    else coarse_pv_mma_kernel<64><<<static_cast<unsigned>(grid), kCmThreads, kPvSmem, s>>>(tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace vsa

@@ -46,27 +46,15 @@ cudaError_t launch_untile(const Dims& d, const uint16_t* xt, uint16_t* x, cudaSt
 cudaError_t launch_pool(const Dims& d, const uint16_t* const* xt, float* const* xbar, int count, cudaStream_t s);
 cudaError_t launch_combine(const Dims& d, const float* o_coarse, const uint16_t* o_fine, const uint16_t* g_coarse,
                            const uint16_t* g_fine, uint16_t* o_tiled, cudaStream_t s);
-// The two halves of launch_coarse: the scores, and softmax(scores) x vbar.
-cudaError_t launch_coarse_scores(const Dims& d, const float* qbar, const float* kbar, float scale, float* scores,
-                                 cudaStream_t s);
-cudaError_t launch_coarse_pv(const Dims& d, const float* scores, const float* vbar, float* o_coarse, cudaStream_t s);
-cudaError_t launch_coarse(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
-                          float* scores, float* o_coarse, cudaStream_t s);
 cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx, cudaStream_t s);
 
 // Largest C whose rows the selection holds in registers; up to it, top-k can
 // also emit each row's work-order signature (uint64 [B, H, C]) in the same
 // pass, and launch_group_sort turns those into the order launch_group gives.
 constexpr int kTopkRegMaxC = 2048;
-cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s);
-
-// The coarse scores, the top-k selection (and each row's work-order key) and, with o_coarse, the
-// coarse output in one launch; the scores stay in shared memory (copied to scores_out when given).
-// Bit-identical scores and selection to launch_coarse_scores + launch_topk_sig.
-bool coarse_select_supported(const Dims& d);
-cudaError_t launch_coarse_select(const Dims& d, const float* qbar, const float* kbar, const float* vbar, float scale,
-                                 int k, int32_t* idx, uint64_t* sig, float* o_coarse, float* scores_out,
-                                 cudaStream_t s);
+// (stats, when non-null: [B, H, C] float2 of each row's maximum and 1 / sum(exp(s - maximum)))
+cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s,
+                            float* stats = nullptr);
 
 // Work order of the fine stage from the coarse scores (C <= kGroupMaxC).
 constexpr int kGroupMaxC = 4096;
@@ -140,8 +128,24 @@ cudaError_t launch_norm_rope(const Dims& d, const NormRopeArgs& a, cudaStream_t 
 cudaError_t launch_gather_heads(const uint16_t* src, int64_t rows, int H, int h0, int hg, uint16_t* dst,
                                 cudaStream_t s);
 
+// xbar (float32 means) and parts (the means split into three bf16 parts, [3][B*H][C][D] per tensor) may
+// each be null.
 cudaError_t launch_pool_tokens(const Dims& d, const uint16_t* const* x, float* const* xbar, int count,
-                               cudaStream_t s);
+                               cudaStream_t s, uint16_t* const* parts = nullptr);
+
+// The coarse stage on the tensor cores: float32 pooled vectors carried as three bf16 parts.
+// launch_split_parts: float32 [B, H, C, D] -> parts [3][B*H][C][D] (split_parts_elems(d) uint16).
+size_t split_parts_elems(const Dims& d);
+cudaError_t launch_split_parts(const Dims& d, const float* x, uint16_t* parts, cudaStream_t s);
+// scores [B, H, C, C] = scale * qbar kbar^T from the parts of qbar and kbar (six partial products per
+// channel step); *why set when a tensor map cannot be encoded.
+cudaError_t launch_coarse_scores_mma(const Dims& d, const uint16_t* q_parts, const uint16_t* k_parts, float scale,
+                                     float* scores, cudaStream_t s, const char** why);
+// stats [B, H, C] float2: each score row's maximum m and 1 / sum(exp(s - m)).
+cudaError_t launch_row_stats(const Dims& d, const float* scores, float* stats, cudaStream_t s);
+// o_coarse [B, H, C, D] = softmax(scores) vbar from the row statistics and the parts of vbar.
+cudaError_t launch_coarse_pv_mma(const Dims& d, const float* scores, const float* stats, const uint16_t* v_parts,
+                                 float* o_coarse, cudaStream_t s, const char** why);
 
 cudaError_t launch_wait_probe(uint64_t limit_ns, cudaStream_t s);
 

@@ -96,9 +96,40 @@ __global__ void __launch_bounds__(kBlock) untile_kernel(Dims d, const uint16_t* 
 // over the warp's lane groups, partial sums are combined with shuffles.
 struct PoolIO {
     const uint16_t* src[3];
-    float* dst[3];
+    float* dst[3];          // float32 means [B, H, C, D], or null
+    uint16_t* parts[3];     // the means as three bf16 parts [3][B*H][C][D], or null
     int count;
 };
+
+// x = hi + mid + lo with each part the bf16 nearest to what the larger parts leave (the residuals are
+// exact in float32); the three parts hold x to within 2^-24 |x| (bits: bf16 patterns).
+__device__ __forceinline__ void split3(float x, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    const __nv_bfloat16 l = __float2bfloat16_rn(r2);
+    hi = __bfloat16_as_ushort(h);
+    mid = __bfloat16_as_ushort(m);
+    lo = __bfloat16_as_ushort(l);
+}
+
+// Eight consecutive float32 values to their three bf16 parts: 16 bytes into each part plane.
+__device__ __forceinline__ void store_parts8(const float (&v)[8], uint16_t* parts, int64_t plane, int64_t off) {
+    uint32_t h[4], m[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        uint16_t h0, m0, l0, h1, m1, l1;
+        split3(v[2 * e], h0, m0, l0);
+        split3(v[2 * e + 1], h1, m1, l1);
+        h[e] = h0 | (uint32_t{h1} << 16);
+        m[e] = m0 | (uint32_t{m1} << 16);
+        l[e] = l0 | (uint32_t{l1} << 16);
+    }
+    *reinterpret_cast<uint4*>(parts + off) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(parts + plane + off) = make_uint4(m[0], m[1], m[2], m[3]);
+    *reinterpret_cast<uint4*>(parts + 2 * plane + off) = make_uint4(l[0], l[1], l[2], l[3]);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kBlock) pool_kernel(Dims d, PoolIO io) {
@@ -170,7 +201,12 @@ __global__ void __launch_bounds__(kPoolThreads) pool_tokens_kernel(Dims d, PoolI
     const int nx = min(kCube, d.X - cx * kCube);
     const int ny = min(kCube, d.Y - cy * kCube);
     const int64_t row = static_cast<int64_t>(d.H) * CH;   // 16-byte chunks per token
-    const uint4* src = reinterpret_cast<const uint4*>(io.src[tensor]) + static_cast<int64_t>(b) * d.N * row + q;
+    // pick the tensor's pointers by value: indexing the parameter arrays with a runtime index would copy them
+    // to the stack
+    const uint16_t* src_t = tensor == 0 ? io.src[0] : tensor == 1 ? io.src[1] : io.src[2];
+    float* dst_t = tensor == 0 ? io.dst[0] : tensor == 1 ? io.dst[1] : io.dst[2];
+    uint16_t* parts_t = tensor == 0 ? io.parts[0] : tensor == 1 ? io.parts[1] : io.parts[2];
+    const uint4* src = reinterpret_cast<const uint4*>(src_t) + static_cast<int64_t>(b) * d.N * row + q;
     const int64_t base_n = (static_cast<int64_t>(ct) * kCube * d.X + cx * kCube) * d.Y + cy * kCube;
     float acc[R][8];
 #pragma unroll
@@ -199,9 +235,28 @@ __global__ void __launch_bounds__(kPoolThreads) pool_tokens_kernel(Dims d, PoolI
     }
     const float inv = 1.0f / static_cast<float>(nt * nx * ny);
     const int64_t bh = static_cast<int64_t>(b) * d.H + h;
-    float4* out = reinterpret_cast<float4*>(io.dst[tensor] + (bh * d.C + c) * D + j * 8);
-    out[0] = make_float4(m[0] * inv, m[1] * inv, m[2] * inv, m[3] * inv);
-    out[1] = make_float4(m[4] * inv, m[5] * inv, m[6] * inv, m[7] * inv);
+    float mean[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mean[e] = m[e] * inv;
+    if (dst_t != nullptr) {
+        float4* out = reinterpret_cast<float4*>(dst_t + (bh * d.C + c) * D + j * 8);
+        out[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
+        out[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
+    }
+    if (parts_t != nullptr)
+        store_parts8(mean, parts_t, static_cast<int64_t>(d.B) * d.H * d.C * D, (bh * d.C + c) * D + j * 8);
+}
+
+// float32 [rows, D] -> three bf16 parts [3][rows][D] (the split of pool_tokens_kernel's means)
+__global__ void __launch_bounds__(kBlock) split_parts_kernel(int64_t groups, const float* __restrict__ x,
+                                                              uint16_t* __restrict__ parts) {
+    for (int64_t g = static_cast<int64_t>(blockIdx.x) * kBlock + threadIdx.x; g < groups;
+         g += static_cast<int64_t>(gridDim.x) * kBlock) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(x) + 2 * g);
+        const float4 b = __ldg(reinterpret_cast<const float4*>(x) + 2 * g + 1);
+        const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        store_parts8(v, parts, groups * 8, g * 8);
+    }
 }
 
 template <int D>
@@ -283,12 +338,20 @@ cudaError_t launch_pool(const Dims& d, const uint16_t* const* xt, float* const* 
     return cudaGetLastError();
 }
 
+cudaError_t launch_split_parts(const Dims& d, const float* x, uint16_t* parts, cudaStream_t s) {
+    const int64_t groups = static_cast<int64_t>(d.B) * d.H * d.C * d.D / 8;
+    const int grid = grid_for((groups + kBlock - 1) / kBlock, 8);
+    split_parts_kernel<<<grid, kBlock, 0, s>>>(groups, x, parts);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_pool_tokens(const Dims& d, const uint16_t* const* x, float* const* xbar, int count,
-                               cudaStream_t s) {
+                               cudaStream_t s, uint16_t* const* parts) {
     PoolIO io{};
     for (int i = 0; i < count; ++i) {
         io.src[i] = x[i];
-        io.dst[i] = xbar[i];
+        io.dst[i] = xbar ? xbar[i] : nullptr;
+        io.parts[i] = parts ? parts[i] : nullptr;
     }
     io.count = count;
     const int64_t cubes = static_cast<int64_t>(count) * d.B * d.C;

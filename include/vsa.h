@@ -120,14 +120,24 @@ vsa_status vsa_pool(const vsa_shape* shape, const vsa_bf16* xt, float* xbar, vsa
 
 /*
  * vsa_coarse — block-level attention over the pooled cubes (same section,
- * part 1): scores = scale * qbar kbar^T, o_coarse = softmax_rows(scores) vbar.
- * float32 arithmetic on CUDA cores.
+ * part 1): scores = scale * qbar kbar^T, o_coarse = softmax_rows(scores) vbar,
+ * both contractions on the tensor cores.  The scores rank the cubes, so they
+ * need float32 accuracy: each float32 input x is carried as three bf16 parts
+ * (hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid), together within
+ * 2^-24 |x|) and each product from its six partial products of size >= 2^-18
+ * (hi*hi, hi*mid, mid*hi, hi*lo, lo*hi, mid*mid; the dropped ones are below
+ * 2^-26), accumulated in float32.  vsa_forward computes the same bits.
  *   qbar, kbar, vbar  [B, H, C, D] float32 (read).
  *   scores            [B, H, C, C] float32 (written): row = query cube.
  *   o_coarse          [B, H, C, D] float32 (written).
+ *   workspace         device buffer of vsa_coarse_workspace_bytes(shape),
+ *                     256-byte aligned (the split inputs and per-row softmax
+ *                     statistics; contents on return unspecified).
  */
+size_t vsa_coarse_workspace_bytes(const vsa_shape* shape);
 vsa_status vsa_coarse(const vsa_shape* shape, const float* qbar, const float* kbar, const float* vbar,
-                      float scale, float* scores, float* o_coarse, vsa_stream_t stream);
+                      float scale, float* scores, float* o_coarse, void* workspace, size_t workspace_bytes,
+                      vsa_stream_t stream);
 
 /*
  * vsa_topk — per query cube, the k key cubes with the highest coarse score
@@ -210,34 +220,6 @@ vsa_status vsa_combine(const vsa_shape* shape, const float* o_coarse, const vsa_
  */
 vsa_status vsa_topk_order(const vsa_shape* shape, const float* scores, int32_t k, int32_t* idx, int32_t* order,
                           uint64_t* sig_scratch, vsa_stream_t stream);
-
-/*
- * vsa_coarse_topk — the coarse stage and the selection in one pass over the
- * pooled cubes (same section, part 1), so the [B, H, C, C] scores never reach
- * global memory (teardown section "Fusion targets launch overhead and
- * memory").  One block per 32 query cubes of one (b, h) computes their rows of
- * scale * qbar kbar^T in shared memory, each score the same float32 sum as
- * vsa_coarse's (identical bits), keeps each row's k best key cubes (identical
- * to vsa_topk on those scores: ties to the lower index, rows ascending) and
- * each row's work-order key (as vsa_topk_order), and, when vbar and o_coarse
- * are given, turns the rows into softmax(scores) in place and writes
- * o_coarse = softmax(scores) vbar (the same values as vsa_coarse's up to
- * float32 rounding order).  With `order`, a second launch sorts the keys into
- * the work order of vsa_topk_order.
- *   qbar, kbar   [B, H, C, D] float32 (read).
- *   vbar         [B, H, C, D] float32 (read), or NULL together with o_coarse.
- *   idx          [B, H, C, k] int32 (written).
- *   order        [B, H, C] int32 (written), or NULL together with sig_scratch.
- *   sig_scratch  [B, H, C] uint64 caller scratch (overwritten), or NULL.
- *   o_coarse     [B, H, C, D] float32 (written), or NULL.
- *   scores       [B, H, C, C] float32, or NULL: a copy of the scores the
- *                kernel ranked (a check of the fusion; it costs the write).
- * Supported for C <= 1536 (a block's 32 score rows must fit in shared memory;
- * VSA_ERR_UNSUPPORTED otherwise: use vsa_coarse and vsa_topk_order).
- */
-vsa_status vsa_coarse_topk(const vsa_shape* shape, const float* qbar, const float* kbar, const float* vbar,
-                           float scale, int32_t k, int32_t* idx, int32_t* order, uint64_t* sig_scratch,
-                           float* o_coarse, float* scores, vsa_stream_t stream);
 
 /*
  * vsa_qk_norm_rope — the pre-attention pass of a Wan DiT block: RMSNorm of each
@@ -338,13 +320,15 @@ size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
 
 /*
  * vsa_forward — the whole attention call on one stream, as eight launches for
- * top-k < C:
- *   vsa_pool_qkv -> vsa_coarse (2) -> vsa_topk_order (2) -> vsa_schedule
- *   -> vsa_fine_fused (the one-tile kernel and its re-run guard)
- * (the second vsa_coarse launch, the coarse output softmax(scores) x V-bar,
- * is skipped when g_coarse is NULL, since only the merge uses it)
+ * top-k < C with a coarse gate:
+ *   vsa_pool_qkv (writing the pooled vectors as their three bf16 parts) ->
+ *   the coarse scores (tensor cores) -> vsa_topk_order (2; the selection pass
+ *   also keeps each row's softmax statistics) -> the coarse output (tensor
+ *   cores; skipped when g_coarse is NULL, since only the merge uses it) ->
+ *   vsa_schedule -> vsa_fine_fused (the one-tile kernel and its re-run guard)
  * (vsa_topk -> vsa_group instead when C > 2048; the grouping step is skipped
- * when C > 4096).  The result equals
+ * when C > 4096).  The scores and the selection are the bits of vsa_coarse and
+ * vsa_topk_order; the result equals
  *   tile -> pool -> coarse -> topk -> group -> fine -> combine -> untile
  * up to the bf16 rounding of O_fine that the staged path makes.
  * When topk == C every cube is selected and the fine stage is dense attention

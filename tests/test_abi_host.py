@@ -97,16 +97,17 @@ def test_forward_rerun_argument_checks():
     assert r.value == 0
 
 
-def test_coarse_topk_argument_checks():
+def test_coarse_workspace_checks():
     s = _shape()
-    p = [ctypes.c_void_p((1 << 40) + i * (1 << 32)) for i in range(8)]
-    call = lambda vbar, order, sig, oc, sh=s: vsa.raw_call("vsa_coarse_topk", ctypes.byref(sh), p[0], p[1], vbar,
-                                                          0.125, 2, p[2], order, sig, oc, None, None)
-    assert call(p[3], None, None, None) == INVALID and "vbar and o_coarse" in vsa.last_error()
-    assert call(None, p[4], None, None) == INVALID and "order and sig_scratch" in vsa.last_error()
-    # C = 6*8*33 = 1584 cubes: the score rows of a block no longer fit in shared memory
-    big = _lib.VsaShape(1, 1, 64, 24, 32, 132)
-    assert call(None, None, None, None, big) == UNSUPPORTED and "1536" in vsa.last_error()
+    need = vsa.raw_call("vsa_coarse_workspace_bytes", ctypes.byref(s))
+    # three float32 inputs as three bf16 parts each, and 8 bytes of softmax statistics per score row
+    up = lambda n: (n + 255) // 256 * 256
+    assert need == 3 * up(3 * 2 * 8 * 128 * 2) + up(2 * 8 * 8)
+    p = [ctypes.c_void_p((1 << 40) + i * (1 << 32)) for i in range(6)]
+    call = lambda ws, n: vsa.raw_call("vsa_coarse", ctypes.byref(s), p[0], p[1], p[2], 0.125, p[3], p[4], ws, n, None)
+    assert call(None, need) == WORKSPACE
+    assert call(p[5], need - 1) == WORKSPACE
+    assert call(ctypes.c_void_p(p[5].value + 16), need) == MISALIGNED
 
 
 def test_overlapping_input_and_output_rejected():
@@ -146,21 +147,19 @@ def test_workspace_checks():
 
 
 def test_workspace_size_480p_matches_layout():
-    # Q, K, V are read in place, so the workspace holds only the pooled q,k,v and o_coarse
-    # (4 x 624*40*128*4 B), the scores (624*624*40*4 B), idx (624*40*32*4 B) and the work order
-    # (624*40*4 B) with its signatures (624*40*8 B), the fine stage's steps and its overflow word, each
-    # rounded up to 256 B
+    # Q, K, V are read in place, so the workspace holds the pooled q, k, v as three bf16 parts each
+    # (3 x 3 x 624*40*128*2 B), the per-row softmax statistics (624*40*8 B), o_coarse (624*40*128*4 B),
+    # the scores (624*624*40*4 B), idx (624*40*32*4 B) and the work order (624*40*4 B) with its
+    # signatures (624*40*8 B), the fine stage's steps and its overflow word, each rounded up to 256 B
     s = vsa.Shape(1, 40, 128, (21, 30, 52)).c()
     up = lambda n: (n + 255) // 256 * 256
-    expect = 4 * up(624 * 40 * 128 * 4) + up(624 * 624 * 40 * 4) + up(624 * 40 * 32 * 4) + up(624 * 40 * 4) \
-        + up(624 * 40 * 8) \
+    coarse = 3 * up(3 * 624 * 40 * 128 * 2) + up(624 * 40 * 8) + up(624 * 40 * 128 * 4) + up(624 * 624 * 40 * 4)
+    expect = coarse + up(624 * 40 * 32 * 4) + up(624 * 40 * 4) + up(624 * 40 * 8) \
         + up(312 * 40 * 32 * 8) \
         + up(4)   # work-order signatures; steps: 312 pairs of query cubes x k steps x 8 B; overflow word
     assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 32) == expect
-
     # every cube selected: dense attention; the coarse buffers are for a coarse gate only
-    assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 624) == 4 * up(624 * 40 * 128 * 4) + \
-        up(624 * 624 * 40 * 4) + up(4)
+    assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 624) == coarse + up(4)
 
 
 def test_probe_limit_checked_before_device():

@@ -592,59 +592,71 @@ def test_topk_order_selection_and_order(case):
                 assert o[bh].tolist() == want, (k, bh)
 
 
-def _check_coarse_topk(s, bars, scale, ks, label):
-    """vsa_coarse_topk against the two-launch path on the same pooled inputs: identical scores (the
-    copy of what it ranked), identical selection and work order, coarse output within float32 rounding."""
-    scores, oc = vsa.coarse(*bars, s, scale)
-    for k in ks:
-        idx, order, oc2, sc2 = vsa.coarse_topk(*bars, s, k, scale, want_scores=True)
-        assert torch.equal(sc2, scores), f"{label}: fused scores differ (k={k})"
-        ref_idx, ref_order = vsa.topk_order(scores, s, k)
-        assert torch.equal(idx, ref_idx), f"{label}: fused selection differs (k={k})"
-        assert torch.equal(order, ref_order), f"{label}: fused work order differs (k={k})"
-        rel = float((oc2 - oc).norm() / oc.norm())
-        assert rel <= 1e-6, f"{label}: coarse output rel L2 {rel:.2e} (k={k})"
-        # without the coarse output, the order or the score copy: the same selection
-        idx2, none_order, none_oc, none_sc = vsa.coarse_topk(bars[0], bars[1], None, s, k, scale, order=False)
-        assert none_order is None and none_oc is None and none_sc is None
-        assert torch.equal(idx2, idx), f"{label}: selection without the coarse output differs (k={k})"
-    return scores, oc
+def _scores_f64(qb: np.ndarray, kb: np.ndarray, scale: float) -> np.ndarray:
+    """Exact-enough reference: the float32 inputs' dot products in float64, scaled."""
+    return scale * np.matmul(qb.astype(np.float64), np.swapaxes(kb.astype(np.float64), -1, -2))
 
 
-def test_coarse_topk_equals_the_two_launch_path(case):
-    """The fused coarse stage + selection on every small and edge case, against vsa_coarse +
-    vsa_topk_order bit for bit, and its coarse output against the oracle's."""
-    w, _, dev, f64 = case
-    s = _shape(w)
+@pytest.mark.parametrize("B,H,D,grid", [(1, 3, 128, (8, 16, 16)), (2, 2, 64, (9, 6, 5)), (1, 2, 128, (21, 30, 52)),
+                                        (1, 1, 128, (3, 2, 4)), (1, 2, 64, (24, 32, 28))],
+                         ids=["C32", "B2_d64_C12", "C624", "C1", "d64_C336"])
+def test_coarse_scores_exact_on_small_integers(B, H, D, grid):
+    """Pooled vectors of small integers: every bf16 part but the first is zero and every dot product is
+    an integer below 2^24, so the split tensor-core product must equal the exact scores bit for bit (a
+    check of the operand layout, the parts, the six partial products and the row/column tails)."""
+    s = vsa.Shape(B, H, D, grid)
     _, C = vsa.shape_info(s)
-    scale = 1 / math.sqrt(w.head_dim)
-    bars = vsa.pool_qkv(dev["q"], dev["k"], dev["v"], s)
-    ks = sorted({1, min(w.topk, C), min(33, C), C})
-    _check_coarse_topk(s, bars, scale, ks, w.name)
-    ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, w.topk, scale)
-    _, _, oc, _ = vsa.coarse_topk(*bars, s, w.topk, scale)
-    rel = np.linalg.norm(from_dev(oc) - ora["o_coarse"]) / np.linalg.norm(ora["o_coarse"])
-    assert rel <= COARSE_REL_L2, rel
+    rng = np.random.default_rng(C + D)
+    q, k = (rng.integers(-8, 9, size=(B, H, C, D)).astype(np.float32) for _ in range(2))
+    v = rng.standard_normal((B, H, C, D)).astype(np.float32)
+    scores, oc = vsa.coarse(*(torch.from_numpy(x).cuda() for x in (q, k, v)), s, 0.125)
+    ref = _scores_f64(q, k, 0.125)
+    assert np.array_equal(from_dev(scores), ref)
+    r_oc = np.matmul(O.softmax_rows(ref), v.astype(np.float64))
+    assert np.linalg.norm(from_dev(oc) - r_oc) / np.linalg.norm(r_oc) <= COARSE_REL_L2
 
 
-@pytest.mark.parametrize("grid,heads", [((8, 16, 16), 3), ((12, 32, 64), 2), ((24, 32, 128), 1)],
-                         ids=["C32", "C384", "C1536"])
-def test_coarse_topk_tie_heavy_pooled_vectors(grid, heads):
-    """Small-integer pooled vectors make many scores exactly equal (integer dot products are exact in
-    float32): the fused selection must break every tie like vsa_topk, for k on the compacted-candidate
-    path (k <= 128) and beyond it, up to C = 1536 (the largest the fused kernel takes)."""
-    s = vsa.Shape(1, heads, 64, grid)
+@pytest.mark.parametrize("D", [64, 128])
+def test_coarse_scores_carry_float32_accuracy(D):
+    """General float32 pooled vectors (three non-zero parts each) across several magnitudes: every score
+    within 2^-19 of the sum of |q_d k_d| from its float64 value (the float32 accumulation of D products
+    alone reaches about 2^-20 of it; a dropped or mis-split middle part would miss by about 2^-9 /
+    sqrt(D)), and the coarse output within the oracle tolerance."""
+    s = vsa.Shape(1, 4, D, (12, 16, 20))
+    _, C = vsa.shape_info(s)
+    rng = np.random.default_rng(D)
+    mag = np.exp(rng.uniform(-6, 6, size=(1, 4, C, 1))).astype(np.float32)
+    q = (rng.standard_normal((1, 4, C, D)) * mag).astype(np.float32)
+    k = (rng.standard_normal((1, 4, C, D)) * np.exp(rng.uniform(-3, 3, size=(1, 4, C, 1)))).astype(np.float32)
+    v = rng.standard_normal((1, 4, C, D)).astype(np.float32)
+    scale = 1 / math.sqrt(D)
+    scores, oc = vsa.coarse(*(torch.from_numpy(x).cuda() for x in (q, k, v)), s, scale)
+    ref = _scores_f64(q, k, scale)
+    bound = scale * np.matmul(np.abs(q.astype(np.float64)), np.swapaxes(np.abs(k.astype(np.float64)), -1, -2))
+    err = np.abs(from_dev(scores) - ref)
+    assert np.all(err <= 2.0 ** -19 * bound), float((err / bound).max())
+    r_oc = np.matmul(O.softmax_rows(ref), v.astype(np.float64))
+    assert np.linalg.norm(from_dev(oc) - r_oc) / np.linalg.norm(r_oc) <= COARSE_REL_L2
+
+
+@pytest.mark.parametrize("C_grid", [(24, 32, 52), (20, 32, 44)], ids=["C624", "C440"])
+def test_topk_every_search_path(C_grid):
+    """The selection on score rows of 440 and 624 cubes, random and tie-heavy, for k on each path of its
+    search (one or up to four keys per lane bounding the k-th largest, a compacted list of up to 128 or
+    256 candidates, the whole row): bit-exact against the oracle's top-k, and the softmax statistics
+    the same pass writes against numpy."""
+    s = vsa.Shape(1, 2, 64, C_grid)
     _, C = vsa.shape_info(s)
     rng = np.random.default_rng(C)
-    mk = lambda: torch.from_numpy(rng.integers(-2, 3, size=(1, heads, C, 64)).astype(np.float32)).cuda()
-    bars = (mk(), mk(), torch.from_numpy(rng.standard_normal((1, heads, C, 64)).astype(np.float32)).cuda())
-    ks = sorted({k for k in (1, 2, 31, 32, 33, 64, 65, 96, 128, 129, 200, C - 1, C) if 1 <= k <= C})
-    _check_coarse_topk(s, bars, 0.125, ks, f"ties C={C}")
-    # every query vector zero: all scores 0, so cubes 0..k-1 for every row
-    zero = torch.zeros_like(bars[0])
-    for k in (k for k in (1, 32, 65) if k <= C):
-        idx, _, _, _ = vsa.coarse_topk(zero, bars[1], None, s, k, 0.125, order=False)
-        assert torch.equal(idx, torch.arange(k, dtype=torch.int32, device="cuda").expand_as(idx)), k
+    shape = (1, 2, C, C)
+    arrays = [rng.standard_normal(shape).astype(np.float32), rng.integers(-3, 4, size=shape).astype(np.float32),
+              np.sort(rng.standard_normal(shape).astype(np.float32), axis=-1)]
+    for a in arrays:
+        dev_a = torch.from_numpy(a).cuda()
+        for k in (1, 2, 31, 32, 33, 64, 65, 97, 128, 129, 300, C - 1, C):
+            idx, order = vsa.topk_order(dev_a, s, k)
+            assert np.array_equal(idx.cpu().numpy(), O.topk(a.astype(np.float64), k)), k
+            assert torch.equal(idx, vsa.topk(dev_a, s, k)), k
 
 
 def _decode_steps(raw: np.ndarray, items: int, stride: int):
