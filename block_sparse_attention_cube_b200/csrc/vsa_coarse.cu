@@ -124,12 +124,6 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 constexpr int kTopM = 4;      // k <= 32 * kTopM: the k-th largest is searched in a compacted candidate list
 constexpr int kTopCand = 8;   // candidates per lane in that list (256 per row)
 
-// Hint: start moving `bytes` (a multiple of 16, 16-byte aligned) at `src` into L2.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
-                 : "memory");
-}
-
 // Writes a row's selection (every key above T, then the lowest-index keys equal to T, ascending
 // index) from keys held key j in lane j % 32, slot j / 32 of n[] (idx_of gives j), and returns the
 // row's work-order key bits (its four smallest selected cubes, 12 bits each from bit 52 down).
@@ -172,30 +166,67 @@ __device__ __forceinline__ uint64_t write_selection(const uint32_t (&n)[N], int 
 // cube's own index, so that sorting the keys puts query cubes whose selections start alike next to
 // each other (the fine stage's tiles are pairs of consecutive cubes, and a tile's steps are the
 // union of its two selections).  When `stats` is non-null, the row's maximum m and
-// 1 / sum(exp(s - m)) are written (the coarse output's softmax).  While a warp works on a row, the
-// next row it will take is prefetched into L2.
-template <int KPL>
+// 1 / sum(exp(s - m)) are written (the coarse output's softmax).
+// 16 bytes global -> shared, asynchronous (cp.async, L2 only); groups committed and awaited per thread.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(reinterpret_cast<uint64_t>(src))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// STAGED (C a multiple of 4, 16-byte aligned scores): each warp copies the next row it will take into
+// the other half of its shared-memory row buffer (cp.async) while it works on the current one, so a
+// row's loads are in flight during the previous row's selection.
+template <int KPL, bool STAGED>
 __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C, int k, const float* __restrict__ scores,
                                                             int32_t* __restrict__ idx, uint64_t* __restrict__ sig,
                                                             float2* __restrict__ stats) {
     __shared__ uint32_t cand_key_all[kThreads / 32][32 * kTopCand];
     __shared__ uint16_t cand_idx_all[kThreads / 32][32 * kTopCand];
+    extern __shared__ __align__(16) float row_buf_all[];   // STAGED: [warp][2][C] floats
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lt_mask = (1u << lane) - 1u;
     uint32_t* cand_key = cand_key_all[warp];
     uint16_t* cand_idx = cand_idx_all[warp];
+    float* row_buf = row_buf_all + static_cast<int64_t>(warp) * 2 * C;
     const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
     const int m = (k + 31) / 32;
-    const bool bulk_prefetch = (C & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
-    for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + warp; row < rows; row += warps) {
+    auto stage = [&](int64_t r, int b) {   // row r's C floats into half b, one 16-byte chunk per lane per step
+        const float* src = scores + r * C;
+        float* dst = row_buf + b * C;
+        for (int q = lane; q < C / 4; q += 32) cp_async16(dst + 4 * q, src + 4 * q);
+        cp_async_commit();
+    };
+    const int64_t first = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + warp;
+    if (STAGED && first < rows) stage(first, 0);
+    int b = 0;
+    for (int64_t row = first; row < rows; row += warps, b ^= 1) {
         const float* s = scores + row * C;
-        if (bulk_prefetch && lane == 0 && row + warps < rows)
-            prefetch_l2_bulk(s + warps * C, static_cast<uint32_t>(C) * 4u);
         uint32_t key[KPL];
+        if constexpr (STAGED) {
+            if (row + warps < rows) {
+                stage(row + warps, b ^ 1);
+                cp_async_wait<1>();   // this lane's copies of the current row have landed
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncwarp();             // ... and every lane's
+            const float* rb = row_buf + b * C;
 #pragma unroll
-        for (int i = 0; i < KPL; ++i) {
-            const int j = lane + 32 * i;
-            key[i] = j < C ? order_key(__ldcs(s + j)) : 0u;   // 0 ranks below every real score
+            for (int i = 0; i < KPL; ++i) {
+                const int j = lane + 32 * i;
+                key[i] = j < C ? order_key(rb[j]) : 0u;   // 0 ranks below every real score
+            }
+            __syncwarp();             // the buffer is free for the copy two rows ahead
+        } else {
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) {
+                const int j = lane + 32 * i;
+                key[i] = j < C ? order_key(__ldcs(s + j)) : 0u;   // 0 ranks below every real score
+            }
         }
         // the lane's largest key and its m-th largest (m <= kTopM), or its smallest real key
         uint32_t lane_max = 0u, lane_m = 0u;
@@ -388,7 +419,25 @@ cudaError_t launch_topk_reg(int64_t rows, int C, int k, const float* scores, int
     const int64_t blocks_needed = (rows + kThreads / 32 - 1) / (kThreads / 32);
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-    topk_reg_kernel<KPL><<<grid, kThreads, 0, s>>>(rows, C, k, scores, idx, sig, reinterpret_cast<float2*>(stats));
+    const bool staged = (C & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
+    if (!staged) {
+        topk_reg_kernel<KPL, false><<<grid, kThreads, 0, s>>>(rows, C, k, scores, idx, sig,
+                                                               reinterpret_cast<float2*>(stats));
+        return cudaGetLastError();
+    }
+    const size_t smem = static_cast<size_t>(kThreads / 32) * 2 * C * 4;   // <= 128 KB for C <= 2048
+    static int configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (!(dev >= 0 && dev < 64 && configured[dev])) {
+        e = cudaFuncSetAttribute(topk_reg_kernel<KPL, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(static_cast<size_t>(kThreads / 32) * 2 * (32 * KPL) * 4));
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = 1;
+    }
+    topk_reg_kernel<KPL, true><<<grid, kThreads, smem, s>>>(rows, C, k, scores, idx, sig,
+                                                             reinterpret_cast<float2*>(stats));
     return cudaGetLastError();
 }
 

@@ -254,11 +254,12 @@ coarse_scores_mma_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_
 
 // ---------------------------------------------------------------- coarse output
 // o_coarse = softmax(scores) vbar, as exp(s - m) vbar / l with each row's maximum m and sum l from
-// row_stats.  One CTA per (b, h, 128 query cubes): four converter warps (one query row per thread,
-// also the TMEM lane quarters of the epilogue) turn each 64-key slice of the row into exp(s - m),
-// split it into three bf16 parts and store them K-major with the 128-byte swizzle (the A operand);
-// a TMA warp brings the same keys' vbar parts (the B operand, MN-major); an MMA warp issues the six
-// partial products per 16-key step into one 128 x D float32 accumulator.
+// row_stats.  One CTA per (b, h, 128 query cubes): eight converter warps (two threads per query row,
+// 32 keys each; the next slice's scores are loaded while the current one is converted) turn each
+// 64-key slice of the rows into exp(s - m), split it into three bf16 parts and store them K-major
+// with the 128-byte swizzle (the A operand); a TMA warp brings the same keys' vbar parts (the B
+// operand, MN-major); an MMA warp issues the six partial products per 16-key step into one 128 x D
+// float32 accumulator, which warps 0-3 scale by 1/l and store.
 constexpr uint32_t kPvA = 3u * 128u * 128u;     // P parts of one 64-key slice: 3 x (128 rows x 128 B)
 constexpr uint32_t kPvB = 3u * 64u * 256u;      // vbar parts of 64 keys x D = 128: 3 x (2 halves x 8 KB)
 constexpr int kPvStages = 2;
@@ -269,6 +270,10 @@ enum PvBar : int { kPvBarAFull = 0, kPvBarAEmpty = 2, kPvBarBFull = 4, kPvBarBEm
                    kPvBarDrain = 9, kPvBars = 10 };
 constexpr uint32_t kPvOffMisc = kPvOffBar + 8u * kPvBars;
 constexpr uint32_t kPvSmem = kPvOffMisc + 16u + 1024u;
+constexpr int kPvConvWarps = 8;                 // warps 0-7 convert (two threads per query row); 0-3 also
+constexpr int kPvTmaWarp = 8;                   // run the epilogue (one TMEM lane quarter each)
+constexpr int kPvMmaWarp = 9;
+constexpr int kPvThreads = 320;
 
 struct PvParams {
     int C, row_tiles;
@@ -280,7 +285,7 @@ struct PvParams {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kCmThreads, 1)
+__global__ void __launch_bounds__(kPvThreads, 1)
 coarse_pv_mma_kernel(const __grid_constant__ CUtensorMap tm_v, const PvParams p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -302,7 +307,7 @@ coarse_pv_mma_kernel(const __grid_constant__ CUtensorMap tm_v, const PvParams p)
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         for (int s = 0; s < kPvStages; ++s) {
-            mbar_init(bar(kPvBarAFull + s), 4);   // one arrival per converter warp
+            mbar_init(bar(kPvBarAFull + s), kPvConvWarps);   // one arrival per converter warp
             mbar_init(bar(kPvBarAEmpty + s), 1);
             mbar_init(bar(kPvBarBFull + s), 1);
             mbar_init(bar(kPvBarBEmpty + s), 1);
@@ -312,7 +317,7 @@ coarse_pv_mma_kernel(const __grid_constant__ CUtensorMap tm_v, const PvParams p)
         fence_mbar_init();
         prefetch_tensormap(&tm_v);
     }
-    if (warp == kCmMmaWarp) {
+    if (warp == kPvMmaWarp) {
         tmem_alloc(base + kPvOffMisc, 128u);
         tmem_relinquish();
     }
@@ -326,7 +331,7 @@ coarse_pv_mma_kernel(const __grid_constant__ CUtensorMap tm_v, const PvParams p)
         }
     };
 
-    if (warp == kCmTmaWarp) {
+    if (warp == kPvTmaWarp) {
         // ------------------------------------------------------------ vbar parts
         if (lane == 0) {
             bool ok = true;
@@ -345,7 +350,7 @@ coarse_pv_mma_kernel(const __grid_constant__ CUtensorMap tm_v, const PvParams p)
                 for (int s = 0; s < kPvStages; ++s)
                     if (issued[s]) drain_wait(bar(kPvBarBFull + s), (issued[s] - 1u) & 1u);
         }
-    } else if (warp == kCmMmaWarp) {
+    } else if (warp == kPvMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);     // P K-major, vbar MN-major
@@ -380,45 +385,52 @@ coarse_pv_mma_kernel(const __grid_constant__ CUtensorMap tm_v, const PvParams p)
         }
     } else {
         // ------------------------------------------------------------ converters, then the epilogue
-        const int r = 32 * warp + lane;
+        const int r = threadIdx.x & 127, hf = threadIdx.x >> 7;   // query row, half of each 64-key slice
         const int gi = i0 + r;
         const bool real = gi < C;
         const float2 st = real ? p.stats[static_cast<int64_t>(bh) * C + gi] : make_float2(0.f, 0.f);
         const float* srow = p.scores + (static_cast<int64_t>(bh) * C + (real ? gi : 0)) * C;
+        // keys 64n + 32hf .. + 31 of the row; past C (or a padding row): -inf, whose exp is 0
+        auto load = [&](int n, float (&x)[32]) {
+            const int jb = 64 * n + 32 * hf;
+            if (real && (C & 3) == 0 && jb + 32 <= C) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 t = *reinterpret_cast<const float4*>(srow + jb + 4 * q);
+                    x[4 * q] = t.x;
+                    x[4 * q + 1] = t.y;
+                    x[4 * q + 2] = t.z;
+                    x[4 * q + 3] = t.w;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = (real && jb + e < C) ? srow[jb + e] : -INFINITY;
+            }
+        };
         bool ok = true;
+        float nxt[32];
+        load(0, nxt);
         for (int n = 0; n < slices; ++n) {
+            float cur[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+            if (n + 1 < slices) load(n + 1, nxt);
             const int slot = n % kPvStages;
             if (!(ok = __all_sync(0xffffffffu, bw.wait(bar(kPvBarAEmpty + slot), ((n / kPvStages) & 1) ^ 1)))) break;
             uint8_t* a = smem + kPvOffA + slot * kPvA + r * 128;
-            const int j0 = 64 * n;
-            const bool vec = real && (C & 3) == 0 && j0 + 64 <= C;   // whole slice in the row, 16-byte aligned
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {                 // 16-byte chunk c: keys j0 + 8c .. j0 + 8c + 7
-                float v[8];
-                if (vec) {
-                    const float4 x0 = *reinterpret_cast<const float4*>(srow + j0 + 8 * c);
-                    const float4 x1 = *reinterpret_cast<const float4*>(srow + j0 + 8 * c + 4);
-                    const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = __expf(xs[e] - st.x);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = j0 + 8 * c + e;
-                        v[e] = (real && j < C) ? __expf(srow[j] - st.x) : 0.f;
-                    }
-                }
+            for (int cq = 0; cq < 4; ++cq) {              // 16-byte chunk c = 4hf + cq: 8 keys
                 uint32_t hw[4], mw[4], lw[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     uint16_t h0, m0, l0, h1, m1, l1;
-                    split3(v[2 * e], h0, m0, l0);
-                    split3(v[2 * e + 1], h1, m1, l1);
+                    split3(__expf(cur[8 * cq + 2 * e] - st.x), h0, m0, l0);
+                    split3(__expf(cur[8 * cq + 2 * e + 1] - st.x), h1, m1, l1);
                     hw[e] = h0 | (uint32_t{h1} << 16);
                     mw[e] = m0 | (uint32_t{m1} << 16);
                     lw[e] = l0 | (uint32_t{l1} << 16);
                 }
-                const int sc = (c ^ (r & 7)) * 16;         // the 128-byte swizzle of row r
+                const int sc = ((4 * hf + cq) ^ (r & 7)) * 16;   // the 128-byte swizzle of row r
                 *reinterpret_cast<uint4*>(a + sc) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                 *reinterpret_cast<uint4*>(a + 16384 + sc) = make_uint4(mw[0], mw[1], mw[2], mw[3]);
                 *reinterpret_cast<uint4*>(a + 32768 + sc) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
@@ -427,7 +439,8 @@ coarse_pv_mma_kernel(const __grid_constant__ CUtensorMap tm_v, const PvParams p)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kPvBarAFull + slot));
         }
-        if (ok && __all_sync(0xffffffffu, bw.wait(bar(kPvBarODone), 0u))) {
+        // warps 0-3 (rows 32 w .. 32 w + 31: their TMEM lane quarter) store the result
+        if (warp < 4 && ok && __all_sync(0xffffffffu, bw.wait(bar(kPvBarODone), 0u))) {
             tc_fence_after();
             const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
             float* orow = p.o_coarse + (static_cast<int64_t>(bh) * C + (real ? gi : 0)) * D;
@@ -449,7 +462,7 @@ coarse_pv_mma_kernel(const __grid_constant__ CUtensorMap tm_v, const PvParams p)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == kCmMmaWarp) {
+    if (warp == kPvMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, 128u);
     }
@@ -594,8 +607,8 @@ cudaError_t launch_coarse_pv_mma(const Dims& d, const float* scores, const float
     }
     const int64_t grid = static_cast<int64_t>(d.B) * d.H * p.row_tiles;
     if (grid > 0x7FFFFFFFll) return cudaErrorInvalidValue;
-    if (d.D == 128) coarse_pv_mma_kernel<128><<<static_cast<unsigned>(grid), kCmThreads, kPvSmem, s>>>(tv, p);
-    else coarse_pv_mma_kernel<64><<<static_cast<unsigned>(grid), kCmThreads, kPvSmem, s>>>(tv, p);
+    if (d.D == 128) coarse_pv_mma_kernel<128><<<static_cast<unsigned>(grid), kPvThreads, kPvSmem, s>>>(tv, p);
+    else coarse_pv_mma_kernel<64><<<static_cast<unsigned>(grid), kPvThreads, kPvSmem, s>>>(tv, p);
     return cudaGetLastError();
 }
 
