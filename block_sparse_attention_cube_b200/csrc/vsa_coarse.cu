@@ -155,12 +155,13 @@ __device__ __forceinline__ uint64_t write_selection(const uint32_t (&n)[N], int 
 }
 
 // Top-k with the row held in registers (KPL keys per lane, key j in lane j % 32, slot j / 32), for
-// C <= 32 * KPL.  For k <= 128 each lane's m = ceil(k / 32) largest keys bound the k-th largest from
-// below (32 m >= k keys reach the smallest of them, lo); when at most 256 keys reach lo they are
-// compacted, with their cube indices and in index order, into a list whose count of keys >= t equals
-// the row's for every t > lo (and both reach k for t <= lo), so the k-th largest key T is built bit
-// by bit from the top over that short list, and the selection (every key above T, then the
-// lowest-index keys equal to T, ascending) is read off the same list; otherwise both run over the
+// C <= 32 * KPL.  For k <= 32 the smallest lane maximum, for k <= 128 the k-th largest among the lanes'
+// m + 1 largest keys (m = ceil(k / 32)), bounds the row's k-th largest from below (lo: at least k real
+// keys reach it); when at most 256 keys reach lo
+// they are compacted, with their cube indices and in index order, into a list whose count of keys
+// >= t equals the row's for every t > lo (and both reach k for t <= lo), so the k-th largest key T
+// is built bit by bit from the top over that short list, and the selection (every key above T, then
+// the lowest-index keys equal to T, ascending) is read off the same list; otherwise both run over the
 // whole row.  Either way the selection is topk_kernel's.  When `sig` is non-null the row's work-order
 // key is written as well: its four smallest selected cubes (12 bits each, C <= 4096) above the
 // cube's own index, so that sorting the keys puts query cubes whose selections start alike next to
@@ -228,50 +229,67 @@ __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C,
                 key[i] = j < C ? order_key(__ldcs(s + j)) : 0u;   // 0 ranks below every real score
             }
         }
-        // the lane's largest key and its m-th largest (m <= kTopM), or its smallest real key
-        uint32_t lane_max = 0u, lane_m = 0u;
-        if (m == 1) {
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) lane_max = max(lane_max, key[i]);
-            lane_m = lane_max;
-        } else if (m == 2) {
-            uint32_t second = 0u;
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) {
-                second = max(second, min(lane_max, key[i]));
-                lane_max = max(lane_max, key[i]);
-            }
-            lane_m = second;
-        } else if (m <= kTopM) {
-            uint32_t top[kTopM] = {0u, 0u, 0u, 0u};   // descending
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) {
-                uint32_t v = key[i];
-#pragma unroll
-                for (int e = 0; e < kTopM; ++e) {
-                    const uint32_t hv = max(top[e], v);
-                    v = min(top[e], v);
-                    top[e] = hv;
-                }
-            }
-            lane_max = top[0];
-            lane_m = m == 3 ? top[2] : top[3];
-        } else {
-            lane_m = 0xFFFFFFFFu;
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) {
-                lane_max = max(lane_max, key[i]);
-                if (lane + 32 * i < C) lane_m = min(lane_m, key[i]);
-            }
-        }
-        const uint32_t hi = __reduce_max_sync(0xffffffffu, lane_max);
-        const uint32_t lo = __reduce_min_sync(0xffffffffu, lane_m);
+        // lo: a lower bound of the k-th largest key.  For k <= 32: the smallest lane maximum (32 keys reach
+        // it); for k <= 32 kTopM: the k-th largest among the lanes' m + 1 largest keys (k real keys reach
+        // it); otherwise the row's smallest key.
+        uint32_t hi, lo;
         int ncand = 0x7FFFFFFF;
         if (m <= kTopM) {
+            uint32_t top[kTopM + 1] = {0u, 0u, 0u, 0u, 0u};   // the lane's m + 1 largest keys, descending
+            if (m == 1) {
+#pragma unroll
+                for (int i = 0; i < KPL; ++i) top[0] = max(top[0], key[i]);
+            } else if (m == 2) {
+#pragma unroll
+                for (int i = 0; i < KPL; ++i) {
+                    uint32_t v = key[i];
+#pragma unroll
+                    for (int e = 0; e < 3; ++e) {
+                        const uint32_t hv = max(top[e], v);
+                        v = min(top[e], v);
+                        top[e] = hv;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < KPL; ++i) {
+                    uint32_t v = key[i];
+#pragma unroll
+                    for (int e = 0; e < kTopM + 1; ++e) {
+                        const uint32_t hv = max(top[e], v);
+                        v = min(top[e], v);
+                        top[e] = hv;
+                    }
+                }
+            }
+            hi = __reduce_max_sync(0xffffffffu, top[0]);
+            if (m == 1) {
+                // k <= 32: the smallest lane maximum already leaves few candidates (a search for a tighter
+                // bound costs more than it saves)
+                lo = __reduce_min_sync(0xffffffffu, top[0]);
+            } else {
+                const uint32_t lane_last = m == 2 ? top[2] : m == 3 ? top[3] : top[4];
+                const uint32_t lo0 = __reduce_min_sync(0xffffffffu, lane_last);   // <= the bound sought
+                if (m == 2) {
+                    const uint32_t t3[3] = {top[0], top[1], top[2]};
+                    lo = kth_key<3>(t3, hi, lo0, k);
+                } else {
+                    lo = kth_key<kTopM + 1>(top, hi, lo0, k);
+                }
+            }
             uint32_t mine = 0;
 #pragma unroll
             for (int i = 0; i < KPL; ++i) mine += (lane + 32 * i < C && key[i] >= lo) ? 1u : 0u;
             ncand = static_cast<int>(__reduce_add_sync(0xffffffffu, mine));
+        } else {
+            uint32_t lane_max = 0u, lane_min = 0xFFFFFFFFu;
+#pragma unroll
+            for (int i = 0; i < KPL; ++i) {
+                lane_max = max(lane_max, key[i]);
+                if (lane + 32 * i < C) lane_min = min(lane_min, key[i]);
+            }
+            hi = __reduce_max_sync(0xffffffffu, lane_max);
+            lo = __reduce_min_sync(0xffffffffu, lane_min);
         }
         int32_t* dst = idx + row * k;
         uint64_t lex;
@@ -291,9 +309,9 @@ __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C,
             uint32_t ck[kTopCand];
 #pragma unroll
             for (int e = 0; e < kTopCand; ++e) ck[e] = lane + 32 * e < ncand ? cand_key[lane + 32 * e] : 0u;
-            const uint32_t T = ncand <= 32 * (kTopCand / 2)
-                                   ? kth_key<kTopCand / 2>(reinterpret_cast<const uint32_t(&)[kTopCand / 2]>(ck), hi, lo, k)
-                                   : kth_key<kTopCand>(ck, hi, lo, k);
+            const uint32_t T = ncand <= 64    ? kth_key<2>(reinterpret_cast<const uint32_t(&)[2]>(ck), hi, lo, k)
+                               : ncand <= 128 ? kth_key<4>(reinterpret_cast<const uint32_t(&)[4]>(ck), hi, lo, k)
+                                              : kth_key<kTopCand>(ck, hi, lo, k);
             uint32_t gt = 0;
 #pragma unroll
             for (int e = 0; e < kTopCand; ++e) gt += ck[e] > T ? 1u : 0u;
