@@ -571,8 +571,8 @@ def run_stages(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--stages", action="store_true", help="stage-by-stage times of one call (profiling case)")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS), help="with --stages")

@@ -205,6 +205,20 @@ def _compare_call(w, dev, f64, k, scale, gates=True):
             check_close(got[b, :, h], ora["out"][b, :, h], f"out[b={b},h={h}] k={k}")
 
 
+@pytest.mark.parametrize("grid,k", [((4, 4, 8400), 4), ((4, 4, 16800), 3)], ids=["C2100", "C4200"])
+def test_forward_beyond_the_register_selection(grid, k):
+    """More cubes than the register-resident selection takes (C > 2048: the shared-memory top-k kernel, the
+    work order from vsa_group, the coarse output's softmax statistics from their own pass) and than the
+    work-order sort takes (C > 4096: no grouping): the whole gated call against the oracle."""
+    w = synth.custom_workload(f"long_{grid[2]}", 1, 1, 64, grid, k, field=True, wid=95 + grid[2] // 8400)
+    x = synth.make_inputs(w)
+    dev = {n: to_dev(v) for n, v in x.items()}
+    f64 = {n: O.bf16_to_f64(v) for n, v in x.items()}
+    _, C = vsa.shape_info(_shape(w))
+    assert C > 2048
+    _compare_call(w, dev, f64, k, 1 / math.sqrt(64))
+
+
 def test_forward_matches_oracle(case):
     w, _, dev, f64 = case
     _compare_call(w, dev, f64, w.topk, 1 / math.sqrt(w.head_dim))
