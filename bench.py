@@ -19,11 +19,12 @@ on the host cores.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
     python bench.py --stages [--workload NAME] [--iters I] [--dense-too] [--staged]
+    python bench.py --calls [--workload NAME] [--iters I]
 
 `--impl reference` times the fp64 CPU oracle, one whole head per step, on
 rank 0 only.  `--stages` runs the launches of one call stage by stage on a
-named workload and prints their median times (a small fixed case to put
-under a profiler).
+named workload and prints their median times, and `--calls` runs whole
+forward calls on it (small fixed cases to put under a profiler).
 """
 from __future__ import annotations
 
@@ -568,6 +569,34 @@ def run_stages(args):
     print(json.dumps({"workload": w.name, "iters": args.iters, "staged": args.staged, "ms": ms}), flush=True)
 
 
+def run_calls(args):
+    """`--iters` whole forward calls on a named workload (gated when it selects), each timed with events:
+    a fixed case whose kernels a profiler can list one by one."""
+    import torch
+
+    import block_sparse_attention_cube_b200 as vsa
+    w = synth.WORKLOADS[args.workload]
+    x = synth.make_inputs(w)
+    d = {k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).cuda() for k, v in x.items()}
+    s = vsa.Shape(w.batch, w.heads, w.head_dim, w.grid)
+    _, C = vsa.shape_info(s)
+    gated = w.topk < C
+    ws = vsa.alloc_workspace(s, w.topk)
+    out = torch.empty_like(d["q"])
+    stream = torch.cuda.current_stream()
+    ms = []
+    for _ in range(args.iters):
+        e0, e1 = _events(torch, 2)
+        e0.record(stream)
+        vsa.forward(d["q"], d["k"], d["v"], s, w.topk, None, d["g_coarse"] if gated else None,
+                    d["g_fine"] if gated else None, workspace=ws, out=out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(round(e0.elapsed_time(e1), 4))
+    vsa.device_status()
+    print(json.dumps({"workload": w.name, "calls": args.iters, "ms": ms}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -575,6 +604,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--stages", action="store_true", help="stage-by-stage times of one call (profiling case)")
+    ap.add_argument("--calls", action="store_true", help="--iters whole forward calls on --workload (profiling case)")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(synth.WORKLOADS), help="with --stages")
     ap.add_argument("--iters", type=int, default=3, help="with --stages")
     ap.add_argument("--dense-too", action="store_true", help="with --stages: add a dense fine-stage launch")
@@ -582,6 +612,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.stages:
         run_stages(args)
+        return 0
+    if args.calls:
+        run_calls(args)
         return 0
     if args.warmup < 3 and args.impl == "cuda":
         ap.error("at least 3 warm-up steps")
