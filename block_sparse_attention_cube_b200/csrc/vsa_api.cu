@@ -272,21 +272,21 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
     const bool sparse = topk < d.C;
     const Carve c = carve(d, topk, gc != nullptr, ws);
     const char* why = nullptr;
-    bool have_stats = false;
     if (sparse || gc != nullptr) {
         // pooled q, k, v straight into their bf16 parts, then the scores on the tensor cores
         const uint16_t* pin[3] = {q, k, v};
         uint16_t* parts[3] = {c.qp, c.kp, c.vp};
         VSA_CUDA(launch_pool_tokens(d, pin, nullptr, 3, s, parts), "pool launch");
-        const cudaError_t e = launch_coarse_scores_mma(d, c.qp, c.kp, scale, c.scores, s, &why);
+        // the softmax statistics of the score rows are needed only for the coarse output
+        const cudaError_t e =
+            launch_coarse_scores_mma(d, c.qp, c.kp, scale, c.scores, gc != nullptr ? c.stats : nullptr, s, &why);
         if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "coarse launch");
     }
     const int32_t* order = nullptr;
     if (sparse) {
         if (d.C <= kTopkRegMaxC && d.C <= kGroupMaxC) {
-            // one pass over the scores gives the selection, the work-order keys and the softmax statistics
-            VSA_CUDA(launch_topk_sig(d, c.scores, topk, c.idx, c.sig, s, c.stats), "topk launch");
-            have_stats = true;
+            // one pass over the scores gives the selection and the work-order keys
+            VSA_CUDA(launch_topk_sig(d, c.scores, topk, c.idx, c.sig, s), "topk launch");
             VSA_CUDA(launch_group_sort(d, c.sig, c.order, s), "group launch");
             order = c.order;
         } else {
@@ -299,7 +299,6 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
     }
     // the coarse output (softmax(scores) x V-bar) is used only by the merge, and only with a coarse gate
     if (gc != nullptr) {
-        if (!have_stats) VSA_CUDA(launch_row_stats(d, c.scores, c.stats, s), "row stats launch");
         const cudaError_t e = launch_coarse_pv_mma(d, c.scores, c.stats, c.vp, c.oc, s, &why);
         if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "coarse launch");
     }
@@ -481,13 +480,12 @@ vsa_status vsa_coarse(const vsa_shape* shape, const float* qbar, const float* kb
     uint16_t* kp = reinterpret_cast<uint16_t*>(w + up(parts_bytes(d)));
     uint16_t* vp = reinterpret_cast<uint16_t*>(w + 2 * up(parts_bytes(d)));
     float* stats = reinterpret_cast<float*>(w + 3 * up(parts_bytes(d)));
-    VSA_CUDA(launch_split_parts(d, qbar, qp, s), "split launch");
-    VSA_CUDA(launch_split_parts(d, kbar, kp, s), "split launch");
-    VSA_CUDA(launch_split_parts(d, vbar, vp, s), "split launch");
+    const float* xin[3] = {qbar, kbar, vbar};
+    uint16_t* pout[3] = {qp, kp, vp};
+    VSA_CUDA(launch_split_parts(d, xin, pout, 3, s), "split launch");
     const char* why = nullptr;
-    cudaError_t e = launch_coarse_scores_mma(d, qp, kp, scale, scores, s, &why);
+    cudaError_t e = launch_coarse_scores_mma(d, qp, kp, scale, scores, stats, s, &why);
     if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "coarse launch");
-    VSA_CUDA(launch_row_stats(d, scores, stats, s), "row stats launch");
     e = launch_coarse_pv_mma(d, scores, stats, vp, o_coarse, s, &why);
     if (e != cudaSuccess) return why ? fail(VSA_ERR_CUDA, "%s", why) : cuda_fail(e, "coarse launch");
     return VSA_OK;

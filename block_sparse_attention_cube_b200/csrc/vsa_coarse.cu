@@ -166,8 +166,7 @@ __device__ __forceinline__ uint64_t write_selection(const uint32_t (&n)[N], int 
 // key is written as well: its four smallest selected cubes (12 bits each, C <= 4096) above the
 // cube's own index, so that sorting the keys puts query cubes whose selections start alike next to
 // each other (the fine stage's tiles are pairs of consecutive cubes, and a tile's steps are the
-// union of its two selections).  When `stats` is non-null, the row's maximum m and
-// 1 / sum(exp(s - m)) are written (the coarse output's softmax).
+// union of its two selections).
 // 16 bytes global -> shared, asynchronous (cp.async, L2 only); groups committed and awaited per thread.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
@@ -183,8 +182,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // row's loads are in flight during the previous row's selection.
 template <int KPL, bool STAGED>
 __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C, int k, const float* __restrict__ scores,
-                                                            int32_t* __restrict__ idx, uint64_t* __restrict__ sig,
-                                                            float2* __restrict__ stats) {
+                                                            int32_t* __restrict__ idx, uint64_t* __restrict__ sig) {
     __shared__ uint32_t cand_key_all[kThreads / 32][32 * kTopCand];
     __shared__ uint16_t cand_idx_all[kThreads / 32][32 * kTopCand];
     extern __shared__ __align__(16) float row_buf_all[];   // STAGED: [warp][2][C] floats
@@ -328,17 +326,6 @@ __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C,
             lex = write_selection<KPL>(key, C, T, need_eq, dst, [&](int i) { return lane + 32 * i; });
         }
         if (sig != nullptr && lane == 0) sig[row] = lex | static_cast<uint64_t>(row % C);
-        if (stats != nullptr) {
-            // the keys decode back to the scores exactly (-0 as +0)
-            const float mx = key_value(hi);
-            float l = 0.f;
-#pragma unroll
-            for (int i = 0; i < KPL; ++i)
-                if (lane + 32 * i < C) l += __expf(key_value(key[i]) - mx);
-#pragma unroll
-            for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-            if (lane == 0) stats[row] = make_float2(mx, 1.0f / l);
-        }
     }
 }
 
@@ -433,14 +420,13 @@ namespace {
 // Register-resident selection for C <= 2048 (a warp holds the row, KPL keys per lane).
 template <int KPL>
 cudaError_t launch_topk_reg(int64_t rows, int C, int k, const float* scores, int32_t* idx, uint64_t* sig,
-                            float* stats, cudaStream_t s) {
+                            cudaStream_t s) {
     const int64_t blocks_needed = (rows + kThreads / 32 - 1) / (kThreads / 32);
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     const int grid = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
     const bool staged = (C & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
     if (!staged) {
-        topk_reg_kernel<KPL, false><<<grid, kThreads, 0, s>>>(rows, C, k, scores, idx, sig,
-                                                               reinterpret_cast<float2*>(stats));
+        topk_reg_kernel<KPL, false><<<grid, kThreads, 0, s>>>(rows, C, k, scores, idx, sig);
         return cudaGetLastError();
     }
     const size_t smem = static_cast<size_t>(kThreads / 32) * 2 * C * 4;   // <= 128 KB for C <= 2048
@@ -454,32 +440,31 @@ cudaError_t launch_topk_reg(int64_t rows, int C, int k, const float* scores, int
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev] = 1;
     }
-    topk_reg_kernel<KPL, true><<<grid, kThreads, smem, s>>>(rows, C, k, scores, idx, sig,
-                                                             reinterpret_cast<float2*>(stats));
+    topk_reg_kernel<KPL, true><<<grid, kThreads, smem, s>>>(rows, C, k, scores, idx, sig);
     return cudaGetLastError();
 }
 
-cudaError_t topk_reg_dispatch(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, float* stats,
+cudaError_t topk_reg_dispatch(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig,
                               cudaStream_t s) {
     const int64_t rows = static_cast<int64_t>(d.B) * d.H * d.C;
     const int kpl = (d.C + 31) / 32;
-    if (kpl <= 4) return launch_topk_reg<4>(rows, d.C, k, scores, idx, sig, stats, s);
-    if (kpl <= 8) return launch_topk_reg<8>(rows, d.C, k, scores, idx, sig, stats, s);
-    if (kpl <= 12) return launch_topk_reg<12>(rows, d.C, k, scores, idx, sig, stats, s);
-    if (kpl <= 16) return launch_topk_reg<16>(rows, d.C, k, scores, idx, sig, stats, s);
-    if (kpl <= 20) return launch_topk_reg<20>(rows, d.C, k, scores, idx, sig, stats, s);
-    if (kpl <= 24) return launch_topk_reg<24>(rows, d.C, k, scores, idx, sig, stats, s);
-    if (kpl <= 32) return launch_topk_reg<32>(rows, d.C, k, scores, idx, sig, stats, s);
-    if (kpl <= 40) return launch_topk_reg<40>(rows, d.C, k, scores, idx, sig, stats, s);
-    if (kpl <= 48) return launch_topk_reg<48>(rows, d.C, k, scores, idx, sig, stats, s);
-    return launch_topk_reg<64>(rows, d.C, k, scores, idx, sig, stats, s);
+    if (kpl <= 4) return launch_topk_reg<4>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 8) return launch_topk_reg<8>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 12) return launch_topk_reg<12>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 16) return launch_topk_reg<16>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 20) return launch_topk_reg<20>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 24) return launch_topk_reg<24>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 32) return launch_topk_reg<32>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 40) return launch_topk_reg<40>(rows, d.C, k, scores, idx, sig, s);
+    if (kpl <= 48) return launch_topk_reg<48>(rows, d.C, k, scores, idx, sig, s);
+    return launch_topk_reg<64>(rows, d.C, k, scores, idx, sig, s);
 }
 
 }  // namespace
 
 cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx, cudaStream_t s) {
     if (d.C > kTopkMaxC) return cudaErrorInvalidValue;
-    if (d.C <= kTopkRegMaxC) return topk_reg_dispatch(d, scores, k, idx, nullptr, nullptr, s);
+    if (d.C <= kTopkRegMaxC) return topk_reg_dispatch(d, scores, k, idx, nullptr, s);
     const int64_t rows = static_cast<int64_t>(d.B) * d.H * d.C;
     const int wpb = topk_warps_per_block(d.C);
     const size_t smem = static_cast<size_t>(wpb) * d.C * 4;
@@ -495,10 +480,9 @@ cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx,
     return cudaGetLastError();
 }
 
-cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s,
-                            float* stats) {
+cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s) {
     if (d.C > kTopkRegMaxC) return cudaErrorInvalidValue;
-    return topk_reg_dispatch(d, scores, k, idx, sig, stats, s);
+    return topk_reg_dispatch(d, scores, k, idx, sig, s);
 }
 
 cudaError_t launch_group_sort(const Dims& d, const uint64_t* sig, int32_t* order, cudaStream_t s) {

@@ -52,9 +52,7 @@ cudaError_t launch_topk(const Dims& d, const float* scores, int k, int32_t* idx,
 // also emit each row's work-order signature (uint64 [B, H, C]) in the same
 // pass, and launch_group_sort turns those into the order launch_group gives.
 constexpr int kTopkRegMaxC = 2048;
-// (stats, when non-null: [B, H, C] float2 of each row's maximum and 1 / sum(exp(s - maximum)))
-cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s,
-                            float* stats = nullptr);
+cudaError_t launch_topk_sig(const Dims& d, const float* scores, int k, int32_t* idx, uint64_t* sig, cudaStream_t s);
 
 // Work order of the fine stage from the coarse scores (C <= kGroupMaxC).
 constexpr int kGroupMaxC = 4096;
@@ -134,15 +132,16 @@ cudaError_t launch_pool_tokens(const Dims& d, const uint16_t* const* x, float* c
                                cudaStream_t s, uint16_t* const* parts = nullptr);
 
 // The coarse stage on the tensor cores: float32 pooled vectors carried as three bf16 parts.
-// launch_split_parts: float32 [B, H, C, D] -> parts [3][B*H][C][D] (split_parts_elems(d) uint16).
+// launch_split_parts: count (1-3) tensors, float32 [B, H, C, D] -> parts [3][B*H][C][D]
+// (split_parts_elems(d) uint16 each), in one launch.
 size_t split_parts_elems(const Dims& d);
-cudaError_t launch_split_parts(const Dims& d, const float* x, uint16_t* parts, cudaStream_t s);
+cudaError_t launch_split_parts(const Dims& d, const float* const* x, uint16_t* const* parts, int count,
+                               cudaStream_t s);
 // scores [B, H, C, C] = scale * qbar kbar^T from the parts of qbar and kbar (six partial products per
-// channel step); *why set when a tensor map cannot be encoded.
+// channel step), and, when stats is non-null, stats [B, H, C] float2: each score row's maximum m and
+// 1 / sum(exp(s - m)); *why set when a tensor map cannot be encoded.
 cudaError_t launch_coarse_scores_mma(const Dims& d, const uint16_t* q_parts, const uint16_t* k_parts, float scale,
-                                     float* scores, cudaStream_t s, const char** why);
-// stats [B, H, C] float2: each score row's maximum m and 1 / sum(exp(s - m)).
-cudaError_t launch_row_stats(const Dims& d, const float* scores, float* stats, cudaStream_t s);
+                                     float* scores, float* stats, cudaStream_t s, const char** why);
 // o_coarse [B, H, C, D] = softmax(scores) vbar from the row statistics and the parts of vbar.
 cudaError_t launch_coarse_pv_mma(const Dims& d, const float* scores, const float* stats, const uint16_t* v_parts,
                                  float* o_coarse, cudaStream_t s, const char** why);

@@ -247,11 +247,23 @@ __global__ void __launch_bounds__(kPoolThreads) pool_tokens_kernel(Dims d, PoolI
         store_parts8(mean, parts_t, static_cast<int64_t>(d.B) * d.H * d.C * D, (bh * d.C + c) * D + j * 8);
 }
 
-// float32 [rows, D] -> three bf16 parts [3][rows][D] (the split of pool_tokens_kernel's means)
-__global__ void __launch_bounds__(kBlock) split_parts_kernel(int64_t groups, const float* __restrict__ x,
-                                                              uint16_t* __restrict__ parts) {
-    for (int64_t g = static_cast<int64_t>(blockIdx.x) * kBlock + threadIdx.x; g < groups;
-         g += static_cast<int64_t>(gridDim.x) * kBlock) {
+// Up to three tensors in one launch: float32 [rows, D] -> three bf16 parts [3][rows][D] each (the
+// split of pool_tokens_kernel's means).
+struct SplitIO {
+    const float* x[3];
+    uint16_t* parts[3];
+    int count;
+};
+
+__global__ void __launch_bounds__(kBlock) split_parts_kernel(int64_t groups, const SplitIO io) {
+    const int64_t total = groups * io.count;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kBlock + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * kBlock) {
+        const int t = static_cast<int>(i / groups);
+        const int64_t g = i - t * groups;
+        // pointers chosen by value: a runtime index into the parameter arrays would go through local memory
+        const float* x = t == 0 ? io.x[0] : t == 1 ? io.x[1] : io.x[2];
+        uint16_t* parts = t == 0 ? io.parts[0] : t == 1 ? io.parts[1] : io.parts[2];
         const float4 a = __ldg(reinterpret_cast<const float4*>(x) + 2 * g);
         const float4 b = __ldg(reinterpret_cast<const float4*>(x) + 2 * g + 1);
         const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -338,10 +350,18 @@ cudaError_t launch_pool(const Dims& d, const uint16_t* const* xt, float* const* 
     return cudaGetLastError();
 }
 
-cudaError_t launch_split_parts(const Dims& d, const float* x, uint16_t* parts, cudaStream_t s) {
+cudaError_t launch_split_parts(const Dims& d, const float* const* x, uint16_t* const* parts, int count,
+                               cudaStream_t s) {
+    if (count < 1 || count > 3) return cudaErrorInvalidValue;
+    SplitIO io{};
+    for (int t = 0; t < count; ++t) {
+        io.x[t] = x[t];
+        io.parts[t] = parts[t];
+    }
+    io.count = count;
     const int64_t groups = static_cast<int64_t>(d.B) * d.H * d.C * d.D / 8;
-    const int grid = grid_for((groups + kBlock - 1) / kBlock, 8);
-    split_parts_kernel<<<grid, kBlock, 0, s>>>(groups, x, parts);
+    const int grid = grid_for((groups * count + kBlock - 1) / kBlock, 8);
+    split_parts_kernel<<<grid, kBlock, 0, s>>>(groups, io);
     return cudaGetLastError();
 }
 

@@ -612,12 +612,15 @@ def _scores_f64(qb: np.ndarray, kb: np.ndarray, scale: float) -> np.ndarray:
 
 
 @pytest.mark.parametrize("B,H,D,grid", [(1, 3, 128, (8, 16, 16)), (2, 2, 64, (9, 6, 5)), (1, 2, 128, (21, 30, 52)),
-                                        (1, 1, 128, (3, 2, 4)), (1, 2, 64, (24, 32, 28))],
-                         ids=["C32", "B2_d64_C12", "C624", "C1", "d64_C336"])
+                                        (1, 1, 128, (3, 2, 4)), (1, 2, 64, (24, 32, 28)), (1, 2, 128, (20, 28, 36)),
+                                        (2, 1, 64, (5, 9, 9))],
+                         ids=["C32", "B2_d64_C12", "C624", "C1", "d64_C336", "C315", "B2_d64_C18"])
 def test_coarse_scores_exact_on_small_integers(B, H, D, grid):
     """Pooled vectors of small integers: every bf16 part but the first is zero and every dot product is
     an integer below 2^24, so the split tensor-core product must equal the exact scores bit for bit (a
-    check of the operand layout, the parts, the six partial products and the row/column tails)."""
+    check of the operand layout, the parts, the six partial products and the row/column tails).  C a
+    multiple of 4 takes the copy-engine paths (scores stored and read back by TMA), C = 1, 315 and 18
+    the per-thread loads and stores."""
     s = vsa.Shape(B, H, D, grid)
     _, C = vsa.shape_info(s)
     rng = np.random.default_rng(C + D)
@@ -630,15 +633,16 @@ def test_coarse_scores_exact_on_small_integers(B, H, D, grid):
     assert np.linalg.norm(from_dev(oc) - r_oc) / np.linalg.norm(r_oc) <= COARSE_REL_L2
 
 
+@pytest.mark.parametrize("grid", [(12, 16, 20), (20, 28, 36)], ids=["C60", "C315"])
 @pytest.mark.parametrize("D", [64, 128])
-def test_coarse_scores_carry_float32_accuracy(D):
+def test_coarse_scores_carry_float32_accuracy(D, grid):
     """General float32 pooled vectors (three non-zero parts each) across several magnitudes: every score
     within 2^-19 of the sum of |q_d k_d| from its float64 value (the float32 accumulation of D products
     alone reaches about 2^-20 of it; a dropped or mis-split middle part would miss by about 2^-9 /
     sqrt(D)), and the coarse output within the oracle tolerance."""
-    s = vsa.Shape(1, 4, D, (12, 16, 20))
+    s = vsa.Shape(1, 4, D, grid)
     _, C = vsa.shape_info(s)
-    rng = np.random.default_rng(D)
+    rng = np.random.default_rng(D + C)
     mag = np.exp(rng.uniform(-6, 6, size=(1, 4, C, 1))).astype(np.float32)
     q = (rng.standard_normal((1, 4, C, D)) * mag).astype(np.float32)
     k = (rng.standard_normal((1, 4, C, D)) * np.exp(rng.uniform(-3, 3, size=(1, 4, C, 1)))).astype(np.float32)
@@ -657,8 +661,7 @@ def test_coarse_scores_carry_float32_accuracy(D):
 def test_topk_every_search_path(C_grid):
     """The selection on score rows of 440 and 624 cubes, random and tie-heavy, for k on each path of its
     search (one or up to four keys per lane bounding the k-th largest, a compacted list of up to 128 or
-    256 candidates, the whole row): bit-exact against the oracle's top-k, and the softmax statistics
-    the same pass writes against numpy."""
+    256 candidates, the whole row): bit-exact against the oracle's top-k."""
     s = vsa.Shape(1, 2, 64, C_grid)
     _, C = vsa.shape_info(s)
     rng = np.random.default_rng(C)
