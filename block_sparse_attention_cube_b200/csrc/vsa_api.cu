@@ -206,7 +206,7 @@ Carve carve(const Dims& d, int k, bool coarse_gate, void* ws) {
         if (d.C <= kTopkRegMaxC) c.sig = reinterpret_cast<uint64_t*>(take(2 * order_bytes(d)));
         if (schedule_supported(d, k)) c.steps = take(schedule_bytes(d, k));
     }
-    c.overflow = reinterpret_cast<int*>(take(sizeof(int)));
+    c.overflow = reinterpret_cast<int*>(take(2 * sizeof(int)));
     c.bytes = off > kAlign ? off : kAlign;
     return c;
 }
@@ -707,7 +707,7 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
                             {steps, steps ? schedule_bytes(d, topk) : 0, "steps"},
                             {o_coarse, o_coarse ? pooled_bytes(d) : 0, "o_coarse"},
                             {g_coarse, g_coarse ? gb : 0, "g_coarse"}, {g_fine, g_fine ? gb : 0, "g_fine"}},
-                           {{out, tb, "out"}, {overflow, steps ? sizeof(int32_t) : 0, "overflow"}}));
+                           {{out, tb, "out"}, {overflow, steps ? 2 * sizeof(int32_t) : 0, "overflow"}}));
     VSA_TRY(check_device());
     return run_fine_fused(d, q, k, v, idx, topk, order, steps, scale, o_coarse, g_coarse, g_fine, out,
                           steps ? overflow : nullptr, as_stream(stream));

@@ -156,6 +156,7 @@ struct FineParams {
     int* status;
     uint64_t limit_ns;
     int* overflow;          // fine_tile_kernel: set to 1 when a probability bound was exceeded (or nullptr)
+    int* work;              // fine_tile_kernel: item counter, zero at launch (nullptr: every gridDim.x-th item)
     const int* run_if;      // fine_kernel: return at once unless *run_if != 0 (or nullptr: always run)
 };
 
@@ -959,6 +960,16 @@ fine_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
 // before item n, until the epilogue has read item n - 2's row sums (SetFree):
 // no group runs more than one item ahead of the epilogue.
 //
+// Work items are claimed, not dealt: the Q/K producer takes the CTA's first
+// item as blockIdx.x and every later one from a counter in the caller's
+// memory (the second word of the overflow pair), then publishes each index in
+// a four-slot shared-memory ring that every other role reads.  Items differ in
+// length (the union of two selections: 16 to 32 steps at top-k 32), and a fixed
+// deal of every 148th item left the longest CTA about 4% behind the mean at
+// Wan 480p; claimed in order, items still run about 148 apart, so the K and V
+// cubes that neighbouring query cubes share stay in L2.  The next index is
+// claimed one item early, so its atomic's latency is hidden.
+//
 // A probability above 2^64 (a later score far above the first
 // maximum) or a non-finite sum raises the overflow word, and the caller then
 // runs fine_kernel, whose online maximum is rescaled per step, over the whole
@@ -978,7 +989,9 @@ constexpr uint32_t kTOffV = kTOffK + kTKStages * kKVBytes;       // [kTVStages]
 constexpr uint32_t kTOffM = kTOffV + kTVStages * kKVBytes;       // [2 items][128] each row's fixed maximum
 constexpr uint32_t kTOffL = kTOffM + 2 * 128 * 4;                // [2 items][kTBufs][128] each group's row sums
 constexpr uint32_t kTOffOC = kTOffL + 2 * kTBufs * 128 * 4;      // [4 epilogue warps][128] coarse outputs
-constexpr uint32_t kTOffBar = kTOffOC + 4 * 128 * 4;
+constexpr int kTItemRing = 4;                                    // items published ahead of the last reader
+constexpr uint32_t kTOffItem = kTOffOC + 4 * 128 * 4;            // [kTItemRing] int32 item indices
+constexpr uint32_t kTOffBar = kTOffItem + kTItemRing * 4;
 constexpr int kTBarQFull = 0;
 constexpr int kTBarQEmpty = 1;
 constexpr int kTBarKFull = 2;                                    // [kTKStages]
@@ -994,7 +1007,12 @@ constexpr int kTBarOFree = kTBarEpi + 2;                         // four arrival
 constexpr int kTBarODone = kTBarOFree + 1;                       // the item's last PV complete (one commit per item)
 constexpr int kTBarSetFree = kTBarODone + 1;                     // [2 items], four arrivals: the set is read
 constexpr int kTBarDrain = kTBarSetFree + 2;                     // [2 issuers]
-constexpr int kTNumBars = kTBarDrain + 2;
+constexpr int kTBarItemFull = kTBarDrain + 2;                    // [kTItemRing]
+constexpr int kTBarItemEmpty = kTBarItemFull + kTItemRing;       // [kTItemRing], kTItemReaders arrivals
+constexpr int kTNumBars = kTBarItemEmpty + kTItemRing;
+// readers of each published item: the S and PV issuers, the V producer, the twelve softmax warps and
+// the four epilogue warps
+constexpr uint32_t kTItemReaders = 1 + 1 + 1 + 12 + 4;
 constexpr uint32_t kTOffMisc = kTOffBar + kTNumBars * 8;         // tmem slot (4 B) + abort flag (4 B)
 constexpr uint32_t kTSmemBytes = kTOffMisc + 16 + 1024;
 constexpr uint32_t kTColO = 384;
@@ -1055,6 +1073,10 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_init(bar(kTBarSetFree + 1), 4);
         mbar_init(bar(kTBarDrain + 0), 1);
         mbar_init(bar(kTBarDrain + 1), 1);
+        for (int i = 0; i < kTItemRing; ++i) {
+            mbar_init(bar(kTBarItemFull + i), 1);
+            mbar_init(bar(kTBarItemEmpty + i), kTItemReaders);
+        }
         fence_mbar_init();
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
@@ -1079,14 +1101,44 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     constexpr int kBoxes = D == 128 ? 4 : 2;
     constexpr unsigned kBoxMask = (1u << kBoxes) - 1u;
+    volatile int32_t* item_ring = reinterpret_cast<volatile int32_t*>(smem + kTOffItem);
+    // The n-th item of this CTA for the lanes of `mask` (lane 0 among them): every lane waits for it
+    // and reads it, lane 0 then releases the slot.  -1: no item is left.
+    auto take_item = [&](int n, unsigned mask, int64_t& it) -> bool {
+        const int slot = n % kTItemRing;
+        const uint32_t par = static_cast<uint32_t>(n / kTItemRing) & 1u;
+        if (!__all_sync(mask, bw.wait(bar(kTBarItemFull + slot), par))) return false;
+        it = item_ring[slot];
+        __syncwarp(mask);
+        if (lane == 0) mbar_arrive(bar(kTBarItemEmpty + slot));   // release: the index is read
+        return true;
+    };
     if (warp == kTTmaWarp) {
         // ------------------------------------------------------------ Q and K producer (lane i: box i)
         if (lane < kBoxes) {
             uint32_t q_issued = 0, k_issued[kTKStages] = {};
             RingPos kp{0, 0};
-            int n_item = 0;
             bool ok = true;
-            for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
+            int64_t claimed = blockIdx.x;   // lane 0: the item this CTA takes next
+            for (int n_item = 0; ok; ++n_item) {
+                // publish the item (or -1 once none is left) and claim the one after it
+                int32_t it32 = -1;
+                if (lane == 0) {
+                    const int slot = n_item % kTItemRing;
+                    ok = bw.wait(bar(kTBarItemEmpty + slot), (static_cast<uint32_t>(n_item / kTItemRing) & 1u) ^ 1u);
+                    if (ok) {
+                        it32 = claimed < p.items ? static_cast<int32_t>(claimed) : -1;
+                        item_ring[slot] = it32;
+                        mbar_arrive(bar(kTBarItemFull + slot));   // release: the index is visible
+                        if (it32 >= 0)
+                            claimed = p.work != nullptr ? static_cast<int64_t>(gridDim.x) + atomicAdd(p.work, 1)
+                                                        : claimed + gridDim.x;
+                    }
+                }
+                ok = __shfl_sync(kBoxMask, ok ? 1 : 0, 0) != 0;
+                it32 = __shfl_sync(kBoxMask, it32, 0);
+                if (!ok || it32 < 0) break;
+                const int64_t it = it32;
                 const Item item = decode_item(it, p);
                 auto load_pair = [&](const CUtensorMap* m, uint32_t dst, int ja, int jb, uint32_t b) {
                     __syncwarp(kBoxMask);   // lane 0's expect_tx first
@@ -1124,9 +1176,10 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const uint64_t fix_k = smem_desc_sw128(0, 16u, 1024u);         // K-major, 8-row groups 1 KB apart
             RingPos kp{0, 0};
             uint32_t uses[kTBufs] = {0u, 0u, 0u};   // S issued into each buffer so far
-            int n_item = 0;
             bool ok = true, issued_any = false;
-            for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
+            for (int n_item = 0; ok; ++n_item) {
+                int64_t it;
+                if (!(ok = take_item(n_item, 1u, it)) || it < 0) break;
                 const uint32_t present = decode_item(it, p).present;
                 if (!(ok = bw.wait(bar(kTBarQFull), n_item & 1))) break;
                 for (int s = 0;; ++s) {
@@ -1165,9 +1218,10 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const uint64_t fix_v = smem_desc_sw128(0, 16384u, 1024u);      // MN-major, d halves 16 KB apart
             RingPos vp{0, 0};
             uint32_t waits[kTBufs] = {0u, 0u, 0u};   // P-full phases consumed per buffer
-            int n_item = 0;
             bool ok = true, issued_any = false;
-            for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
+            for (int n_item = 0; ok; ++n_item) {
+                int64_t it;
+                if (!(ok = take_item(n_item, 1u, it)) || it < 0) break;
                 const uint32_t present = decode_item(it, p).present;
                 for (int s = 0;; ++s) {
                     const StepRec r = tile_step(p, it, s, present);
@@ -1205,7 +1259,9 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             uint32_t v_issued[kTVStages] = {};
             RingPos vp{0, 0};
             bool ok = true;
-            for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x) {
+            for (int n_item = 0; ok; ++n_item) {
+                int64_t it;
+                if (!(ok = take_item(n_item, kBoxMask, it)) || it < 0) break;
                 const Item item = decode_item(it, p);
                 for (int s = 0;; ++s) {
                     const StepRec r = tile_step(p, it, s, item.present);
@@ -1270,8 +1326,9 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             return tok;
         };
-        int n_item = 0;
-        for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
+        for (int n_item = 0; ok; ++n_item) {
+            int64_t it;
+            if (!(ok = take_item(n_item, 0xffffffffu, it)) || it < 0) break;
             const Item item = decode_item(it, p);
             const int ip = n_item & 1;
             const uint32_t ipar = static_cast<uint32_t>(n_item >> 1) & 1u;
@@ -1302,8 +1359,14 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     ocr = oc_w;
                 }
             }
-            const int64_t nxt = it + gridDim.x;
-            if (nxt < p.items && q == 0 && lane < 3) {
+            // the next item, when it is already published (a look at its slot, no wait)
+            int64_t nxt = -1;
+            {
+                const int ns = (n_item + 1) % kTItemRing;
+                if (mbar_try_wait(bar(kTBarItemFull + ns), static_cast<uint32_t>((n_item + 1) / kTItemRing) & 1u))
+                    nxt = item_ring[ns];
+            }
+            if (nxt >= 0 && nxt < p.items && q == 0 && lane < 3) {
                 if (lane < 2 && p.steps != nullptr && 128 * lane < 8 * p.steps_stride)
                     prefetch_l1(reinterpret_cast<const uint8_t*>(p.steps + nxt * p.steps_stride) + 128 * lane);
                 if (lane == 2 && p.order != nullptr) {
@@ -1380,8 +1443,9 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const bool mine = bw.wait(b, par);
             return __all_sync(0xffffffffu, mine);
         };
-        int n_item = 0;
-        for (int64_t it = blockIdx.x; ok && it < p.items; it += gridDim.x, ++n_item) {
+        for (int n_item = 0; ok; ++n_item) {
+            int64_t it;
+            if (!(ok = take_item(n_item, 0xffffffffu, it)) || it < 0) break;
             const Item item = decode_item(it, p);
             // The groups go on to the next item while the epilogue warps write this one, so the
             // maxima, the row sums and their barriers alternate between two sets by item parity.
@@ -1869,7 +1933,8 @@ cudaError_t launch_fine(const Dims& d, const FineArgs& a, cudaStream_t s, const 
             return cudaErrorInvalidValue;
         }
         pt.overflow = ovf;
-        cudaError_t e = cudaMemsetAsync(ovf, 0, sizeof(int), s);
+        pt.work = ovf + 1;   // the item counter beside the overflow flag
+        cudaError_t e = cudaMemsetAsync(ovf, 0, 2 * sizeof(int), s);
         if (e != cudaSuccess) return e;
         const int gt = static_cast<int>(pt.items < sm_count() ? pt.items : sm_count());
         if (gt > 0) {

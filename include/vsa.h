@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define VSA_ABI_VERSION 2
+#define VSA_ABI_VERSION 3
 
 typedef uint16_t vsa_bf16;
 typedef void* vsa_stream_t;
@@ -276,8 +276,12 @@ vsa_status vsa_pool_qkv(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf1
  *   o_coarse   [B, H, C, D] float32, or NULL (no coarse term; g_coarse ignored).
  *   g_coarse, g_fine  [B, N, H] bf16 or NULL (g_coarse = 0, g_fine = 1).
  *   out        [B, N, H, D] bf16 (written at every real token).
- *   overflow   one int32 of caller-owned device memory; required with
- *              `steps` (VSA_ERR_INVALID_ARGUMENT otherwise), ignored without.
+ *   overflow   two int32 of caller-owned device memory (4-byte aligned);
+ *              required with `steps` (VSA_ERR_INVALID_ARGUMENT otherwise),
+ *              ignored without.  overflow[0] is the overflow word below;
+ *              overflow[1] is the one-tile kernel's work counter (its CTAs
+ *              claim work items from it, so that items of unequal length
+ *              balance across the SMs), cleared by the call with word 0.
  *              With steps the stage runs on the one-tile kernel, which keeps
  *              each query row's first selected maximum fixed for the whole row
  *              (teardown section "Fixed-max softmax is a numerical contract"):

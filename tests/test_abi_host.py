@@ -37,7 +37,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert vsa.abi_version() == 2
+    assert vsa.abi_version() == 3
     for code, name in _lib.STATUS_NAMES.items():
         assert _lib.load().vsa_status_string(code).decode() == name
 
@@ -156,10 +156,10 @@ def test_workspace_size_480p_matches_layout():
     coarse = 3 * up(3 * 624 * 40 * 128 * 2) + up(624 * 40 * 8) + up(624 * 40 * 128 * 4) + up(624 * 624 * 40 * 4)
     expect = coarse + up(624 * 40 * 32 * 4) + up(624 * 40 * 4) + up(624 * 40 * 8) \
         + up(312 * 40 * 32 * 8) \
-        + up(4)   # work-order signatures; steps: 312 pairs of query cubes x k steps x 8 B; overflow word
+        + up(8)   # work-order signatures; steps: 312 pairs of query cubes x k steps x 8 B; overflow pair
     assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 32) == expect
     # every cube selected: dense attention; the coarse buffers are for a coarse gate only
-    assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 624) == coarse + up(4)
+    assert vsa.raw_call("vsa_workspace_bytes", ctypes.byref(s), 624) == coarse + up(8)
 
 
 def test_probe_limit_checked_before_device():

@@ -336,7 +336,8 @@ def test_overflow_scores_through_the_forward_call(dense):
 def test_overflow_word_of_the_fused_fine_call():
     """vsa_fine_fused with precomputed steps reports its overflow in the caller's word: 1 on the x16
     inputs (and the re-run's result matches the oracle), 0 on the plain inputs; a stale 1 left in
-    the word is cleared by the next call."""
+    the word is cleared by the next call.  The second word is the kernel's work counter: every item
+    past the first one of each CTA is claimed from it exactly once, so it ends at the item count."""
     w = synth.WORKLOADS["padded_7x15x16"]
     plain = synth.make_inputs(w)
     scaled = dict(plain)
@@ -353,6 +354,8 @@ def test_overflow_word_of_the_fused_fine_call():
         got = from_dev(vsa.fine_fused(dev["q"], dev["k"], dev["v"], s, idx, scale, steps=vsa.schedule(idx, s),
                                       overflow=word))
         assert int(word[0].item()) == expect
+        _, C = vsa.shape_info(s)
+        assert int(word[1].item()) == w.batch * w.heads * ((C + 1) // 2)
         ref = O.untile(ora["o_fine"], w.grid)
         for b in range(w.batch):
             for h in range(w.heads):
