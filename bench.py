@@ -1,9 +1,11 @@
 """Benchmark of the B200 VSA / dense attention path at the Wan 480p workload.
 
 One step = one VSA call (grid 21x30x52 -> 39,936 padded tokens, 624 cubes,
-40 heads, d=128, top-k 32 cubes, gated coarse + fine output) followed by one
-dense attention call on the same Q/K/V (every cube selected, no gates), both
-through the library's C ABI on one stream with inputs resident in HBM.
+40 heads, d=128, top-k 32 cubes, gated coarse + fine output) and one dense
+attention call on the same Q/K/V (every cube selected, no gates), both
+through the library's C ABI on one stream with inputs resident in HBM; the
+timed region runs the K steps' VSA calls back to back, then their dense
+calls (the two kinds alternating are reported on their own afterwards).
 
 Prints one JSON line.  `value` is the median milliseconds per VSA call (whole
 job: with N GPUs, N independent calls complete per step, so value = step
@@ -298,7 +300,7 @@ def stage_times(vsa, torch, d, w, iters: int, warmup: int, dense_too: bool = Fal
                 mark("fine_dense")
         else:
             if dense:
-                vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out)
+                vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out, overflow=word)
                 mark("fine")
             else:
                 bars = vsa.pool_qkv(d["q"], d["k"], d["v"], s)
@@ -313,7 +315,7 @@ def stage_times(vsa, torch, d, w, iters: int, warmup: int, dense_too: bool = Fal
                                out=out, steps=steps, overflow=word)
                 mark("fine")
             if dense_too:
-                vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out)
+                vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale, out=out, overflow=word)
                 mark("fine_dense")
         torch.cuda.synchronize()
         if it >= warmup:
@@ -416,20 +418,29 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     out = torch.empty_like(d["q"])
     out_d = torch.empty_like(d["q"])
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+    def vsa_call():
         vsa.forward(d["q"], d["k"], d["v"], s, w.topk, scale, d["g_coarse"], d["g_fine"], workspace=ws, out=out)
-        if ev is not None:
-            ev[1].record(stream)
-        vsa.forward(d["q"], d["k"], d["v"], s, C, scale, workspace=ws_dense, out=out_d)
-        if ev is not None:
-            ev[2].record(stream)
 
-    for _ in range(args.warmup):
-        step()
+    def dense_call():
+        vsa.forward(d["q"], d["k"], d["v"], s, C, scale, workspace=ws_dense, out=out_d)
+
+    def block(fn, evs=None):
+        # the calls of one kind back to back, each between two events when evs is given
+        for i in range(len(evs) if evs is not None else args.warmup):
+            if evs is not None:
+                evs[i][0].record(stream)
+            fn()
+            if evs is not None:
+                evs[i][1].record(stream)
+
+    # A step is one VSA call and one dense call; the K steps' VSA calls run back to back, then their
+    # dense calls (in a DiT every layer's attention is of one kind).  Alternating the two made each
+    # call run at the clock the other's power draw left behind: that is reported separately below.
+    block(vsa_call)
+    block(dense_call)
     vsa.device_status()
-    evs = [_events(torch, 3) for _ in range(args.steps)]
+    ev_v = [_events(torch, 2) for _ in range(args.steps)]
+    ev_d = [_events(torch, 2) for _ in range(args.steps)]
     t_start, t_end = _events(torch, 2)
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else f"GPU-{uuid}")
@@ -439,8 +450,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     sampler.start()
     time.sleep(0.3)
     t_start.record(stream)
-    for i in range(args.steps):
-        step(evs[i])
+    block(vsa_call, ev_v)
+    block(dense_call, ev_d)
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -448,19 +459,37 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
         dist.barrier()
     vsa.device_status()
     step_ms = t_start.elapsed_time(t_end) / args.steps
-    vsa_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
-    dense_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    vsa_ms = statistics.median(a.elapsed_time(b) for a, b in ev_v)
+    dense_ms = statistics.median(a.elapsed_time(b) for a, b in ev_d)
     step_ms_max = reduce_max(step_ms, world)
     vsa_ms_max = reduce_max(vsa_ms, world)
     dense_ms_max = reduce_max(dense_ms, world)
+
+    # ---- the same calls alternating (after the timed region): each call then follows the other kind
+    pairs = max(5, args.steps // 5)
+    ev_alt = [_events(torch, 3) for _ in range(pairs)]
+    for e in ev_alt:
+        e[0].record(stream)
+        vsa_call()
+        e[1].record(stream)
+        dense_call()
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    interleaved = {"pairs": pairs,
+                   "vsa_ms": round(statistics.median(e[0].elapsed_time(e[1]) for e in ev_alt), 4),
+                   "dense_ms": round(statistics.median(e[1].elapsed_time(e[2]) for e in ev_alt), 4),
+                   "note": "VSA and dense calls alternating, after the timed region; not part of value"}
     rerun = vsa.forward_rerun(s, w.topk, ws, has_g_coarse=True)
+    rerun_dense = vsa.forward_rerun(s, C, ws_dense, has_g_coarse=False)
 
     peaks, peaks_src = load_peaks()
     bf16_peak = float(peaks["bf16_tflops"])
     hbm_peak = float(peaks["hbm_gbs"])
 
-    # ---- per-stage breakdown: the launches of vsa_forward, one by one through the entry points
-    stage_ms = stage_times(vsa, torch, d, w, args.steps, args.warmup, dense_too=True)
+    # ---- per-stage breakdown: the launches of vsa_forward, one by one through the entry points; like
+    # the timed region, the VSA calls' stages back to back, then the dense calls' fine stage
+    stage_ms = stage_times(vsa, torch, d, w, args.steps, args.warmup)
+    stage_ms["fine_dense"] = stage_times(vsa, torch, d, wd, max(5, args.steps // 5), 3)["fine"]
 
     # ---- the memory-bound entry points one launch at a time
     mem = memory_kernels(vsa, torch, d, w, hbm_peak, max(10, args.steps))
@@ -516,17 +545,21 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                    "padded_tokens": npad, "cubes": C, "heads": w.heads, "head_dim": w.head_dim, "topk": w.topk,
                    "dense_call": {"workload": DENSE_WORKLOAD, "topk": C},
                    "l2": "no flush: 1.0 GB of Q/K/V per call exceeds the 126 MB L2",
-                   "timing": "median of the timed calls (CUDA events on the launching stream)",
+                   "timing": "median of the timed calls (CUDA events on the launching stream); the K VSA "
+                             "calls back to back, then the K dense calls",
                    "parallelism": f"{world} independent replicas (weak scaling)"},
         "dense_ms_per_call": round(whole_job_ms_per_call(dense_ms_max, 1, world), 4),
         "stage_ms": stage_ms,
-        "fixed_max_rerun": rerun,
+        "fixed_max_rerun": {"vsa": rerun, "dense": rerun_dense},
+        "interleaved": interleaved,
         "fine": {"executed_tflop": round(fine_flops / 1e12, 4), "tflops": round(fine_tflops, 1),
                  "frac_bf16_peak": round(fine_tflops / bf16_peak, 4),
                  "dense_equivalent_tflops": round(dense_equivalent_flops(w.batch, w.heads, w.tokens, w.head_dim)
                                                   / (stage_ms["fine"] * 1e-3) / 1e12, 1)},
         "dense_fine": {"executed_tflop": round(dense_flops / 1e12, 3), "tflops": round(dense_tflops, 1),
                        "frac_bf16_peak": round(dense_tflops / bf16_peak, 4),
+                       "kernel": "fine_tile_kernel<128, tokens> (the one-tile kernel over blocks of real tokens)",
+                       "traffic": traffic_for(fine_src, "fine_kernel_wan480p_dense"),
                        "per_launch": "4*B*H*(64*ceil(N/64))^2*D: blocks of 64 real tokens, no padding"},
         "roofline": {"kernel": "fine_tile_kernel<128, cubes> (VSA, top-k 32)", "bound": "tensor",
                      "achieved": round(fine_tflops, 2),
@@ -546,8 +579,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                 "api": "vsa_forward_host (pinned host q/k/v/gates in, host out; copies pipelined by head groups)"},
         # per step, VSA call: pool, coarse scores, coarse softmax x V, top-k, order sort, schedule, fine
         # (one-tile kernel) and the re-run guard (fine_kernel, which returns at once unless the one-tile
-        # kernel overflowed) = 8; dense call: fine = 1
-        "gpu_launches": 9 * args.steps,
+        # kernel overflowed) = 8; dense call: the one-tile kernel and its re-run guard = 2
+        "gpu_launches": 10 * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
         "context": {"pages_dense_call_ms_b200": 17.0, "pages_vsa_kernel_ms_b200_k78": 4.719,

@@ -229,16 +229,17 @@ def fine_fused(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, shape: Shape, 
     """Fine attention + gated merge on the token layout, written as [B,N,H,D] (idx None: dense attention).
 
     `steps` (from schedule()) replaces the kernel's own walk of the selection; the fixed-maximum
-    kernel that then runs reports an overflow (and the re-run it caused) in `overflow`, int32 on the
-    device with at least two elements: [0] the overflow word, [1] the kernel's work counter
-    (allocated here when omitted)."""
+    kernel that then runs (and runs for dense attention) reports an overflow (and the re-run it
+    caused) in `overflow`, int32 on the device with at least two elements: [0] the overflow word,
+    [1] the kernel's work counter (allocated here when omitted)."""
     scale = default_scale(shape) if scale is None else scale
     kk = int(idx.shape[-1]) if idx is not None else 0
     if out is None:
         out = torch.empty_like(q)
-    if steps is not None and overflow is None:
+    fixed_max = steps is not None or idx is None   # the one-tile kernel: sparse with steps, and dense
+    if fixed_max and overflow is None:
         overflow = torch.empty(4, dtype=torch.int32, device=q.device)
-    if steps is not None and overflow.numel() < 2:
+    if fixed_max and overflow.numel() < 2:
         raise ValueError("overflow needs two int32 elements (the overflow word and the work counter)")
     _check(_L.vsa_fine_fused(ctypes.byref(shape.c()), _ptr(q, torch.bfloat16, "q"), _ptr(k, torch.bfloat16, "k"),
                              _ptr(v, torch.bfloat16, "v"), _ptr(idx, torch.int32, "idx"), kk,

@@ -693,7 +693,10 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
     VSA_TRY(opt_ptr(steps, "steps"));
     if (steps && !idx) return fail(VSA_ERR_INVALID_ARGUMENT, "steps given without idx");
     VSA_TRY(opt_ptr(overflow, "overflow"));
-    if (steps && !overflow) return fail(VSA_ERR_INVALID_ARGUMENT, "steps given without an overflow word");
+    // the fixed-maximum kernel runs with precomputed steps and for dense attention
+    const bool fixed_max = steps != nullptr || idx == nullptr;
+    if (fixed_max && !overflow)
+        return fail(VSA_ERR_INVALID_ARGUMENT, "%s without an overflow word", steps ? "steps given" : "dense attention");
     if (steps && d.C > kScheduleMaxC)
         return fail(VSA_ERR_UNSUPPORTED, "precomputed steps support at most %d cubes (got %d)", kScheduleMaxC, d.C);
     VSA_TRY(opt_ptr(o_coarse, "o_coarse"));
@@ -707,10 +710,10 @@ vsa_status vsa_fine_fused(const vsa_shape* shape, const vsa_bf16* q, const vsa_b
                             {steps, steps ? schedule_bytes(d, topk) : 0, "steps"},
                             {o_coarse, o_coarse ? pooled_bytes(d) : 0, "o_coarse"},
                             {g_coarse, g_coarse ? gb : 0, "g_coarse"}, {g_fine, g_fine ? gb : 0, "g_fine"}},
-                           {{out, tb, "out"}, {overflow, steps ? 2 * sizeof(int32_t) : 0, "overflow"}}));
+                           {{out, tb, "out"}, {overflow, fixed_max ? 2 * sizeof(int32_t) : 0, "overflow"}}));
     VSA_TRY(check_device());
     return run_fine_fused(d, q, k, v, idx, topk, order, steps, scale, o_coarse, g_coarse, g_fine, out,
-                          steps ? overflow : nullptr, as_stream(stream));
+                          fixed_max ? overflow : nullptr, as_stream(stream));
 }
 
 size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk) {
@@ -756,7 +759,7 @@ vsa_status vsa_forward_rerun(const vsa_shape* shape, int32_t topk, int32_t has_g
     VSA_TRY(need_ptr(workspace, "workspace"));
     *rerun = 0;
     const Carve c = carve(d, topk, has_g_coarse != 0, const_cast<void*>(workspace));
-    if (topk == d.C || c.steps == nullptr) return VSA_OK;   // no fixed-maximum stage ran
+    if (topk < d.C && c.steps == nullptr) return VSA_OK;   // the sparse stage walked the selection: no fixed maximum
     cudaError_t e = cudaStreamSynchronize(as_stream(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
     int value = 0;

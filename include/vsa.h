@@ -277,13 +277,15 @@ vsa_status vsa_pool_qkv(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf1
  *   g_coarse, g_fine  [B, N, H] bf16 or NULL (g_coarse = 0, g_fine = 1).
  *   out        [B, N, H, D] bf16 (written at every real token).
  *   overflow   two int32 of caller-owned device memory (4-byte aligned);
- *              required with `steps` (VSA_ERR_INVALID_ARGUMENT otherwise),
- *              ignored without.  overflow[0] is the overflow word below;
- *              overflow[1] is the one-tile kernel's work counter (its CTAs
- *              claim work items from it, so that items of unequal length
- *              balance across the SMs), cleared by the call with word 0.
- *              With steps the stage runs on the one-tile kernel, which keeps
- *              each query row's first selected maximum fixed for the whole row
+ *              required with `steps` and with idx == NULL
+ *              (VSA_ERR_INVALID_ARGUMENT otherwise), ignored otherwise.
+ *              overflow[0] is the overflow word below; overflow[1] is the
+ *              one-tile kernel's work counter (its CTAs claim work items from
+ *              it, so that items of unequal length balance across the SMs),
+ *              cleared by the call with word 0.
+ *              With steps, and for dense attention, the stage runs on the
+ *              one-tile kernel, which keeps each query row's first selected
+ *              (dense: first block's) maximum fixed for the whole row
  *              (teardown section "Fixed-max softmax is a numerical contract"):
  *              the call clears the word, the kernel sets it to 1 when a
  *              probability would exceed 2^64 or a row sum is not finite, and a
@@ -326,8 +328,8 @@ size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
  * vsa_forward — the whole attention call on one stream, as eight launches for
  * top-k < C with a coarse gate:
  *   vsa_pool_qkv (writing the pooled vectors as their three bf16 parts) ->
- *   the coarse scores (tensor cores) -> vsa_topk_order (2; the selection pass
- *   also keeps each row's softmax statistics) -> the coarse output (tensor
+ *   the coarse scores (tensor cores; with g_coarse they also keep each row's
+ *   softmax statistics) -> vsa_topk_order (2) -> the coarse output (tensor
  *   cores; skipped when g_coarse is NULL, since only the merge uses it) ->
  *   vsa_schedule -> vsa_fine_fused (the one-tile kernel and its re-run guard)
  * (vsa_topk -> vsa_group instead when C > 2048; the grouping step is skipped
@@ -338,7 +340,8 @@ size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
  * When topk == C every cube is selected and the fine stage is dense attention
  * over the real tokens: vsa_fine_fused with idx == NULL, preceded by
  * vsa_pool_qkv -> vsa_coarse only when g_coarse is given.  With both gates
- * NULL that is dense attention in one launch.
+ * NULL that is dense attention in two launches (the one-tile kernel and its
+ * re-run guard, which returns at once unless the fixed maxima overflowed).
  *   q, k, v      [B, N, H, D] bf16 token layout (read).
  *   g_coarse, g_fine  [B, N, H] bf16 or NULL (see vsa_combine).
  *   workspace    device buffer of at least vsa_workspace_bytes(shape, topk),
@@ -357,9 +360,10 @@ vsa_status vsa_forward(const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16
  * re-run its fine stage with online rescaling because the fixed per-row
  * maxima overflowed (see the `overflow` argument of vsa_fine_fused; the
  * forward call keeps that word in its workspace).  Synchronizes `stream`,
- * then sets *rerun to 1 or 0.  A dense call (topk == C), which rescales
- * online from the start, and a call whose fine stage walked the selection
- * itself (no precomputed steps) always give 0 without touching the device.
+ * then sets *rerun to 1 or 0.  A sparse call whose fine stage walked the
+ * selection itself (no precomputed steps: C above the schedule's limit),
+ * which rescales online from the start, always gives 0 without touching the
+ * device.
  */
 vsa_status vsa_forward_rerun(const vsa_shape* shape, int32_t topk, int32_t has_g_coarse, const void* workspace,
                              int32_t* rerun, vsa_stream_t stream);

@@ -82,6 +82,10 @@ def test_fine_fused_steps_need_an_overflow_word():
     st = vsa.raw_call("vsa_fine_fused", ctypes.byref(s), p[0], p[1], p[2], p[3], 2, None, p[4], 0.125,
                       None, None, None, p[5], ctypes.c_void_p(p[6].value + 4), None)
     assert st == MISALIGNED and "overflow" in vsa.last_error()
+    # dense attention (idx NULL) runs on the same fixed-maximum kernel: it needs the word too
+    st = vsa.raw_call("vsa_fine_fused", ctypes.byref(s), p[0], p[1], p[2], None, 0, None, None, 0.125,
+                      None, None, None, p[5], None, None)
+    assert st == INVALID and "dense attention without an overflow word" in vsa.last_error()
 
 
 def test_forward_rerun_argument_checks():
@@ -91,9 +95,11 @@ def test_forward_rerun_argument_checks():
     assert vsa.raw_call("vsa_forward_rerun", ctypes.byref(s), 2, 1, ws, None, None) == INVALID
     assert vsa.raw_call("vsa_forward_rerun", ctypes.byref(s), 0, 1, ws, ctypes.byref(r), None) == INVALID
     assert vsa.raw_call("vsa_forward_rerun", ctypes.byref(s), 2, 1, None, ctypes.byref(r), None) == INVALID
-    # dense call (top-k = C): no fixed-maximum stage, answered without touching the device
-    _, c = vsa.shape_info(vsa.Shape(s.batch, s.heads, s.head_dim, (s.grid_t, s.grid_h, s.grid_w)))
-    assert vsa.raw_call("vsa_forward_rerun", ctypes.byref(s), c, 0, ws, ctypes.byref(r), None) == 0
+    # a sparse call with more cubes than the precomputed schedule holds (32,000: its per-warp marks
+    # exceed 48 KB of shared memory) walks the selection itself with online rescaling: no fixed-maximum
+    # stage ran, so the answer comes without touching the device
+    big = _shape(grid=(80, 160, 160))
+    assert vsa.raw_call("vsa_forward_rerun", ctypes.byref(big), 2, 0, ws, ctypes.byref(r), None) == 0
     assert r.value == 0
 
 

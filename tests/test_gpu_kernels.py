@@ -301,7 +301,9 @@ def test_overflow_scores_through_the_forward_call(dense):
     """The fused call on the same scaled inputs.  Sparse: the one-tile kernel's fixed per-row maxima
     overflow, it raises its overflow word and the call re-runs the fine stage with the online
     rescaling kernel; the word must read 1 here and 0 for the unscaled inputs, and both results must
-    match the oracle.  Dense: the two-tile kernel raises a row's maximum itself (no re-run)."""
+    match the oracle.  Dense attention runs on the same kernel with each row's first 64-key block's
+    maximum fixed: the same guard, the same re-run (the x16 rows exceed that maximum by far more than
+    2^64 allows, the plain rows by at most 2^17)."""
     w = synth.WORKLOADS["padded_7x15x16"]
     plain = synth.make_inputs(w)
     x = dict(plain)
@@ -322,7 +324,7 @@ def test_overflow_scores_through_the_forward_call(dense):
         if dense:
             ref, lse = O.dense(f64["q"], f64["k"], f64["v"], w.grid, scale)
             assert (lse.max() > 100) == scaled
-            assert not rerun
+            assert rerun == scaled, f"dense overflow re-run {'missing' if scaled else 'fired'}"
         else:
             ora = O.forward(f64["q"], f64["k"], f64["v"], w.grid, k, scale, f64["g_coarse"], f64["g_fine"])
             ref = ora["out"]
