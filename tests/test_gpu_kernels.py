@@ -425,7 +425,8 @@ def test_one_tile_kernel_with_many_items_per_cta():
     SM, so every CTA carries several items and the per-item hand-overs between the softmax groups, the
     epilogue warps and the next item's first steps happen many times.  The fused fine stage with
     precomputed steps (the one-tile kernel) must match the oracle on every head and give the same bits
-    on every one of 20 repeated launches; the whole forward call must repeat bit for bit too."""
+    on every one of 20 repeated launches; the whole forward call must repeat bit for bit too, and so
+    must dense attention on the same kernel."""
     w = synth.custom_workload("many_items_8x8x8", 1, 160, 64, (8, 8, 8), 2, field=True, wid=97)
     x = synth.make_inputs(w)
     d = {k: to_dev(v) for k, v in x.items()}
@@ -447,6 +448,15 @@ def test_one_tile_kernel_with_many_items_per_cta():
     for rep in range(5):
         b = vsa.forward(d["q"], d["k"], d["v"], s, w.topk, scale, d["g_coarse"], d["g_fine"])
         assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"forward call {rep} differs"
+    # dense attention on the same kernel: 160 heads x 4 items of four 64-token blocks, claimed by the CTAs
+    r_dense, _ = O.dense(f64["q"], f64["k"], f64["v"], w.grid, scale)
+    dense = vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale)
+    got = from_dev(dense)
+    for h in range(w.heads):
+        check_close(got[0, :, h], r_dense[0, :, h], f"many items dense h={h}")
+    for rep in range(10):
+        again = vsa.fine_fused(d["q"], d["k"], d["v"], s, None, scale)
+        assert torch.equal(again.view(torch.int16), dense.view(torch.int16)), f"dense launch {rep} differs"
 
 
 HOST_CASES = {
