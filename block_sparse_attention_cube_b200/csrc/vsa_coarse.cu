@@ -12,11 +12,11 @@ namespace {
 constexpr int kThreads = 256;
 
 // Order-preserving map float -> uint32 (larger float, larger key); -0 is
-// folded onto +0 so that equal scores compare equal.
+// folded onto +0 (-0 + 0 = +0) so that equal scores compare equal.  Every
+// score's key is at least 0x007FFFFF (that of -inf), so 0 ranks below all.
 __device__ __forceinline__ uint32_t order_key(float f) {
-    if (f == 0.0f) f = 0.0f;
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    const uint32_t u = __float_as_uint(f + 0.0f);
+    return u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
 }
 
 __device__ __forceinline__ void top3_insert(uint64_t (&t)[3], uint64_t v) {
@@ -275,10 +275,23 @@ __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C,
                     lo = kth_key<kTopM + 1>(top, hi, lo0, k);
                 }
             }
-            uint32_t mine = 0;
+            // a lane holding only padding (C < 32) has maximum 0; lo >= 1 keeps padding keys out of every
+            // count below (real keys are all >= 1, and at least k of them reach lo)
+            lo = max(lo, 1u);
+            // the keys >= lo, with their cube indices and in index order, into the candidate list while it
+            // has room; ncand counts them all
+            ncand = 0;
 #pragma unroll
-            for (int i = 0; i < KPL; ++i) mine += (lane + 32 * i < C && key[i] >= lo) ? 1u : 0u;
-            ncand = static_cast<int>(__reduce_add_sync(0xffffffffu, mine));
+            for (int i = 0; i < KPL; ++i) {
+                const bool f = key[i] >= lo;
+                const uint32_t bal = __ballot_sync(0xffffffffu, f);
+                const int pos = ncand + __popc(bal & lt_mask);
+                if (f && pos < 32 * kTopCand) {
+                    cand_key[pos] = key[i];
+                    cand_idx[pos] = static_cast<uint16_t>(lane + 32 * i);
+                }
+                ncand += __popc(bal);
+            }
         } else {
             uint32_t lane_max = 0u, lane_min = 0xFFFFFFFFu;
 #pragma unroll
@@ -292,17 +305,6 @@ __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C,
         int32_t* dst = idx + row * k;
         uint64_t lex;
         if (ncand <= 32 * kTopCand) {
-            int base = 0;
-#pragma unroll
-            for (int i = 0; i < KPL; ++i) {
-                const bool f = lane + 32 * i < C && key[i] >= lo;
-                const uint32_t bal = __ballot_sync(0xffffffffu, f);
-                if (f) {
-                    cand_key[base + __popc(bal & lt_mask)] = key[i];
-                    cand_idx[base + __popc(bal & lt_mask)] = static_cast<uint16_t>(lane + 32 * i);
-                }
-                base += __popc(bal);
-            }
             __syncwarp();
             uint32_t ck[kTopCand];
 #pragma unroll
@@ -318,6 +320,7 @@ __global__ void __launch_bounds__(kThreads) topk_reg_kernel(int64_t rows, int C,
                                             [&](int e) { return lane + 32 * e < ncand ? int(cand_idx[lane + 32 * e]) : 0; });
             __syncwarp();
         } else {
+            // (padding keys are 0: below lo, so below T)
             const uint32_t T = kth_key<KPL>(key, hi, lo, k);
             uint32_t gt = 0;
 #pragma unroll
