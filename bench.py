@@ -4,7 +4,7 @@ One step = one VSA call (grid 21x30x52 -> 39,936 padded tokens, 624 cubes,
 40 heads, d=128, top-k 32 cubes, gated coarse + fine output) and one dense
 attention call on the same Q/K/V (every cube selected, no gates), both
 through the library's C ABI on one stream with inputs resident in HBM; the
-timed region runs the K steps' VSA calls back to back, then their dense
+timed region runs the K steps' dense calls back to back, then their VSA
 calls (the two kinds alternating are reported on their own afterwards).
 
 Prints one JSON line.  `value` is the median milliseconds per VSA call (whole
@@ -433,9 +433,11 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
             if evs is not None:
                 evs[i][1].record(stream)
 
-    # A step is one VSA call and one dense call; the K steps' VSA calls run back to back, then their
-    # dense calls (in a DiT every layer's attention is of one kind).  Alternating the two made each
-    # call run at the clock the other's power draw left behind: that is reported separately below.
+    # A step is one VSA call and one dense call; the K steps' dense calls run back to back, then their
+    # VSA calls (in a DiT every layer's attention is of one kind), so the VSA block starts at the clock
+    # the dense block's power draw leaves.  Alternating the two made each call run at the clock the
+    # other kind left behind: that is reported separately below.  Each kind's per-stage breakdown
+    # follows its own block: the VSA stages right after the timed region, then the dense fine stage.
     block(vsa_call)
     block(dense_call)
     vsa.device_status()
@@ -450,8 +452,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     sampler.start()
     time.sleep(0.3)
     t_start.record(stream)
-    block(vsa_call, ev_v)
     block(dense_call, ev_d)
+    block(vsa_call, ev_v)
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -465,7 +467,19 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     vsa_ms_max = reduce_max(vsa_ms, world)
     dense_ms_max = reduce_max(dense_ms, world)
 
-    # ---- the same calls alternating (after the timed region): each call then follows the other kind
+    rerun = vsa.forward_rerun(s, w.topk, ws, has_g_coarse=True)
+    rerun_dense = vsa.forward_rerun(s, C, ws_dense, has_g_coarse=False)
+
+    peaks, peaks_src = load_peaks()
+    bf16_peak = float(peaks["bf16_tflops"])
+    hbm_peak = float(peaks["hbm_gbs"])
+
+    # ---- per-stage breakdown: the launches of vsa_forward, one by one through the entry points; the VSA
+    # calls' stages back to back right after the VSA block, then the dense calls' fine stage
+    stage_ms = stage_times(vsa, torch, d, w, args.steps, args.warmup)
+    stage_ms["fine_dense"] = stage_times(vsa, torch, d, wd, max(5, args.steps // 5), 3)["fine"]
+
+    # ---- the same calls alternating (after the stage breakdown): each call follows the other kind
     pairs = max(5, args.steps // 5)
     ev_alt = [_events(torch, 3) for _ in range(pairs)]
     for e in ev_alt:
@@ -478,18 +492,7 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
     interleaved = {"pairs": pairs,
                    "vsa_ms": round(statistics.median(e[0].elapsed_time(e[1]) for e in ev_alt), 4),
                    "dense_ms": round(statistics.median(e[1].elapsed_time(e[2]) for e in ev_alt), 4),
-                   "note": "VSA and dense calls alternating, after the timed region; not part of value"}
-    rerun = vsa.forward_rerun(s, w.topk, ws, has_g_coarse=True)
-    rerun_dense = vsa.forward_rerun(s, C, ws_dense, has_g_coarse=False)
-
-    peaks, peaks_src = load_peaks()
-    bf16_peak = float(peaks["bf16_tflops"])
-    hbm_peak = float(peaks["hbm_gbs"])
-
-    # ---- per-stage breakdown: the launches of vsa_forward, one by one through the entry points; like
-    # the timed region, the VSA calls' stages back to back, then the dense calls' fine stage
-    stage_ms = stage_times(vsa, torch, d, w, args.steps, args.warmup)
-    stage_ms["fine_dense"] = stage_times(vsa, torch, d, wd, max(5, args.steps // 5), 3)["fine"]
+                   "note": "VSA and dense calls alternating, after the stage breakdown; not part of value"}
 
     # ---- the memory-bound entry points one launch at a time
     mem = memory_kernels(vsa, torch, d, w, hbm_peak, max(10, args.steps))
@@ -545,8 +548,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int):
                    "padded_tokens": npad, "cubes": C, "heads": w.heads, "head_dim": w.head_dim, "topk": w.topk,
                    "dense_call": {"workload": DENSE_WORKLOAD, "topk": C},
                    "l2": "no flush: 1.0 GB of Q/K/V per call exceeds the 126 MB L2",
-                   "timing": "median of the timed calls (CUDA events on the launching stream); the K VSA "
-                             "calls back to back, then the K dense calls",
+                   "timing": "median of the timed calls (CUDA events on the launching stream); the K dense "
+                             "calls back to back, then the K VSA calls",
                    "parallelism": f"{world} independent replicas (weak scaling)"},
         "dense_ms_per_call": round(whole_job_ms_per_call(dense_ms_max, 1, world), 4),
         "stage_ms": stage_ms,
