@@ -133,6 +133,35 @@ vsa_status lib_stream(int which, cudaStream_t* out) {
 // vsa_forward_host: head groups per call (the copies of one overlap the compute of another)
 constexpr int kHostGroups = 8;
 
+// The head ranges [h0, h0 + hn) of one vsa_forward_host call.  Every upload but the first overlaps
+// compute, so the call takes about all its uploads plus the last group's compute and download: with 27 or
+// more heads the last three groups hold 4, 2 and 1 heads and the others split the rest evenly, largest
+// first (Wan's 40 heads: 7 7 7 6 6 4 2 1); with fewer heads, groups of ceil(H / kHostGroups).  Copies of
+// 256-byte rows (one head) still run at about 52 GB/s against 55 for whole rows, measured on B200.
+struct HostPlan {
+    int n = 0, largest = 0;
+    int h0[kHostGroups] = {}, hn[kHostGroups] = {};
+};
+
+HostPlan host_plan(int H) {
+    HostPlan pl;
+    if (H >= 27) {
+        const int rest = H - 7, nr = kHostGroups - 3;
+        for (int i = 0; i < nr; ++i) pl.hn[pl.n++] = rest / nr + (i < rest % nr ? 1 : 0);
+        pl.hn[pl.n++] = 4;
+        pl.hn[pl.n++] = 2;
+        pl.hn[pl.n++] = 1;
+    } else {
+        const int hg = (H + kHostGroups - 1) / kHostGroups;
+        for (int h = 0; h < H; h += hg) pl.hn[pl.n++] = H - h < hg ? H - h : hg;
+    }
+    for (int i = 0, h = 0; i < pl.n; h += pl.hn[i], ++i) {
+        pl.h0[i] = h;
+        if (pl.hn[i] > pl.largest) pl.largest = pl.hn[i];
+    }
+    return pl;
+}
+
 // Events of one vsa_forward_host call, destroyed when it returns (CUDA keeps a recorded event
 // alive until the work it marks is done).
 struct EventSet {
@@ -311,11 +340,11 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
                           gf, out, c.overflow, s);
 }
 
-// vsa_forward_host's pipeline over head groups of hg heads (see vsa_forward_host): uploads on up_s,
+// vsa_forward_host's pipeline over the head groups of `pl` (see vsa_forward_host): uploads on up_s,
 // compute on s, downloads on down_s, ordered by events; `stream` waits for the last download.
 vsa_status forward_host_groups(const Dims& d, const vsa_shape* shape, const vsa_bf16* q, const vsa_bf16* k,
                                const vsa_bf16* v, const vsa_bf16* g_coarse, const vsa_bf16* g_fine, int32_t topk,
-                               float scale, void* workspace, int hg, size_t fwd_g, size_t gate_g,
+                               float scale, void* workspace, const HostPlan& pl, size_t fwd_g, size_t gate_g,
                                uint16_t* dq, uint16_t* dk, uint16_t* dv, uint16_t* dout, uint16_t* dgc,
                                uint16_t* dgf, vsa_bf16* out, cudaStream_t s, cudaStream_t up_s,
                                cudaStream_t down_s) {
@@ -323,7 +352,7 @@ vsa_status forward_host_groups(const Dims& d, const vsa_shape* shape, const vsa_
     const int64_t rows = static_cast<int64_t>(d.B) * d.N;
     const size_t gb = gate_bytes(d);
     vsa_shape sg = *shape;
-    const int groups = (d.H + hg - 1) / hg;
+    const int groups = pl.n;
     EventSet ev;
     VSA_CUDA(ev.create(2 * groups + 2), "create events");
     uint16_t* cgc = dgc ? reinterpret_cast<uint16_t*>(w + fwd_g) : nullptr;
@@ -336,7 +365,7 @@ vsa_status forward_host_groups(const Dims& d, const vsa_shape* shape, const vsa_
     if (dgf) VSA_CUDA(cudaMemcpyAsync(dgf, g_fine, gb, cudaMemcpyHostToDevice, up_s), "copy g_fine to device");
     const size_t row_all = static_cast<size_t>(d.H) * d.D * 2;
     for (int gi = 0; gi < groups; ++gi) {
-        const int h0 = gi * hg, hn = d.H - h0 < hg ? d.H - h0 : hg;
+        const int h0 = pl.h0[gi], hn = pl.hn[gi];
         const size_t off = static_cast<size_t>(rows) * h0 * d.D;   // elements before this group's block
         const size_t row_g = static_cast<size_t>(hn) * d.D * 2;
         const size_t src_off = static_cast<size_t>(h0) * d.D;
@@ -808,7 +837,8 @@ vsa_status vsa_forward_host(const vsa_shape* shape, const vsa_bf16* q, const vsa
     // [B, N, hn, D], one after the other in the staging buffers; its gates are gathered on the device
     // from the whole arrays into the part of the forward workspace that the smaller call leaves free.
     const int64_t rows = static_cast<int64_t>(d.B) * d.N;
-    int hg = d.H >= 2 ? (d.H + kHostGroups - 1) / kHostGroups : d.H;
+    const HostPlan pl = host_plan(d.H);
+    int hg = pl.largest;   // the largest group sizes the per-group workspace and gate staging
     Dims dg{};
     vsa_shape sg = *shape;
     sg.heads = hg;
@@ -833,7 +863,7 @@ vsa_status vsa_forward_host(const vsa_shape* shape, const vsa_bf16* q, const vsa
     cudaStream_t up_s = nullptr, down_s = nullptr;
     VSA_TRY(lib_stream(0, &up_s));
     VSA_TRY(lib_stream(1, &down_s));
-    const vsa_status st = forward_host_groups(d, shape, q, k, v, g_coarse, g_fine, topk, scale, workspace, hg, fwd_g,
+    const vsa_status st = forward_host_groups(d, shape, q, k, v, g_coarse, g_fine, topk, scale, workspace, pl, fwd_g,
                                               gate_g, dq, dk, dv, dout, dgc, dgf, out, s, up_s, down_s);
     if (st != VSA_OK) {
         // best effort: whatever the copy streams still hold comes before anything later on `stream`

@@ -381,7 +381,9 @@ size_t vsa_workspace_bytes_host(const vsa_shape* shape, int32_t topk);
  * `stream`, and its output is copied back into its head range of `out`; the
  * copies run on two copy streams of the library's, ordered against `stream`
  * by events, so the uploads of one group and the download of another overlap
- * the compute of a third.  The gates are copied whole and gathered per group
+ * the compute of a third.  With 27 or more heads the last groups shrink (4,
+ * 2, 1 heads), so little compute and download follow the last upload.  The
+ * gates are copied whole and gathered per group
  * on the device.  The result is bit-identical to vsa_forward on the same
  * inputs.  Everything already enqueued on `stream` happens before the copies,
  * and the call's last copy is complete when `stream` reaches the point after

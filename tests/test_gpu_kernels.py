@@ -461,10 +461,12 @@ def test_one_tile_kernel_with_many_items_per_cta():
 
 HOST_CASES = {
     # name: (workload, gates): 4 heads -> four groups of one head; 1 head -> one group (no pipeline);
-    # 11 heads -> groups of two heads with a last group of one, no gates; B = 2, d = 64
+    # 11 heads -> groups of two heads with a last group of one, no gates; B = 2, d = 64; 40 heads ->
+    # groups of 7 7 7 6 6 4 2 1 heads (the shrinking tail)
     "padded_4_heads": ("padded_7x15x16", True),
     "one_head": (("one_head_7x15x16", 1, 1, 128, (7, 15, 16), 8), True),
     "eleven_heads_no_gates": (("eleven_heads_9x6x5", 2, 11, 64, (9, 6, 5), 4), False),
+    "forty_heads": (("forty_heads_7x15x16", 1, 40, 64, (7, 15, 16), 8), True),
 }
 
 
