@@ -1480,10 +1480,12 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             float mx = -INFINITY;
 #pragma unroll 1
                             for (int ch = 0; ch < 4; ++ch) {
+                                const uint64_t vm = ch < 2 ? vm_a : vm_b;
+                                const uint32_t w = static_cast<uint32_t>(vm >> (32 * (ch & 1)));
+                                if (w == 0u) continue;   // warp-uniform: no key of the chunk counts
                                 uint32_t sc[32];
                                 tmem_ld32_wait(tS + 32u * ch, sc);
-                                const uint64_t vm = ch < 2 ? vm_a : vm_b;
-                                mask32(sc, static_cast<uint32_t>(vm >> (32 * (ch & 1))));
+                                mask32(sc, w);
                                 mx = fmaxf(mx, max32(sc));
                             }
                             m = mx == -INFINITY ? 0.f : mx * c;
@@ -1499,13 +1501,22 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         float sum = 0.f;
 #pragma unroll 1
                         for (int ch = 0; ch < 4; ++ch) {
-                            uint32_t sc[32];
-                            tmem_ld32_wait(tS + 32u * ch, sc);
                             const uint64_t vm = ch < 2 ? vm_a : vm_b;
-                            mask32(sc, static_cast<uint32_t>(vm >> (32 * (ch & 1))));
+                            const uint32_t w = static_cast<uint32_t>(vm >> (32 * (ch & 1)));
                             uint32_t pk[16];
-                            sum += probs32(sc, c, m, pk);
-                            // P of keys 32ch.. over columns 16ch..: scores there were already read
+                            if (w == 0u) {
+                                // warp-uniform: the chunk's 32 keys are outside this row's selection (a key
+                                // cube only the other query cube of the tile selected): P = 0, no exponentials
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                            } else {
+                                uint32_t sc[32];
+                                tmem_ld32_wait(tS + 32u * ch, sc);
+                                mask32(sc, w);
+                                sum += probs32(sc, c, m, pk);
+                            }
+                            // P of keys 32ch.. over columns 16ch..: scores there were already read (or,
+                            // for a skipped chunk 0, are not needed)
                             tmem_st16(tS + 16u * ch, pk);
                         }
                         if (!(sum <= kSumLimit) && p.overflow != nullptr) *p.overflow = 1;
