@@ -1482,7 +1482,7 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             for (int ch = 0; ch < 4; ++ch) {
                                 const uint64_t vm = ch < 2 ? vm_a : vm_b;
                                 const uint32_t w = static_cast<uint32_t>(vm >> (32 * (ch & 1)));
-                                if (w == 0u) continue;   // warp-uniform: no key of the chunk counts
+                                if (LM == kLoadCubes && w == 0u) continue;   // warp-uniform: no key counts
                                 uint32_t sc[32];
                                 tmem_ld32_wait(tS + 32u * ch, sc);
                                 mask32(sc, w);
@@ -1504,9 +1504,10 @@ fine_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             const uint64_t vm = ch < 2 ? vm_a : vm_b;
                             const uint32_t w = static_cast<uint32_t>(vm >> (32 * (ch & 1)));
                             uint32_t pk[16];
-                            if (w == 0u) {
+                            if (LM == kLoadCubes && w == 0u) {
                                 // warp-uniform: the chunk's 32 keys are outside this row's selection (a key
-                                // cube only the other query cube of the tile selected): P = 0, no exponentials
+                                // cube only the other query cube of the tile selected): P = 0, no exponentials.
+                                // (Dense blocks are selected by every row: the dense kernel keeps no such test.)
 #pragma unroll
                                 for (int j = 0; j < 16; ++j) pk[j] = 0u;
                             } else {
