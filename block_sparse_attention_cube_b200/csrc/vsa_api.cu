@@ -305,7 +305,8 @@ vsa_status run_forward(const Dims& d, const uint16_t* q, const uint16_t* k, cons
         // pooled q, k, v straight into their bf16 parts, then the scores on the tensor cores
         const uint16_t* pin[3] = {q, k, v};
         uint16_t* parts[3] = {c.qp, c.kp, c.vp};
-        VSA_CUDA(launch_pool_tokens(d, pin, nullptr, 3, s, parts), "pool launch");
+        // v-bar feeds only the coarse output, which only the coarse gate uses: without it v is not pooled
+        VSA_CUDA(launch_pool_tokens(d, pin, nullptr, gc != nullptr ? 3 : 2, s, parts), "pool launch");
         // the softmax statistics of the score rows are needed only for the coarse output
         const cudaError_t e =
             launch_coarse_scores_mma(d, c.qp, c.kp, scale, c.scores, gc != nullptr ? c.stats : nullptr, s, &why);

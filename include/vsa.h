@@ -327,7 +327,8 @@ size_t vsa_workspace_bytes(const vsa_shape* shape, int32_t topk);
 /*
  * vsa_forward — the whole attention call on one stream, as eight launches for
  * top-k < C with a coarse gate:
- *   vsa_pool_qkv (writing the pooled vectors as their three bf16 parts) ->
+ *   vsa_pool_qkv (writing the pooled vectors as their three bf16 parts; v only
+ *   with g_coarse, since only the coarse output uses it) ->
  *   the coarse scores (tensor cores; with g_coarse they also keep each row's
  *   softmax statistics) -> vsa_topk_order (2) -> the coarse output (tensor
  *   cores; skipped when g_coarse is NULL, since only the merge uses it) ->
