@@ -15,6 +15,9 @@ namespace vsa {
 namespace {
 
 constexpr int kBlock = 256;
+// Resident blocks per SM that the copy kernels' register bounds guarantee; their
+// grids are sized to exactly that many per SM.
+constexpr int kLayoutPerSm = 8;
 
 struct CubeTask {
     int tensor;
@@ -47,31 +50,38 @@ __device__ __forceinline__ int64_t token_of(const Dims& d, const CubeTask& t, in
     return (static_cast<int64_t>(tt) * d.X + xx) * d.Y + yy;
 }
 
+// A thread's PER row loads are all issued before its first store.
 template <int D>
-__global__ void __launch_bounds__(kBlock) tile_kernel(Dims d, Bf16Triple io) {
+__global__ void __launch_bounds__(kBlock, kLayoutPerSm) tile_kernel(Dims d, Bf16Triple io) {
     constexpr int CH = D / 8;                   // 16-byte chunks per row
     constexpr int PER = kCubeTokens * CH / kBlock;
+    constexpr int ROWS = kBlock / CH;           // rows covered by one pass of the block
+    static_assert(kBlock % CH == 0, "a thread's column chunk must stay fixed across its rows");
     const int64_t total = static_cast<int64_t>(d.B) * d.H * d.C * io.count;
+    const int j = threadIdx.x % CH, o0 = threadIdx.x / CH;
     for (int64_t task = blockIdx.x; task < total; task += gridDim.x) {
         const CubeTask t = decode_task(task, d);
-        const uint4* src = reinterpret_cast<const uint4*>(io.src[t.tensor]);
-        uint4* dst = reinterpret_cast<uint4*>(io.dst[t.tensor]);
+        // pointers chosen by value: a runtime index into the parameter arrays would go through local memory
+        const uint16_t* src_t = t.tensor == 0 ? io.src[0] : t.tensor == 1 ? io.src[1] : io.src[2];
+        uint16_t* dst_t = t.tensor == 0 ? io.dst[0] : t.tensor == 1 ? io.dst[1] : io.dst[2];
+        const uint4* src = reinterpret_cast<const uint4*>(src_t);
+        uint4* dst = reinterpret_cast<uint4*>(dst_t);
         const int64_t out_row0 = t.bh * d.Npad + static_cast<int64_t>(t.c) * kCubeTokens;
+        uint4 v[PER];
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
-            const int q = threadIdx.x + i * kBlock;
-            const int o = q / CH, j = q % CH;
-            const int64_t n = token_of(d, t, o);
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (n >= 0) v = __ldcs(src + ((static_cast<int64_t>(t.b) * d.N + n) * d.H + t.h) * CH + j);
-            dst[(out_row0 + o) * CH + j] = v;
+            const int64_t n = token_of(d, t, o0 + i * ROWS);
+            v[i] = n >= 0 ? __ldcs(src + ((static_cast<int64_t>(t.b) * d.N + n) * d.H + t.h) * CH + j)
+                          : make_uint4(0u, 0u, 0u, 0u);
         }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) dst[(out_row0 + o0 + i * ROWS) * CH + j] = v[i];
     }
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBlock) untile_kernel(Dims d, const uint16_t* __restrict__ xt,
-                                                        uint16_t* __restrict__ x) {
+__global__ void __launch_bounds__(kBlock, kLayoutPerSm) untile_kernel(Dims d, const uint16_t* __restrict__ xt,
+                                                                      uint16_t* __restrict__ x) {
     constexpr int CH = D / 8;
     constexpr int PER = kCubeTokens * CH / kBlock;
     const int64_t total = static_cast<int64_t>(d.B) * d.H * d.C;
@@ -271,46 +281,67 @@ __global__ void __launch_bounds__(kBlock) split_parts_kernel(int64_t groups, con
     }
 }
 
+// Each thread keeps one 16-byte column chunk j of the cube's rows (kBlock is a
+// multiple of the chunks per row), so its eight coarse values are loaded once
+// per cube.  All of a cube's loads (O_f rows, gates) are issued before any
+// arithmetic: the gate loads are scattered (one 2-byte value per 80-byte row of
+// the [B, N, H] layout), and issuing them one row at a time behind each O_f
+// load left too few bytes in flight to cover HBM latency.  The registers that
+// hold them allow kCombinePerSm resident blocks per SM, and the grid is sized to
+// exactly that many: a grid-stride grid larger than the resident blocks would
+// leave its last blocks to run alone after the first wave.
+constexpr int kCombinePerSm = 5;
+
 template <int D>
-__global__ void __launch_bounds__(kBlock) combine_kernel(Dims d, const float* __restrict__ o_coarse,
-                                                         const uint16_t* __restrict__ o_fine,
-                                                         const uint16_t* __restrict__ g_coarse,
-                                                         const uint16_t* __restrict__ g_fine,
-                                                         uint16_t* __restrict__ o_tiled) {
+__global__ void __launch_bounds__(kBlock, kCombinePerSm) combine_kernel(Dims d, const float* __restrict__ o_coarse,
+                                                                        const uint16_t* __restrict__ o_fine,
+                                                                        const uint16_t* __restrict__ g_coarse,
+                                                                        const uint16_t* __restrict__ g_fine,
+                                                                        uint16_t* __restrict__ o_tiled) {
     constexpr int CH = D / 8;
     constexpr int PER = kCubeTokens * CH / kBlock;
+    constexpr int ROWS = kBlock / CH;   // rows covered by one pass of the block
+    static_assert(kBlock % CH == 0, "a thread's column chunk must stay fixed across its rows");
     const int64_t total = static_cast<int64_t>(d.B) * d.H * d.C;
     const uint4* of = reinterpret_cast<const uint4*>(o_fine);
     uint4* out = reinterpret_cast<uint4*>(o_tiled);
+    const int j = threadIdx.x % CH, o0 = threadIdx.x / CH;
     for (int64_t task = blockIdx.x; task < total; task += gridDim.x) {
         const CubeTask t = decode_task(task, d);
         const int64_t row0 = t.bh * d.Npad + static_cast<int64_t>(t.c) * kCubeTokens;
         const float4* oc = reinterpret_cast<const float4*>(o_coarse + (t.bh * d.C + t.c) * D);
+        int n[PER];   // token of each row, -1 for padding (below 2^30: at most 2^24 cubes)
+        uint4 f[PER];
+        float gc[PER], gf[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) n[i] = static_cast<int>(token_of(d, t, o0 + i * ROWS));
+#pragma unroll
+        for (int i = 0; i < PER; ++i)
+            f[i] = n[i] >= 0 ? __ldcs(of + (row0 + o0 + i * ROWS) * CH + j) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
-            const int q = threadIdx.x + i * kBlock;
-            const int o = q / CH, j = q % CH;
-            const int64_t n = token_of(d, t, o);
+            const int64_t g = (static_cast<int64_t>(t.b) * d.N + (n[i] >= 0 ? n[i] : 0)) * d.H + t.h;
+            gc[i] = g_coarse && n[i] >= 0 ? __uint_as_float(static_cast<uint32_t>(g_coarse[g]) << 16) : 0.f;
+            gf[i] = g_fine && n[i] >= 0 ? __uint_as_float(static_cast<uint32_t>(g_fine[g]) << 16) : 1.f;
+        }
+        const float4 c0 = __ldg(oc + 2 * j), c1 = __ldg(oc + 2 * j + 1);
+        const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
             uint4 r = make_uint4(0u, 0u, 0u, 0u);
-            if (n >= 0) {
-                const int64_t g = (static_cast<int64_t>(t.b) * d.N + n) * d.H + t.h;
-                const float gc = g_coarse ? __uint_as_float(static_cast<uint32_t>(g_coarse[g]) << 16) : 0.f;
-                const float gf = g_fine ? __uint_as_float(static_cast<uint32_t>(g_fine[g]) << 16) : 1.f;
-                const float4 c0 = __ldg(oc + 2 * j), c1 = __ldg(oc + 2 * j + 1);
-                const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                const uint4 f = __ldcs(of + (row0 + o) * CH + j);
-                const uint32_t fw[4] = {f.x, f.y, f.z, f.w};
+            if (n[i] >= 0) {
+                const uint32_t fw[4] = {f[i].x, f[i].y, f[i].z, f[i].w};
                 uint32_t ow[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float lo = gc * cv[2 * e] + gf * __uint_as_float(fw[e] << 16);
-                    const float hi = gc * cv[2 * e + 1] + gf * __uint_as_float(fw[e] & 0xFFFF0000u);
+                    const float lo = fmaf(gc[i], cv[2 * e], gf[i] * __uint_as_float(fw[e] << 16));
+                    const float hi = fmaf(gc[i], cv[2 * e + 1], gf[i] * __uint_as_float(fw[e] & 0xFFFF0000u));
                     const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
                     ow[e] = *reinterpret_cast<const uint32_t*>(&p);
                 }
                 r = make_uint4(ow[0], ow[1], ow[2], ow[3]);
             }
-            out[(row0 + o) * CH + j] = r;
+            out[(row0 + o0 + i * ROWS) * CH + j] = r;
         }
     }
 }
@@ -323,14 +354,14 @@ int grid_for(int64_t tasks, int per_sm) {
 }  // namespace
 
 cudaError_t launch_tile(const Dims& d, const Bf16Triple& t, cudaStream_t s) {
-    const int grid = grid_for(static_cast<int64_t>(d.B) * d.H * d.C * t.count, 8);
+    const int grid = grid_for(static_cast<int64_t>(d.B) * d.H * d.C * t.count, kLayoutPerSm);
     if (d.D == 128) tile_kernel<128><<<grid, kBlock, 0, s>>>(d, t);
     else tile_kernel<64><<<grid, kBlock, 0, s>>>(d, t);
     return cudaGetLastError();
 }
 
 cudaError_t launch_untile(const Dims& d, const uint16_t* xt, uint16_t* x, cudaStream_t s) {
-    const int grid = grid_for(static_cast<int64_t>(d.B) * d.H * d.C, 8);
+    const int grid = grid_for(static_cast<int64_t>(d.B) * d.H * d.C, kLayoutPerSm);
     if (d.D == 128) untile_kernel<128><<<grid, kBlock, 0, s>>>(d, xt, x);
     else untile_kernel<64><<<grid, kBlock, 0, s>>>(d, xt, x);
     return cudaGetLastError();
@@ -405,7 +436,7 @@ cudaError_t launch_gather_heads(const uint16_t* src, int64_t rows, int H, int h0
 
 cudaError_t launch_combine(const Dims& d, const float* o_coarse, const uint16_t* o_fine, const uint16_t* g_coarse,
                            const uint16_t* g_fine, uint16_t* o_tiled, cudaStream_t s) {
-    const int grid = grid_for(static_cast<int64_t>(d.B) * d.H * d.C, 8);
+    const int grid = grid_for(static_cast<int64_t>(d.B) * d.H * d.C, kCombinePerSm);
     if (d.D == 128) combine_kernel<128><<<grid, kBlock, 0, s>>>(d, o_coarse, o_fine, g_coarse, g_fine, o_tiled);
     else combine_kernel<64><<<grid, kBlock, 0, s>>>(d, o_coarse, o_fine, g_coarse, g_fine, o_tiled);
     return cudaGetLastError();
